@@ -1,0 +1,38 @@
+// Internal launchers shared between the kernel files and the C-ABI layer.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "kvs.h"
+#include "kvs_common.cuh"
+
+namespace kvs {
+
+// Window statistics: (m, l) per window query, o_bar and alpha_bar into the score workspace.
+cudaError_t launch_window_stats(const kvs_cache_desc& d, const void* K, const void* V,
+                                const float* logn, const int32_t* len, const void* Qw, int W,
+                                const ScoreLayout& Ly, char* ws, cudaStream_t st);
+
+// Pair norms, merge weight and score from alpha_bar / o_bar.
+cudaError_t launch_pair_score(const kvs_cache_desc& d, const void* K, const void* V,
+                              const int32_t* len, const int32_t* cand_begin, int n_recent,
+                              const ScoreLayout& Ly, char* ws, float* score, float* w_b,
+                              cudaStream_t st);
+
+// Selection to the budget, then merge + compaction (out-of-place or in-place).
+cudaError_t launch_select(const kvs_cache_desc& d, const float* score, const int32_t* len,
+                          const int32_t* cand_begin, int n_recent, const int32_t* target,
+                          int scope, const MergeLayout& Ly, char* ws, cudaStream_t st);
+
+cudaError_t launch_merge(const kvs_cache_desc& d, const void* K, const void* V, const float* logn,
+                         const float* score, const float* w_b, int scope, int T_cap_out,
+                         bool inplace, void* K_out, void* V_out, float* logn_out,
+                         int32_t* len_out, uint8_t* dbg_sel, int32_t* dbg_off, float* dbg_km,
+                         const MergeLayout& Ly, char* ws, cudaStream_t st);
+
+// Split-K GQA decode with fused split combine and optional append.
+cudaError_t launch_decode(const kvs_cache_desc& d, const void* q, void* K, void* V, float* logn,
+                          int32_t* len, const void* k_new, const void* v_new, void* out,
+                          const DecodeLayout& Ly, char* ws, cudaStream_t st);
+
+}  // namespace kvs

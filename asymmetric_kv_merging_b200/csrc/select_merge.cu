@@ -1,0 +1,648 @@
+// Pair selection to the budget, merge and compaction of one round.
+//
+// Merge rule: KVSlimmer deep dive ("论文专题讲解：KVSlimmer：非对称 KV 合并的数学与工程"),
+// §数学主线四 forward-only merged Key, k* = k_a + w_b (k_b - k_a). Values are kept
+// (核心判断: merge homogeneous Keys, preserve heterogeneous Values): a merged row stores
+// the count-weighted mean value and log(count) as a logit bias, which is exactly
+// attention over the original rows sharing k*.
+//
+// select_kernel (one CTA per selection unit):
+//   R = min(P, max(0, len - target)); the threshold key is the R-th smallest
+//   (score_key, index) found by a 4-pass 8-bit radix select; then per block of
+//   kMergePairsPerBlock pairs the counts of keys below / equal to the threshold,
+//   exclusive-scanned in unit order (h, p), give every merge CTA its offsets.
+// merge_kernel (out-of-place): one CTA per (head, pair block) plus copy CTAs for
+//   the protected prefix and suffix; a block-level ballot scan gives each pair's
+//   output row; rows move as 16-byte vectors, merged rows are computed in fp32.
+// merge_inplace_kernel: one CTA per head walks the span in order, staging each
+//   chunk in shared memory before writing it to lower (or equal) rows.
+#include "kvs_common.cuh"
+#include "kvs_kernels.h"
+
+namespace kvs {
+
+constexpr int kSelThreads = 1024;
+constexpr int kMergeThreads = 256;
+constexpr int kCopyRows = 256;
+// Pairs staged per in-place step: 32 for rows up to 256 bytes, 16 for 512-byte rows,
+// so the staging buffers stay within the default 48 KB of shared memory.
+template <typename T, int D>
+constexpr int inplace_chunk() { return D * (int)sizeof(T) <= 256 ? 32 : 16; }
+
+__device__ __forceinline__ int head_pairs(int L, int c0, int n_recent) {
+  int s = L - n_recent - c0;
+  return s > 0 ? s / 2 : 0;
+}
+
+// Block-wide exclusive scan of one int per thread (blockDim = kSelThreads).
+__device__ __forceinline__ int block_excl_scan(int v, int* warp_tot, int& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < (int)(blockDim.x >> 5) ? warp_tot[lane] : 0;
+    int wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int n = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += n;
+    }
+    warp_tot[lane] = wi - w;          // exclusive warp offsets
+    if (lane == 31) warp_tot[32] = wi;
+  }
+  __syncthreads();
+  int r = warp_tot[warp] + incl - v;
+  total = warp_tot[32];
+  __syncthreads();
+  return r;
+}
+
+__global__ void __launch_bounds__(kSelThreads)
+select_kernel(const float* __restrict__ score, const int32_t* __restrict__ len,
+              const int32_t* __restrict__ cand_begin, int n_recent,
+              const int32_t* __restrict__ target, int scope, int H_kv, int T_cap, int nblk,
+              SelUnit* __restrict__ sel, HeadInfo* __restrict__ hinfo, int2* __restrict__ blk,
+              int32_t* __restrict__ flags) {
+  __shared__ int hist[256];
+  __shared__ int warp_tot[33];
+  __shared__ int s_digit, s_before, s_R, s_P, s_bad;
+  const int u = blockIdx.x, tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
+  const int nh = scope == KVS_SCOPE_POOLED ? H_kv : 1;
+  const int h_first = scope == KVS_SCOPE_POOLED ? u * H_kv : u;
+  const int pstride = T_cap / 2;
+
+  if (tid == 0) {
+    long long tot_len = 0, tot_P = 0;
+    int bad = 0;
+    for (int i = 0; i < nh; ++i) {
+      const int hh = h_first + i;
+      const int L = len[hh], c0 = cand_begin[hh];
+      if (L < 0 || L > T_cap || c0 < 0) bad = 1;
+      const int P = bad ? 0 : head_pairs(L, c0, n_recent);
+      hinfo[hh].len_in = L;
+      hinfo[hh].P = P;
+      hinfo[hh].c0 = c0;
+      tot_len += L;
+      tot_P += P;
+    }
+    long long want = tot_len - (long long)target[u];
+    if (want < 0) want = 0;
+    if (want > tot_P) want = tot_P;
+    s_R = bad ? 0 : (int)want;
+    s_P = (int)tot_P;
+    s_bad = bad;
+    if (bad) {
+      set_flag(flags, KVS_FLAG_BAD_LENGTH);
+      for (int i = 0; i < nh; ++i) hinfo[h_first + i].len_in = -1;
+    }
+  }
+  __syncthreads();
+  if (s_bad) return;
+  const int R = s_R, Ptot = s_P;
+
+  uint32_t thr;
+  int need_eq;
+  if (R == 0) {
+    thr = 0u;
+    need_eq = 0;
+  } else if (R == Ptot) {
+    thr = 0xffffffffu;
+    need_eq = 0;
+  } else {
+    uint32_t prefix = 0u, pmask = 0u;
+    int rank = R;   // 1-based rank of the threshold among the unit's keys
+    for (int pass = 0; pass < 4; ++pass) {
+      const int shift = 24 - 8 * pass;
+      for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0;
+      __syncthreads();
+      for (int i = 0; i < nh; ++i) {
+        const int hh = h_first + i;
+        const int P = hinfo[hh].P;
+        const float* sc = score + (size_t)hh * pstride;
+        for (int p0 = 0; p0 < P; p0 += kSelThreads) {
+          const int p = p0 + tid;
+          const bool in = p < P;
+          const uint32_t key = in ? score_key(sc[p]) : 0u;
+          const bool match = in && ((key & pmask) == prefix);
+          const unsigned dg = (key >> shift) & 255u;
+          // aggregate equal digits inside the warp before the shared atomic
+          const unsigned peers = __match_any_sync(0xffffffffu, match ? dg : 0x100u + lane);
+          if (match && (__ffs(peers) - 1) == lane) atomicAdd(&hist[dg], __popc(peers));
+        }
+      }
+      __syncthreads();
+      if (warp == 0) {
+        int c[8], sum = 0;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) { c[k] = hist[lane * 8 + k]; sum += c[k]; }
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          int n = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += n;
+        }
+        const int excl = incl - sum;
+        if (excl < rank && rank <= incl) {
+          int acc = excl;
+          for (int k = 0; k < 8; ++k) {
+            if (rank <= acc + c[k]) { s_digit = lane * 8 + k; s_before = acc; break; }
+            acc += c[k];
+          }
+        }
+      }
+      __syncthreads();
+      prefix |= (uint32_t)s_digit << shift;
+      pmask |= 0xffu << shift;
+      rank -= s_before;
+      __syncthreads();
+    }
+    thr = prefix;
+    need_eq = rank;
+  }
+
+  // Per block counts of keys below / equal to the threshold, (h, block) order.
+  const int nent = nh * nblk;
+  for (int e0 = 0; e0 < nent; e0 += kSelThreads / 32) {
+    const int e = e0 + warp;
+    if (e < nent) {
+      const int i = e / nblk, j = e - i * nblk;
+      const int hh = h_first + i;
+      const int P = hinfo[hh].P;
+      const float* sc = score + (size_t)hh * pstride;
+      int lt = 0, eq = 0;
+      for (int k = 0; k < kMergePairsPerBlock; k += 32) {
+        const int p = j * kMergePairsPerBlock + k + lane;
+        const bool in = p < P;
+        const uint32_t key = in ? score_key(sc[p]) : 0u;
+        lt += __popc(__ballot_sync(0xffffffffu, in && key < thr));
+        eq += __popc(__ballot_sync(0xffffffffu, in && key == thr));
+      }
+      if (lane == 0) blk[(size_t)hh * nblk + j] = make_int2(lt, eq);
+    }
+  }
+  __syncthreads();
+  // Unit-wide exclusive scans of both counts.
+  int carry_lt = 0, carry_eq = 0;
+  for (int e0 = 0; e0 < nent; e0 += kSelThreads) {
+    const int e = e0 + tid;
+    const int i = e / nblk, j = e - i * nblk;
+    int2 v = make_int2(0, 0);
+    if (e < nent) v = blk[(size_t)(h_first + i) * nblk + j];
+    int tl, te;
+    const int xl = block_excl_scan(v.x, warp_tot, tl);
+    const int xe = block_excl_scan(v.y, warp_tot, te);
+    if (e < nent) blk[(size_t)(h_first + i) * nblk + j] = make_int2(carry_lt + xl, carry_eq + xe);
+    carry_lt += tl;
+    carry_eq += te;
+  }
+  __syncthreads();
+  // Per head: scan values at its first block and its merged-pair count.
+  if (tid < nh) {
+    const int hh = h_first + tid;
+    const int2 first = blk[(size_t)hh * nblk];
+    const int2 next = (tid + 1 < nh) ? blk[(size_t)(hh + 1) * nblk] : make_int2(carry_lt, carry_eq);
+    const int lt_h = next.x - first.x;
+    const int eq_sel = min(need_eq, next.y) - min(need_eq, first.y);
+    hinfo[hh].lt0 = first.x;
+    hinfo[hh].eq0 = first.y;
+    hinfo[hh].R = lt_h + eq_sel;
+  }
+  if (tid == 0) {
+    sel[u].thr_key = thr;
+    sel[u].need_eq = need_eq;
+    sel[u].R = R;
+    sel[u].P = Ptot;
+  }
+}
+
+// Copy `rows` consecutive rows of K, V (and logn) from row `src` to row `dst`.
+template <typename T, int D>
+__device__ __forceinline__ void copy_rows(const T* __restrict__ Kh, const T* __restrict__ Vh,
+                                          const float* __restrict__ lnh, T* __restrict__ Ko,
+                                          T* __restrict__ Vo, float* __restrict__ lno, int src,
+                                          int dst, int rows) {
+  constexpr int VPR = D * (int)sizeof(T) / 16;
+  const int nvec = rows * VPR;
+  for (int i = threadIdx.x; i < nvec; i += blockDim.x) {
+    const int r = i / VPR, c = i - r * VPR;
+    const size_t so = ((size_t)(src + r) * D) * sizeof(T) + (size_t)c * 16;
+    const size_t dof = ((size_t)(dst + r) * D) * sizeof(T) + (size_t)c * 16;
+    store_raw(reinterpret_cast<char*>(Ko) + dof, load_raw(reinterpret_cast<const char*>(Kh) + so));
+    store_raw(reinterpret_cast<char*>(Vo) + dof, load_raw(reinterpret_cast<const char*>(Vh) + so));
+  }
+  for (int r = threadIdx.x; r < rows; r += blockDim.x) lno[dst + r] = lnh ? lnh[src + r] : 0.f;
+}
+
+// Selection flags and output rows of up to 128 consecutive pairs (threads < 128).
+struct PairPlan {
+  int off;
+  bool sel;
+};
+
+__device__ __forceinline__ PairPlan plan_pair(int t, int pbase, int P, const float* sc,
+                                              const SelUnit& su, int lt_before, int eq_unit,
+                                              const HeadInfo& hi, int* s_cnt) {
+  // s_cnt: 8 ints of shared scratch (4 warps x {lt, eq}); all 128 threads call this.
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int p = pbase + t;
+  const bool in = p < P;
+  const uint32_t key = in ? score_key(sc[p]) : 0xffffffffu;
+  const bool lt = in && key < su.thr_key;
+  const bool eq = in && key == su.thr_key;
+  const unsigned blt = __ballot_sync(0xffffffffu, lt);
+  const unsigned beq = __ballot_sync(0xffffffffu, eq);
+  if (lane == 0) { s_cnt[warp * 2] = __popc(blt); s_cnt[warp * 2 + 1] = __popc(beq); }
+  asm volatile("bar.sync 1, 128;");
+  int wl = 0, we = 0;
+  for (int w = 0; w < warp; ++w) { wl += s_cnt[w * 2]; we += s_cnt[w * 2 + 1]; }
+  const unsigned lower = (1u << lane) - 1u;
+  const int lt_rank = wl + __popc(blt & lower);
+  const int eq_rank = we + __popc(beq & lower);
+  const int eqg = eq_unit + eq_rank;
+  PairPlan pp;
+  pp.sel = lt || (eq && eqg < su.need_eq);
+  const int sel_before = lt_before + lt_rank + min(su.need_eq, eqg) - min(su.need_eq, hi.eq0);
+  pp.off = hi.c0 + 2 * p - sel_before;
+  asm volatile("bar.sync 1, 128;");
+  return pp;
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kMergeThreads)
+merge_kernel(const T* __restrict__ K, const T* __restrict__ V, const float* __restrict__ logn,
+             const float* __restrict__ score, const float* __restrict__ w_b, int scope, int H_kv,
+             int T_cap, int T_cap_out, int nblk, const SelUnit* __restrict__ sel,
+             const HeadInfo* __restrict__ hinfo, const int2* __restrict__ blk,
+             T* __restrict__ K_out, T* __restrict__ V_out, float* __restrict__ logn_out,
+             int32_t* __restrict__ len_out, uint8_t* __restrict__ dbg_sel,
+             int32_t* __restrict__ dbg_off, float* __restrict__ dbg_km,
+             int32_t* __restrict__ flags) {
+  constexpr int MB = kMergePairsPerBlock;
+  constexpr int VN = Vec16<T>::n;
+  constexpr int LPR = D / VN;
+  __shared__ int s_off[MB];
+  __shared__ unsigned char s_sel[MB];
+  __shared__ float s_w[MB];
+  __shared__ int s_cnt[8];
+
+  const int head = blockIdx.y;
+  const HeadInfo hi = hinfo[head];
+  if (hi.len_in < 0) return;
+  const int u = scope == KVS_SCOPE_POOLED ? head / H_kv : head;
+  const SelUnit su = sel[u];
+  const int L = hi.len_in, P = hi.P, R = hi.R, c0 = hi.c0;
+  const int L_out = L - R;
+  if (L_out > T_cap_out) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) set_flag(flags, KVS_FLAG_OUT_CAPACITY);
+    return;
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0) len_out[head] = L_out;
+
+  const T* Kh = K + (size_t)head * T_cap * D;
+  const T* Vh = V + (size_t)head * T_cap * D;
+  const float* lnh = logn ? logn + (size_t)head * T_cap : nullptr;
+  T* Ko = K_out + (size_t)head * T_cap_out * D;
+  T* Vo = V_out + (size_t)head * T_cap_out * D;
+  float* lno = logn_out + (size_t)head * T_cap_out;
+  const int x = blockIdx.x;
+
+  if (x >= nblk) {   // protected rows: prefix [0, c0) in place, suffix shifted down by R
+    const int ct = x - nblk;
+    const int r0 = ct * kCopyRows;
+    const int pre = min(c0, L);     // a span start past the end leaves only [0, L)
+    if (r0 < pre) copy_rows<T, D>(Kh, Vh, lnh, Ko, Vo, lno, r0, r0, min(kCopyRows, pre - r0));
+    const int s0 = c0 + 2 * P + r0;
+    if (s0 < L) copy_rows<T, D>(Kh, Vh, lnh, Ko, Vo, lno, s0, s0 - R, min(kCopyRows, L - s0));
+    return;
+  }
+
+  const int pbase = x * MB;
+  if (pbase >= P) return;
+  const float* sc = score + (size_t)head * (T_cap / 2);
+  const float* wb = w_b + (size_t)head * (T_cap / 2);
+  if (threadIdx.x < MB) {
+    const int2 bs = blk[(size_t)head * nblk + x];
+    const int t = threadIdx.x;
+    const PairPlan pp = plan_pair(t, pbase, P, sc, su, bs.x - hi.lt0, bs.y, hi, s_cnt);
+    s_off[t] = pp.off;
+    s_sel[t] = pp.sel ? 1 : 0;
+    const int p = pbase + t;
+    s_w[t] = (p < P) ? wb[p] : 0.f;
+    if (p < P) {
+      if (dbg_sel) dbg_sel[(size_t)head * (T_cap / 2) + p] = pp.sel ? 1 : 0;
+      if (dbg_off) dbg_off[(size_t)head * (T_cap / 2) + p] = pp.off;
+    }
+  }
+  __syncthreads();
+
+  const int nvalid = min(MB, P - pbase);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  constexpr int WARPS = kMergeThreads / 32;
+  if constexpr (LPR <= 16) {
+    constexpr int PPI = 16 / LPR;                   // pairs per warp iteration
+    const int slot = lane / (2 * LPR), r = (lane / LPR) & 1, c = lane % LPR;
+    for (int base = warp * PPI; base < nvalid; base += WARPS * PPI) {
+      const int t = base + slot;
+      const bool valid = t < nvalid;
+      const int p = pbase + t;
+      const int row = c0 + 2 * p + r;
+      uint4 kr = make_uint4(0, 0, 0, 0), vr = make_uint4(0, 0, 0, 0);
+      float lr = 0.f;
+      if (valid) {
+        kr = load_raw(Kh + (size_t)row * D + c * VN);
+        vr = load_raw(Vh + (size_t)row * D + c * VN);
+        lr = lnh ? lnh[row] : 0.f;
+      }
+      uint4 kp, vp;
+      kp.x = __shfl_xor_sync(0xffffffffu, kr.x, LPR); kp.y = __shfl_xor_sync(0xffffffffu, kr.y, LPR);
+      kp.z = __shfl_xor_sync(0xffffffffu, kr.z, LPR); kp.w = __shfl_xor_sync(0xffffffffu, kr.w, LPR);
+      vp.x = __shfl_xor_sync(0xffffffffu, vr.x, LPR); vp.y = __shfl_xor_sync(0xffffffffu, vr.y, LPR);
+      vp.z = __shfl_xor_sync(0xffffffffu, vr.z, LPR); vp.w = __shfl_xor_sync(0xffffffffu, vr.w, LPR);
+      const float lp = __shfl_xor_sync(0xffffffffu, lr, LPR);
+      if (!valid) continue;
+      const int off = s_off[t];
+      if (s_sel[t]) {
+        if (r == 0) {
+          float ka[VN], kb[VN], va[VN], vb[VN], ko[VN], vo[VN];
+          load_vec(reinterpret_cast<const T*>(&kr), ka);
+          load_vec(reinterpret_cast<const T*>(&kp), kb);
+          load_vec(reinterpret_cast<const T*>(&vr), va);
+          load_vec(reinterpret_cast<const T*>(&vp), vb);
+          const float w = s_w[t];
+          const float na = expf(lr), nb = expf(lp);
+          const float inv = 1.f / (na + nb);
+#pragma unroll
+          for (int e = 0; e < VN; ++e) {
+            ko[e] = fmaf(w, kb[e] - ka[e], ka[e]);
+            vo[e] = (na * va[e] + nb * vb[e]) * inv;
+          }
+          store_vec(Ko + (size_t)off * D + c * VN, ko);
+          store_vec(Vo + (size_t)off * D + c * VN, vo);
+          if (c == 0) lno[off] = logf(na + nb);
+          if (dbg_km) {
+            float* dk = dbg_km + ((size_t)head * (T_cap / 2) + p) * D + c * VN;
+#pragma unroll
+            for (int e = 0; e < VN; e += 4) *reinterpret_cast<float4*>(dk + e) = make_float4(ko[e], ko[e + 1], ko[e + 2], ko[e + 3]);
+          }
+        }
+      } else {
+        store_raw(Ko + (size_t)(off + r) * D + c * VN, kr);
+        store_raw(Vo + (size_t)(off + r) * D + c * VN, vr);
+        if (c == 0) lno[off + r] = lr;
+      }
+    }
+  } else {
+    // LPR == 32: one lane holds the same 16-byte slice of both rows.
+    for (int t = warp; t < nvalid; t += WARPS) {
+      const int p = pbase + t;
+      const int a = c0 + 2 * p;
+      const uint4 ka_r = load_raw(Kh + (size_t)a * D + lane * VN);
+      const uint4 kb_r = load_raw(Kh + (size_t)(a + 1) * D + lane * VN);
+      const uint4 va_r = load_raw(Vh + (size_t)a * D + lane * VN);
+      const uint4 vb_r = load_raw(Vh + (size_t)(a + 1) * D + lane * VN);
+      const float la = lnh ? lnh[a] : 0.f, lb = lnh ? lnh[a + 1] : 0.f;
+      const int off = s_off[t];
+      if (s_sel[t]) {
+        float ka[VN], kb[VN], va[VN], vb[VN], ko[VN], vo[VN];
+        load_vec(reinterpret_cast<const T*>(&ka_r), ka);
+        load_vec(reinterpret_cast<const T*>(&kb_r), kb);
+        load_vec(reinterpret_cast<const T*>(&va_r), va);
+        load_vec(reinterpret_cast<const T*>(&vb_r), vb);
+        const float w = s_w[t];
+        const float na = expf(la), nb = expf(lb);
+        const float inv = 1.f / (na + nb);
+#pragma unroll
+        for (int e = 0; e < VN; ++e) {
+          ko[e] = fmaf(w, kb[e] - ka[e], ka[e]);
+          vo[e] = (na * va[e] + nb * vb[e]) * inv;
+        }
+        store_vec(Ko + (size_t)off * D + lane * VN, ko);
+        store_vec(Vo + (size_t)off * D + lane * VN, vo);
+        if (lane == 0) lno[off] = logf(na + nb);
+        if (dbg_km) {
+          float* dk = dbg_km + ((size_t)head * (T_cap / 2) + p) * D + lane * VN;
+#pragma unroll
+          for (int e = 0; e < VN; e += 4) *reinterpret_cast<float4*>(dk + e) = make_float4(ko[e], ko[e + 1], ko[e + 2], ko[e + 3]);
+        }
+      } else {
+        store_raw(Ko + (size_t)off * D + lane * VN, ka_r);
+        store_raw(Ko + (size_t)(off + 1) * D + lane * VN, kb_r);
+        store_raw(Vo + (size_t)off * D + lane * VN, va_r);
+        store_raw(Vo + (size_t)(off + 1) * D + lane * VN, vb_r);
+        if (lane == 0) { lno[off] = la; lno[off + 1] = lb; }
+      }
+    }
+  }
+}
+
+// In-place variant: one CTA per head; each chunk is read completely into shared
+// memory before any of its rows is written, and rows only move to lower indices,
+// so no unread row is ever overwritten.
+template <typename T, int D>
+__global__ void __launch_bounds__(kMergeThreads)
+merge_inplace_kernel(T* __restrict__ K, T* __restrict__ V, float* __restrict__ logn,
+                     const float* __restrict__ score, const float* __restrict__ w_b, int scope,
+                     int H_kv, int T_cap, const SelUnit* __restrict__ sel,
+                     const HeadInfo* __restrict__ hinfo, int32_t* __restrict__ len,
+                     uint8_t* __restrict__ dbg_sel, int32_t* __restrict__ dbg_off,
+                     float* __restrict__ dbg_km, int32_t* __restrict__ flags) {
+  constexpr int CH = inplace_chunk<T, D>();
+  constexpr int VPR = D * (int)sizeof(T) / 16;
+  constexpr int VN = Vec16<T>::n;
+  extern __shared__ __align__(16) unsigned char ism[];
+  uint4* sK = reinterpret_cast<uint4*>(ism);                 // [2*CH][VPR]
+  uint4* sV = sK + 2 * CH * VPR;                             // [2*CH][VPR]
+  float* sL = reinterpret_cast<float*>(sV + 2 * CH * VPR);   // [2*CH]
+  __shared__ int s_off[32];
+  __shared__ unsigned char s_sel[32];
+  __shared__ float s_w[32];
+  __shared__ int s_lt, s_eq;
+
+  const int head = blockIdx.x;
+  const HeadInfo hi = hinfo[head];
+  if (hi.len_in < 0) return;
+  const int L = hi.len_in, P = hi.P, R = hi.R, c0 = hi.c0;
+  if (L - c0 > kInplaceMaxSpan) {
+    if (threadIdx.x == 0) set_flag(flags, KVS_FLAG_INPLACE_SPAN);
+    return;
+  }
+  const int u = scope == KVS_SCOPE_POOLED ? head / H_kv : head;
+  const SelUnit su = sel[u];
+  T* Kh = K + (size_t)head * T_cap * D;
+  T* Vh = V + (size_t)head * T_cap * D;
+  float* lnh = logn + (size_t)head * T_cap;
+  const float* sc = score + (size_t)head * (T_cap / 2);
+  const float* wb = w_b + (size_t)head * (T_cap / 2);
+  const int tid = threadIdx.x, lane = tid & 31;
+  if (tid == 0) { s_lt = 0; s_eq = hi.eq0; }
+  __syncthreads();
+
+  if (R > 0) {
+    for (int pb = 0; pb < P; pb += CH) {
+      const int np = min(CH, P - pb);
+      if (tid < 32) {   // one warp plans the chunk (CH <= 32)
+        const int p = pb + lane;
+        const bool in = lane < np;
+        const uint32_t key = in ? score_key(sc[p]) : 0xffffffffu;
+        const bool lt = in && key < su.thr_key;
+        const bool eq = in && key == su.thr_key;
+        const unsigned blt = __ballot_sync(0xffffffffu, lt);
+        const unsigned beq = __ballot_sync(0xffffffffu, eq);
+        const unsigned lower = (1u << lane) - 1u;
+        const int eqg = s_eq + __popc(beq & lower);
+        const bool sl = lt || (eq && eqg < su.need_eq);
+        const int sel_before = s_lt + __popc(blt & lower) + min(su.need_eq, eqg) -
+                               min(su.need_eq, hi.eq0);
+        const int off = c0 + 2 * p - sel_before;
+        s_off[lane] = off;
+        s_sel[lane] = sl ? 1 : 0;
+        s_w[lane] = in ? wb[p] : 0.f;
+        if (in) {
+          if (dbg_sel) dbg_sel[(size_t)head * (T_cap / 2) + p] = sl ? 1 : 0;
+          if (dbg_off) dbg_off[(size_t)head * (T_cap / 2) + p] = off;
+        }
+        __syncwarp();
+        if (lane == 0) { s_lt += __popc(blt); s_eq += __popc(beq); }
+      }
+      const int row0 = c0 + 2 * pb;
+      for (int i = tid; i < 2 * np * VPR; i += blockDim.x) {
+        const int r = i / VPR, c = i - r * VPR;
+        sK[i] = *reinterpret_cast<const uint4*>(Kh + (size_t)(row0 + r) * D + c * VN);
+        sV[i] = *reinterpret_cast<const uint4*>(Vh + (size_t)(row0 + r) * D + c * VN);
+      }
+      for (int r = tid; r < 2 * np; r += blockDim.x) sL[r] = lnh[row0 + r];
+      __syncthreads();
+      for (int i = tid; i < np * VPR; i += blockDim.x) {
+        const int t = i / VPR, c = i - t * VPR;
+        const int off = s_off[t];
+        const uint4 ka_r = sK[(2 * t) * VPR + c], kb_r = sK[(2 * t + 1) * VPR + c];
+        const uint4 va_r = sV[(2 * t) * VPR + c], vb_r = sV[(2 * t + 1) * VPR + c];
+        if (s_sel[t]) {
+          float ka[VN], kb[VN], va[VN], vb[VN], ko[VN], vo[VN];
+          load_vec(reinterpret_cast<const T*>(&ka_r), ka);
+          load_vec(reinterpret_cast<const T*>(&kb_r), kb);
+          load_vec(reinterpret_cast<const T*>(&va_r), va);
+          load_vec(reinterpret_cast<const T*>(&vb_r), vb);
+          const float w = s_w[t];
+          const float na = expf(sL[2 * t]), nb = expf(sL[2 * t + 1]);
+          const float inv = 1.f / (na + nb);
+#pragma unroll
+          for (int e = 0; e < VN; ++e) {
+            ko[e] = fmaf(w, kb[e] - ka[e], ka[e]);
+            vo[e] = (na * va[e] + nb * vb[e]) * inv;
+          }
+          store_vec(Kh + (size_t)off * D + c * VN, ko);
+          store_vec(Vh + (size_t)off * D + c * VN, vo);
+          if (c == 0) lnh[off] = logf(na + nb);
+          if (dbg_km) {
+            float* dk = dbg_km + ((size_t)head * (T_cap / 2) + pb + t) * D + c * VN;
+#pragma unroll
+            for (int e = 0; e < VN; e += 4) *reinterpret_cast<float4*>(dk + e) = make_float4(ko[e], ko[e + 1], ko[e + 2], ko[e + 3]);
+          }
+        } else {
+          *reinterpret_cast<uint4*>(Kh + (size_t)off * D + c * VN) = ka_r;
+          *reinterpret_cast<uint4*>(Kh + (size_t)(off + 1) * D + c * VN) = kb_r;
+          *reinterpret_cast<uint4*>(Vh + (size_t)off * D + c * VN) = va_r;
+          *reinterpret_cast<uint4*>(Vh + (size_t)(off + 1) * D + c * VN) = vb_r;
+          if (c == 0) { lnh[off] = sL[2 * t]; lnh[off + 1] = sL[2 * t + 1]; }
+        }
+      }
+      __syncthreads();
+    }
+    // suffix rows move down by R, chunk by chunk in increasing order
+    for (int s0 = c0 + 2 * P; s0 < L; s0 += 2 * CH) {
+      const int nr = min(2 * CH, L - s0);
+      for (int i = tid; i < nr * VPR; i += blockDim.x) {
+        const int r = i / VPR, c = i - r * VPR;
+        sK[i] = *reinterpret_cast<const uint4*>(Kh + (size_t)(s0 + r) * D + c * VN);
+        sV[i] = *reinterpret_cast<const uint4*>(Vh + (size_t)(s0 + r) * D + c * VN);
+      }
+      for (int r = tid; r < nr; r += blockDim.x) sL[r] = lnh[s0 + r];
+      __syncthreads();
+      for (int i = tid; i < nr * VPR; i += blockDim.x) {
+        const int r = i / VPR, c = i - r * VPR;
+        *reinterpret_cast<uint4*>(Kh + (size_t)(s0 + r - R) * D + c * VN) = sK[i];
+        *reinterpret_cast<uint4*>(Vh + (size_t)(s0 + r - R) * D + c * VN) = sV[i];
+      }
+      for (int r = tid; r < nr; r += blockDim.x) lnh[s0 + r - R] = sL[r];
+      __syncthreads();
+    }
+  } else if (dbg_sel || dbg_off) {
+    for (int p = tid; p < P; p += blockDim.x) {
+      if (dbg_sel) dbg_sel[(size_t)head * (T_cap / 2) + p] = 0;
+      if (dbg_off) dbg_off[(size_t)head * (T_cap / 2) + p] = c0 + 2 * p;
+    }
+  }
+  __syncthreads();
+  if (tid == 0) len[head] = L - R;
+}
+
+cudaError_t launch_select(const kvs_cache_desc& d, const float* score, const int32_t* len,
+                          const int32_t* cand_begin, int n_recent, const int32_t* target,
+                          int scope, const MergeLayout& Ly, char* ws, cudaStream_t st) {
+  const int units = scope == KVS_SCOPE_POOLED ? d.B : d.B * d.H_kv;
+  select_kernel<<<units, kSelThreads, 0, st>>>(
+      score, len, cand_begin, n_recent, target, scope, d.H_kv, d.T_cap, Ly.nblk,
+      reinterpret_cast<SelUnit*>(ws + Ly.sel), reinterpret_cast<HeadInfo*>(ws + Ly.head),
+      reinterpret_cast<int2*>(ws + Ly.blk), reinterpret_cast<int32_t*>(ws));
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+template <typename T, int D>
+static cudaError_t launch_merge_t(const kvs_cache_desc& d, const void* K, const void* V,
+                                  const float* logn, const float* score, const float* w_b,
+                                  int scope, int T_cap_out, bool inplace, void* K_out,
+                                  void* V_out, float* logn_out, int32_t* len_out,
+                                  uint8_t* dbg_sel, int32_t* dbg_off, float* dbg_km,
+                                  const MergeLayout& Ly, char* ws, cudaStream_t st) {
+  const int heads = d.B * d.H_kv;
+  const SelUnit* sel = reinterpret_cast<const SelUnit*>(ws + Ly.sel);
+  const HeadInfo* hinfo = reinterpret_cast<const HeadInfo*>(ws + Ly.head);
+  const int2* blk = reinterpret_cast<const int2*>(ws + Ly.blk);
+  int32_t* flags = reinterpret_cast<int32_t*>(ws);
+  if (inplace) {
+    constexpr int VPR = D * (int)sizeof(T) / 16;
+    constexpr int CH = inplace_chunk<T, D>();
+    constexpr size_t smem = (size_t)2 * (2 * CH * VPR) * 16 + 2 * CH * sizeof(float);
+    static_assert(smem + 512 <= 48 * 1024, "in-place staging must fit the default shared-memory limit");
+    auto kfn = merge_inplace_kernel<T, D>;
+    kfn<<<heads, kMergeThreads, smem, st>>>((T*)K_out, (T*)V_out, logn_out, score, w_b, scope,
+                                            d.H_kv, d.T_cap, sel, hinfo, len_out, dbg_sel,
+                                            dbg_off, dbg_km, flags);
+    count_launches(1);
+    return cudaGetLastError();
+  }
+  const int ncopy = (d.T_cap + kCopyRows - 1) / kCopyRows;
+  dim3 grid(Ly.nblk + ncopy, heads);
+  merge_kernel<T, D><<<grid, kMergeThreads, 0, st>>>(
+      (const T*)K, (const T*)V, logn, score, w_b, scope, d.H_kv, d.T_cap, T_cap_out, Ly.nblk,
+      sel, hinfo, blk, (T*)K_out, (T*)V_out, logn_out, len_out, dbg_sel, dbg_off, dbg_km, flags);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_merge(const kvs_cache_desc& d, const void* K, const void* V, const float* logn,
+                         const float* score, const float* w_b, int scope, int T_cap_out,
+                         bool inplace, void* K_out, void* V_out, float* logn_out,
+                         int32_t* len_out, uint8_t* dbg_sel, int32_t* dbg_off, float* dbg_km,
+                         const MergeLayout& Ly, char* ws, cudaStream_t st) {
+#define KVS_MERGE_ARGS K, V, logn, score, w_b, scope, T_cap_out, inplace, K_out, V_out, logn_out, \
+                       len_out, dbg_sel, dbg_off, dbg_km, Ly, ws, st
+  if (d.dtype == KVS_BF16) {
+    if (d.d == 128) return launch_merge_t<bf16, 128>(d, KVS_MERGE_ARGS);
+    return launch_merge_t<bf16, 64>(d, KVS_MERGE_ARGS);
+  }
+  if (d.d == 128) return launch_merge_t<float, 128>(d, KVS_MERGE_ARGS);
+  return launch_merge_t<float, 64>(d, KVS_MERGE_ARGS);
+#undef KVS_MERGE_ARGS
+}
+
+}  // namespace kvs

@@ -74,8 +74,9 @@ class Workload:
 
     @property
     def T_cap(self) -> int:
-        """Cache capacity: prefill plus room for every decode append."""
-        return self.T + self.n_decode
+        """Cache capacity: prefill plus room for every decode append, rounded up to even."""
+        c = self.T + self.n_decode
+        return c + c % 2
 
 
 WORKLOADS = [
@@ -202,6 +203,7 @@ def make_layer(w: Workload, layer: int = 0, device="cpu", T_cap: Optional[int] =
     if lens is None:
         lens = sequence_lengths(w)
     T_cap = T_cap if T_cap is not None else int(lens.max()) + w.n_decode
+    T_cap += T_cap % 2            # caches hold an even number of rows (whole pairs)
     dt = w.torch_dtype
     W_K = [projection(w.d_model, w.d, False, gen, device) for _ in range(w.H_kv)]
     W_V = [projection(w.d_model, w.d, True, gen, device) for _ in range(w.H_kv)]

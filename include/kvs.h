@@ -1,0 +1,200 @@
+/*
+ * kvs.h -- C ABI of the KVSlimmer asymmetric-KV-merging hot path on B200 (sm_100a).
+ *
+ * The method: "论文专题讲解：KVSlimmer：非对称 KV 合并的数学与工程" (blog deep dive of
+ * arXiv 2603.00907) and the abstract pages of "KVSlimmer: Theoretical Insights and
+ * Practical Optimizations for Asymmetric KV Merging". Adjacent Keys (k_m, k_m+1) of
+ * a cache K = [k_1..k_n] are merged with forward-only closed-form weights (§数学主线二,
+ * §数学主线四); Values are preserved (核心判断: merge homogeneous Keys, keep
+ * heterogeneous Values); decode attention runs over the merged cache (Figure 5,
+ * decoder stage).
+ *
+ * Data layout (all device memory, row-major, caller-owned):
+ *   cache K, V      [B, H_kv, T_cap, d]   element type kvs_dtype (fp32 or bf16)
+ *   log-count logn  [B, H_kv, T_cap]      fp32; log(number of original tokens a row
+ *                                         stands for); 0 for unmerged rows. NULL on
+ *                                         input means "all counts are 1".
+ *   lengths len     [B, H_kv]             int32; valid prefix of each head's rows
+ *   window queries  [B, H_q, W, d]        query head hq belongs to KV head hq / G,
+ *                                         G = H_q / H_kv; query j sits at cache
+ *                                         position len - W + j and sees positions
+ *                                         <= its own.
+ *   decode queries  [B, H_q, d]; decode output [B, H_q, d] (same dtype as the cache)
+ *   pair arrays     [B, H_kv, T_cap / 2]  fp32, indexed by pair p; pair p of a head is
+ *                                         the rows (c0 + 2p, c0 + 2p + 1), c0 = cand_begin.
+ *
+ * Candidate span of a head: [cand_begin, len - n_recent). Rows before it (sink
+ * tokens; the pages keep 32, §实验设置) and after it (the recent window, §工程上怎么用)
+ * are never merged. P = max(0, (len - n_recent - cand_begin) / 2) pairs; an odd
+ * leftover row is never merged.
+ *
+ * Streams and memory: every call is asynchronous on `stream`, allocates nothing,
+ * keeps no state between calls and never synchronises, unless its comment says
+ * otherwise. Pointers must be 16-byte aligned (cache, query and output tensors)
+ * or 4-byte aligned (int32 / fp32 arrays); the workspace 256-byte aligned.
+ *
+ * Errors: argument errors are found on the host and returned before anything is
+ * launched. Launch failures return KVS_ERR_CUDA. Conditions only the device can
+ * see (a length outside [0, T_cap], an output that would not fit) are skipped by
+ * the kernels and recorded as bits in the workspace's device flag word, read with
+ * kvs_device_flags().
+ */
+#ifndef KVS_H_
+#define KVS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  KVS_OK = 0,
+  KVS_ERR_INVALID_ARG = 1,   /* NULL pointer, non-positive size, misalignment, bad W / n_recent */
+  KVS_ERR_UNSUPPORTED = 2,   /* head dim, dtype, group size or window size not built */
+  KVS_ERR_BUDGET = 3,        /* (device flag) a budget that the candidate pairs cannot reach */
+  KVS_ERR_WORKSPACE = 4,     /* workspace NULL, too small or not 256-byte aligned */
+  KVS_ERR_ALIAS = 5,         /* an output overlaps an input in a way the call does not allow */
+  KVS_ERR_CUDA = 6           /* a CUDA runtime call or kernel launch failed */
+} kvs_status;
+
+typedef enum { KVS_F32 = 0, KVS_BF16 = 1 } kvs_dtype;
+
+/* Shape of a cache. d in {64, 128}; H_q a multiple of H_kv with G = H_q / H_kv <= 8;
+   T_cap even. */
+typedef struct {
+  int32_t B, H_kv, H_q, d, T_cap;
+  int32_t dtype; /* kvs_dtype */
+} kvs_cache_desc;
+
+typedef struct CUstream_st* kvs_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+
+enum { KVS_OP_SCORE = 0, KVS_OP_MERGE = 1, KVS_OP_DECODE = 2 };
+enum { KVS_SCOPE_HEAD = 0, KVS_SCOPE_POOLED = 1 };
+
+/* Device flag bits (see kvs_device_flags). */
+enum {
+  KVS_FLAG_BAD_LENGTH = 1,      /* a len[] value was < 0 or > T_cap; that head was skipped */
+  KVS_FLAG_OUT_CAPACITY = 2,    /* a merged head or an append did not fit the output capacity */
+  KVS_FLAG_INPLACE_SPAN = 4,    /* in-place merge on a span longer than it supports; head skipped */
+  KVS_FLAG_NONFINITE_STATS = 8  /* a window query had no finite softmax normaliser */
+};
+
+/*
+ * Bytes of workspace `op` needs for caches of shape `desc` (and window W for
+ * KVS_OP_SCORE). Returns 0 for an invalid shape. Every layout begins with the
+ * same persistent region: the device flag word (first 256 bytes) and one decode
+ * arrival counter per KV head (the next 256-byte-aligned block). Zero the whole
+ * workspace once (cudaMemset) before its first use; every call leaves the
+ * persistent region valid for the next call, so one zeroed workspace, sized for
+ * the largest op, serves all three ops on one stream. Calls that share a
+ * workspace must not overlap in time.
+ */
+size_t kvs_workspace_size(const kvs_cache_desc* desc, int32_t W, int32_t op);
+
+/*
+ * kvs_score_pairs -- one scoring pass: window statistics, then every candidate
+ * pair's forward-only Hessian norms, merge weight and score.
+ *
+ *   alpha_bar_t = mean over the window queries of softmax_t(q k_t^T / sqrt(d) + logn_t)
+ *   o_bar       = mean over the window queries of o_q = sum_t alpha_t v_t
+ *       (attention forward: §数学主线三; averaging the window: the one-query formulas
+ *        of the pages applied to the window mean)
+ *   N11 = |a_a (1 - 2 a_a)| |v_a - o_bar|,  N22 = |a_b (1 - 2 a_b)| |v_b - o_bar|,
+ *   N12 = a_a a_b |v_a + v_b - 2 o_bar|      (|c11|, |c22|, |c12| of §数学主线四)
+ *   D = N11 - 2 N12 + N22;  w_b = (N22 - N12) / D;
+ *   score = |k_b - k_a|^2 (N11 N22 - N12^2) / D  (minimum of the §数学主线二 objective
+ *       with the forward-only scalars); when D <= 1e-6 (N11 + N22) or a term is not
+ *       finite: w_b = 1/2, score = |k_b - k_a|^2 (N11 + 2 N12 + N22) / 4.
+ *
+ * In:  K, V [B,H_kv,T_cap,d]; logn (nullable); len [B*H_kv]; cand_begin [B*H_kv];
+ *      n_recent >= 0; Q_win [B,H_q,W,d], 1 <= W, G*W <= 256.
+ * Out: score, w_b [B,H_kv,T_cap/2] fp32 (entries p >= P of a head are not written).
+ * Workspace: kvs_workspace_size(desc, W, KVS_OP_SCORE) bytes.
+ */
+kvs_status kvs_score_pairs(const kvs_cache_desc* desc, const void* K, const void* V,
+                           const float* logn, const int32_t* len, const int32_t* cand_begin,
+                           int32_t n_recent, const void* Q_win, int32_t W,
+                           float* score, float* w_b,
+                           void* ws, size_t ws_bytes, kvs_stream_t stream);
+
+/*
+ * kvs_merge_compact -- one merge round: select pairs to the budget, merge them,
+ * and compact the cache (order preserved).
+ *
+ * Each unit merges R = min(P_unit, max(0, len_unit - target_unit)) pairs: the R
+ * with the smallest (score, index); NaN scores rank as +inf, -0 as +0. With
+ * scope KVS_SCOPE_HEAD a unit is one (b, h) and target has B*H_kv entries; with
+ * KVS_SCOPE_POOLED a unit is one sequence b across its H_kv heads, target has B
+ * entries (total rows over the heads), and the index order is (h, p).
+ * A selected pair (a, b) becomes one row at the pair's slot:
+ *   k* = k_a + w_b (k_b - k_a)                              (§数学主线四)
+ *   v* = (n_a v_a + n_b v_b) / (n_a + n_b),  logn* = log(n_a + n_b),  n = exp(logn)
+ *       (Values preserved: attention over the merged row equals attention over the
+ *        n_a + n_b original rows sharing k*)
+ * len_out = len - R. Repeating rounds reaches the budget exactly.
+ *
+ * Out-of-place (K_out != K): outputs must not overlap inputs (KVS_ERR_ALIAS).
+ * In-place (K_out == K, V_out == V, logn_out == logn, len_out == len): allowed when
+ * every head's span len - cand_begin is at most 8192 rows; rows before cand_begin
+ * are left untouched. Longer spans set KVS_FLAG_INPLACE_SPAN and are skipped.
+ *
+ * In:  the cache (logn nullable), len, cand_begin, n_recent, score and w_b from
+ *      kvs_score_pairs for the same cache, target, scope.
+ * Out: K_out, V_out [B,H_kv,T_cap_out,d]; logn_out [B,H_kv,T_cap_out]; len_out [B*H_kv].
+ *      Optional (nullable): dbg_selected [B,H_kv,T_cap/2] u8 (1 = merged);
+ *      dbg_out_offset [B,H_kv,T_cap/2] i32 (output row of the pair's first row);
+ *      dbg_kmerged_f32 [B,H_kv,T_cap/2,d] fp32 (merged key before rounding).
+ * Workspace: kvs_workspace_size(desc, 0, KVS_OP_MERGE) bytes.
+ */
+kvs_status kvs_merge_compact(const kvs_cache_desc* desc, const void* K, const void* V,
+                             const float* logn, const int32_t* len, const int32_t* cand_begin,
+                             int32_t n_recent, const float* score, const float* w_b,
+                             const int32_t* target, int32_t scope, int32_t T_cap_out,
+                             void* K_out, void* V_out, float* logn_out, int32_t* len_out,
+                             uint8_t* dbg_selected, int32_t* dbg_out_offset,
+                             float* dbg_kmerged_f32, void* ws, size_t ws_bytes,
+                             kvs_stream_t stream);
+
+/*
+ * kvs_decode_attn -- one decode step of GQA attention over the merged cache
+ * (attention of §数学主线三 with the log-count bias; the decoder stage of Figure 5).
+ *
+ *   out[b, hq] = sum_t softmax_t(q[b,hq] . k_t / sqrt(d) + logn_t) v_t over the
+ *   rows t < len[b, hq / G], plus the appended row when k_new is given.
+ *
+ * If k_new and v_new are non-NULL ([B, H_kv, d]), the step first appends them
+ * (count 1) at row len of every head: the row is attended, written into K, V
+ * (and logn = 0 when logn is non-NULL) and len is incremented by 1. A head whose
+ * len == T_cap cannot take the row: it sets KVS_FLAG_OUT_CAPACITY and is not
+ * changed (its output is still written, without the new row).
+ * In:  q [B,H_q,d]; K, V; logn (nullable); len [B*H_kv].
+ * Out: out [B,H_q,d] (cache dtype); K, V, logn, len updated when appending.
+ * Workspace: kvs_workspace_size(desc, 0, KVS_OP_DECODE) bytes; its counters must be
+ * zero at the first call (each call leaves them zero).
+ */
+kvs_status kvs_decode_attn(const kvs_cache_desc* desc, const void* q, void* K, void* V,
+                           float* logn, int32_t* len, const void* k_new, const void* v_new,
+                           void* out, void* ws, size_t ws_bytes, kvs_stream_t stream);
+
+/*
+ * kvs_device_flags -- read (and optionally clear) the device flag word of a
+ * workspace. Synchronises `stream`. Host pointer `flags` receives the bits.
+ */
+kvs_status kvs_device_flags(void* ws, int32_t* flags, int32_t clear, kvs_stream_t stream);
+
+/* Static string for a status code. */
+const char* kvs_status_str(kvs_status s);
+
+/* Library version, for the binding's load check. */
+int32_t kvs_version(void);
+
+/* Number of kernels this process has launched through the library so far
+   (host-side count at launch time; replays of a captured CUDA graph do not add). */
+int64_t kvs_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KVS_H_ */

@@ -40,6 +40,12 @@ reason, in the design notes):
   R8 window position: window query j sits at cache position len - W + j and
      attends positions <= its own (causal). Queries with a negative position
      are left out of the average.
+  R9 storage: a cache is stored in its element type between rounds. Merged
+     rows are rounded to that type (bf16: to fp32, then round-to-nearest-even
+     on the upper 16 bits) and log counts to fp32 before the next round reads
+     them; arithmetic inside a round stays fp64.
+  R10 empty cache: decode attention over a head with no rows (and no appended
+     row) returns the zero vector.
 """
 
 from __future__ import annotations
@@ -51,6 +57,29 @@ from typing import List, Optional, Sequence
 import numpy as np
 
 DEGENERATE_REL = 1e-6
+
+
+# ---------------------------------------------------------------------------
+# Storage precision of a cache (reading R9)
+# ---------------------------------------------------------------------------
+
+def storage_round(x, storage="f64"):
+    """Round fp64 values to what a cache of element type `storage` holds."""
+    x = np.asarray(x, dtype=np.float64)
+    if storage == "f64":
+        return x
+    f32 = x.astype(np.float32)
+    if storage == "f32":
+        return f32.astype(np.float64)
+    if storage == "bf16":
+        bits = f32.view(np.uint32).astype(np.uint64)
+        nan = np.isnan(f32)
+        lsb = (bits >> 16) & 1
+        rounded = ((bits + 0x7FFF + lsb) >> 16) << 16
+        out = rounded.astype(np.uint32).view(np.float32)
+        out = np.where(nan, np.float32(np.nan), out)
+        return out.astype(np.float64)
+    raise ValueError(storage)
 
 
 # ---------------------------------------------------------------------------
@@ -305,14 +334,15 @@ class HeadMerge:
     k_merged: np.ndarray        # (P, d) merged keys (rows of unselected pairs are zero)
 
 
-def merge_compact_head(K, V, log_n, length, cand_begin, n_recent, selected, w_b):
+def merge_compact_head(K, V, log_n, length, cand_begin, n_recent, selected, w_b, storage="f64"):
     """Merge the selected pairs and compact one KV head, order preserved.
 
     Selected pair (a, b):  k* = k_a + w_b (k_b - k_a)      ([KVS] §数学主线四, reading R7)
                            v* = (n_a v_a + n_b v_b) / (n_a + n_b),
                            log n* = log(n_a + n_b)          (reading R5)
     Unselected pairs, protected prefix [0, c0), the odd leftover and the
-    recent suffix are copied unchanged.
+    recent suffix are copied unchanged. Merged rows are rounded to `storage`
+    (reading R9); ``k_merged`` keeps the unrounded fp64 keys.
     """
     K = np.asarray(K, dtype=np.float64)
     V = np.asarray(V, dtype=np.float64)
@@ -334,7 +364,9 @@ def merge_compact_head(K, V, log_n, length, cand_begin, n_recent, selected, w_b)
             n_a, n_b = math.exp(ln[a]), math.exp(ln[b])
             v_star = (n_a * V[a] + n_b * V[b]) / (n_a + n_b)
             k_merged[p] = k_star
-            out_K.append(k_star); out_V.append(v_star); out_ln.append(math.log(n_a + n_b))
+            out_K.append(storage_round(k_star, storage))
+            out_V.append(storage_round(v_star, storage))
+            out_ln.append(float(storage_round(math.log(n_a + n_b), "f64" if storage == "f64" else "f32")))
         else:
             out_K.extend([K[a], K[b]]); out_V.extend([V[a], V[b]]); out_ln.extend([ln[a], ln[b]])
     for t in range(max(c0, 0) + 2 * P, length):
@@ -399,7 +431,7 @@ class RoundResult:
     R: np.ndarray                 # pairs merged per unit
 
 
-def merge_round(cache, Q_win, W, cand_begin, n_recent, target, scope="head"):
+def merge_round(cache, Q_win, W, cand_begin, n_recent, target, scope="head", storage="f64"):
     """One scoring + selection + merge round over a whole cache.
 
     Q_win: (B, H_q, W, d); query head hq belongs to KV head hq // G.
@@ -440,14 +472,15 @@ def merge_round(cache, Q_win, W, cand_begin, n_recent, target, scope="head"):
         raise ValueError(scope)
     merges = [[merge_compact_head(cache.K[b][h], cache.V[b][h], cache.log_n[b][h],
                                   cache.length(b, h), cand_begin[b, h], n_recent,
-                                  selected[b][h], scores[b][h].w_b)
+                                  selected[b][h], scores[b][h].w_b, storage)
                for h in range(H)] for b in range(B)]
     out = Cache([[m.K for m in row] for row in merges], [[m.V for m in row] for row in merges],
                 [[m.log_n for m in row] for row in merges])
     return RoundResult(cache=out, scores=scores, selected=selected, merges=merges, R=R)
 
 
-def compress(cache, Q_win, W, cand_begin, n_recent, target, scope="head", max_rounds=64):
+def compress(cache, Q_win, W, cand_begin, n_recent, target, scope="head", max_rounds=64,
+             storage="f64"):
     """Repeat merge rounds until every unit reaches its budget exactly (reading R4)."""
     rounds = []
     for _ in range(max_rounds):
@@ -458,7 +491,7 @@ def compress(cache, Q_win, W, cand_begin, n_recent, target, scope="head", max_ro
             done = np.all(lens.sum(axis=1) == np.asarray(target).reshape(-1))
         if done:
             return cache, rounds
-        r = merge_round(cache, Q_win, W, cand_begin, n_recent, target, scope)
+        r = merge_round(cache, Q_win, W, cand_begin, n_recent, target, scope, storage)
         if np.all(r.R == 0):
             raise ValueError("budget unreachable: no candidate pairs left")
         rounds.append(r)
@@ -472,6 +505,8 @@ def decode_attention(q_heads, K, V, log_n, length):
     q_heads = np.asarray(q_heads, dtype=np.float64)
     K = np.asarray(K, dtype=np.float64)[:length]
     V = np.asarray(V, dtype=np.float64)[:length]
+    if length == 0:   # reading R10: attention over no rows is the zero vector
+        return np.zeros_like(q_heads)
     ln = None if log_n is None else np.asarray(log_n, dtype=np.float64)[:length]
     return np.array([attention_output(softmax(attention_logits(q, K, ln)), V) for q in q_heads])
 

@@ -1,0 +1,397 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle, on the
+same seeded inputs, for all five workloads and the edge cases."""
+
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from asymmetric_kv_merging_b200 import inputs
+
+from parity import GpuCache, Stats, compare_decode, compare_round, gpu_round, storage_of, to_oracle_cache
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def kvs():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from asymmetric_kv_merging_b200 import build
+    build.build()
+    from asymmetric_kv_merging_b200 import kvs as mod
+    return mod
+
+
+def _workspace(kvs, B, H, H_q, d, T_cap, dtype, W=32):
+    return kvs.workspace(kvs.make_desc(B, H, H_q, d, T_cap, dtype), W)
+
+
+def compress_both(kvs, w, li, batch=None, ratio=None, stats=None, Q_override=None):
+    """Compress on the GPU (all sequences) and in the oracle (sequences `batch`),
+    comparing every round."""
+    dev = torch.device("cuda")
+    B, H, T_cap, d = li.K.shape
+    ratio = ratio or w.ratio
+    batch = list(range(B)) if batch is None else list(batch)
+    g = GpuCache(li.K.to(dev), li.V.to(dev), li.lens.to(dev))
+    o = to_oracle_cache(g, batch=batch)
+    lens = li.lens.view(B, H).cpu().numpy().astype(np.int64)
+    if w.scope == "pooled":
+        target_np = (lens // ratio).sum(axis=1)
+        scope, scope_code = "pooled", kvs.SCOPE_POOLED
+    else:
+        target_np = lens // ratio
+        scope, scope_code = "head", kvs.SCOPE_HEAD
+    target = torch.tensor(target_np.reshape(-1), dtype=torch.int32, device=dev)
+    cand = torch.full((B * H,), w.sink, dtype=torch.int32, device=dev)
+    Q = (li.Q_win if Q_override is None else Q_override).to(dev)
+    Qo = Q.double().cpu().numpy()[batch]
+    ws = _workspace(kvs, B, H, w.H_q, d, T_cap, li.K.dtype, w.W)
+    stats = stats or Stats()
+    for _ in range(16):
+        cur = g.lens.view(B, H).cpu().numpy()
+        done = (cur.sum(axis=1) <= target_np) if scope == "pooled" else (cur <= target_np)
+        if np.all(done):
+            break
+        r = oracle.merge_round(o, Qo, w.W, np.full((len(batch), H), w.sink), w.W,
+                               target_np[batch], scope, storage_of(li.K.dtype))
+        gout, gres = gpu_round(g, w.H_q, Q, w.W, cand, w.W, target, scope_code, ws)
+        compare_round(r, gres, gout, g, o, li.K.dtype, scope, batch, stats)
+        g, o = gout, r.cache
+    else:
+        raise AssertionError("compression did not finish")
+    lens_out = g.lens.view(B, H).cpu().numpy()
+    if scope == "pooled":
+        assert np.array_equal(lens_out.sum(axis=1), target_np)
+    else:
+        assert np.array_equal(lens_out, target_np)
+    assert kvs.device_flags(ws) == 0
+    return g, o, stats, ws
+
+
+def decode_both(kvs, w, li, g, o, steps, batch=None, stats=None, ws=None, check=True):
+    dev = torch.device("cuda")
+    B, H, T_cap, d = g.K.shape
+    batch = list(range(B)) if batch is None else list(batch)
+    desc = kvs.make_desc(B, H, w.H_q, d, T_cap, g.K.dtype)
+    ws = ws if ws is not None else kvs.workspace(desc, w.W)
+    out = torch.empty(B, w.H_q, d, dtype=g.K.dtype, device=dev)
+    for s in steps:
+        q = li.q_dec[s].to(dev).contiguous()
+        kn = li.k_new[s].to(dev).contiguous()
+        vn = li.v_new[s].to(dev).contiguous()
+        kvs.decode_attn(desc, q, g.K, g.V, g.logn, g.lens, out, ws, kn, vn)
+        oo, o = oracle.decode_step(o, q.double().cpu().numpy()[batch],
+                                   kn.double().cpu().numpy()[batch], vn.double().cpu().numpy()[batch])
+        if check:
+            compare_decode(oo, out, g.K.dtype, w.G, stats, batch)
+    assert kvs.device_flags(ws) == 0
+    return g, o
+
+
+# --------------------------------------------------------------------------- workload 0
+
+@pytest.mark.parametrize("q_scale", [1.0, 6.0])
+def test_workload0_tiny_fp32_pipeline(kvs, q_scale):
+    w = inputs.workload(0)
+    li = inputs.make_layer(w, 0, q_scale=q_scale)
+    g, o, stats, ws = compress_both(kvs, w, li)
+    g, o = decode_both(kvs, w, li, g, o, range(w.n_decode), stats=stats, ws=ws)
+    print("workload 0", q_scale, stats.report())
+    assert stats.merged_compared > 0 and not stats.diverged_heads
+
+
+def test_peaked_attention_exercises_degenerate_pairs(kvs):
+    """Strongly peaked window attention gives pairs with alpha near 1/2 and D <= 0."""
+    w = inputs.small_workload(inputs.workload(0), T=192, n_decode=2)
+    li = inputs.make_layer(w, 0, q_scale=40.0)
+    stats = Stats()
+    compress_both(kvs, w, li, stats=stats)
+    print(stats.report())
+
+
+# --------------------------------------------------------------------------- workload 1
+
+def test_workload1_llama_layer_full_size(kvs):
+    w = inputs.workload(1)
+    li = inputs.make_layer(w, 0, device="cuda")
+    g, o, stats, ws = compress_both(kvs, w, li)
+    g, o = decode_both(kvs, w, li, g, o, range(w.n_decode), stats=stats, ws=ws)
+    print("workload 1", stats.report())
+    assert stats.merged_compared > 8 * 16000
+    assert len(stats.diverged_heads) <= 1
+
+
+# --------------------------------------------------------------------------- workload 2
+
+@pytest.mark.parametrize("layer", [0, 31])
+def test_workload2_128k_layer_sample(kvs, layer):
+    """One layer of the 32-layer 128K workload, at full size: every round and a few
+    decode steps (the bench times all 32 layers with the same kernels)."""
+    w = inputs.workload(2)
+    li = inputs.make_layer(w, layer, device="cuda")
+    g, o, stats, ws = compress_both(kvs, w, li)
+    g, o = decode_both(kvs, w, li, g, o, range(4), stats=stats, ws=ws)
+    print("workload 2 layer", layer, stats.report())
+    assert len(stats.diverged_heads) <= 1
+
+
+# --------------------------------------------------------------------------- workload 3
+
+def test_workload3_pooled_budget_sample(kvs):
+    """Batch 8 on the GPU; the oracle checks sequences 0 and 5 of layer 0."""
+    w = inputs.workload(3)
+    li = inputs.make_layer(w, 0, device="cuda")
+    batch = [0, 5]
+    g, o, stats, ws = compress_both(kvs, w, li, batch=batch)
+    lens = g.lens.view(w.B, w.H_kv).cpu().numpy()
+    assert len(set(lens.reshape(-1).tolist())) > 1          # ragged per-head lengths
+    g, o = decode_both(kvs, w, li, g, o, range(w.n_decode), batch=batch, stats=stats, ws=ws)
+    print("workload 3", stats.report())
+
+
+# --------------------------------------------------------------------------- workload 4
+
+def test_workload4_serving_mix_sample(kvs):
+    """Ragged batch of 16: 8x compression, 256 decode steps with an in-place
+    re-merge of the newest 64 rows every 64 steps; the oracle follows sequences 0 and 9."""
+    w = inputs.workload(4)
+    li = inputs.make_layer(w, 0, device="cuda")
+    batch = [0, 9]
+    g, o, stats, ws = compress_both(kvs, w, li, batch=batch)
+    dev = torch.device("cuda")
+    B, H, T_cap, d = g.K.shape
+    for seg in range(w.n_decode // w.remerge_every):
+        s0 = seg * w.remerge_every
+        g, o = decode_both(kvs, w, li, g, o, range(s0, s0 + w.remerge_every), batch=batch,
+                           stats=stats, ws=ws, check=(seg % 2 == 0))
+        # re-merge the newest segment in place: 64 -> 8 rows, window = last 32 decode queries
+        Qw = li.q_dec[s0 + w.remerge_every - w.W: s0 + w.remerge_every].to(dev)
+        Qw = Qw.permute(1, 2, 0, 3).contiguous()                    # [B, H_q, W, d]
+        Qo = Qw.double().cpu().numpy()[batch]
+        for _ in range(3):
+            cand = (g.lens - w.remerge_every // (2 ** _)).contiguous()
+            lens_now = g.lens.view(B, H).cpu().numpy()
+            seg_len = w.remerge_every // (2 ** _)
+            target_np = lens_now - seg_len // 2
+            target = torch.tensor(target_np.reshape(-1), dtype=torch.int32, device=dev)
+            gin = GpuCache(g.K.clone(), g.V.clone(), g.lens.clone(), g.logn.clone())
+            oc = o.lengths() - seg_len
+            r = oracle.merge_round(o, Qo, w.W, oc, 0, target_np[batch], "head",
+                                   storage_of(g.K.dtype))
+            gout, gres = gpu_round(g, w.H_q, Qw, w.W, cand, 0, target, kvs.SCOPE_HEAD, ws,
+                                   inplace=True)
+            compare_round(r, gres, gout, gin, o, g.K.dtype, "head", batch, stats)
+            g, o = gout, r.cache
+    print("workload 4", stats.report())
+    assert kvs.device_flags(ws) == 0
+
+
+# --------------------------------------------------------------------------- selection
+
+def _selection_case(kvs, scope, B, H, L, c0, n_recent, R_list, ties, seed, dtype=torch.bfloat16, d=128):
+    dev = torch.device("cuda")
+    T_cap = L + 6 + L % 2
+    g = torch.Generator().manual_seed(seed)
+    K = torch.randn(B, H, T_cap, d, generator=g).to(dtype)
+    V = torch.randn(B, H, T_cap, d, generator=g).to(dtype)
+    logn = torch.log(torch.randint(1, 4, (B, H, T_cap), generator=g).float())
+    lens = torch.full((B * H,), L, dtype=torch.int32)
+    P = max(0, (L - n_recent - c0) // 2)
+    score = torch.zeros(B, H, T_cap // 2)
+    w_b = torch.zeros(B, H, T_cap // 2)
+    for i in range(B * H):
+        b, h = divmod(i, H)
+        score[b, h, :P] = inputs.random_scores(P, seed * 100 + i, ties=ties, with_nan=True)
+        w_b[b, h, :P] = inputs.random_weights(P, seed * 100 + i)
+    desc = kvs.make_desc(B, H, 4 * H, d, T_cap, dtype)
+    ws = kvs.workspace(desc, 32)
+    cand = torch.full((B * H,), c0, dtype=torch.int32)
+    for R in R_list:
+        if scope == kvs.SCOPE_POOLED:
+            target = torch.full((B,), H * L - R, dtype=torch.int32)
+        else:
+            target = torch.full((B * H,), L - R, dtype=torch.int32)
+        outs = {}
+        for inplace in (False, True):
+            Kd, Vd, ld, lnd = K.to(dev), V.to(dev), lens.to(dev), logn.to(dev)
+            sel = torch.zeros(B, H, T_cap // 2, dtype=torch.uint8, device=dev)
+            off = torch.full((B, H, T_cap // 2), -1, dtype=torch.int32, device=dev)
+            if inplace:
+                Ko, Vo, lo, lno = Kd, Vd, ld, lnd
+            else:
+                Ko, Vo = torch.zeros_like(Kd), torch.zeros_like(Vd)
+                lo, lno = torch.zeros_like(ld), torch.zeros_like(lnd)
+            kvs.merge_compact(desc, Kd, Vd, lnd, ld, cand.to(dev), n_recent, score.to(dev),
+                              w_b.to(dev), target.to(dev), scope, T_cap, Ko, Vo, lno, lo, ws,
+                              sel, off)
+            torch.cuda.synchronize()
+            outs[inplace] = (Ko.cpu(), Vo.cpu(), lno.cpu(), lo.cpu(), sel.cpu(), off.cpu())
+        assert kvs.device_flags(ws) == 0
+        # oracle on the same fp32 scores: bit-exact selection and offsets
+        Ko, Vo, lno, lo, sel, off = outs[False]
+        for b in range(B):
+            if scope == kvs.SCOPE_POOLED:
+                pooled = np.concatenate([score[b, h, :P].double().numpy() for h in range(H)])
+                mask = oracle.select_pairs(pooled, R).reshape(H, P)
+            for h in range(H):
+                sc = score[b, h, :P].double().numpy()
+                m_sel = mask[h] if scope == kvs.SCOPE_POOLED else oracle.select_pairs(sc, R)
+                np.testing.assert_array_equal(sel[b, h, :P].numpy().astype(bool), m_sel)
+                m = oracle.merge_compact_head(K[b, h].double().numpy(), V[b, h].double().numpy(),
+                                              logn[b, h].double().numpy(), L, c0, n_recent, m_sel,
+                                              w_b[b, h, :P].double().numpy(),
+                                              storage_of(dtype))
+                np.testing.assert_array_equal(off[b, h, :P].numpy(), m.out_offset)
+                assert int(lo[b * H + h]) == m.length
+                n = m.length
+                np.testing.assert_allclose(Ko[b, h, :n].double().numpy(), m.K, rtol=2e-2, atol=1e-2)
+                np.testing.assert_allclose(Vo[b, h, :n].double().numpy(), m.V, rtol=2e-2, atol=1e-2)
+                np.testing.assert_allclose(lno[b, h, :n].double().numpy(), m.log_n, atol=2e-6)
+                merged = np.zeros(n, bool)
+                merged[m.out_offset[m_sel]] = True
+                np.testing.assert_array_equal(Ko[b, h, :n][~merged].double().numpy(), m.K[~merged])
+        # in-place gives the same rows as out-of-place
+        Ki, Vi, lni, li_, seli, offi = outs[True]
+        assert torch.equal(li_, lo) and torch.equal(seli, sel) and torch.equal(offi, off)
+        for b in range(B):
+            for h in range(H):
+                n = int(lo[b * H + h])
+                assert torch.equal(Ki[b, h, :n], Ko[b, h, :n]) and torch.equal(Vi[b, h, :n], Vo[b, h, :n])
+                assert torch.equal(lni[b, h, :n], lno[b, h, :n])
+                assert torch.equal(Ki[b, h, :c0], K[b, h, :c0])
+
+
+@pytest.mark.parametrize("ties", [False, True])
+def test_selection_per_head_exact(kvs, ties):
+    L, c0, nr = 700, 32, 32
+    P = (L - nr - c0) // 2
+    _selection_case(kvs, kvs.SCOPE_HEAD, 2, 3, L, c0, nr, [0, 1, 17, P // 2, P - 1, P], ties, 1)
+
+
+@pytest.mark.parametrize("ties", [False, True])
+def test_selection_pooled_exact(kvs, ties):
+    L, c0, nr = 501, 7, 10
+    P = (L - nr - c0) // 2
+    _selection_case(kvs, kvs.SCOPE_POOLED, 2, 4, L, c0, nr, [0, 5, 4 * P // 3, 4 * P - 1, 4 * P],
+                    ties, 2)
+
+
+def test_selection_spans_many_blocks_fp32_d64(kvs):
+    L = 128 * 2 * 9 + 77       # several merge blocks and a ragged tail
+    _selection_case(kvs, kvs.SCOPE_HEAD, 1, 2, L, 32, 32, [300, 1000], False, 3,
+                    dtype=torch.float32, d=64)
+
+
+# --------------------------------------------------------------------------- decode
+
+@pytest.mark.parametrize("dtype,d,G", [(torch.bfloat16, 128, 4), (torch.float32, 64, 2),
+                                       (torch.bfloat16, 64, 8), (torch.float32, 128, 1)])
+def test_decode_ragged_with_append(kvs, dtype, d, G):
+    dev = torch.device("cuda")
+    B, H = 3, 2
+    lens = torch.tensor([[0, 1], [777, 64], [4097, 2000]], dtype=torch.int32)
+    T_cap = 4200
+    g = torch.Generator().manual_seed(7)
+    K = (torch.randn(B, H, T_cap, d, generator=g)).to(dtype)
+    V = torch.randn(B, H, T_cap, d, generator=g).to(dtype)
+    logn = torch.log(torch.randint(1, 5, (B, H, T_cap), generator=g).float())
+    q = (torch.randn(3, B, H * G, d, generator=g) * 3).to(dtype)
+    kn = torch.randn(3, B, H, d, generator=g).to(dtype)
+    vn = torch.randn(3, B, H, d, generator=g).to(dtype)
+    gc = GpuCache(K.to(dev), V.to(dev), lens.to(dev), logn.to(dev))
+    o = to_oracle_cache(gc)
+    desc = kvs.make_desc(B, H, H * G, d, T_cap, dtype)
+    ws = kvs.workspace(desc, 32)
+    out = torch.empty(B, H * G, d, dtype=dtype, device=dev)
+    # a step without append first
+    kvs.decode_attn(desc, q[0].to(dev), gc.K, gc.V, gc.logn, gc.lens, out, ws)
+    oo, _ = oracle.decode_step(o, q[0].double().numpy())
+    compare_decode(oo, out, dtype, G)
+    for s in range(3):
+        kvs.decode_attn(desc, q[s].to(dev), gc.K, gc.V, gc.logn, gc.lens, out, ws,
+                        kn[s].to(dev), vn[s].to(dev))
+        oo, o = oracle.decode_step(o, q[s].double().numpy(), kn[s].double().numpy(),
+                                   vn[s].double().numpy())
+        compare_decode(oo, out, dtype, G)
+    assert torch.equal(gc.lens.cpu().view(B, H), lens + 3)
+    assert kvs.device_flags(ws) == 0
+
+
+def test_decode_append_at_capacity_sets_flag(kvs):
+    dev = torch.device("cuda")
+    desc = kvs.make_desc(1, 1, 4, 128, 64, torch.bfloat16)
+    K = torch.randn(1, 1, 64, 128, device=dev).to(torch.bfloat16)
+    V = torch.randn_like(K)
+    lens = torch.tensor([64], dtype=torch.int32, device=dev)
+    ws = kvs.workspace(desc, 32)
+    out = torch.empty(1, 4, 128, dtype=torch.bfloat16, device=dev)
+    kn = torch.randn(1, 1, 128, device=dev).to(torch.bfloat16)
+    kvs.decode_attn(desc, torch.randn(1, 4, 128, device=dev).to(torch.bfloat16), K, V, None, lens,
+                    out, ws, kn, kn)
+    assert kvs.device_flags(ws, clear=True) == kvs.FLAG_OUT_CAPACITY
+    assert int(lens.item()) == 64
+    assert kvs.device_flags(ws) == 0
+
+
+# --------------------------------------------------------------------------- edge cases
+
+def test_edge_cases_short_and_empty_spans(kvs):
+    """Heads with no candidate pairs, odd spans, a cache shorter than the window,
+    and a budget already met, in one batch."""
+    dev = torch.device("cuda")
+    w = inputs.small_workload(inputs.workload(0), B=1, H_kv=6, H_q=12, T=200, n_decode=0)
+    g0 = torch.Generator().manual_seed(3)
+    T_cap = 256
+    K = torch.randn(1, 6, T_cap, 64, generator=g0)
+    V = torch.randn(1, 6, T_cap, 64, generator=g0)
+    Q = torch.randn(1, 12, 32, 64, generator=g0) * 2
+    lens = torch.tensor([[200, 65, 64, 20, 0, 97]], dtype=torch.int32)   # 64: P = 0; 20 < W
+    li = inputs.LayerInputs(K=K, V=V, lens=lens, Q_win=Q, q_dec=None, k_new=None, v_new=None)
+    gc = GpuCache(K.to(dev), V.to(dev), lens.to(dev))
+    o = to_oracle_cache(gc)
+    cand = torch.full((6,), 32, dtype=torch.int32, device=dev)
+    target_np = np.array([[100, 60, 64, 20, 0, 90]])
+    target = torch.tensor(target_np.reshape(-1), dtype=torch.int32, device=dev)
+    ws = kvs.workspace(kvs.make_desc(1, 6, 12, 64, T_cap, torch.float32), 32)
+    stats = Stats()
+    for _ in range(4):
+        r = oracle.merge_round(o, Q.double().numpy(), 32, np.full((1, 6), 32), 32, target_np,
+                               "head", "f32")
+        gout, gres = gpu_round(gc, 12, Q.to(dev), 32, cand, 32, target, kvs.SCOPE_HEAD, ws)
+        compare_round(r, gres, gout, gc, o, torch.float32, "head", None, stats)
+        gc, o = gout, r.cache
+    assert kvs.device_flags(ws) == 0
+    # the 65-row head has a one-row span (no pairs): its budget is unreachable
+    assert gc.lens.cpu().tolist() == [100, 65, 64, 20, 0, 90]
+
+
+def test_bad_length_and_capacity_flags(kvs):
+    dev = torch.device("cuda")
+    desc = kvs.make_desc(1, 2, 4, 64, 128, torch.float32)
+    K = torch.randn(1, 2, 128, 64, device=dev)
+    V = torch.randn_like(K)
+    lens = torch.tensor([129, 100], dtype=torch.int32, device=dev)      # head 0 invalid
+    Q = torch.randn(1, 4, 32, 64, device=dev)
+    cand = torch.full((2,), 32, dtype=torch.int32, device=dev)
+    ws = kvs.workspace(desc, 32)
+    score = torch.zeros(1, 2, 64, device=dev)
+    w_b = torch.zeros_like(score)
+    kvs.score_pairs(desc, K, V, None, lens, cand, 32, Q, 32, score, w_b, ws)
+    assert kvs.device_flags(ws, clear=True) & kvs.FLAG_BAD_LENGTH
+    lens = torch.tensor([128, 100], dtype=torch.int32, device=dev)
+    kvs.score_pairs(desc, K, V, None, lens, cand, 32, Q, 32, score, w_b, ws)
+    assert kvs.device_flags(ws) == 0
+    # the output capacity (96 rows) is too small for head 0 (128 - 8 merged = 120 rows)
+    Ko = torch.zeros(1, 2, 96, 64, device=dev)
+    Vo = torch.zeros_like(Ko)
+    lno = torch.zeros(1, 2, 96, device=dev)
+    lo = torch.zeros(2, dtype=torch.int32, device=dev)
+    target = torch.tensor([120, 50], dtype=torch.int32, device=dev)
+    kvs.merge_compact(desc, K, V, None, lens, cand, 32, score, w_b, target, kvs.SCOPE_HEAD, 96,
+                      Ko, Vo, lno, lo, ws)
+    assert kvs.device_flags(ws, clear=True) == kvs.FLAG_OUT_CAPACITY
+    assert int(lo[1]) == 82   # head 1: 100 rows, all 18 pairs merged

@@ -39,7 +39,7 @@ def test_layer_shapes_and_determinism():
     w = inputs.small_workload(inputs.WORKLOADS[0], T=96, n_decode=3)
     a = inputs.make_layer(w, 0)
     b = inputs.make_layer(w, 0)
-    assert a.K.shape == (1, 2, 99, 64) and a.Q_win.shape == (1, 4, 32, 64)
+    assert a.K.shape == (1, 2, 100, 64) and a.Q_win.shape == (1, 4, 32, 64)   # 96 + 3, even
     assert a.q_dec.shape == (3, 1, 4, 64) and a.k_new.shape == (3, 1, 2, 64)
     assert torch.equal(a.K, b.K) and torch.equal(a.Q_win, b.Q_win)
     assert torch.all(a.K[:, :, 96:] == 0)

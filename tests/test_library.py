@@ -1,0 +1,132 @@
+"""The C-ABI library loads, exports every entry point include/kvs.h declares, and
+rejects bad arguments on the host (no GPU needed: nothing here launches)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def kvs():
+    from asymmetric_kv_merging_b200 import build
+    build.build()
+    from asymmetric_kv_merging_b200 import kvs as mod
+    return mod
+
+
+def header_functions():
+    with open(os.path.join(ROOT, "include", "kvs.h")) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[A-Za-z_0-9]+\s*\*?\s*(kvs_[a-z_0-9]+)\s*\(",
+                                 text, re.M)))
+
+
+def test_every_declared_function_is_exported(kvs):
+    names = header_functions()
+    assert {"kvs_score_pairs", "kvs_merge_compact", "kvs_decode_attn", "kvs_workspace_size"} <= set(names)
+    lib = ctypes.CDLL(kvs.library_path())
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(kvs.EXPORTS) <= set(names)
+
+
+def test_status_strings(kvs):
+    for code in range(7):
+        assert kvs.status_str(code)
+    assert kvs.status_str(0) == "ok"
+
+
+def test_workspace_sizes(kvs):
+    d = kvs.make_desc(1, 8, 32, 128, 32768, kvs.BF16)
+    for op in (kvs.OP_SCORE, kvs.OP_MERGE, kvs.OP_DECODE):
+        n = kvs.workspace_size(d, 32, op)
+        assert n > 0 and n % 256 == 0
+    # alpha_bar alone needs one fp32 per cached row
+    assert kvs.workspace_size(d, 32, kvs.OP_SCORE) >= 8 * 32768 * 4
+    bad = kvs.make_desc(1, 8, 32, 96, 32768, kvs.BF16)           # head dim 96 not built
+    assert kvs.workspace_size(bad, 32, kvs.OP_SCORE) == 0
+    assert kvs.workspace_size(kvs.make_desc(1, 8, 24, 128, 64, kvs.BF16), 32, kvs.OP_DECODE) == 0
+    assert kvs.workspace_size(d, 32, 7) == 0
+
+
+FAKE = 1 << 40          # aligned fake device addresses: validation never dereferences
+
+
+def _fake(i):
+    return ctypes.c_void_p(FAKE + i * (1 << 34))
+
+
+def _score(kvs, desc, **over):
+    args = dict(K=_fake(1), V=_fake(2), logn=None, len=_fake(3), cb=_fake(4), n_recent=32,
+                Q=_fake(5), W=32, score=_fake(6), w_b=_fake(7), ws=_fake(8), ws_bytes=1 << 40)
+    args.update(over)
+    return kvs._lib.kvs_score_pairs(ctypes.byref(desc), args["K"], args["V"], args["logn"],
+                                    args["len"], args["cb"], args["n_recent"], args["Q"],
+                                    args["W"], args["score"], args["w_b"], args["ws"],
+                                    args["ws_bytes"], None)
+
+
+def test_score_pairs_host_validation(kvs):
+    d = kvs.make_desc(1, 8, 32, 128, 1024, kvs.BF16)
+    assert _score(kvs, d, K=None) == 1                                   # NULL
+    assert _score(kvs, d, K=ctypes.c_void_p(FAKE + 8)) == 1              # misaligned
+    assert _score(kvs, d, W=0) == 1
+    assert _score(kvs, d, n_recent=-1) == 1
+    assert _score(kvs, d, W=33) == 2                                     # G*W > 128
+    assert _score(kvs, kvs.make_desc(1, 8, 32, 80, 1024, kvs.BF16)) == 2
+    assert _score(kvs, kvs.make_desc(1, 8, 32, 128, 1023, kvs.BF16)) == 1  # odd T_cap
+    assert _score(kvs, kvs.make_desc(1, 8, 32, 128, 1024, 5)) == 2
+    assert _score(kvs, d, ws_bytes=1024) == 4
+    assert _score(kvs, d, ws=None) == 4
+    assert _score(kvs, d, ws=ctypes.c_void_p(FAKE + 128)) == 4           # not 256-aligned
+    assert _score(kvs, d, score=_fake(1)) == 5                           # score over K
+
+
+def _merge(kvs, desc, **over):
+    a = dict(K=_fake(1), V=_fake(2), logn=_fake(9), len=_fake(3), cb=_fake(4), n_recent=32,
+             score=_fake(6), w_b=_fake(7), target=_fake(10), scope=0, T_out=desc.T_cap,
+             K_out=_fake(11), V_out=_fake(12), ln_out=_fake(13), len_out=_fake(14),
+             dsel=None, doff=None, dkm=None, ws=_fake(8), ws_bytes=1 << 40)
+    a.update(over)
+    return kvs._lib.kvs_merge_compact(
+        ctypes.byref(desc), a["K"], a["V"], a["logn"], a["len"], a["cb"], a["n_recent"], a["score"],
+        a["w_b"], a["target"], a["scope"], a["T_out"], a["K_out"], a["V_out"], a["ln_out"],
+        a["len_out"], a["dsel"], a["doff"], a["dkm"], a["ws"], a["ws_bytes"], None)
+
+
+def test_merge_compact_host_validation(kvs):
+    d = kvs.make_desc(2, 8, 32, 128, 4096, kvs.BF16)
+    assert _merge(kvs, d, target=None) == 1
+    assert _merge(kvs, d, scope=2) == 1
+    assert _merge(kvs, d, T_out=0) == 1
+    assert _merge(kvs, d, K_out=_fake(2)) == 5                 # K_out over V
+    assert _merge(kvs, d, dsel=_fake(6)) == 5                  # debug output over score
+    assert _merge(kvs, d, V_out=_fake(11)) == 5                # two outputs overlap
+    # in-place needs every cache buffer in place and a log-count array
+    assert _merge(kvs, d, K_out=_fake(1), V_out=_fake(12)) == 5
+    assert _merge(kvs, d, K_out=_fake(1), V_out=_fake(2), ln_out=_fake(9), len_out=_fake(3),
+                  ws_bytes=16) == 4
+    assert _merge(kvs, d, K_out=_fake(1), V_out=_fake(2), logn=None, ln_out=None,
+                  len_out=_fake(3)) == 1
+    assert _merge(kvs, d, ws_bytes=256) == 4
+
+
+def test_decode_host_validation(kvs):
+    d = kvs.make_desc(1, 8, 32, 128, 4096, kvs.BF16)
+    lib = kvs._lib
+
+    def call(**o):
+        a = dict(q=_fake(1), K=_fake(2), V=_fake(3), logn=None, len=_fake(4), kn=None, vn=None,
+                 out=_fake(5), ws=_fake(6), ws_bytes=1 << 40)
+        a.update(o)
+        return lib.kvs_decode_attn(ctypes.byref(d), a["q"], a["K"], a["V"], a["logn"], a["len"],
+                                   a["kn"], a["vn"], a["out"], a["ws"], a["ws_bytes"], None)
+
+    assert call(q=None) == 1
+    assert call(kn=_fake(7)) == 1                               # k_new without v_new
+    assert call(out=_fake(2)) == 5                              # output over K
+    assert call(ws_bytes=100) == 4

@@ -134,3 +134,14 @@ def test_pooled_scope_budget_and_global_selection():
         assert R == last.R[b]
         # exactly the R smallest of the pooled scores
         assert np.all(pooled[chosen].max(initial=-np.inf) <= pooled[~chosen].min(initial=np.inf))
+
+
+def test_storage_rounding_matches_torch_conversions():
+    import torch
+    rng = np.random.default_rng(5)
+    x = np.concatenate([rng.normal(size=2000) * 10.0 ** rng.integers(-8, 8, size=2000),
+                        [0.0, -0.0, 1.0, 1.00390625, 1.001953125, 65504.0, 3.0e38]])
+    for storage, tdt in (("bf16", torch.bfloat16), ("f32", torch.float32)):
+        ref = torch.tensor(x, dtype=torch.float64).to(torch.float32).to(tdt).to(torch.float64).numpy()
+        got = oracle.storage_round(x, storage)
+        assert np.array_equal(got, ref), storage

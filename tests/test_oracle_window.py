@@ -96,3 +96,8 @@ def test_decode_step_appends_then_attends():
         for g in range(2):
             _, o = loop_attention_row(q[0, 2 * h + g], Kf, Vf, [0.0] * (L + 1), L)
             np.testing.assert_allclose(out[0, 2 * h + g], o, rtol=1e-12)
+
+
+def test_decode_over_an_empty_cache_is_zero():
+    out = oracle.decode_attention(np.ones((2, 4)), np.zeros((0, 4)), np.zeros((0, 4)), None, 0)
+    assert out.shape == (2, 4) and np.all(out == 0)

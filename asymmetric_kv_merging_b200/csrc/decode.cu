@@ -196,6 +196,10 @@ static cudaError_t launch_decode_t(const kvs_cache_desc& d, const void* q, void*
 cudaError_t launch_decode(const kvs_cache_desc& d, const void* q, void* K, void* V, float* logn,
                           int32_t* len, const void* k_new, const void* v_new, void* out,
                           const DecodeLayout& Ly, char* ws, cudaStream_t st) {
+  // bf16 caches take the TMA + tensor-core kernel; fp32 caches (and caches too large
+  // for 32-bit TMA row coordinates) the CUDA-core kernel below
+  if (decode_tc_supported(d))
+    return launch_decode_tc(d, q, K, V, logn, len, k_new, v_new, out, Ly, ws, st);
   if (d.dtype == KVS_BF16) {
     if (d.d == 128) return launch_decode_t<bf16, 128>(d, q, K, V, logn, len, k_new, v_new, out, Ly, ws, st);
     return launch_decode_t<bf16, 64>(d, q, K, V, logn, len, k_new, v_new, out, Ly, ws, st);

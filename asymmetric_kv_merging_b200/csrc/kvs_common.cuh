@@ -184,7 +184,6 @@ inline MergeLayout merge_layout(const kvs_cache_desc& d) {
 
 inline DecodeLayout decode_layout(const kvs_cache_desc& d) {
   DecodeLayout L;
-  size_t heads = (size_t)d.B * d.H_kv;
   size_t qheads = (size_t)d.B * d.H_q;
   L.nsplit = decode_splits(d);
   L.counters = kWsAlign;

@@ -35,4 +35,10 @@ cudaError_t launch_decode(const kvs_cache_desc& d, const void* q, void* K, void*
                           int32_t* len, const void* k_new, const void* v_new, void* out,
                           const DecodeLayout& Ly, char* ws, cudaStream_t st);
 
+// The same step for bf16 caches on the TMA + tensor-core kernel.
+bool decode_tc_supported(const kvs_cache_desc& d);
+cudaError_t launch_decode_tc(const kvs_cache_desc& d, const void* q, void* K, void* V, float* logn,
+                             int32_t* len, const void* k_new, const void* v_new, void* out,
+                             const DecodeLayout& Ly, char* ws, cudaStream_t st);
+
 }  // namespace kvs

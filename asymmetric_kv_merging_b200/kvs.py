@@ -24,6 +24,7 @@ F32, BF16 = 0, 1
 OP_SCORE, OP_MERGE, OP_DECODE = 0, 1, 2
 SCOPE_HEAD, SCOPE_POOLED = 0, 1
 FLAG_BAD_LENGTH, FLAG_OUT_CAPACITY, FLAG_INPLACE_SPAN, FLAG_NONFINITE_STATS = 1, 2, 4, 8
+FLAG_TIMEOUT = 16
 
 STATUS = {0: "KVS_OK", 1: "KVS_ERR_INVALID_ARG", 2: "KVS_ERR_UNSUPPORTED", 3: "KVS_ERR_BUDGET",
           4: "KVS_ERR_WORKSPACE", 5: "KVS_ERR_ALIAS", 6: "KVS_ERR_CUDA"}

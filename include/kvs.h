@@ -78,7 +78,8 @@ enum {
   KVS_FLAG_BAD_LENGTH = 1,      /* a len[] value was < 0 or > T_cap; that head was skipped */
   KVS_FLAG_OUT_CAPACITY = 2,    /* a merged head or an append did not fit the output capacity */
   KVS_FLAG_INPLACE_SPAN = 4,    /* in-place merge on a span longer than it supports; head skipped */
-  KVS_FLAG_NONFINITE_STATS = 8  /* a window query had no finite softmax normaliser */
+  KVS_FLAG_NONFINITE_STATS = 8, /* a window query had no finite softmax normaliser */
+  KVS_FLAG_TIMEOUT = 16         /* a pipeline wait gave up (bounded waits); results invalid */
 };
 
 /*

@@ -30,7 +30,8 @@ STATUS = {0: "KVS_OK", 1: "KVS_ERR_INVALID_ARG", 2: "KVS_ERR_UNSUPPORTED", 3: "K
           4: "KVS_ERR_WORKSPACE", 5: "KVS_ERR_ALIAS", 6: "KVS_ERR_CUDA"}
 
 EXPORTS = ("kvs_workspace_size", "kvs_score_pairs", "kvs_merge_compact", "kvs_decode_attn",
-           "kvs_device_flags", "kvs_status_str", "kvs_version", "kvs_launch_count")
+           "kvs_device_flags", "kvs_status_str", "kvs_version", "kvs_launch_count",
+           "kvs_decode_attn_static", "kvs_static_scratch_bytes")
 
 
 class CacheDesc(ctypes.Structure):
@@ -60,6 +61,9 @@ _lib.kvs_merge_compact.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, 
                                    _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
 _lib.kvs_decode_attn.restype = ctypes.c_int
 _lib.kvs_decode_attn.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+_lib.kvs_decode_attn_static.restype = ctypes.c_int
+_lib.kvs_decode_attn_static.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+_lib.kvs_static_scratch_bytes.restype = _sz
 _lib.kvs_device_flags.restype = ctypes.c_int
 _lib.kvs_device_flags.argtypes = [_vp, ctypes.POINTER(_i32), _i32, _vp]
 
@@ -161,3 +165,15 @@ def status_str(code: int) -> str:
 def launch_count() -> int:
     """Kernels launched through the library by this process (host-side count)."""
     return int(_lib.kvs_launch_count())
+
+
+def decode_attn_static(desc, q, K, V, logn, lens, out, k_new=None, v_new=None, stream=None):
+    """kvs_decode_attn on the library's built-in scratch buffer: allocates nothing."""
+    _check(_lib.kvs_decode_attn_static(ctypes.byref(desc), _ptr(q), _ptr(K), _ptr(V), _ptr(logn),
+                                       _ptr(lens), _ptr(k_new), _ptr(v_new), _ptr(out),
+                                       _stream(stream)),
+           "kvs_decode_attn_static")
+
+
+def static_scratch_bytes() -> int:
+    return int(_lib.kvs_static_scratch_bytes())

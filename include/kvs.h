@@ -180,6 +180,33 @@ kvs_status kvs_decode_attn(const kvs_cache_desc* desc, const void* q, void* K, v
                            void* out, void* ws, size_t ws_bytes, kvs_stream_t stream);
 
 /*
+ * kvs_decode_attn_static -- kvs_decode_attn without a caller-provided workspace.
+ * The pages have no counterpart to this entry point; it exists for callers that
+ * cannot allocate device memory at call time: a runtime whose memory plan is fixed
+ * before it starts serving, a host framework that only hands a plugin a stream, or
+ * code that must not let an allocation synchronise the device mid-step.
+ *
+ * It computes exactly what kvs_decode_attn computes (same kernels, same arguments
+ * minus ws / ws_bytes) using a scratch buffer built into the library: a device
+ * array of kvs_static_scratch_bytes() bytes (4 MiB) that every GPU which loads the
+ * library holds until the process exits. Shapes whose decode workspace
+ * (kvs_workspace_size(desc, 0, KVS_OP_DECODE)) exceeds it return KVS_ERR_WORKSPACE
+ * and launch nothing. It allocates nothing: no cudaMalloc, no cudaFree.
+ *
+ * The first call on a device looks up the buffer's device address for that device
+ * (make that call outside any stream capture); every call then clears the buffer's
+ * flag word and arrival counters on `stream` before launching. All calls share the
+ * one buffer: calls that overlap on the GPU (other streams, other host threads)
+ * race on it, and the buffer keeps the last call's contents.
+ */
+kvs_status kvs_decode_attn_static(const kvs_cache_desc* desc, const void* q, void* K, void* V,
+                                  float* logn, int32_t* len, const void* k_new,
+                                  const void* v_new, void* out, kvs_stream_t stream);
+
+/* Size in bytes of the scratch buffer kvs_decode_attn_static uses. */
+size_t kvs_static_scratch_bytes(void);
+
+/*
  * kvs_device_flags -- read (and optionally clear) the device flag word of a
  * workspace. Synchronises `stream`. Host pointer `flags` receives the bits.
  */

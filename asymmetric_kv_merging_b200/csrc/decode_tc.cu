@@ -37,7 +37,7 @@ struct TcShape {
 };
 
 template <int D, int G>
-__global__ void __launch_bounds__(kTcThreads)
+__global__ void __launch_bounds__(kTcThreads, 2)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                  const bf16* __restrict__ q, bf16* K, bf16* V, float* logn, int32_t* len,
                  const bf16* __restrict__ k_new, const bf16* __restrict__ v_new,
@@ -116,6 +116,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
       for (int i = issued > kTcStages ? issued - kTcStages : 0; i < issued; ++i)
         if (!mbar_wait(&full[i % kTcStages], (i / kTcStages) & 1)) set_flag(flags, KVS_FLAG_TIMEOUT);
     }
+    __syncwarp();   // reconverge before the CTA-wide barrier after the main loop
   } else {
     // ---------------- consumers: 16 rows of each stage per warp ----------------
     const int grp = lane >> 2, tig = lane & 3;       // MMA fragment row / column pair
@@ -136,9 +137,24 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     const float* lnh = logn ? logn + (size_t)head * T_cap : nullptr;
     const int r0 = warp * 16;                        // this warp's rows inside a stage
     const uint32_t ring = smem_u32(base);
+    // log-counts of this lane's four rows of a tile, fetched one tile ahead so the
+    // global-memory latency overlaps the previous tile's work (rows 8j + 2 tig + e;
+    // the row index is even, so each pair is one aligned 8-byte load)
+    auto fetch_ln = [&](int tile, float2 (&dst)[2]) {
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int tok = t0 + tile * kTcTile + r0 + 8 * j + 2 * tig;
+        dst[j] = (lnh && tile < ntiles && tok < t1) ? *reinterpret_cast<const float2*>(lnh + tok)
+                                                    : make_float2(0.f, 0.f);
+      }
+    };
+    float2 ln_cur[2], ln_next[2];
+    fetch_ln(0, ln_cur);
     for (int i = 0; i < ntiles; ++i) {
+      fetch_ln(i + 1, ln_next);
       const int s = i % kTcStages;
-      if (!mbar_wait(&full[s], (i / kTcStages) & 1)) {
+      // ldmatrix / mma are warp-collective: the whole warp leaves together
+      if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (i / kTcStages) & 1))) {
         set_flag(flags, KVS_FLAG_TIMEOUT);
         break;
       }
@@ -180,7 +196,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
           for (int e = 0; e < 2; ++e) {
             const int tok = tok0 + 8 * j + 2 * tig + e;
             float sv = -INFINITY;
-            if (tok < t1) sv = fmaf(sc[j][e], qscale, lnh ? lnh[tok] * kLog2e : 0.f);
+            const float lnv = e ? ln_cur[j].y : ln_cur[j].x;
+            if (tok < t1) sv = fmaf(sc[j][e], qscale, lnv * kLog2e);
             p[j][e] = sv;
             mloc = fmaxf(mloc, sv);
           }
@@ -221,6 +238,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
+      ln_cur[0] = ln_next[0];
+      ln_cur[1] = ln_next[1];
     }
   }
 
@@ -250,7 +269,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
 // Host side: tensor maps over the whole cache ([B*H_kv*T_cap rows, d] bf16) and launch
 // ---------------------------------------------------------------------------
 
-static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (!fn) {
     void* p = nullptr;
@@ -263,14 +282,13 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// 2D map: inner dimension d (contiguous), outer dimension `rows`; boxes of 64 x 64
-// elements (128 bytes x 64 rows) with 128-byte swizzling; rows past the end read as 0.
-static bool encode_rows_map(CUtensorMap* map, const void* base, unsigned long long rows, int d) {
+bool encode_rows_map(CUtensorMap* map, const void* base, unsigned long long rows, int d,
+                     int box_rows) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
   cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)d * sizeof(bf16)};
-  cuuint32_t box[2] = {64, (cuuint32_t)kTcTile};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -311,7 +329,7 @@ cudaError_t launch_decode_tc(const kvs_cache_desc& d, const void* q, void* K, vo
                              const DecodeLayout& Ly, char* ws, cudaStream_t st) {
   const unsigned long long rows = (unsigned long long)d.B * d.H_kv * (unsigned long long)d.T_cap;
   CUtensorMap mK, mV;
-  if (!encode_rows_map(&mK, K, rows, d.d) || !encode_rows_map(&mV, V, rows, d.d))
+  if (!encode_rows_map(&mK, K, rows, d.d, kTcTile) || !encode_rows_map(&mV, V, rows, d.d, kTcTile))
     return cudaErrorInvalidValue;
   const int G = d.H_q / d.H_kv;
 #define KVS_TC(DD, GG) \

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include "kvs.h"
 #include "kvs_common.cuh"
@@ -34,6 +35,18 @@ cudaError_t launch_merge(const kvs_cache_desc& d, const void* K, const void* V, 
 cudaError_t launch_decode(const kvs_cache_desc& d, const void* q, void* K, void* V, float* logn,
                           int32_t* len, const void* k_new, const void* v_new, void* out,
                           const DecodeLayout& Ly, char* ws, cudaStream_t st);
+
+// Driver entry point for tensor maps, and a 2D map over a [rows, d] bf16 array with
+// boxes of 64 elements x box_rows rows and 128-byte swizzling (rows past the end read 0).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
+bool encode_rows_map(CUtensorMap* map, const void* base, unsigned long long rows, int d,
+                     int box_rows);
+
+// Window statistics for bf16 caches on tcgen05 (G*W <= 128), same outputs as above.
+bool window_tc_supported(const kvs_cache_desc& d, int W);
+cudaError_t launch_window_stats_tc(const kvs_cache_desc& d, const void* K, const void* V,
+                                   const float* logn, const int32_t* len, const void* Qw, int W,
+                                   const ScoreLayout& Ly, char* ws, cudaStream_t st);
 
 // The same step for bf16 caches on the TMA + tensor-core kernel.
 bool decode_tc_supported(const kvs_cache_desc& d);

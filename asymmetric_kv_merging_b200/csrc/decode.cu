@@ -161,9 +161,10 @@ decode_kernel(const T* __restrict__ q, T* K, T* V, float* logn, int32_t* len,
 #pragma unroll
     for (int k = 0; k < CPL; ++k) s_acc[warp][g][lane * CPL + k] = acc[g][k];
   __syncthreads();
-  decode_epilogue<T, D, G, kDecWarps>(s_m, s_l, s_acc, qs, s_new, &s_last, tid, kDecThreads, head,
-                                      split, nsplit, L, bad, T_cap, K, V, logn, len, k_new, v_new,
-                                      out, counters, part_ml, part_acc, flags);
+  static_assert(kDecWarps * G * D >= 2 * G * 64 + 2 * G, "combine scratch fits s_acc");
+  decode_epilogue<T, D, G, kDecWarps>(s_m, s_l, s_acc, qs, s_new, &s_last, &s_acc[0][0][0], tid,
+                                      kDecThreads, head, split, nsplit, L, bad, T_cap, K, V, logn,
+                                      len, k_new, v_new, out, counters, part_ml, part_acc, flags);
 }
 
 template <typename T, int D>

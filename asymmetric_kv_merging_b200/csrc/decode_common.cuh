@@ -20,11 +20,14 @@ __device__ __forceinline__ void store_out<bf16>(bf16* p, float v) { *p = __float
 // All `nthreads` threads of the CTA call this after __syncthreads(); the warp partials
 // sm[NW][G], sl[NW][G], sacc[NW][G][D] live in shared memory. qs[G][D] holds the
 // scaled queries (fp32, log2 domain). Query head g of KV head `head` (= b*H_kv + h)
-// is head*G + g. Returns after the CTA's part is done.
+// is head*G + g. `scratch` is shared memory for 2*G*nsplit + 2*G floats that may
+// overlap sacc (sacc is consumed before scratch is written). Returns after the CTA's
+// part is done.
 template <typename T, int D, int G, int NW>
 __device__ __forceinline__ void decode_epilogue(
     const float (*sm)[G], const float (*sl)[G], const float (*sacc)[G][D], const float (*qs)[D],
-    float* s_new, int* s_last, int tid, int nthreads, int head, int split, int nsplit, int L,
+    float* s_new, int* s_last, float* scratch, int tid, int nthreads, int head, int split,
+    int nsplit, int L,
     bool bad, int T_cap, T* K, T* V, float* logn, int32_t* len, const T* k_new,
     const T* v_new, T* out, int32_t* counters, float* part_ml, float* part_acc,
     int32_t* flags) {
@@ -70,32 +73,55 @@ __device__ __forceinline__ void decode_epilogue(
       if (lane == 0) s_new[g] = sp;   // appended rows have count 1: no bias
     }
   }
+  // The combine must not wait on one L2 round trip per split: stage every split's
+  // (m, l) in shared memory with one parallel pass, turn them into scale factors,
+  // then reduce the accumulators four columns per thread with independent loads.
+  float* f_m = scratch;                    // [G * nsplit]   split maxima, then scale factors
+  float* f_l = scratch + G * nsplit;       // [G * nsplit]   split sums
+  float* g_stat = f_l + G * nsplit;        // [G][2]         combined (M, 1/L)
+  for (int i = tid; i < G * nsplit; i += nthreads) {
+    const float2 ml = __ldcg(reinterpret_cast<const float2*>(pml) + i);
+    f_m[i] = ml.x;
+    f_l[i] = ml.y;
+  }
   __syncthreads();
-  for (int i = tid; i < G * D; i += nthreads) {
-    const int g = i / D, c = i - g * D;
-    float M = -INFINITY;
+  for (int g = tid; g < G; g += nthreads) {
+    float M = (append && fits) ? s_new[g] : -INFINITY;
+    for (int s = 0; s < nsplit; ++s)
+      if (f_l[g * nsplit + s] > 0.f) M = fmaxf(M, f_m[g * nsplit + s]);
+    float Ls = (append && fits && M > -INFINITY) ? exp2f(s_new[g] - M) : 0.f;
     for (int s = 0; s < nsplit; ++s) {
-      const float ls = __ldcg(pml + ((size_t)g * nsplit + s) * 2 + 1);
-      if (ls > 0.f) M = fmaxf(M, __ldcg(pml + ((size_t)g * nsplit + s) * 2));
+      const float ls = f_l[g * nsplit + s];
+      const float f = (ls > 0.f && M > -INFINITY) ? exp2f(f_m[g * nsplit + s] - M) : 0.f;
+      f_m[g * nsplit + s] = f;               // now the scale factor of split s
+      Ls = fmaf(ls, f, Ls);
     }
-    if (append && fits) M = fmaxf(M, s_new[g]);
-    float Ls = 0.f, A = 0.f;
-    if (M > -INFINITY) {
-      for (int s = 0; s < nsplit; ++s) {
-        const float ls = __ldcg(pml + ((size_t)g * nsplit + s) * 2 + 1);
-        if (ls > 0.f) {
-          const float f = exp2f(__ldcg(pml + ((size_t)g * nsplit + s) * 2) - M);
-          Ls = fmaf(ls, f, Ls);
-          A = fmaf(__ldcg(pacc + ((size_t)g * nsplit + s) * D + c), f, A);
-        }
-      }
-      if (append && fits) {
-        const float f = exp2f(s_new[g] - M);
-        Ls += f;
-        A = fmaf(to_f32(vn[c]), f, A);
+    g_stat[2 * g] = M;
+    g_stat[2 * g + 1] = Ls > 0.f ? 1.f / Ls : 0.f;
+  }
+  __syncthreads();
+  for (int e = tid; e < G * (D / 4); e += nthreads) {
+    const int g = e / (D / 4), c = (e - g * (D / 4)) * 4;
+    float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4* src = reinterpret_cast<const float4*>(pacc + (size_t)g * nsplit * D + c);
+#pragma unroll 8
+    for (int s = 0; s < nsplit; ++s) {
+      const float f = f_m[g * nsplit + s];
+      if (f != 0.f) {
+        const float4 v = __ldcg(src + (size_t)s * (D / 4));
+        A.x = fmaf(v.x, f, A.x); A.y = fmaf(v.y, f, A.y);
+        A.z = fmaf(v.z, f, A.z); A.w = fmaf(v.w, f, A.w);
       }
     }
-    store_out<T>(out + ((size_t)head * G + g) * D + c, Ls > 0.f ? A / Ls : 0.f);
+    if (append && fits) {
+      const float f = exp2f(s_new[g] - g_stat[2 * g]);
+      A.x = fmaf(to_f32(vn[c]), f, A.x); A.y = fmaf(to_f32(vn[c + 1]), f, A.y);
+      A.z = fmaf(to_f32(vn[c + 2]), f, A.z); A.w = fmaf(to_f32(vn[c + 3]), f, A.w);
+    }
+    const float inv = g_stat[2 * g + 1];
+    T* o = out + ((size_t)head * G + g) * D + c;
+    store_out<T>(o, A.x * inv); store_out<T>(o + 1, A.y * inv);
+    store_out<T>(o + 2, A.z * inv); store_out<T>(o + 3, A.w * inv);
   }
   if (append) {
     if (fits) {

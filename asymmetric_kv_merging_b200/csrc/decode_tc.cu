@@ -59,6 +59,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
 
   const int head = blockIdx.y, split = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  pdl_trigger();
+  pdl_wait();     // nothing above this line touches global memory
   int L = len[head];
   const bool bad = L < 0 || L > T_cap;
   if (bad) {
@@ -260,9 +262,14 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     }
   }
   __syncthreads();
-  decode_epilogue<bf16, D, G, kTcConsumers>(s_m, s_l, s_acc, qs, s_new, &s_last, tid, kTcThreads,
-                                            head, split, nsplit, L, bad, T_cap, K, V, logn, len,
-                                            k_new, v_new, out, counters, part_ml, part_acc, flags);
+  // the combine scratch sits in the ring after the warp partials
+  float* scratch = reinterpret_cast<float*>(base) + kTcConsumers * G * D;
+  static_assert((kTcConsumers * G * D + 2 * G * 64 + 2 * G) * 4 <= kTcStages * S::kStageBytes,
+                "combine scratch fits the ring");
+  decode_epilogue<bf16, D, G, kTcConsumers>(s_m, s_l, s_acc, qs, s_new, &s_last, scratch, tid,
+                                            kTcThreads, head, split, nsplit, L, bad, T_cap, K, V,
+                                            logn, len, k_new, v_new, out, counters, part_ml,
+                                            part_acc, flags);
 }
 
 // ---------------------------------------------------------------------------
@@ -314,14 +321,25 @@ static cudaError_t launch_tc(const kvs_cache_desc& d, const CUtensorMap& mK, con
       return cudaErrorInvalidValue;
     attr = true;
   }
-  dim3 grid(Ly.nsplit, d.B * d.H_kv);
-  kfn<<<grid, kTcThreads, TcShape<D>::kSmem, st>>>(
-      mK, mV, (const bf16*)q, (bf16*)K, (bf16*)V, logn, len, (const bf16*)k_new,
-      (const bf16*)v_new, (bf16*)out, d.T_cap, Ly.nsplit, reinterpret_cast<int32_t*>(ws + Ly.counters),
-      reinterpret_cast<float*>(ws + Ly.part_ml), reinterpret_cast<float*>(ws + Ly.part_acc),
-      reinterpret_cast<int32_t*>(ws));
+  // programmatic serialization lets this grid launch while the previous one drains;
+  // the kernel waits for it (griddepcontrol.wait) before any global-memory access
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(Ly.nsplit, d.B * d.H_kv);
+  cfg.blockDim = dim3(kTcThreads);
+  cfg.dynamicSmemBytes = TcShape<D>::kSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(
+      &cfg, kfn, mK, mV, (const bf16*)q, (bf16*)K, (bf16*)V, logn, len, (const bf16*)k_new,
+      (const bf16*)v_new, (bf16*)out, d.T_cap, Ly.nsplit,
+      reinterpret_cast<int32_t*>(ws + Ly.counters), reinterpret_cast<float*>(ws + Ly.part_ml),
+      reinterpret_cast<float*>(ws + Ly.part_acc), reinterpret_cast<int32_t*>(ws));
   count_launches(1);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_decode_tc(const kvs_cache_desc& d, const void* q, void* K, void* V, float* logn,

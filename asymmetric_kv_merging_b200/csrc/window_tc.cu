@@ -69,7 +69,7 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   __shared__ volatile int s_abort;               // set when any wait gives up
   __shared__ float red[kWtSoft][kWtKeys];        // per-warp column sums (pass B)
   __shared__ float abar[kWtKeys];                // alpha_bar of the tile's keys (pass B)
-  __shared__ float ored[(D == 64) ? 2 * 64 : 1]; // row-group partials of o_bar (d = 64)
+  __shared__ float ored[256];                    // row-group partials of o_bar (pass B)
 
   const int unit = blockIdx.y, split = blockIdx.x;
   const int b = unit / H_kv, h = unit - b * H_kv;
@@ -197,7 +197,7 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       const float M0 = stats[((size_t)unit * Qn + r) * 2], L0 = stats[((size_t)unit * Qn + r) * 2 + 1];
       if (L0 > 0.f && isfinite(L0) && isfinite(M0)) { Mr = M0; invL = 1.f / L0; }
     }
-    float oacc = 0.f;                             // pass B: o_bar partial of one column
+    float oacc2[2] = {0.f, 0.f};                  // pass B: o_bar partials of a column pair
     // this thread's key of each tile: its log-count is fetched one tile ahead
     float ln_next = (lnh && t0 + st < t1) ? lnh[t0 + st] : 0.f;
     for (int i = 0; i < ntiles; ++i) {
@@ -230,23 +230,38 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         lns[buf][st] = ln_cur * kLog2e;
         named_bar(1, kWtSoft * 32);
       }
-      // logits in the log2 domain; the causal window and the split end are masked
+      // logits in the log2 domain. Only the split's last tile and the last W cache
+      // positions need masks (split end, causal window); interior tiles skip them.
+      const bool interior = tb + kWtKeys <= t1 && tb + kWtKeys - 1 <= L - W;
+      if (interior && live && row_ok) {
 #pragma unroll
-      for (int j = 0; j < kWtKeys; ++j) {
-        const int t = tb + j;
-        const bool vis = live && row_ok && t < t1 && t <= pos;
-        sv[j] = vis ? fmaf(sv[j], qscale, lnh ? lns[buf][j] : 0.f) : -INFINITY;
+        for (int j = 0; j < kWtKeys; ++j) sv[j] = fmaf(sv[j], qscale, lnh ? lns[buf][j] : 0.f);
+      } else {
+#pragma unroll
+        for (int j = 0; j < kWtKeys; ++j) {
+          const int t = tb + j;
+          const bool vis = live && row_ok && t < t1 && t <= pos;
+          sv[j] = vis ? fmaf(sv[j], qscale, lnh ? lns[buf][j] : 0.f) : -INFINITY;
+        }
       }
       if constexpr (!MASS) {
-        float tmax = -INFINITY;
+        // eight independent chains instead of one 128-long dependency chain
+        float tm[8];
 #pragma unroll
-        for (int j = 0; j < kWtKeys; ++j) tmax = fmaxf(tmax, sv[j]);
+        for (int k = 0; k < 8; ++k) tm[k] = sv[k];
+#pragma unroll
+        for (int j = 8; j < kWtKeys; ++j) tm[j & 7] = fmaxf(tm[j & 7], sv[j]);
+        const float tmax = fmaxf(fmaxf(fmaxf(tm[0], tm[1]), fmaxf(tm[2], tm[3])),
+                                 fmaxf(fmaxf(tm[4], tm[5]), fmaxf(tm[6], tm[7])));
         const float m_new = fmaxf(m, tmax);
         if (m_new > -INFINITY) {
-          float ps = 0.f;
+          float ps[8];
 #pragma unroll
-          for (int j = 0; j < kWtKeys; ++j) ps += exp2f(sv[j] - m_new);
-          l = l * exp2f(m - m_new) + ps;
+          for (int k = 0; k < 8; ++k) ps[k] = 0.f;
+#pragma unroll
+          for (int j = 0; j < kWtKeys; ++j) ps[j & 7] += exp2f(sv[j] - m_new);
+          const float psum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+          l = l * exp2f(m - m_new) + psum;
           m = m_new;
         }
       } else {
@@ -279,15 +294,34 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         bool vlive = mbar_wait_ab(&v_full[vs], (i / VS) & 1, &s_abort);
         named_bar(1, kWtSoft * 32);
         if (vlive) {
-          // o_bar partial: thread st takes column st % D over every (128 / D)-th row
+          // o_bar partial: thread st takes the column pair (2 cp, 2 cp + 1), cp = st % (D/2),
+          // over rows j = rg, rg + NRG, ... (rg = st / (D/2)); two accumulators per column
+          constexpr int NRG = 256 / D;
           const unsigned char* vt = base + S::kVOff + vs * S::kTile;
-          const int c = st % D, cc = c & 63, bx = c >> 6;
+          const int cp = st % (D / 2), rg = st / (D / 2);
+          const int cc = (2 * cp) & 63, bx = (2 * cp) >> 6;
           const int nvalid = min(kWtKeys, t1 - tb);
-          for (int j = st / D; j < nvalid; j += kWtKeys / D) {
-            const bf16 x = *reinterpret_cast<const bf16*>(
+          float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
+          int j = rg;
+          for (; j + NRG < nvalid; j += 2 * NRG) {
+            const uint32_t x = *reinterpret_cast<const uint32_t*>(
                 vt + bx * S::kBox + j * 128 + ((((cc >> 3) ^ (j & 7)) << 4) + (cc & 7) * 2));
-            oacc = fmaf(abar[j], __bfloat162float(x), oacc);
+            const int j2 = j + NRG;
+            const uint32_t y = *reinterpret_cast<const uint32_t*>(
+                vt + bx * S::kBox + j2 * 128 + ((((cc >> 3) ^ (j2 & 7)) << 4) + (cc & 7) * 2));
+            a0 = fmaf(abar[j], bf16_lo(x), a0);
+            a1 = fmaf(abar[j], bf16_hi(x), a1);
+            b0 = fmaf(abar[j2], bf16_lo(y), b0);
+            b1 = fmaf(abar[j2], bf16_hi(y), b1);
           }
+          if (j < nvalid) {
+            const uint32_t x = *reinterpret_cast<const uint32_t*>(
+                vt + bx * S::kBox + j * 128 + ((((cc >> 3) ^ (j & 7)) << 4) + (cc & 7) * 2));
+            a0 = fmaf(abar[j], bf16_lo(x), a0);
+            a1 = fmaf(abar[j], bf16_hi(x), a1);
+          }
+          oacc2[0] += a0 + b0;
+          oacc2[1] += a1 + b1;
         } else {
           set_flag(flags, KVS_FLAG_TIMEOUT);
         }
@@ -301,12 +335,19 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         part_ml[(((size_t)unit * nsplit + split) * Qn + r) * 2 + 0] = m;
         part_ml[(((size_t)unit * nsplit + split) * Qn + r) * 2 + 1] = l;
       }
-    } else if constexpr (D == 128) {
-      opart[((size_t)unit * nsplit + split) * D + st] = oacc;
     } else {
-      ored[st] = oacc;
+      // combine the row groups of each column pair
+      constexpr int NRG = 256 / D;
+      const int cp = st % (D / 2), rg = st / (D / 2);
+      ored[rg * D + 2 * cp] = oacc2[0];
+      ored[rg * D + 2 * cp + 1] = oacc2[1];
       named_bar(1, kWtSoft * 32);
-      if (st < D) opart[((size_t)unit * nsplit + split) * D + st] = ored[st] + ored[st + D];
+      if (st < D) {
+        float a = 0.f;
+#pragma unroll
+        for (int k = 0; k < NRG; ++k) a += ored[k * D + st];
+        opart[((size_t)unit * nsplit + split) * D + st] = a;
+      }
     }
   }
 

@@ -102,16 +102,16 @@ __device__ __forceinline__ void decode_epilogue(
   __syncthreads();
   for (int e = tid; e < G * (D / 4); e += nthreads) {
     const int g = e / (D / 4), c = (e - g * (D / 4)) * 4;
+    // every split wrote its accumulator (zeros when it saw no rows), so the loads need
+    // no guard and sixteen of them can be in flight at once
     float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
     const float4* src = reinterpret_cast<const float4*>(pacc + (size_t)g * nsplit * D + c);
-#pragma unroll 8
+#pragma unroll 16
     for (int s = 0; s < nsplit; ++s) {
       const float f = f_m[g * nsplit + s];
-      if (f != 0.f) {
-        const float4 v = __ldcg(src + (size_t)s * (D / 4));
-        A.x = fmaf(v.x, f, A.x); A.y = fmaf(v.y, f, A.y);
-        A.z = fmaf(v.z, f, A.z); A.w = fmaf(v.w, f, A.w);
-      }
+      const float4 v = __ldcg(src + (size_t)s * (D / 4));
+      A.x = fmaf(v.x, f, A.x); A.y = fmaf(v.y, f, A.y);
+      A.z = fmaf(v.z, f, A.z); A.w = fmaf(v.w, f, A.w);
     }
     if (append && fits) {
       const float f = exp2f(s_new[g] - g_stat[2 * g]);

@@ -126,15 +126,26 @@ select_kernel(const float* __restrict__ score, const int32_t* __restrict__ len,
         const int hh = h_first + i;
         const int P = hinfo[hh].P;
         const float* sc = score + (size_t)hh * pstride;
-        for (int p0 = 0; p0 < P; p0 += kSelThreads) {
-          const int p = p0 + tid;
-          const bool in = p < P;
-          const uint32_t key = in ? score_key(sc[p]) : 0u;
-          const bool match = in && ((key & pmask) == prefix);
-          const unsigned dg = (key >> shift) & 255u;
-          // aggregate equal digits inside the warp before the shared atomic
-          const unsigned peers = __match_any_sync(0xffffffffu, match ? dg : 0x100u + lane);
-          if (match && (__ffs(peers) - 1) == lane) atomicAdd(&hist[dg], __popc(peers));
+        // eight independent loads per thread are in flight before any is used
+        constexpr int kBatch = 8;
+        for (int p0 = 0; p0 < P; p0 += kSelThreads * kBatch) {
+          float v[kBatch];
+#pragma unroll
+          for (int k = 0; k < kBatch; ++k) {
+            const int p = p0 + k * kSelThreads + tid;
+            v[k] = p < P ? sc[p] : 0.f;
+          }
+#pragma unroll
+          for (int k = 0; k < kBatch; ++k) {
+            const int p = p0 + k * kSelThreads + tid;
+            const bool in = p < P;
+            const uint32_t key = in ? score_key(v[k]) : 0u;
+            const bool match = in && ((key & pmask) == prefix);
+            const unsigned dg = (key >> shift) & 255u;
+            // aggregate equal digits inside the warp before the shared atomic
+            const unsigned peers = __match_any_sync(0xffffffffu, match ? dg : 0x100u + lane);
+            if (match && (__ffs(peers) - 1) == lane) atomicAdd(&hist[dg], __popc(peers));
+          }
         }
       }
       __syncthreads();
@@ -169,25 +180,44 @@ select_kernel(const float* __restrict__ score, const int32_t* __restrict__ len,
 
   // Per block counts of keys below / equal to the threshold, (h, block) order.
   const int nent = nh * nblk;
-  for (int e0 = 0; e0 < nent; e0 += kSelThreads / 32) {
-    const int e = e0 + warp;
-    if (e < nent) {
+  if (R == 0 || R == Ptot) {
+    // nothing or everything is merged: every count follows from P alone, no score is read
+    for (int e = tid; e < nent; e += kSelThreads) {
       const int i = e / nblk, j = e - i * nblk;
       const int hh = h_first + i;
       const int P = hinfo[hh].P;
-      const float* sc = score + (size_t)hh * pstride;
-      int lt = 0, eq = 0;
-      for (int k = 0; k < kMergePairsPerBlock; k += 32) {
-        const int p = j * kMergePairsPerBlock + k + lane;
-        const bool in = p < P;
-        const uint32_t key = in ? score_key(sc[p]) : 0u;
-        lt += __popc(__ballot_sync(0xffffffffu, in && key < thr));
-        eq += __popc(__ballot_sync(0xffffffffu, in && key == thr));
-      }
-      if (lane == 0) blk[(size_t)hh * nblk + j] = make_int2(lt, eq);
+      const int in_blk = max(0, min(kMergePairsPerBlock, P - j * kMergePairsPerBlock));
+      blk[(size_t)hh * nblk + j] = make_int2(R == 0 ? 0 : in_blk, 0);
     }
+    __syncthreads();
+  } else {
+    for (int e0 = 0; e0 < nent; e0 += kSelThreads / 32) {
+      const int e = e0 + warp;
+      if (e < nent) {
+        const int i = e / nblk, j = e - i * nblk;
+        const int hh = h_first + i;
+        const int P = hinfo[hh].P;
+        const float* sc = score + (size_t)hh * pstride;
+        int lt = 0, eq = 0;
+        float v[kMergePairsPerBlock / 32];
+#pragma unroll
+        for (int k = 0; k < kMergePairsPerBlock / 32; ++k) {
+          const int p = j * kMergePairsPerBlock + k * 32 + lane;
+          v[k] = p < P ? sc[p] : 0.f;
+        }
+#pragma unroll
+        for (int k = 0; k < kMergePairsPerBlock / 32; ++k) {
+          const int p = j * kMergePairsPerBlock + k * 32 + lane;
+          const bool in = p < P;
+          const uint32_t key = in ? score_key(v[k]) : 0u;
+          lt += __popc(__ballot_sync(0xffffffffu, in && key < thr));
+          eq += __popc(__ballot_sync(0xffffffffu, in && key == thr));
+        }
+        if (lane == 0) blk[(size_t)hh * nblk + j] = make_int2(lt, eq);
+      }
+    }
+    __syncthreads();
   }
-  __syncthreads();
   // Unit-wide exclusive scans of both counts.
   int carry_lt = 0, carry_eq = 0;
   for (int e0 = 0; e0 < nent; e0 += kSelThreads) {

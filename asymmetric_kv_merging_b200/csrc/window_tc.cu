@@ -14,8 +14,9 @@
 // Warp roles: warp 0 issues TMA tile loads (128-byte swizzle, no multicast) of Q once
 // and of K (and V) per 128-key tile into mbarrier-guarded rings; warp 1 owns the
 // tensor memory (two 128-column fp32 S buffers) and one thread issues tcgen05.mma
-// with smem descriptors, committing to mbarriers; warps 2-5 read S rows from tensor
-// memory (one row per thread) and do the softmax arithmetic. Every wait is bounded.
+// with smem descriptors, committing to mbarriers; warps 2-9 read S rows from tensor
+// memory (one row, half of the keys, per thread) and do the softmax arithmetic.
+// Every wait is bounded.
 #include <cudaTypedefs.h>
 
 #include "kvs_common.cuh"
@@ -26,7 +27,7 @@ namespace kvs {
 
 constexpr int kWtKeys = 128;            // keys per tile: MMA N
 constexpr int kWtRows = 128;            // window-query rows, padded: MMA M
-constexpr int kWtSoft = 4;              // softmax warps (one TMEM lane quarter each)
+constexpr int kWtSoft = 8;              // softmax warps (two per TMEM lane quarter)
 constexpr int kWtThreads = (2 + kWtSoft) * 32;
 constexpr uint32_t kWtTmemCols = 256;   // two S buffers of 128 fp32 columns
 
@@ -67,9 +68,9 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   uint64_t* v_empty = v_full + VS;               // VS
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_abort;               // set when any wait gives up
-  __shared__ float red[kWtSoft][kWtKeys];        // per-warp column sums (pass B)
+  __shared__ float red[4][kWtKeys];              // column sums per lane quarter (pass B)
   __shared__ float abar[kWtKeys];                // alpha_bar of the tile's keys (pass B)
-  __shared__ float ored[256];                    // row-group partials of o_bar (pass B)
+  __shared__ float ored[2 * kWtSoft * 32];       // row-group partials of o_bar (pass B)
 
   const int unit = blockIdx.y, split = blockIdx.x;
   const int b = unit / H_kv, h = unit - b * H_kv;
@@ -181,38 +182,46 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     }
     __syncwarp();
   } else {
-    // ---------------- softmax warps: one window-query row (TMEM lane) per thread ----
-    const int quarter = warp & 3;                 // warps 2..5 own lane quarters 2, 3, 0, 1
+    // ---------------- softmax warps: two per TMEM lane quarter ----------------
+    // warp 2 + sw (sw = 0..7) reads lane quarter (warp & 3), i.e. window-query rows
+    // 32 * quarter + lane, and the key columns [NC * half, NC * half + NC) of each tile
+    constexpr int NC = kWtKeys / (kWtSoft / 4);   // 64 key columns per softmax warp
+    constexpr int NST = kWtSoft * 32;             // 256 softmax threads
+    const int sw = warp - 2;
+    const int quarter = warp & 3;
+    const int half = sw >> 2;
+    const int c0w = half * NC;
     const int r = quarter * 32 + lane;            // window-query row of the KV head
-    const int st = tid - 64;                      // index among the 128 softmax threads
+    const int st = tid - 64;                      // index among the softmax threads
     const int pos = L - W + (r % W);              // last cache position row r attends
     const bool row_ok = r < Qn && pos >= 0;
     const int Qv = G * min(W, L);                 // window queries with a position >= 0
     const float qscale = kLog2e / sqrtf((float)D);
     const float* lnh = logn ? logn + (size_t)unit * T_cap : nullptr;
-    __shared__ float lns[2][kWtKeys];             // log2(e) * logn of the tile's keys
-    float m = -INFINITY, l = 0.f;                 // pass A: running row statistics
+    __shared__ __align__(16) float lns[2][kWtKeys];   // log2(e) * logn of the tile's keys
+    __shared__ float rowstat[kWtRows][2];         // pass A: second half's (m, l) per row
+    float m = -INFINITY, l = 0.f;                 // pass A: running statistics of the half-row
     float Mr = 0.f, invL = 0.f;                   // pass B: final row statistics
     if (MASS && row_ok) {
       const float M0 = stats[((size_t)unit * Qn + r) * 2], L0 = stats[((size_t)unit * Qn + r) * 2 + 1];
       if (L0 > 0.f && isfinite(L0) && isfinite(M0)) { Mr = M0; invL = 1.f / L0; }
     }
     float oacc2[2] = {0.f, 0.f};                  // pass B: o_bar partials of a column pair
-    // this thread's key of each tile: its log-count is fetched one tile ahead
-    float ln_next = (lnh && t0 + st < t1) ? lnh[t0 + st] : 0.f;
+    // each tile's log-counts are fetched one tile ahead (threads st < 128, one key each)
+    float ln_next = (lnh && st < kWtKeys && t0 + st < t1) ? lnh[t0 + st] : 0.f;
     for (int i = 0; i < ntiles; ++i) {
       const int buf = i & 1;
       const int tb = t0 + i * kWtKeys;
       const float ln_cur = ln_next;
-      if (lnh) ln_next = (tb + kWtKeys + st < t1) ? lnh[tb + kWtKeys + st] : 0.f;
+      if (lnh && st < kWtKeys) ln_next = (tb + kWtKeys + st < t1) ? lnh[tb + kWtKeys + st] : 0.f;
       bool live = mbar_wait_ab(&s_full[buf], (i / 2) & 1, &s_abort);
       live = __all_sync(0xffffffffu, live);       // tcgen05.ld is warp-collective
-      float sv[kWtKeys];
+      float sv[NC];
       if (live) {
         tc_fence_after();
-        const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * kWtKeys);
+        const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * kWtKeys + c0w);
 #pragma unroll
-        for (int c = 0; c < kWtKeys / 32; ++c) {
+        for (int c = 0; c < NC / 32; ++c) {
           float part[32];
           tmem_ld32(ta + c * 32, part);
 #pragma unroll
@@ -221,36 +230,47 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       } else {
         set_flag(flags, KVS_FLAG_TIMEOUT);
 #pragma unroll
-        for (int j = 0; j < kWtKeys; ++j) sv[j] = 0.f;
+        for (int j = 0; j < NC; ++j) sv[j] = 0.f;
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&s_empty[buf]);  // the S buffer may be overwritten now
+      if (lane == 0) mbar_arrive(&s_empty[buf]);  // this warp is done with the S buffer
       if (lnh) {
-        lns[buf][st] = ln_cur * kLog2e;
-        named_bar(1, kWtSoft * 32);
+        if (st < kWtKeys) lns[buf][st] = ln_cur * kLog2e;
+        named_bar(1, NST);
       }
       // logits in the log2 domain. Only the split's last tile and the last W cache
       // positions need masks (split end, causal window); interior tiles skip them.
       const bool interior = tb + kWtKeys <= t1 && tb + kWtKeys - 1 <= L - W;
       if (interior && live && row_ok) {
+        if (lnh) {
 #pragma unroll
-        for (int j = 0; j < kWtKeys; ++j) sv[j] = fmaf(sv[j], qscale, lnh ? lns[buf][j] : 0.f);
+          for (int j = 0; j < NC; j += 4) {
+            const float4 lv = *reinterpret_cast<const float4*>(&lns[buf][c0w + j]);
+            sv[j] = fmaf(sv[j], qscale, lv.x);
+            sv[j + 1] = fmaf(sv[j + 1], qscale, lv.y);
+            sv[j + 2] = fmaf(sv[j + 2], qscale, lv.z);
+            sv[j + 3] = fmaf(sv[j + 3], qscale, lv.w);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < NC; ++j) sv[j] *= qscale;
+        }
       } else {
 #pragma unroll
-        for (int j = 0; j < kWtKeys; ++j) {
-          const int t = tb + j;
+        for (int j = 0; j < NC; ++j) {
+          const int t = tb + c0w + j;
           const bool vis = live && row_ok && t < t1 && t <= pos;
-          sv[j] = vis ? fmaf(sv[j], qscale, lnh ? lns[buf][j] : 0.f) : -INFINITY;
+          sv[j] = vis ? fmaf(sv[j], qscale, lnh ? lns[buf][c0w + j] : 0.f) : -INFINITY;
         }
       }
       if constexpr (!MASS) {
-        // eight independent chains instead of one 128-long dependency chain
+        // eight independent chains instead of one long dependency chain
         float tm[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) tm[k] = sv[k];
 #pragma unroll
-        for (int j = 8; j < kWtKeys; ++j) tm[j & 7] = fmaxf(tm[j & 7], sv[j]);
+        for (int j = 8; j < NC; ++j) tm[j & 7] = fmaxf(tm[j & 7], sv[j]);
         const float tmax = fmaxf(fmaxf(fmaxf(tm[0], tm[1]), fmaxf(tm[2], tm[3])),
                                  fmaxf(fmaxf(tm[4], tm[5]), fmaxf(tm[6], tm[7])));
         const float m_new = fmaxf(m, tmax);
@@ -259,7 +279,7 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 #pragma unroll
           for (int k = 0; k < 8; ++k) ps[k] = 0.f;
 #pragma unroll
-          for (int j = 0; j < kWtKeys; ++j) ps[j & 7] += exp2f(sv[j] - m_new);
+          for (int j = 0; j < NC; ++j) ps[j & 7] += exp2f(sv[j] - m_new);
           const float psum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
           l = l * exp2f(m - m_new) + psum;
           m = m_new;
@@ -268,7 +288,7 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         // normalised probabilities; column sums over this warp's 32 rows by a
         // transpose-reduce: after it, lane j holds the sum of column j of each 32-column block
 #pragma unroll
-        for (int c = 0; c < kWtKeys / 32; ++c) {
+        for (int c = 0; c < NC / 32; ++c) {
           float v[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = exp2f(sv[c * 32 + j] - Mr) * invL;
@@ -282,21 +302,23 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
               v[k] = keep + __shfl_xor_sync(0xffffffffu, give, o);
             }
           }
-          red[quarter][c * 32 + lane] = v[0];
+          red[quarter][c0w + c * 32 + lane] = v[0];
         }
-        named_bar(1, kWtSoft * 32);
-        const int t = tb + st;
-        float a = (red[0][st] + red[1][st] + red[2][st] + red[3][st]) / (float)(Qv > 0 ? Qv : 1);
-        a = (t < t1 && Qv > 0) ? a : 0.f;
-        if (t < t1) alpha[(size_t)unit * T_cap + t] = a;
-        abar[st] = a;
+        named_bar(1, NST);
+        if (st < kWtKeys) {
+          const int t = tb + st;
+          float a = (red[0][st] + red[1][st] + red[2][st] + red[3][st]) / (float)(Qv > 0 ? Qv : 1);
+          a = (t < t1 && Qv > 0) ? a : 0.f;
+          if (t < t1) alpha[(size_t)unit * T_cap + t] = a;
+          abar[st] = a;
+        }
         const int vs = i % VS;
         bool vlive = mbar_wait_ab(&v_full[vs], (i / VS) & 1, &s_abort);
-        named_bar(1, kWtSoft * 32);
+        named_bar(1, NST);
         if (vlive) {
           // o_bar partial: thread st takes the column pair (2 cp, 2 cp + 1), cp = st % (D/2),
           // over rows j = rg, rg + NRG, ... (rg = st / (D/2)); two accumulators per column
-          constexpr int NRG = 256 / D;
+          constexpr int NRG = 2 * NST / D;
           const unsigned char* vt = base + S::kVOff + vs * S::kTile;
           const int cp = st % (D / 2), rg = st / (D / 2);
           const int cc = (2 * cp) & 63, bx = (2 * cp) >> 6;
@@ -331,17 +353,23 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     }
     // per-split outputs
     if constexpr (!MASS) {
-      if (r < Qn) {
-        part_ml[(((size_t)unit * nsplit + split) * Qn + r) * 2 + 0] = m;
-        part_ml[(((size_t)unit * nsplit + split) * Qn + r) * 2 + 1] = l;
+      // merge the two half-rows of each window query
+      if (half == 1) { rowstat[r][0] = m; rowstat[r][1] = l; }
+      named_bar(1, NST);
+      if (half == 0 && r < Qn) {
+        const float m1 = rowstat[r][0], l1 = rowstat[r][1];
+        const float M = fmaxf(m, m1);
+        const float Ls = M > -INFINITY ? l * exp2f(m - M) + l1 * exp2f(m1 - M) : 0.f;
+        part_ml[(((size_t)unit * nsplit + split) * Qn + r) * 2 + 0] = M;
+        part_ml[(((size_t)unit * nsplit + split) * Qn + r) * 2 + 1] = Ls;
       }
     } else {
       // combine the row groups of each column pair
-      constexpr int NRG = 256 / D;
+      constexpr int NRG = 2 * NST / D;
       const int cp = st % (D / 2), rg = st / (D / 2);
       ored[rg * D + 2 * cp] = oacc2[0];
       ored[rg * D + 2 * cp + 1] = oacc2[1];
-      named_bar(1, kWtSoft * 32);
+      named_bar(1, NST);
       if (st < D) {
         float a = 0.f;
 #pragma unroll

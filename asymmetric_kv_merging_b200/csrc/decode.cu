@@ -52,8 +52,8 @@ __global__ void __launch_bounds__(kDecThreads)
 decode_kernel(const T* __restrict__ q, T* K, T* V, float* logn, int32_t* len,
               const T* __restrict__ k_new,
               const T* __restrict__ v_new, T* __restrict__ out, int H_kv, int T_cap, int nsplit,
-              int32_t* __restrict__ counters, float* __restrict__ part_ml,
-              float* __restrict__ part_acc, int32_t* __restrict__ flags) {
+              int32_t* __restrict__ counters, float* __restrict__ part,
+              int32_t* __restrict__ flags) {
   constexpr int VN = Vec16<T>::n;
   constexpr int VPR = D / VN;              // 16-byte vectors per row
   constexpr int CPL = D / 32;              // output columns per lane
@@ -61,6 +61,8 @@ decode_kernel(const T* __restrict__ q, T* K, T* V, float* logn, int32_t* len,
   __shared__ float s_m[kDecWarps][G], s_l[kDecWarps][G];
   __shared__ __align__(16) float s_acc[kDecWarps][G][D];
   __shared__ float s_new[G];
+  __shared__ float s_fac[G][kMaxDecodeSplits];
+  __shared__ float s_gstat[G][2];
   __shared__ int s_last;
 
   const int head = blockIdx.y, split = blockIdx.x;
@@ -161,10 +163,12 @@ decode_kernel(const T* __restrict__ q, T* K, T* V, float* logn, int32_t* len,
 #pragma unroll
     for (int k = 0; k < CPL; ++k) s_acc[warp][g][lane * CPL + k] = acc[g][k];
   __syncthreads();
-  static_assert(kDecWarps * G * D >= 2 * G * 64 + 2 * G, "combine scratch fits s_acc");
-  decode_epilogue<T, D, G, kDecWarps>(s_m, s_l, s_acc, qs, s_new, &s_last, &s_acc[0][0][0], tid,
-                                      kDecThreads, head, split, nsplit, L, bad, T_cap, K, V, logn,
-                                      len, k_new, v_new, out, counters, part_ml, part_acc, flags);
+  // the (m, l) staging of the last CTA overlays s_acc, which is consumed by then
+  static_assert(kDecWarps * G * D >= 2 * G * kMaxDecodeSplits, "(m, l) staging fits s_acc");
+  const DecodeSmem<D, G, kDecWarps> S{s_m, s_l, s_acc, qs, s_new, s_fac, s_gstat, &s_last};
+  const DecodeArgs<T> a{head, split, nsplit, L, T_cap, bad, K, V, logn, len, k_new, v_new,
+                        out, counters, part, flags};
+  decode_epilogue<T, D, G, kDecWarps>(S, &s_acc[0][0][0], a, tid, kDecThreads);
 }
 
 template <typename T, int D>
@@ -176,12 +180,11 @@ static cudaError_t launch_decode_t(const kvs_cache_desc& d, const void* q, void*
   dim3 grid(Ly.nsplit, d.B * d.H_kv);
   int32_t* flags = reinterpret_cast<int32_t*>(ws);
   int32_t* counters = reinterpret_cast<int32_t*>(ws + Ly.counters);
-  float* pml = reinterpret_cast<float*>(ws + Ly.part_ml);
-  float* pacc = reinterpret_cast<float*>(ws + Ly.part_acc);
+  float* part = reinterpret_cast<float*>(ws + Ly.part);
 #define KVS_DEC(GG)                                                                         \
   decode_kernel<T, D, GG><<<grid, kDecThreads, 0, st>>>(                                   \
       (const T*)q, (T*)K, (T*)V, logn, len, (const T*)k_new, (const T*)v_new, (T*)out,      \
-      d.H_kv, d.T_cap, Ly.nsplit, counters, pml, pacc, flags)
+      d.H_kv, d.T_cap, Ly.nsplit, counters, part, flags)
   switch (G) {
     case 1: KVS_DEC(1); break;
     case 2: KVS_DEC(2); break;

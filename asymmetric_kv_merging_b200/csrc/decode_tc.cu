@@ -33,7 +33,10 @@ struct TcShape {
   static constexpr int kBoxBytes = kTcTile * 128;          // one box of one stage
   static constexpr int kTileBytes = kBoxes * kBoxBytes;    // K (or V) rows of one stage
   static constexpr int kStageBytes = 2 * kTileBytes;       // K then V
-  static constexpr int kSmem = kTcStages * kStageBytes + 2 * kTcStages * 8 + 1024;
+  static constexpr int kRingBytes = kTcStages * kStageBytes;
+  static constexpr int kSmem = kRingBytes + (2 * kTcStages + 1) * 8 + 1024;
+  // the combine stages all splits of at least one query head in the ring
+  static_assert(kMaxDecodeSplits * (D + kPartPad) * 4 <= kRingBytes, "combine staging");
 };
 
 template <int D, int G>
@@ -41,18 +44,21 @@ __global__ void __launch_bounds__(kTcThreads, 2)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                  const bf16* __restrict__ q, bf16* K, bf16* V, float* logn, int32_t* len,
                  const bf16* __restrict__ k_new, const bf16* __restrict__ v_new,
-                 bf16* __restrict__ out, int T_cap, int nsplit, int32_t* counters,
-                 float* part_ml, float* part_acc, int32_t* flags) {
+                 bf16* __restrict__ out, int T_cap, int nsplit, int32_t* counters, float* part,
+                 int32_t* flags) {
   using S = TcShape<D>;
-  static_assert(G * D * 4 * kTcConsumers <= kTcStages * S::kStageBytes, "epilogue overlay");
+  static_assert(kTcConsumers * G * D * 4 <= kTcStages * S::kStageBytes, "warp partials fit the ring");
   extern __shared__ unsigned char dsm[];
   unsigned char* base = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(dsm) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(base + kTcStages * S::kStageBytes);
   uint64_t* empty = full + kTcStages;
+  uint64_t* cbar = empty + kTcStages;              // the combine's bulk copies
   __shared__ __align__(16) float qs[G][D];
   __shared__ float s_m[kTcConsumers][G], s_l[kTcConsumers][G];
   __shared__ float s_new[G];
+  __shared__ float s_fac[G][kMaxDecodeSplits];
+  __shared__ float s_gstat[G][2];
   __shared__ int s_last;
   // after the main loop the stage buffers hold the consumer warps' partial outputs
   float(*s_acc)[G][D] = reinterpret_cast<float(*)[G][D]>(base);
@@ -83,14 +89,18 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kTcConsumers);
     }
+    mbar_init(cbar, 1);
     fence_mbar_init();
   }
   __syncthreads();
 
-  float m_run = -INFINITY, l_run = 0.f;
-  float O[D / 8][4];
+  // per consumer lane: two query-head columns n0 = 2 tig, n1 = 2 tig + 1 of the
+  // transposed problem (running max, this lane's share of the sum) and the
+  // transposed output O^T[d][n] for d = 16 j + grp (+8)
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+  float O[D / 16][4];
 #pragma unroll
-  for (int n = 0; n < D / 8; ++n) O[n][0] = O[n][1] = O[n][2] = O[n][3] = 0.f;
+  for (int j = 0; j < D / 16; ++j) O[j][0] = O[j][1] = O[j][2] = O[j][3] = 0.f;
 
   if (warp == kTcConsumers) {
     // ---------------- producer: one thread issues every TMA load ----------------
@@ -121,36 +131,34 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     __syncwarp();   // reconverge before the CTA-wide barrier after the main loop
   } else {
     // ---------------- consumers: 16 rows of each stage per warp ----------------
-    const int grp = lane >> 2, tig = lane & 3;       // MMA fragment row / column pair
+    // The problem is computed transposed so that the 16 cache rows fill the MMA's M
+    // dimension and the G query heads its N = 8 columns: S^T = K Q^T, O^T += V^T P^T.
+    const int grp = lane >> 2, tig = lane & 3;       // fragment row / column pair
     const int mi = lane >> 3, ri = lane & 7;         // ldmatrix: matrix index, row in matrix
-    // query A fragments: row grp (< G) of the 16-row tile, k pairs (2 tig, +1) and (+8);
-    // rows 8..15 of the tile are padding and stay zero
-    uint32_t qa[D / 16][2];
+    // B operand of S^T = K Q^T: column n = grp holds query head grp (zero past G)
+    uint32_t qb[D / 16][2];
 #pragma unroll
     for (int ks = 0; ks < D / 16; ++ks) {
       if (grp < G) {
         const bf16* qr = q + ((size_t)head * G + grp) * D + ks * 16 + tig * 2;
-        qa[ks][0] = *reinterpret_cast<const uint32_t*>(qr);
-        qa[ks][1] = *reinterpret_cast<const uint32_t*>(qr + 8);
+        qb[ks][0] = *reinterpret_cast<const uint32_t*>(qr);
+        qb[ks][1] = *reinterpret_cast<const uint32_t*>(qr + 8);
       } else {
-        qa[ks][0] = qa[ks][1] = 0u;
+        qb[ks][0] = qb[ks][1] = 0u;
       }
     }
     const float* lnh = logn ? logn + (size_t)head * T_cap : nullptr;
     const int r0 = warp * 16;                        // this warp's rows inside a stage
     const uint32_t ring = smem_u32(base);
-    // log-counts of this lane's four rows of a tile, fetched one tile ahead so the
-    // global-memory latency overlaps the previous tile's work (rows 8j + 2 tig + e;
-    // the row index is even, so each pair is one aligned 8-byte load)
-    auto fetch_ln = [&](int tile, float2 (&dst)[2]) {
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const int tok = t0 + tile * kTcTile + r0 + 8 * j + 2 * tig;
-        dst[j] = (lnh && tile < ntiles && tok < t1) ? *reinterpret_cast<const float2*>(lnh + tok)
-                                                    : make_float2(0.f, 0.f);
-      }
+    // log-counts of this lane's rows grp and grp + 8, fetched one tile ahead so the
+    // global-memory latency overlaps the previous tile's work
+    auto fetch_ln = [&](int tile, float2& dst) {
+      const int tok = t0 + tile * kTcTile + r0 + grp;
+      const bool live = lnh && tile < ntiles;
+      dst.x = (live && tok < t1) ? lnh[tok] : 0.f;
+      dst.y = (live && tok + 8 < t1) ? lnh[tok + 8] : 0.f;
     };
-    float2 ln_cur[2], ln_next[2];
+    float2 ln_cur, ln_next;
     fetch_ln(0, ln_cur);
     for (int i = 0; i < ntiles; ++i) {
       fetch_ln(i + 1, ln_next);
@@ -178,98 +186,93 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
           fence_proxy_async_smem();
           __syncwarp();
         }
-        // logits of the 16 rows: two 8-row n-tiles
-        float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        // S^T (16 rows x 8 columns): A = the K rows, two accumulators to halve the chain
+        float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
-          const int row = r0 + ((mi >> 1) << 3) + ri;
-          const int el = ks * 16 + ((mi & 1) << 3);
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4(kb + (el >> 6) * S::kBoxBytes + swz128(row, (el & 63) >> 3), b0, b1, b2, b3);
-          mma_bf16_16816(sc[0], qa[ks][0], 0u, qa[ks][1], 0u, b0, b1);
-          mma_bf16_16816(sc[1], qa[ks][0], 0u, qa[ks][1], 0u, b2, b3);
+          const int row = r0 + ((mi & 1) << 3) + ri;
+          const int el = ks * 16 + ((mi >> 1) << 3);
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(kb + (el >> 6) * S::kBoxBytes + swz128(row, (el & 63) >> 3), a0, a1, a2, a3);
+          if (ks & 1)
+            mma_bf16_16816(sb, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
+          else
+            mma_bf16_16816(sa, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
         }
-        // online softmax on row grp: this lane holds rows tok0 + 8j + 2 tig + e
-        float p[2][2];
-        float mloc = -INFINITY;
+        // this lane: rows grp (x0: n0, x1: n1) and grp + 8 (x2: n0, x3: n1)
+        const bool v0 = grp < nval, v1 = grp + 8 < nval;
+        const float x0 = v0 ? fmaf(sa[0] + sb[0], qscale, ln_cur.x * kLog2e) : -INFINITY;
+        const float x1 = v0 ? fmaf(sa[1] + sb[1], qscale, ln_cur.x * kLog2e) : -INFINITY;
+        const float x2 = v1 ? fmaf(sa[2] + sb[2], qscale, ln_cur.y * kLog2e) : -INFINITY;
+        const float x3 = v1 ? fmaf(sa[3] + sb[3], qscale, ln_cur.y * kLog2e) : -INFINITY;
+        // column maxima over the 16 rows: the 8 lanes sharing tig
+        float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int tok = tok0 + 8 * j + 2 * tig + e;
-            float sv = -INFINITY;
-            const float lnv = e ? ln_cur[j].y : ln_cur[j].x;
-            if (tok < t1) sv = fmaf(sc[j][e], qscale, lnv * kLog2e);
-            p[j][e] = sv;
-            mloc = fmaxf(mloc, sv);
-          }
+        for (int off = 4; off < 32; off <<= 1) {
+          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
         }
-        mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 1));
-        mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 2));
-        const float m_new = fmaxf(m_run, mloc);
-        const float corr = exp2f(m_run - m_new);
-        float psum = 0.f;
-#pragma unroll
-        for (int j = 0; j < 2; ++j)
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            p[j][e] = exp2f(p[j][e] - m_new);
-            psum += p[j][e];
-          }
-        psum += __shfl_xor_sync(0xffffffffu, psum, 1);
-        psum += __shfl_xor_sync(0xffffffffu, psum, 2);
-        l_run = l_run * corr + psum;
-        m_run = m_new;
-#pragma unroll
-        for (int n = 0; n < D / 8; ++n) {
-          O[n][0] *= corr;
-          O[n][1] *= corr;
-        }
-        // P (bf16) as the A operand: k = the 16 rows, row grp; padding rows zero
-        const uint32_t pa0 = pack_bf16x2(p[0][0], p[0][1]);
-        const uint32_t pa2 = pack_bf16x2(p[1][0], p[1][1]);
+        const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+        const float b0 = mn0 == -INFINITY ? 0.f : mn0;     // all -inf so far: keep zeros
+        const float b1 = mn1 == -INFINITY ? 0.f : mn1;
+        const float c0 = exp2f(m0 - b0), c1 = exp2f(m1 - b1);
+        const float p0 = exp2f(x0 - b0), p1 = exp2f(x1 - b1);
+        const float p2 = exp2f(x2 - b0), p3 = exp2f(x3 - b1);
+        l0 = fmaf(l0, c0, p0 + p2);
+        l1 = fmaf(l1, c1, p1 + p3);
+        m0 = mn0;
+        m1 = mn1;
+        // P^T as the B operand: transpose the two 8x8 bf16 blocks (rows 0-7, 8-15)
+        const uint32_t pb0 = movmatrix_trans(pack_bf16x2(p0, p1));
+        const uint32_t pb1 = movmatrix_trans(pack_bf16x2(p2, p3));
 #pragma unroll
         for (int j = 0; j < D / 16; ++j) {
-          const int row = r0 + ((mi & 1) << 3) + ri;
-          const int el = j * 16 + ((mi >> 1) << 3);
-          uint32_t v0, v1, v2, v3;
-          ldsm_x4_trans(vb + (el >> 6) * S::kBoxBytes + swz128(row, (el & 63) >> 3), v0, v1, v2, v3);
-          mma_bf16_16816(O[2 * j], pa0, 0u, pa2, 0u, v0, v1);
-          mma_bf16_16816(O[2 * j + 1], pa0, 0u, pa2, 0u, v2, v3);
+          const int row = r0 + ((mi >> 1) << 3) + ri;
+          const int el = j * 16 + ((mi & 1) << 3);
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4_trans(vb + (el >> 6) * S::kBoxBytes + swz128(row, (el & 63) >> 3), a0, a1, a2, a3);
+          O[j][0] *= c0; O[j][1] *= c1; O[j][2] *= c0; O[j][3] *= c1;
+          mma_bf16_16816(O[j], a0, a1, a2, a3, pb0, pb1);
         }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
-      ln_cur[0] = ln_next[0];
-      ln_cur[1] = ln_next[1];
+      ln_cur = ln_next;
+    }
+    // the lanes sharing tig hold disjoint rows' shares of the column sums
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, off);
     }
   }
 
   // every TMA write has landed and every read is done: reuse the ring for partials
   __syncthreads();
   if (warp < kTcConsumers) {
-    const int grp = lane >> 2, tig = lane & 3;
-    if (grp < G) {
+    const int grp = lane >> 2, n0 = 2 * (lane & 3), n1 = n0 + 1;
 #pragma unroll
-      for (int n = 0; n < D / 8; ++n) {
-        s_acc[warp][grp][n * 8 + tig * 2] = O[n][0];
-        s_acc[warp][grp][n * 8 + tig * 2 + 1] = O[n][1];
+    for (int j = 0; j < D / 16; ++j) {
+      if (n0 < G) {
+        s_acc[warp][n0][16 * j + grp] = O[j][0];
+        s_acc[warp][n0][16 * j + grp + 8] = O[j][2];
       }
-      if (tig == 0) {
-        s_m[warp][grp] = m_run;
-        s_l[warp][grp] = l_run;
+      if (n1 < G) {
+        s_acc[warp][n1][16 * j + grp] = O[j][1];
+        s_acc[warp][n1][16 * j + grp + 8] = O[j][3];
       }
+    }
+    if (grp == 0) {
+      if (n0 < G) { s_m[warp][n0] = m0; s_l[warp][n0] = l0; }
+      if (n1 < G) { s_m[warp][n1] = m1; s_l[warp][n1] = l1; }
     }
   }
   __syncthreads();
-  // the combine scratch sits in the ring after the warp partials
-  float* scratch = reinterpret_cast<float*>(base) + kTcConsumers * G * D;
-  static_assert((kTcConsumers * G * D + 2 * G * 64 + 2 * G) * 4 <= kTcStages * S::kStageBytes,
-                "combine scratch fits the ring");
-  decode_epilogue<bf16, D, G, kTcConsumers>(s_m, s_l, s_acc, qs, s_new, &s_last, scratch, tid,
-                                            kTcThreads, head, split, nsplit, L, bad, T_cap, K, V,
-                                            logn, len, k_new, v_new, out, counters, part_ml,
-                                            part_acc, flags);
+  const DecodeSmem<D, G, kTcConsumers> Sm{s_m, s_l, s_acc, qs, s_new, s_fac, s_gstat, &s_last};
+  const DecodeArgs<bf16> a{head, split, nsplit, L, T_cap, bad, K, V, logn, len, k_new, v_new,
+                           out, counters, part, flags};
+  decode_epilogue_staged<bf16, D, G, kTcConsumers>(Sm, base, S::kRingBytes, cbar, a,
+                                                   tid, kTcThreads);
 }
 
 // ---------------------------------------------------------------------------
@@ -336,8 +339,8 @@ static cudaError_t launch_tc(const kvs_cache_desc& d, const CUtensorMap& mK, con
   const cudaError_t e = cudaLaunchKernelEx(
       &cfg, kfn, mK, mV, (const bf16*)q, (bf16*)K, (bf16*)V, logn, len, (const bf16*)k_new,
       (const bf16*)v_new, (bf16*)out, d.T_cap, Ly.nsplit,
-      reinterpret_cast<int32_t*>(ws + Ly.counters), reinterpret_cast<float*>(ws + Ly.part_ml),
-      reinterpret_cast<float*>(ws + Ly.part_acc), reinterpret_cast<int32_t*>(ws));
+      reinterpret_cast<int32_t*>(ws + Ly.counters), reinterpret_cast<float*>(ws + Ly.part),
+      reinterpret_cast<int32_t*>(ws));
   count_launches(1);
   return e != cudaSuccess ? e : cudaGetLastError();
 }

@@ -125,8 +125,12 @@ struct MergeLayout {
   size_t sel, head, blk, total;
   int nblk;
 };
+// Decode split partials: one row of kPartPad + d floats per (query head, split),
+// query-head major, so that every split of a query head is one contiguous block:
+// [acc[0..d) | m | l | pad | pad]. Rows are 16-byte multiples (d in {64, 128}).
+constexpr int kPartPad = 4;
 struct DecodeLayout {
-  size_t counters, part_ml, part_acc, total;
+  size_t counters, part, total;
   int nsplit;
 };
 
@@ -139,12 +143,14 @@ inline int window_splits(const kvs_cache_desc& d) {
   return s < 1 ? 1 : s;
 }
 
+constexpr int kMaxDecodeSplits = 64;      // the combine gives each lane two splits
+
 inline int decode_splits(const kvs_cache_desc& d) {
   int units = d.B * d.H_kv;
   int s = (kTargetCtas + units - 1) / units;
   int cap = d.T_cap / 128 > 1 ? d.T_cap / 128 : 1;
   if (s > cap) s = cap;
-  if (s > 64) s = 64;
+  if (s > kMaxDecodeSplits) s = kMaxDecodeSplits;
   return s < 1 ? 1 : s;
 }
 
@@ -187,9 +193,9 @@ inline DecodeLayout decode_layout(const kvs_cache_desc& d) {
   size_t qheads = (size_t)d.B * d.H_q;
   L.nsplit = decode_splits(d);
   L.counters = kWsAlign;
-  L.part_ml = persistent_bytes(d);
-  L.part_acc = align_up(L.part_ml + qheads * L.nsplit * 2 * sizeof(float), kWsAlign);
-  L.total = align_up(L.part_acc + qheads * L.nsplit * (size_t)d.d * sizeof(float), kWsAlign);
+  L.part = persistent_bytes(d);
+  L.total = align_up(L.part + qheads * L.nsplit * (size_t)(d.d + kPartPad) * sizeof(float),
+                     kWsAlign);
   return L;
 }
 

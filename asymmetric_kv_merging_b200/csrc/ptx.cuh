@@ -209,4 +209,40 @@ __device__ __forceinline__ void named_bar(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// Transpose an 8x8 matrix of 16-bit elements held one row pair per lane (lane l:
+// row l/4, columns 2(l%4), 2(l%4)+1) into the same fragment layout of its transpose.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t a) {
+  uint32_t d;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
+  return d;
+}
+
+// Untiled bulk copy global -> shared (no multicast), completing `bytes` of transaction
+// count on `bar`. Both addresses 16-byte aligned, `bytes` a multiple of 16.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Order this thread's generic-proxy view of global memory before its later async-proxy
+// (bulk copy) accesses.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Device-scope fetch-and-add with acquire-release semantics. Issued by one thread after
+// a CTA barrier it publishes every write the CTA made before the barrier, and makes
+// every write published by earlier arrivals visible to this CTA after the next barrier.
+__device__ __forceinline__ int atom_add_acq_rel_gpu(int32_t* p, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;"
+               : "=r"(old)
+               : "l"(reinterpret_cast<uint64_t>(p)), "r"(v)
+               : "memory");
+  return old;
+}
+
 }  // namespace kvs

@@ -286,4 +286,95 @@ __device__ __forceinline__ void decode_epilogue_staged(const DecodeSmem<D, G, NW
   finish_head<T, D>(a, append, fits, tid, nthreads);
 }
 
+// Epilogue of a cluster launch in which the C CTAs of a cluster are all the splits of
+// one KV head: no global partials, no arrival counter, no last CTA. The CTA merges its
+// warps into cp [G][D] and cml [G][2] (its own shared memory); after a cluster barrier
+// each CTA combines a slice of the G*D output columns by reading every CTA's partial
+// through distributed shared memory, and the CTA of rank 0 appends the new row. A
+// second barrier keeps every CTA's shared memory alive until all reads are done.
+template <typename T, int D, int G, int NW>
+__device__ __forceinline__ void decode_epilogue_cluster(const DecodeSmem<D, G, NW>& S, float* cp,
+                                                        float* cml, uint32_t C, uint32_t rank,
+                                                        const DecodeArgs<T>& a, int tid,
+                                                        int nthreads) {
+  const int lane = tid & 31, warp = tid >> 5, nwarps = nthreads / 32;
+  const bool append = a.k_new != nullptr && a.v_new != nullptr && !a.bad;
+  const bool fits = a.L < a.T_cap;
+  const bool attend_new = append && fits;
+  for (int i = tid; i < G * D; i += nthreads) {
+    const int g = i / D, c = i - g * D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, S.sm[w][g]);
+    float Ls = 0.f, A = 0.f;
+    if (M > -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < NW; ++w) {
+        const float f = exp2f(S.sm[w][g] - M);
+        Ls = fmaf(S.sl[w][g], f, Ls);
+        A = fmaf(S.sacc[w][g][c], f, A);
+      }
+    }
+    cp[i] = A;
+    if (c == 0) {
+      cml[2 * g] = M;
+      cml[2 * g + 1] = Ls;
+    }
+  }
+  if (attend_new) appended_logits<T, D, G, NW>(S, a.k_new + (size_t)a.head * D, warp, lane, nwarps);
+  cluster_arrive();
+  cluster_wait();                              // every CTA's partial is visible
+  // (m, l) of every CTA of the cluster, staged locally: ml[(j * G + g) * 2 + {0, 1}]
+  float* ml = &S.fac[0][0];                    // C * G * 2 <= 16 * G * 2 floats
+  const uint32_t cml_s = smem_u32(cml), cp_s = smem_u32(cp);
+  for (int i = tid; i < (int)C * G * 2; i += nthreads) {
+    const int j = i / (G * 2);
+    ml[i] = ld_cluster_f32(cluster_map(cml_s + (uint32_t)(i - j * G * 2) * 4u, (uint32_t)j));
+  }
+  __syncthreads();
+  const int lo = (int)((uint32_t)(G * D) * rank / C), hi = (int)((uint32_t)(G * D) * (rank + 1) / C);
+  const T* vn = attend_new ? a.v_new + (size_t)a.head * D : nullptr;
+  for (int col = lo + tid; col < hi; col += nthreads) {
+    const int g = col / D, c = col - g * D;
+    const float sn = attend_new ? S.s_new[g] : -INFINITY;
+    float M = sn;
+    for (uint32_t j = 0; j < C; ++j)
+      if (ml[(j * G + g) * 2 + 1] > 0.f) M = fmaxf(M, ml[(j * G + g) * 2]);
+    float Ls = 0.f, A = 0.f;
+    if (M > -INFINITY) {
+#pragma unroll 16
+      for (uint32_t j = 0; j < C; ++j) {
+        const float lj = ml[(j * G + g) * 2 + 1];
+        const float f = lj > 0.f ? exp2f(ml[(j * G + g) * 2] - M) : 0.f;
+        Ls = fmaf(lj, f, Ls);
+        A = fmaf(ld_cluster_f32(cluster_map(cp_s + (uint32_t)col * 4u, j)), f, A);
+      }
+      if (vn) {
+        const float f = exp2f(sn - M);
+        Ls += f;
+        A = fmaf(to_f32(vn[c]), f, A);
+      }
+    }
+    store_out<T>(a.out + ((size_t)a.head * G + g) * D + c, Ls > 0.f ? A / Ls : 0.f);
+  }
+  cluster_arrive();                            // this CTA's remote reads are done
+  if (rank == 0) {
+    if (append) {
+      if (fits) {
+        const T* kn = a.k_new + (size_t)a.head * D;
+        const T* vnn = a.v_new + (size_t)a.head * D;
+        for (int c = tid; c < D; c += nthreads) {
+          a.K[((size_t)a.head * a.T_cap + a.L) * D + c] = kn[c];
+          a.V[((size_t)a.head * a.T_cap + a.L) * D + c] = vnn[c];
+        }
+        if (tid == 0 && a.logn) a.logn[(size_t)a.head * a.T_cap + a.L] = 0.f;
+        if (tid == 0) a.len[a.head] = a.L + 1;
+      } else if (tid == 0) {
+        set_flag(a.flags, KVS_FLAG_OUT_CAPACITY);
+      }
+    }
+  }
+  cluster_wait();                              // no CTA leaves while its partial is read
+}
+
 }  // namespace kvs

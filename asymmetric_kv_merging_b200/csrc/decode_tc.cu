@@ -5,15 +5,27 @@
 // §数学主线三) with the log-count logit bias of merged rows; the decoder stage the
 // pages time (Figure 5). The step is HBM-bound (about 4 flop per byte), so the
 // design goal is to keep every byte of K and V moving: one producer warp issues
-// 2D TMA tile loads (128-byte swizzle, no multicast) of 64 cache rows of K and V
-// into a 3-stage ring of shared-memory buffers guarded by mbarriers; four consumer
-// warps each take 16 rows of a stage, compute the logits of the G query heads with
-// m16n8k16 MMAs (the G heads padded to the 16-row A tile), run the online softmax
-// in registers, and accumulate P V with a second set of MMAs whose A operand is the
-// probability tile repacked from the logit accumulators. Two CTAs fit on an SM, and
-// the grid covers every (KV head, split) once. The split partials are combined by
-// the last CTA to arrive (decode_common.cuh); no CTA waits on another.
+// 2D TMA tile loads (128-byte swizzle, no multicast, L2 evict-first) of 16 * NC
+// cache rows of K and V into a ring of shared-memory stages guarded by mbarriers;
+// NC consumer warps each take 16 rows of a stage. The problem is computed
+// transposed so that the cache rows fill the MMA's M dimension and the G query
+// heads its N = 8 columns: S^T = K Q^T by m16n8k16 MMAs, the online softmax on the
+// accumulator fragments, the probability tile transposed in registers (movmatrix)
+// and O^T += V^T P^T by a second set of MMAs.
+//
+// Two launch shapes share the main loop:
+//  - split grid (NC = 4, two CTAs per SM, nsplit splits per KV head): each CTA
+//    publishes a partial row, and the last CTA of a head to arrive combines them
+//    (decode_common.cuh); no CTA waits on another;
+//  - cluster grid (NC = 8, one CTA per SM): the C splits of a KV head form one
+//    thread-block cluster and combine their partials through distributed shared
+//    memory, with no global partials and no arrival counter. Used when every head's
+//    cluster fits on the GPU at once (few heads, as in single-sequence decode).
 #include <cudaTypedefs.h>
+
+#include <map>
+#include <mutex>
+#include <utility>
 
 #include "decode_common.cuh"
 #include "kvs_common.cuh"
@@ -22,43 +34,48 @@
 
 namespace kvs {
 
-constexpr int kTcTile = 64;                        // cache rows per pipeline stage
-constexpr int kTcStages = 3;
-constexpr int kTcConsumers = 4;                    // consumer warps, 16 rows each
-constexpr int kTcThreads = (kTcConsumers + 1) * 32;
 
-template <int D>
+template <int D, int NC, int STAGES>
 struct TcShape {
+  static constexpr int kTile = 16 * NC;                    // cache rows per stage
+  static constexpr int kThreads = (NC + 1) * 32;           // NC consumers + 1 producer
   static constexpr int kBoxes = D / 64;                    // 128-byte boxes per row
-  static constexpr int kBoxBytes = kTcTile * 128;          // one box of one stage
+  static constexpr int kBoxBytes = kTile * 128;            // one box of one stage
   static constexpr int kTileBytes = kBoxes * kBoxBytes;    // K (or V) rows of one stage
   static constexpr int kStageBytes = 2 * kTileBytes;       // K then V
-  static constexpr int kRingBytes = kTcStages * kStageBytes;
-  static constexpr int kSmem = kRingBytes + (2 * kTcStages + 1) * 8 + 1024;
-  // the combine stages all splits of at least one query head in the ring
+  static constexpr int kRingBytes = STAGES * kStageBytes;
+  static constexpr int kSmem = kRingBytes + (2 * STAGES + 1) * 8 + 1024;
+  // the split combine stages all splits of at least one query head in the ring
   static_assert(kMaxDecodeSplits * (D + kPartPad) * 4 <= kRingBytes, "combine staging");
 };
 
-template <int D, int G>
-__global__ void __launch_bounds__(kTcThreads, 2)
+// the two launch shapes
+template <int D> using SplitShape = TcShape<D, 4, 3>;
+template <int D> using ClusterShape = TcShape<D, 8, D == 64 ? 6 : 3>;
+constexpr int kMaxClusterSize = 16;
+
+template <int D, int G, int NC, int STAGES, bool kCluster>
+__global__ void __launch_bounds__((NC + 1) * 32, kCluster ? 1 : 2)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                  const bf16* __restrict__ q, bf16* K, bf16* V, float* logn, int32_t* len,
                  const bf16* __restrict__ k_new, const bf16* __restrict__ v_new,
                  bf16* __restrict__ out, int T_cap, int nsplit, int32_t* counters, float* part,
                  int32_t* flags) {
-  using S = TcShape<D>;
-  static_assert(kTcConsumers * G * D * 4 <= kTcStages * S::kStageBytes, "warp partials fit the ring");
+  using S = TcShape<D, NC, STAGES>;
+  constexpr int kTile = S::kTile, kThreads = S::kThreads;
+  static_assert((NC + 1) * G * D * 4 <= S::kRingBytes, "warp and CTA partials fit the ring");
   extern __shared__ unsigned char dsm[];
   unsigned char* base = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(dsm) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(base + kTcStages * S::kStageBytes);
-  uint64_t* empty = full + kTcStages;
-  uint64_t* cbar = empty + kTcStages;              // the combine's bulk copies
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + S::kRingBytes);
+  uint64_t* empty = full + STAGES;
+  uint64_t* cbar = empty + STAGES;                 // the split combine's bulk copies
   __shared__ __align__(16) float qs[G][D];
-  __shared__ float s_m[kTcConsumers][G], s_l[kTcConsumers][G];
+  __shared__ float s_m[NC][G], s_l[NC][G];
   __shared__ float s_new[G];
   __shared__ float s_fac[G][kMaxDecodeSplits];
   __shared__ float s_gstat[G][2];
+  __shared__ float s_cml[G][2];
   __shared__ int s_last;
   // after the main loop the stage buffers hold the consumer warps' partial outputs
   float(*s_acc)[G][D] = reinterpret_cast<float(*)[G][D]>(base);
@@ -73,21 +90,23 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     if (split == 0 && tid == 0) set_flag(flags, KVS_FLAG_BAD_LENGTH);
     L = 0;
   }
-  int chunk = (L + nsplit - 1) / nsplit;
-  chunk = (chunk + kTcTile - 1) / kTcTile * kTcTile;
-  const int t0 = split * chunk, t1 = min(L, t0 + chunk);
-  const int ntiles = t1 > t0 ? (t1 - t0 + kTcTile - 1) / kTcTile : 0;
+  // whole tiles per split, the remainder spread one tile each (at most one tile of
+  // imbalance, whatever the length)
+  const long long T = (L + kTile - 1) / kTile;
+  const int tb = (int)(split * T / nsplit), te = (int)((split + 1) * T / nsplit);
+  const int t0 = tb * kTile, t1 = min(L, te * kTile);
+  const int ntiles = t1 > t0 ? te - tb : 0;
   const int row0 = head * T_cap + t0;            // B*H_kv*T_cap < 2^31 (host check)
 
   const float qscale = kLog2e / sqrtf((float)D);
-  for (int i = tid; i < G * D; i += kTcThreads) {
+  for (int i = tid; i < G * D; i += kThreads) {
     const int g = i / D, c = i - g * D;
     qs[g][c] = to_f32(q[((size_t)head * G + g) * D + c]) * qscale;
   }
   if (tid == 0) {
-    for (int s = 0; s < kTcStages; ++s) {
+    for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kTcConsumers);
+      mbar_init(&empty[s], NC);
     }
     mbar_init(cbar, 1);
     fence_mbar_init();
@@ -102,15 +121,16 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
 #pragma unroll
   for (int j = 0; j < D / 16; ++j) O[j][0] = O[j][1] = O[j][2] = O[j][3] = 0.f;
 
-  if (warp == kTcConsumers) {
+  if (warp == NC) {
     // ---------------- producer: one thread issues every TMA load ----------------
     if (lane == 0) {
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
+      const uint64_t once = policy_evict_first();   // K and V are read once per step
       int issued = 0;
       for (int i = 0; i < ntiles; ++i) {
-        const int s = i % kTcStages;
-        if (i >= kTcStages && !mbar_wait(&empty[s], ((i / kTcStages) - 1) & 1)) {
+        const int s = i % STAGES;
+        if (i >= STAGES && !mbar_wait(&empty[s], ((i / STAGES) - 1) & 1)) {
           set_flag(flags, KVS_FLAG_TIMEOUT);
           break;
         }
@@ -118,21 +138,20 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
         mbar_arrive_expect_tx(&full[s], S::kStageBytes);
 #pragma unroll
         for (int bx = 0; bx < S::kBoxes; ++bx) {
-          tma_load_2d(st + bx * S::kBoxBytes, &tmK, bx * 64, row0 + i * kTcTile, &full[s]);
-          tma_load_2d(st + S::kTileBytes + bx * S::kBoxBytes, &tmV, bx * 64, row0 + i * kTcTile,
-                      &full[s]);
+          tma_load_2d_hint(st + bx * S::kBoxBytes, &tmK, bx * 64, row0 + i * kTile, &full[s],
+                           once);
+          tma_load_2d_hint(st + S::kTileBytes + bx * S::kBoxBytes, &tmV, bx * 64,
+                           row0 + i * kTile, &full[s], once);
         }
         issued = i + 1;
       }
       // the last load issued into each stage must land before the buffers are reused
-      for (int i = issued > kTcStages ? issued - kTcStages : 0; i < issued; ++i)
-        if (!mbar_wait(&full[i % kTcStages], (i / kTcStages) & 1)) set_flag(flags, KVS_FLAG_TIMEOUT);
+      for (int i = issued > STAGES ? issued - STAGES : 0; i < issued; ++i)
+        if (!mbar_wait(&full[i % STAGES], (i / STAGES) & 1)) set_flag(flags, KVS_FLAG_TIMEOUT);
     }
     __syncwarp();   // reconverge before the CTA-wide barrier after the main loop
   } else {
     // ---------------- consumers: 16 rows of each stage per warp ----------------
-    // The problem is computed transposed so that the 16 cache rows fill the MMA's M
-    // dimension and the G query heads its N = 8 columns: S^T = K Q^T, O^T += V^T P^T.
     const int grp = lane >> 2, tig = lane & 3;       // fragment row / column pair
     const int mi = lane >> 3, ri = lane & 7;         // ldmatrix: matrix index, row in matrix
     // B operand of S^T = K Q^T: column n = grp holds query head grp (zero past G)
@@ -153,7 +172,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     // log-counts of this lane's rows grp and grp + 8, fetched one tile ahead so the
     // global-memory latency overlaps the previous tile's work
     auto fetch_ln = [&](int tile, float2& dst) {
-      const int tok = t0 + tile * kTcTile + r0 + grp;
+      const int tok = t0 + tile * kTile + r0 + grp;
       const bool live = lnh && tile < ntiles;
       dst.x = (live && tok < t1) ? lnh[tok] : 0.f;
       dst.y = (live && tok + 8 < t1) ? lnh[tok + 8] : 0.f;
@@ -162,15 +181,15 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     fetch_ln(0, ln_cur);
     for (int i = 0; i < ntiles; ++i) {
       fetch_ln(i + 1, ln_next);
-      const int s = i % kTcStages;
+      const int s = i % STAGES;
       // ldmatrix / mma are warp-collective: the whole warp leaves together
-      if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (i / kTcStages) & 1))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (i / STAGES) & 1))) {
         set_flag(flags, KVS_FLAG_TIMEOUT);
         break;
       }
       const uint32_t kb = ring + s * S::kStageBytes;
       const uint32_t vb = kb + S::kTileBytes;
-      const int tok0 = t0 + i * kTcTile + r0;
+      const int tok0 = t0 + i * kTile + r0;
       const int nval = min(16, t1 - tok0);
       if (nval > 0) {
         if (nval < 16) {
@@ -249,7 +268,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
 
   // every TMA write has landed and every read is done: reuse the ring for partials
   __syncthreads();
-  if (warp < kTcConsumers) {
+  if (warp < NC) {
     const int grp = lane >> 2, n0 = 2 * (lane & 3), n1 = n0 + 1;
 #pragma unroll
     for (int j = 0; j < D / 16; ++j) {
@@ -268,12 +287,18 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     }
   }
   __syncthreads();
-  const DecodeSmem<D, G, kTcConsumers> Sm{s_m, s_l, s_acc, qs, s_new, s_fac, s_gstat, &s_last};
+  const DecodeSmem<D, G, NC> Sm{s_m, s_l, s_acc, qs, s_new, s_fac, s_gstat, &s_last};
   const DecodeArgs<bf16> a{head, split, nsplit, L, T_cap, bad, K, V, logn, len, k_new, v_new,
                            out, counters, part, flags};
-  decode_epilogue_staged<bf16, D, G, kTcConsumers>(Sm, base, S::kRingBytes, cbar, a,
-                                                   tid, kTcThreads);
+  if constexpr (kCluster) {
+    // the CTA partial goes after the warp partials in the ring
+    decode_epilogue_cluster<bf16, D, G, NC>(Sm, &s_acc[NC][0][0], &s_cml[0][0], (uint32_t)nsplit,
+                                            cluster_ctarank(), a, tid, kThreads);
+  } else {
+    decode_epilogue_staged<bf16, D, G, NC>(Sm, base, S::kRingBytes, cbar, a, tid, kThreads);
+  }
 }
+
 
 // ---------------------------------------------------------------------------
 // Host side: tensor maps over the whole cache ([B*H_kv*T_cap rows, d] bf16) and launch
@@ -311,50 +336,117 @@ bool decode_tc_supported(const kvs_cache_desc& d) {
          tensor_map_encoder() != nullptr;
 }
 
+// Cluster size for a cluster launch over `units` KV heads on the current device, or
+// 0 when the split grid is to be used: the largest C <= 16 with C * units <= SM count
+// for which the occupancy calculator places all `units` clusters at once.
 template <int D, int G>
-static cudaError_t launch_tc(const kvs_cache_desc& d, const CUtensorMap& mK, const CUtensorMap& mV,
-                             const void* q, void* K, void* V, float* logn, int32_t* len,
-                             const void* k_new, const void* v_new, void* out,
-                             const DecodeLayout& Ly, char* ws, cudaStream_t st) {
-  auto kfn = decode_tc_kernel<D, G>;
+static int cluster_size_for(int units) {
+  using CS = ClusterShape<D>;
+  auto kfn = decode_tc_kernel<D, G, 8, (D == 64 ? 6 : 3), true>;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  static std::mutex mu;
+  static std::map<std::pair<int, int>, int> cache;
+  std::lock_guard<std::mutex> lock(mu);
+  const auto key = std::make_pair(dev, units);
+  const auto it = cache.find(key);
+  if (it != cache.end()) return it->second;
+  int sms = 0;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int C = units > 0 ? sms / units : 0;
+  if (C > kMaxClusterSize) C = kMaxClusterSize;
+  if (cudaFuncSetAttribute((const void*)kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           CS::kSmem) != cudaSuccess)
+    C = 0;
+  if (C > 8 && cudaFuncSetAttribute((const void*)kfn,
+                                    cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+    C = 8;
+  for (; C >= 2; --C) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(C, units);
+    cfg.blockDim = dim3(CS::kThreads);
+    cfg.dynamicSmemBytes = CS::kSmem;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = C;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, (const void*)kfn, &cfg) == cudaSuccess && n >= units) break;
+  }
+  (void)cudaGetLastError();   // a refused query leaves no error behind
+  if (C < 2) C = 0;
+  cache[key] = C;
+  return C;
+}
+
+template <int D, int G, int NC, int STAGES, bool kCluster>
+static cudaError_t launch_shape(const kvs_cache_desc& d, const void* q, void* K, void* V,
+                                float* logn, int32_t* len, const void* k_new, const void* v_new,
+                                void* out, int nsplit, const DecodeLayout& Ly, char* ws,
+                                cudaStream_t st) {
+  using S = TcShape<D, NC, STAGES>;
+  auto kfn = decode_tc_kernel<D, G, NC, STAGES, kCluster>;
   static bool attr = false;   // set once per process, before any capture
   if (!attr) {
     if (cudaFuncSetAttribute((const void*)kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             TcShape<D>::kSmem) != cudaSuccess)
+                             S::kSmem) != cudaSuccess)
+      return cudaErrorInvalidValue;
+    if (kCluster && nsplit > 8 &&
+        cudaFuncSetAttribute((const void*)kfn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+            cudaSuccess)
       return cudaErrorInvalidValue;
     attr = true;
   }
+  const unsigned long long rows = (unsigned long long)d.B * d.H_kv * (unsigned long long)d.T_cap;
+  CUtensorMap mK, mV;
+  if (!encode_rows_map(&mK, K, rows, d.d, S::kTile) || !encode_rows_map(&mV, V, rows, d.d, S::kTile))
+    return cudaErrorInvalidValue;
   // programmatic serialization lets this grid launch while the previous one drains;
   // the kernel waits for it (griddepcontrol.wait) before any global-memory access
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(Ly.nsplit, d.B * d.H_kv);
-  cfg.blockDim = dim3(kTcThreads);
-  cfg.dynamicSmemBytes = TcShape<D>::kSmem;
+  cfg.gridDim = dim3(nsplit, d.B * d.H_kv);
+  cfg.blockDim = dim3(S::kThreads);
+  cfg.dynamicSmemBytes = S::kSmem;
   cfg.stream = st;
-  cudaLaunchAttribute pdl[1];
-  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  pdl[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = pdl;
-  cfg.numAttrs = 1;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  at[1].id = cudaLaunchAttributeClusterDimension;
+  at[1].val.clusterDim.x = nsplit;
+  at[1].val.clusterDim.y = 1;
+  at[1].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = kCluster ? 2 : 1;
   const cudaError_t e = cudaLaunchKernelEx(
       &cfg, kfn, mK, mV, (const bf16*)q, (bf16*)K, (bf16*)V, logn, len, (const bf16*)k_new,
-      (const bf16*)v_new, (bf16*)out, d.T_cap, Ly.nsplit,
+      (const bf16*)v_new, (bf16*)out, d.T_cap, nsplit,
       reinterpret_cast<int32_t*>(ws + Ly.counters), reinterpret_cast<float*>(ws + Ly.part),
       reinterpret_cast<int32_t*>(ws));
   count_launches(1);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
+template <int D, int G>
+static cudaError_t launch_tc(const kvs_cache_desc& d, const void* q, void* K, void* V,
+                             float* logn, int32_t* len, const void* k_new, const void* v_new,
+                             void* out, const DecodeLayout& Ly, char* ws, cudaStream_t st) {
+  const int C = cluster_size_for<D, G>(d.B * d.H_kv);
+  if (C >= 2)
+    return launch_shape<D, G, 8, (D == 64 ? 6 : 3), true>(d, q, K, V, logn, len, k_new, v_new, out,
+                                                          C, Ly, ws, st);
+  return launch_shape<D, G, 4, 3, false>(d, q, K, V, logn, len, k_new, v_new, out, Ly.nsplit, Ly,
+                                         ws, st);
+}
+
 cudaError_t launch_decode_tc(const kvs_cache_desc& d, const void* q, void* K, void* V, float* logn,
                              int32_t* len, const void* k_new, const void* v_new, void* out,
                              const DecodeLayout& Ly, char* ws, cudaStream_t st) {
-  const unsigned long long rows = (unsigned long long)d.B * d.H_kv * (unsigned long long)d.T_cap;
-  CUtensorMap mK, mV;
-  if (!encode_rows_map(&mK, K, rows, d.d, kTcTile) || !encode_rows_map(&mV, V, rows, d.d, kTcTile))
-    return cudaErrorInvalidValue;
   const int G = d.H_q / d.H_kv;
 #define KVS_TC(DD, GG) \
-  if (d.d == DD && G == GG) return launch_tc<DD, GG>(d, mK, mV, q, K, V, logn, len, k_new, v_new, out, Ly, ws, st)
+  if (d.d == DD && G == GG) return launch_tc<DD, GG>(d, q, K, V, logn, len, k_new, v_new, out, Ly, ws, st)
   KVS_TC(128, 1); KVS_TC(128, 2); KVS_TC(128, 4); KVS_TC(128, 8);
   KVS_TC(64, 1); KVS_TC(64, 2); KVS_TC(64, 4); KVS_TC(64, 8);
 #undef KVS_TC

@@ -286,95 +286,122 @@ __device__ __forceinline__ void decode_epilogue_staged(const DecodeSmem<D, G, NW
   finish_head<T, D>(a, append, fits, tid, nthreads);
 }
 
-// Epilogue of a cluster launch in which the C CTAs of a cluster are all the splits of
-// one KV head: no global partials, no arrival counter, no last CTA. The CTA merges its
-// warps into cp [G][D] and cml [G][2] (its own shared memory); after a cluster barrier
-// each CTA combines a slice of the G*D output columns by reading every CTA's partial
-// through distributed shared memory, and the CTA of rank 0 appends the new row. A
-// second barrier keeps every CTA's shared memory alive until all reads are done.
+// Shared-memory inbox of a cluster combine: the partial columns and (m, l) that the C
+// CTAs of a cluster push to the CTA owning an output slice. A dedicated region (not
+// the ring), because peers may push while this CTA is still streaming.
+template <int D, int G>
+struct __align__(16) ClusterInbox {
+  float acc[G * D + kMaxClusterSize];                   // [C][G*D/C + 1]
+  float ml[kMaxClusterSize][G][2];                      // [C][G] (m, l)
+};
+
+// Output slice of rank r among C CTAs: columns [G*D*r/C, G*D*(r+1)/C).
+__device__ __forceinline__ int slice_lo(int n, int r, int C) { return (int)((unsigned)n * r / C); }
+__device__ __forceinline__ int slice_owner(int n, int col, int C) {
+  return (int)(((unsigned)(col + 1) * C - 1) / n);
+}
+
+// Cluster combine of a decode step in which the C CTAs of a cluster are all the splits
+// of one KV head: no global partials, no arrival counter, no last CTA. Every CTA
+// merges its warp partials and pushes each column to the CTA owning that column's
+// output slice (distributed shared-memory stores into the owner's inbox), and its
+// (m, l) to every CTA; after one cluster barrier each CTA combines its slice from its
+// own inbox, and the CTA of rank 0 appends the new row. Nothing is read remotely, so
+// a CTA may leave as soon as its slice is written.
+//
+// `dry`: run the same instructions with every store aimed at this CTA's scratch
+// (`inbox` and `out` point there, head is 0) and without barriers or the append,
+// from a single warp while the other warps stream. A kernel launch starts with cold
+// instruction caches; the dry run pulls this code in before the real combine needs it.
 template <typename T, int D, int G, int NW>
-__device__ __forceinline__ void decode_epilogue_cluster(const DecodeSmem<D, G, NW>& S, float* cp,
-                                                        float* cml, uint32_t C, uint32_t rank,
-                                                        const DecodeArgs<T>& a, int tid,
-                                                        int nthreads) {
+__device__ __noinline__ void cluster_combine(
+    float (*sm)[G], float (*sl)[G], float (*sacc)[G][D], float (*qs)[D], float* s_cml,
+    float* s_new, ClusterInbox<D, G>* inbox, int C, int rank, int tid, int nthreads, bool dry,
+    int head, int L, int T_cap, bool append, T* K, T* V, float* logn, int32_t* len,
+    const T* k_new, const T* v_new, T* out, int32_t* flags) {
+  constexpr int N = G * D;
   const int lane = tid & 31, warp = tid >> 5, nwarps = nthreads / 32;
-  const bool append = a.k_new != nullptr && a.v_new != nullptr && !a.bad;
-  const bool fits = a.L < a.T_cap;
+  const bool fits = L < T_cap;
   const bool attend_new = append && fits;
-  for (int i = tid; i < G * D; i += nthreads) {
-    const int g = i / D, c = i - g * D;
+  const int slice_w = N / C + 1;                       // inbox row stride (>= any slice)
+  // this CTA's (m, l) per query head
+  for (int g = tid; g < G; g += nthreads) {
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < NW; ++w) M = fmaxf(M, S.sm[w][g]);
-    float Ls = 0.f, A = 0.f;
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, sm[w][g]);
+    float Ls = 0.f;
     if (M > -INFINITY) {
 #pragma unroll
-      for (int w = 0; w < NW; ++w) {
-        const float f = exp2f(S.sm[w][g] - M);
-        Ls = fmaf(S.sl[w][g], f, Ls);
-        A = fmaf(S.sacc[w][g][c], f, A);
-      }
+      for (int w = 0; w < NW; ++w) Ls = fmaf(sl[w][g], exp2f(sm[w][g] - M), Ls);
     }
-    cp[i] = A;
-    if (c == 0) {
-      cml[2 * g] = M;
-      cml[2 * g + 1] = Ls;
+    s_cml[2 * g] = M;
+    s_cml[2 * g + 1] = Ls;
+  }
+  if (attend_new) appended_logits<T, D, G, NW>(DecodeSmem<D, G, NW>{sm, sl, sacc, qs, s_new, nullptr, nullptr, nullptr},
+                                               k_new + (size_t)head * D, warp, lane, nwarps);
+  if (!dry) __syncthreads();
+  const uint32_t in_acc = smem_u32(inbox->acc), in_ml = smem_u32(&inbox->ml[0][0][0]);
+  // push (m, l) of every query head to every CTA: ml[rank][g] in CTA j
+  for (int k = tid; k < C * G; k += nthreads) {
+    const int j = k / G, g = k - j * G;
+    const uint32_t dst = cluster_map(in_ml + (uint32_t)((rank * G + g) * 2) * 4u, dry ? rank : j);
+    st_cluster_f32x2(dst, s_cml[2 * g], s_cml[2 * g + 1]);
+  }
+  // merge the warps column by column and push each column to its owner
+  for (int i = tid; i < N; i += nthreads) {
+    const int g = i / D, c = i - g * D;
+    const float M = s_cml[2 * g];
+    float A = 0.f;
+    if (M > -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < NW; ++w) A = fmaf(sacc[w][g][c], exp2f(sm[w][g] - M), A);
     }
+    const int owner = slice_owner(N, i, C);
+    const int at = rank * slice_w + (i - slice_lo(N, owner, C));
+    st_cluster_f32(cluster_map(in_acc + (uint32_t)at * 4u, dry ? rank : owner), A);
   }
-  if (attend_new) appended_logits<T, D, G, NW>(S, a.k_new + (size_t)a.head * D, warp, lane, nwarps);
-  cluster_arrive();
-  cluster_wait();                              // every CTA's partial is visible
-  // (m, l) of every CTA of the cluster, staged locally: ml[(j * G + g) * 2 + {0, 1}]
-  float* ml = &S.fac[0][0];                    // C * G * 2 <= 16 * G * 2 floats
-  const uint32_t cml_s = smem_u32(cml), cp_s = smem_u32(cp);
-  for (int i = tid; i < (int)C * G * 2; i += nthreads) {
-    const int j = i / (G * 2);
-    ml[i] = ld_cluster_f32(cluster_map(cml_s + (uint32_t)(i - j * G * 2) * 4u, (uint32_t)j));
+  if (!dry) {
+    cluster_arrive();
+    cluster_wait();                                    // every push to this CTA landed
   }
-  __syncthreads();
-  const int lo = (int)((uint32_t)(G * D) * rank / C), hi = (int)((uint32_t)(G * D) * (rank + 1) / C);
-  const T* vn = attend_new ? a.v_new + (size_t)a.head * D : nullptr;
+  // combine this CTA's slice from its inbox
+  const int lo = slice_lo(N, rank, C), hi = slice_lo(N, rank + 1, C);
   for (int col = lo + tid; col < hi; col += nthreads) {
     const int g = col / D, c = col - g * D;
-    const float sn = attend_new ? S.s_new[g] : -INFINITY;
+    const float sn = attend_new ? s_new[g] : -INFINITY;
     float M = sn;
-    for (uint32_t j = 0; j < C; ++j)
-      if (ml[(j * G + g) * 2 + 1] > 0.f) M = fmaxf(M, ml[(j * G + g) * 2]);
+    for (int j = 0; j < C; ++j)
+      if (inbox->ml[j][g][1] > 0.f) M = fmaxf(M, inbox->ml[j][g][0]);
     float Ls = 0.f, A = 0.f;
     if (M > -INFINITY) {
-#pragma unroll 16
-      for (uint32_t j = 0; j < C; ++j) {
-        const float lj = ml[(j * G + g) * 2 + 1];
-        const float f = lj > 0.f ? exp2f(ml[(j * G + g) * 2] - M) : 0.f;
+      for (int j = 0; j < C; ++j) {
+        const float lj = inbox->ml[j][g][1];
+        const float f = lj > 0.f ? exp2f(inbox->ml[j][g][0] - M) : 0.f;
         Ls = fmaf(lj, f, Ls);
-        A = fmaf(ld_cluster_f32(cluster_map(cp_s + (uint32_t)col * 4u, j)), f, A);
+        A = fmaf(inbox->acc[j * slice_w + (col - lo)], f, A);
       }
-      if (vn) {
+      if (attend_new) {
         const float f = exp2f(sn - M);
         Ls += f;
-        A = fmaf(to_f32(vn[c]), f, A);
+        A = fmaf(to_f32(v_new[(size_t)head * D + c]), f, A);
       }
     }
-    store_out<T>(a.out + ((size_t)a.head * G + g) * D + c, Ls > 0.f ? A / Ls : 0.f);
+    store_out<T>(out + ((size_t)head * G + g) * D + c, Ls > 0.f ? A / Ls : 0.f);
   }
-  cluster_arrive();                            // this CTA's remote reads are done
-  if (rank == 0) {
-    if (append) {
-      if (fits) {
-        const T* kn = a.k_new + (size_t)a.head * D;
-        const T* vnn = a.v_new + (size_t)a.head * D;
-        for (int c = tid; c < D; c += nthreads) {
-          a.K[((size_t)a.head * a.T_cap + a.L) * D + c] = kn[c];
-          a.V[((size_t)a.head * a.T_cap + a.L) * D + c] = vnn[c];
-        }
-        if (tid == 0 && a.logn) a.logn[(size_t)a.head * a.T_cap + a.L] = 0.f;
-        if (tid == 0) a.len[a.head] = a.L + 1;
-      } else if (tid == 0) {
-        set_flag(a.flags, KVS_FLAG_OUT_CAPACITY);
+  if (!dry && rank == 0 && append) {
+    if (fits) {
+      const T* kn = k_new + (size_t)head * D;
+      const T* vn = v_new + (size_t)head * D;
+      for (int c = tid; c < D; c += nthreads) {
+        K[((size_t)head * T_cap + L) * D + c] = kn[c];
+        V[((size_t)head * T_cap + L) * D + c] = vn[c];
       }
+      if (tid == 0 && logn) logn[(size_t)head * T_cap + L] = 0.f;
+      if (tid == 0) len[head] = L + 1;
+    } else if (tid == 0) {
+      set_flag(flags, KVS_FLAG_OUT_CAPACITY);
     }
   }
-  cluster_wait();                              // no CTA leaves while its partial is read
 }
 
 }  // namespace kvs

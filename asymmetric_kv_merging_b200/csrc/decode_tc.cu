@@ -24,6 +24,7 @@
 #include <cudaTypedefs.h>
 
 #include <map>
+#include <type_traits>
 #include <mutex>
 #include <utility>
 
@@ -35,10 +36,10 @@
 namespace kvs {
 
 
-template <int D, int NC, int STAGES>
+template <int D, int NC, int STAGES, int EXTRA>
 struct TcShape {
   static constexpr int kTile = 16 * NC;                    // cache rows per stage
-  static constexpr int kThreads = (NC + 1) * 32;           // NC consumers + 1 producer
+  static constexpr int kThreads = (NC + 1 + EXTRA) * 32;   // consumers, producer, extra
   static constexpr int kBoxes = D / 64;                    // 128-byte boxes per row
   static constexpr int kBoxBytes = kTile * 128;            // one box of one stage
   static constexpr int kTileBytes = kBoxes * kBoxBytes;    // K (or V) rows of one stage
@@ -49,21 +50,20 @@ struct TcShape {
   static_assert(kMaxDecodeSplits * (D + kPartPad) * 4 <= kRingBytes, "combine staging");
 };
 
-// the two launch shapes
-template <int D> using SplitShape = TcShape<D, 4, 3>;
-template <int D> using ClusterShape = TcShape<D, 8, D == 64 ? 6 : 3>;
-constexpr int kMaxClusterSize = 16;
+// the two launch shapes (the cluster shape adds the warp that pre-runs the combine)
+template <int D> using SplitShape = TcShape<D, 4, 3, 0>;
+template <int D> using ClusterShape = TcShape<D, 8, D == 64 ? 6 : 3, 1>;
 
 template <int D, int G, int NC, int STAGES, bool kCluster>
-__global__ void __launch_bounds__((NC + 1) * 32, kCluster ? 1 : 2)
+__global__ void __launch_bounds__((NC + (kCluster ? 2 : 1)) * 32, kCluster ? 1 : 2)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                  const bf16* __restrict__ q, bf16* K, bf16* V, float* logn, int32_t* len,
                  const bf16* __restrict__ k_new, const bf16* __restrict__ v_new,
                  bf16* __restrict__ out, int T_cap, int nsplit, int32_t* counters, float* part,
                  int32_t* flags) {
-  using S = TcShape<D, NC, STAGES>;
+  using S = TcShape<D, NC, STAGES, kCluster ? 1 : 0>;
   constexpr int kTile = S::kTile, kThreads = S::kThreads;
-  static_assert((NC + 1) * G * D * 4 <= S::kRingBytes, "warp and CTA partials fit the ring");
+  static_assert(NC * G * D * 4 <= S::kRingBytes, "warp partials fit the ring");
   extern __shared__ unsigned char dsm[];
   unsigned char* base = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(dsm) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -77,13 +77,14 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
   __shared__ float s_gstat[G][2];
   __shared__ float s_cml[G][2];
   __shared__ int s_last;
+  // cluster shape: the inbox peers push into, and the scratch of the warm-up run
+  using Inbox = std::conditional_t<kCluster, ClusterInbox<D, G>, char>;
+  __shared__ Inbox s_inbox[2];
   // after the main loop the stage buffers hold the consumer warps' partial outputs
   float(*s_acc)[G][D] = reinterpret_cast<float(*)[G][D]>(base);
 
   const int head = blockIdx.y, split = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  pdl_trigger();
-  pdl_wait();     // nothing above this line touches global memory
   int L = len[head];
   const bool bad = L < 0 || L > T_cap;
   if (bad) {
@@ -121,7 +122,14 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
 #pragma unroll
   for (int j = 0; j < D / 16; ++j) O[j][0] = O[j][1] = O[j][2] = O[j][3] = 0.f;
 
-  if (warp == NC) {
+  if (kCluster && warp == NC + 1) {
+    // ---------------- warm-up: the combine's code, dry, while the others stream ----
+    if constexpr (kCluster)
+      cluster_combine<bf16, D, G, NC>(s_m, s_l, s_acc, qs, &s_cml[0][0], s_new, &s_inbox[1], nsplit,
+                                      (int)cluster_ctarank(), lane, 32, /*dry=*/true, 0, L, T_cap,
+                                      k_new != nullptr && v_new != nullptr && !bad, K, V, logn, len,
+                                      k_new, v_new, reinterpret_cast<bf16*>(&s_inbox[1]), flags);
+  } else if (warp == NC) {
     // ---------------- producer: one thread issues every TMA load ----------------
     if (lane == 0) {
       prefetch_tmap(&tmK);
@@ -150,7 +158,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
         if (!mbar_wait(&full[i % STAGES], (i / STAGES) & 1)) set_flag(flags, KVS_FLAG_TIMEOUT);
     }
     __syncwarp();   // reconverge before the CTA-wide barrier after the main loop
-  } else {
+  } else if (warp < NC) {
     // ---------------- consumers: 16 rows of each stage per warp ----------------
     const int grp = lane >> 2, tig = lane & 3;       // fragment row / column pair
     const int mi = lane >> 3, ri = lane & 7;         // ldmatrix: matrix index, row in matrix
@@ -291,9 +299,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
   const DecodeArgs<bf16> a{head, split, nsplit, L, T_cap, bad, K, V, logn, len, k_new, v_new,
                            out, counters, part, flags};
   if constexpr (kCluster) {
-    // the CTA partial goes after the warp partials in the ring
-    decode_epilogue_cluster<bf16, D, G, NC>(Sm, &s_acc[NC][0][0], &s_cml[0][0], (uint32_t)nsplit,
-                                            cluster_ctarank(), a, tid, kThreads);
+    cluster_combine<bf16, D, G, NC>(s_m, s_l, s_acc, qs, &s_cml[0][0], s_new, &s_inbox[0], nsplit,
+                                    (int)cluster_ctarank(), tid, kThreads, /*dry=*/false, head, L,
+                                    T_cap, k_new != nullptr && v_new != nullptr && !bad, K, V, logn,
+                                    len, k_new, v_new, out, flags);
   } else {
     decode_epilogue_staged<bf16, D, G, NC>(Sm, base, S::kRingBytes, cbar, a, tid, kThreads);
   }
@@ -387,7 +396,7 @@ static cudaError_t launch_shape(const kvs_cache_desc& d, const void* q, void* K,
                                 float* logn, int32_t* len, const void* k_new, const void* v_new,
                                 void* out, int nsplit, const DecodeLayout& Ly, char* ws,
                                 cudaStream_t st) {
-  using S = TcShape<D, NC, STAGES>;
+  using S = TcShape<D, NC, STAGES, kCluster ? 1 : 0>;
   auto kfn = decode_tc_kernel<D, G, NC, STAGES, kCluster>;
   static bool attr = false;   // set once per process, before any capture
   if (!attr) {
@@ -404,22 +413,21 @@ static cudaError_t launch_shape(const kvs_cache_desc& d, const void* q, void* K,
   CUtensorMap mK, mV;
   if (!encode_rows_map(&mK, K, rows, d.d, S::kTile) || !encode_rows_map(&mV, V, rows, d.d, S::kTile))
     return cudaErrorInvalidValue;
-  // programmatic serialization lets this grid launch while the previous one drains;
-  // the kernel waits for it (griddepcontrol.wait) before any global-memory access
+  // Plain stream order: letting the next grid launch early (programmatic dependent
+  // launch) measured 1-2 us slower per step here, since its CTAs take SM slots and
+  // cluster places while this grid's combine still runs.
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(nsplit, d.B * d.H_kv);
   cfg.blockDim = dim3(S::kThreads);
   cfg.dynamicSmemBytes = S::kSmem;
   cfg.stream = st;
-  cudaLaunchAttribute at[2];
-  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  at[0].val.programmaticStreamSerializationAllowed = 1;
-  at[1].id = cudaLaunchAttributeClusterDimension;
-  at[1].val.clusterDim.x = nsplit;
-  at[1].val.clusterDim.y = 1;
-  at[1].val.clusterDim.z = 1;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = nsplit;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
   cfg.attrs = at;
-  cfg.numAttrs = kCluster ? 2 : 1;
+  cfg.numAttrs = kCluster ? 1 : 0;
   const cudaError_t e = cudaLaunchKernelEx(
       &cfg, kfn, mK, mV, (const bf16*)q, (bf16*)K, (bf16*)V, logn, len, (const bf16*)k_new,
       (const bf16*)v_new, (bf16*)out, d.T_cap, nsplit,

@@ -144,6 +144,7 @@ inline int window_splits(const kvs_cache_desc& d) {
 }
 
 constexpr int kMaxDecodeSplits = 64;      // the combine gives each lane two splits
+constexpr int kMaxClusterSize = 16;       // CTAs of one KV head in a cluster launch
 
 inline int decode_splits(const kvs_cache_desc& d) {
   int units = d.B * d.H_kv;

@@ -266,6 +266,13 @@ __device__ __forceinline__ float4 ld_cluster_f32x4(uint32_t addr) {
   return v;
 }
 
+__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+__device__ __forceinline__ void st_cluster_f32x2(uint32_t addr, float a, float b) {
+  asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(a), "f"(b) : "memory");
+}
+
 // Transpose an 8x8 matrix of 16-bit elements held one row pair per lane (lane l:
 // row l/4, columns 2(l%4), 2(l%4)+1) into the same fragment layout of its transpose.
 __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t a) {

@@ -45,7 +45,12 @@ struct TcShape {
   static constexpr int kTileBytes = kBoxes * kBoxBytes;    // K (or V) rows of one stage
   static constexpr int kStageBytes = 2 * kTileBytes;       // K then V
   static constexpr int kRingBytes = STAGES * kStageBytes;
-  static constexpr int kSmem = kRingBytes + (2 * STAGES + 1) * 8 + 1024;
+  // log-counts of a stage: kTile + 4 floats from a 16-byte aligned start (TMA needs
+  // the start coordinate of an fp32 box to be a multiple of 4), one slot per stage
+  static constexpr int kLnBox = kTile + 4;
+  static constexpr int kLnSlot = 1024;
+  static_assert(kLnBox * 4 <= kLnSlot, "log-count slot");
+  static constexpr int kSmem = kRingBytes + STAGES * kLnSlot + (2 * STAGES + 1) * 8 + 1024;
   // the split combine stages all splits of at least one query head in the ring
   static_assert(kMaxDecodeSplits * (D + kPartPad) * 4 <= kRingBytes, "combine staging");
 };
@@ -57,6 +62,7 @@ template <int D> using ClusterShape = TcShape<D, 8, D == 64 ? 6 : 3, 1>;
 template <int D, int G, int NC, int STAGES, bool kCluster>
 __global__ void __launch_bounds__((NC + (kCluster ? 2 : 1)) * 32, kCluster ? 1 : 2)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                 const __grid_constant__ CUtensorMap tmL, int ln_lead,
                  const bf16* __restrict__ q, bf16* K, bf16* V, float* logn, int32_t* len,
                  const bf16* __restrict__ k_new, const bf16* __restrict__ v_new,
                  bf16* __restrict__ out, int T_cap, int nsplit, int32_t* counters, float* part,
@@ -67,7 +73,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
   extern __shared__ unsigned char dsm[];
   unsigned char* base = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(dsm) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(base + S::kRingBytes);
+  unsigned char* ln_ring = base + S::kRingBytes;   // STAGES log-count slots
+  uint64_t* full = reinterpret_cast<uint64_t*>(ln_ring + STAGES * S::kLnSlot);
   uint64_t* empty = full + STAGES;
   uint64_t* cbar = empty + STAGES;                 // the split combine's bulk copies
   __shared__ __align__(16) float qs[G][D];
@@ -98,6 +105,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
   const int t0 = tb * kTile, t1 = min(L, te * kTile);
   const int ntiles = t1 > t0 ? te - tb : 0;
   const int row0 = head * T_cap + t0;            // B*H_kv*T_cap < 2^31 (host check)
+  // log-counts of tile i start at element e = ln_lead + row0 + i * kTile of the
+  // log-count map; its box starts at e rounded down to a multiple of 4 (so every
+  // tile's offset is (ln_lead + row0) & 3, kTile being a multiple of 4)
+  const bool has_ln = logn != nullptr;
+  const int ln_off = (ln_lead + row0) & 3;
 
   const float qscale = kLog2e / sqrtf((float)D);
   for (int i = tid; i < G * D; i += kThreads) {
@@ -134,6 +146,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     if (lane == 0) {
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
+      if (has_ln) prefetch_tmap(&tmL);
       const uint64_t once = policy_evict_first();   // K and V are read once per step
       int issued = 0;
       for (int i = 0; i < ntiles; ++i) {
@@ -143,7 +156,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
           break;
         }
         unsigned char* st = base + s * S::kStageBytes;
-        mbar_arrive_expect_tx(&full[s], S::kStageBytes);
+        mbar_arrive_expect_tx(&full[s], S::kStageBytes + (has_ln ? S::kLnBox * 4 : 0));
+        if (has_ln)
+          tma_load_1d_hint(ln_ring + s * S::kLnSlot, &tmL, ln_lead + row0 + i * kTile - ln_off,
+                           &full[s], once);
 #pragma unroll
         for (int bx = 0; bx < S::kBoxes; ++bx) {
           tma_load_2d_hint(st + bx * S::kBoxBytes, &tmK, bx * 64, row0 + i * kTile, &full[s],
@@ -174,21 +190,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
         qb[ks][0] = qb[ks][1] = 0u;
       }
     }
-    const float* lnh = logn ? logn + (size_t)head * T_cap : nullptr;
     const int r0 = warp * 16;                        // this warp's rows inside a stage
     const uint32_t ring = smem_u32(base);
-    // log-counts of this lane's rows grp and grp + 8, fetched one tile ahead so the
-    // global-memory latency overlaps the previous tile's work
-    auto fetch_ln = [&](int tile, float2& dst) {
-      const int tok = t0 + tile * kTile + r0 + grp;
-      const bool live = lnh && tile < ntiles;
-      dst.x = (live && tok < t1) ? lnh[tok] : 0.f;
-      dst.y = (live && tok + 8 < t1) ? lnh[tok + 8] : 0.f;
-    };
-    float2 ln_cur, ln_next;
-    fetch_ln(0, ln_cur);
     for (int i = 0; i < ntiles; ++i) {
-      fetch_ln(i + 1, ln_next);
       const int s = i % STAGES;
       // ldmatrix / mma are warp-collective: the whole warp leaves together
       if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (i / STAGES) & 1))) {
@@ -225,6 +229,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
             mma_bf16_16816(sb, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
           else
             mma_bf16_16816(sa, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
+        }
+        // log-counts of this lane's rows grp and grp + 8 (landed with the stage)
+        float2 ln_cur = make_float2(0.f, 0.f);
+        if (has_ln) {
+          const float* lns = reinterpret_cast<const float*>(ln_ring + s * S::kLnSlot) + ln_off + r0;
+          ln_cur = make_float2(lns[grp], lns[grp + 8]);
         }
         // this lane: rows grp (x0: n0, x1: n1) and grp + 8 (x2: n0, x3: n1)
         const bool v0 = grp < nval, v1 = grp + 8 < nval;
@@ -264,7 +274,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
-      ln_cur = ln_next;
     }
     // the lanes sharing tig hold disjoint rows' shares of the column sums
 #pragma unroll
@@ -339,6 +348,25 @@ bool encode_rows_map(CUtensorMap* map, const void* base, unsigned long long rows
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 1D map over the log-counts, starting at the 16-byte boundary at or below `logn`;
+// *lead = the elements between that boundary and logn (0..3). Elements past the end
+// read as zero; the few before logn lie in the same 16-byte chunk, so the same page.
+static bool encode_ln_map(CUtensorMap* map, const float* logn, unsigned long long n, int box,
+                          int* lead) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  const uintptr_t a = reinterpret_cast<uintptr_t>(logn);
+  const uintptr_t b = a & ~static_cast<uintptr_t>(15);
+  *lead = (int)((a - b) / sizeof(float));
+  cuuint64_t dims[1] = {(cuuint64_t)(n + *lead)};
+  cuuint64_t strides[1] = {0};
+  cuuint32_t boxd[1] = {(cuuint32_t)box};
+  cuuint32_t estr[1] = {1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 1, reinterpret_cast<void*>(b), dims, strides,
+             boxd, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool decode_tc_supported(const kvs_cache_desc& d) {
   const unsigned long long rows = (unsigned long long)d.B * d.H_kv * (unsigned long long)d.T_cap;
   return d.dtype == KVS_BF16 && (d.d == 64 || d.d == 128) && rows < (1ull << 31) &&
@@ -410,9 +438,15 @@ static cudaError_t launch_shape(const kvs_cache_desc& d, const void* q, void* K,
     attr = true;
   }
   const unsigned long long rows = (unsigned long long)d.B * d.H_kv * (unsigned long long)d.T_cap;
-  CUtensorMap mK, mV;
+  CUtensorMap mK, mV, mL;
   if (!encode_rows_map(&mK, K, rows, d.d, S::kTile) || !encode_rows_map(&mV, V, rows, d.d, S::kTile))
     return cudaErrorInvalidValue;
+  int ln_lead = 0;
+  if (logn) {
+    if (!encode_ln_map(&mL, logn, rows, S::kLnBox, &ln_lead)) return cudaErrorInvalidValue;
+  } else {
+    mL = mK;   // never read
+  }
   // Plain stream order: letting the next grid launch early (programmatic dependent
   // launch) measured 1-2 us slower per step here, since its CTAs take SM slots and
   // cluster places while this grid's combine still runs.
@@ -429,7 +463,7 @@ static cudaError_t launch_shape(const kvs_cache_desc& d, const void* q, void* K,
   cfg.attrs = at;
   cfg.numAttrs = kCluster ? 1 : 0;
   const cudaError_t e = cudaLaunchKernelEx(
-      &cfg, kfn, mK, mV, (const bf16*)q, (bf16*)K, (bf16*)V, logn, len, (const bf16*)k_new,
+      &cfg, kfn, mK, mV, mL, ln_lead, (const bf16*)q, (bf16*)K, (bf16*)V, logn, len, (const bf16*)k_new,
       (const bf16*)v_new, (bf16*)out, d.T_cap, nsplit,
       reinterpret_cast<int32_t*>(ws + Ly.counters), reinterpret_cast<float*>(ws + Ly.part),
       reinterpret_cast<int32_t*>(ws));

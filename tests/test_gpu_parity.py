@@ -321,6 +321,38 @@ def test_decode_ragged_with_append(kvs, dtype, d, G):
     assert kvs.device_flags(ws) == 0
 
 
+@pytest.mark.parametrize("B,H", [(1, 2), (40, 2)])      # few heads: cluster grid; many: split grid
+@pytest.mark.parametrize("lead", [0, 1, 3])
+def test_decode_log_counts_at_any_4_byte_offset(kvs, B, H, lead):
+    """The log-counts may start at any 4-byte boundary (a view into a larger buffer):
+    the TMA map over them starts at the 16-byte boundary below and skips `lead`."""
+    dev = torch.device("cuda")
+    d, G, T_cap = 128, 4, 1000
+    g = torch.Generator().manual_seed(100 + lead)
+    lens = torch.randint(0, T_cap - 1, (B, H), generator=g, dtype=torch.int32)
+    lens[0, 0] = T_cap - 1
+    K = torch.randn(B, H, T_cap, d, generator=g).to(torch.bfloat16)
+    V = torch.randn(B, H, T_cap, d, generator=g).to(torch.bfloat16)
+    logn = torch.log(torch.randint(1, 9, (B, H, T_cap), generator=g).float())
+    buf = torch.zeros(B * H * T_cap + 4, device=dev)
+    ln_view = buf[lead:lead + B * H * T_cap].view(B, H, T_cap)
+    ln_view.copy_(logn.to(dev))
+    assert (ln_view.data_ptr() % 16) == 4 * lead
+    q = (torch.randn(B, H * G, d, generator=g) * 3).to(torch.bfloat16)
+    kn = torch.randn(B, H, d, generator=g).to(torch.bfloat16)
+    vn = torch.randn(B, H, d, generator=g).to(torch.bfloat16)
+    gc = GpuCache(K.to(dev), V.to(dev), lens.to(dev), ln_view)
+    o = to_oracle_cache(gc)
+    desc = kvs.make_desc(B, H, H * G, d, T_cap, torch.bfloat16)
+    ws = kvs.workspace(desc, 32)
+    out = torch.empty(B, H * G, d, dtype=torch.bfloat16, device=dev)
+    kvs.decode_attn(desc, q.to(dev), gc.K, gc.V, ln_view, gc.lens, out, ws, kn.to(dev), vn.to(dev))
+    oo, o = oracle.decode_step(o, q.double().numpy(), kn.double().numpy(), vn.double().numpy())
+    compare_decode(oo, out, torch.bfloat16, G)
+    assert torch.equal(gc.lens.cpu().view(B, H), lens + 1)
+    assert kvs.device_flags(ws) == 0
+
+
 def test_decode_append_at_capacity_sets_flag(kvs):
     dev = torch.device("cuda")
     desc = kvs.make_desc(1, 1, 4, 128, 64, torch.bfloat16)

@@ -500,7 +500,7 @@ def main():
             "clocks": clk,
             "e2e": e2e,
             "gpu_launches": (rn.launches_merge + rn.launches_decode) * args.steps,
-            "roofline": {"kernel": "decode_kernel (split-K GQA decode)", "bound": "hbm",
+            "roofline": {"kernel": "decode_tc_kernel (GQA decode, one thread-block cluster per KV head)", "bound": "hbm",
                          "achieved": achieved, "peak": peak, "peak_kind": peak_kind,
                          "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
                          "bytes_per_launch": rn.decode_bytes_per_launch(),

@@ -174,6 +174,9 @@ kvs_status kvs_merge_compact(const kvs_cache_desc* desc, const void* K, const vo
  * Out: out [B,H_q,d] (cache dtype); K, V, logn, len updated when appending.
  * Workspace: kvs_workspace_size(desc, 0, KVS_OP_DECODE) bytes; its counters must be
  * zero at the first call (each call leaves them zero).
+ * The first call for a device and a B*H_kv sets kernel attributes and asks the CUDA
+ * occupancy calculator which launch shape fits (host calls only, cached): make it
+ * outside any stream capture.
  */
 kvs_status kvs_decode_attn(const kvs_cache_desc* desc, const void* q, void* K, void* V,
                            float* logn, int32_t* len, const void* k_new, const void* v_new,

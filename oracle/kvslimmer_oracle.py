@@ -202,7 +202,10 @@ def pair_norms(alpha_a, alpha_b, v_a, v_b, o):
     return n11, n12, n22
 
 
-def weight_and_score(n11, n12, n22, k_a, k_b):
+FORMS = ("full", "diagonal")
+
+
+def weight_and_score(n11, n12, n22, k_a, k_b, form="full"):
     """Merge weight w_b of the second key and the pair's score (vectorised).
 
     With the effective scalars (g11, g12, g22) = (N11, -N12, N22) -- the
@@ -212,13 +215,30 @@ def weight_and_score(n11, n12, n22, k_a, k_b):
     |k_b - k_a|^2 (N11 N22 - N12^2) / D (the score, reading R3).
     Degenerate pairs use w_b = 1/2 and the objective there,
     |k_b - k_a|^2 (N11 + 2 N12 + N22) / 4 (reading R6).
+
+    form="diagonal" is the ablation without the coupling term (g12 = 0, the
+    per-key weighting of AsymKV that §数学主线二 contrasts with): the objective
+    N11 |k - k_a|^2 + N22 |k - k_b|^2 has its minimiser at
+    k* = (N11 k_a + N22 k_b) / (N11 + N22), i.e. w_b = N22 / (N11 + N22), and
+    minimum value |k_b - k_a|^2 N11 N22 / (N11 + N22); degenerate (N11 + N22 not
+    positive or a term not finite): w_b = 1/2, score |k_b - k_a|^2 (N11 + N22) / 4.
     Returns (w_b, score, degenerate_mask, D).
     """
+    if form not in FORMS:
+        raise ValueError(form)
     n11 = np.asarray(n11, dtype=np.float64)
     n12 = np.asarray(n12, dtype=np.float64)
     n22 = np.asarray(n22, dtype=np.float64)
     delta = np.asarray(k_b, dtype=np.float64) - np.asarray(k_a, dtype=np.float64)
     delta_sq = np.sum(delta * delta, axis=-1)
+    if form == "diagonal":
+        D = n11 + n22
+        with np.errstate(invalid="ignore", divide="ignore", over="ignore"):
+            ok = np.isfinite(n11) & np.isfinite(n22) & np.isfinite(D) & (D > 0.0)
+            safe_D = np.where(ok, D, 1.0)
+            w_b = np.where(ok, n22 / safe_D, 0.5)
+            score = np.where(ok, delta_sq * n11 * n22 / safe_D, delta_sq * D / 4.0)
+        return w_b, score, ~ok, D
     D = n11 - 2.0 * n12 + n22
     with np.errstate(invalid="ignore", divide="ignore", over="ignore"):
         ok = (np.isfinite(n11) & np.isfinite(n12) & np.isfinite(n22) & np.isfinite(D)
@@ -296,8 +316,8 @@ class HeadScores:
     o_bar: np.ndarray
 
 
-def score_head(K, V, log_n, length, cand_begin, n_recent, Q_heads, W):
-    """Score every candidate pair of one KV head."""
+def score_head(K, V, log_n, length, cand_begin, n_recent, Q_heads, W, form="full"):
+    """Score every candidate pair of one KV head (form: see weight_and_score)."""
     K = np.asarray(K, dtype=np.float64)
     V = np.asarray(V, dtype=np.float64)
     alpha_bar, o_bar = window_statistics(Q_heads, K, V, log_n, length, W)
@@ -305,7 +325,7 @@ def score_head(K, V, log_n, length, cand_begin, n_recent, Q_heads, W):
     a = int(cand_begin) + 2 * np.arange(P)
     b = a + 1
     n11, n12, n22 = pair_norms(alpha_bar[a], alpha_bar[b], V[a], V[b], o_bar)
-    w_b, score, degen, D = weight_and_score(n11, n12, n22, K[a], K[b])
+    w_b, score, degen, D = weight_and_score(n11, n12, n22, K[a], K[b], form)
     return HeadScores(score=score, w_b=w_b, n11=n11, n12=n12, n22=n22, D=D,
                       degenerate=degen, alpha_bar=alpha_bar, o_bar=o_bar)
 
@@ -431,7 +451,8 @@ class RoundResult:
     R: np.ndarray                 # pairs merged per unit
 
 
-def merge_round(cache, Q_win, W, cand_begin, n_recent, target, scope="head", storage="f64"):
+def merge_round(cache, Q_win, W, cand_begin, n_recent, target, scope="head", storage="f64",
+                form="full"):
     """One scoring + selection + merge round over a whole cache.
 
     Q_win: (B, H_q, W, d); query head hq belongs to KV head hq // G.
@@ -444,7 +465,7 @@ def merge_round(cache, Q_win, W, cand_begin, n_recent, target, scope="head", sto
     G = Q_win.shape[1] // H
     cand_begin = np.asarray(cand_begin).reshape(B, H)
     scores = [[score_head(cache.K[b][h], cache.V[b][h], cache.log_n[b][h], cache.length(b, h),
-                          cand_begin[b, h], n_recent, Q_win[b, h * G:(h + 1) * G], W)
+                          cand_begin[b, h], n_recent, Q_win[b, h * G:(h + 1) * G], W, form)
                for h in range(H)] for b in range(B)]
     selected = [[None] * H for _ in range(B)]
     if scope == "head":
@@ -480,7 +501,7 @@ def merge_round(cache, Q_win, W, cand_begin, n_recent, target, scope="head", sto
 
 
 def compress(cache, Q_win, W, cand_begin, n_recent, target, scope="head", max_rounds=64,
-             storage="f64"):
+             storage="f64", form="full"):
     """Repeat merge rounds until every unit reaches its budget exactly (reading R4)."""
     rounds = []
     for _ in range(max_rounds):
@@ -491,7 +512,7 @@ def compress(cache, Q_win, W, cand_begin, n_recent, target, scope="head", max_ro
             done = np.all(lens.sum(axis=1) == np.asarray(target).reshape(-1))
         if done:
             return cache, rounds
-        r = merge_round(cache, Q_win, W, cand_begin, n_recent, target, scope, storage)
+        r = merge_round(cache, Q_win, W, cand_begin, n_recent, target, scope, storage, form)
         if np.all(r.R == 0):
             raise ValueError("budget unreachable: no candidate pairs left")
         rounds.append(r)

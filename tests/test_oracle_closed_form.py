@@ -140,3 +140,64 @@ def test_merged_keys_of_a_scored_head_are_objective_minimisers():
                        method="BFGS", options={"gtol": 1e-14})
         np.testing.assert_allclose(m.k_merged[p], res.x, rtol=1e-5, atol=1e-7)
         np.testing.assert_allclose(m.K[m.out_offset[p]], res.x, rtol=1e-5, atol=1e-7)
+
+
+# ----------------------------------------------------------------- diagonal-only ablation
+
+def _diagonal_objective(k, a, b, n11, n22):
+    # the objective without the coupling term, written out by hand
+    return n11 * np.sum((k - a) ** 2) + n22 * np.sum((k - b) ** 2)
+
+
+@pytest.mark.parametrize("seed", range(5))
+def test_diagonal_form_matches_numerical_minimiser(seed):
+    """form="diagonal" (g12 = 0): weight and score are the minimiser and minimum of
+    N11 |k - k_a|^2 + N22 |k - k_b|^2, whatever N12 is."""
+    rng = np.random.default_rng(100 + seed)
+    d = 6
+    a, b = rng.normal(size=d), rng.normal(size=d)
+    n11, n22 = rng.uniform(0.05, 3.0, size=2)
+    n12 = rng.uniform(0.0, 2.0)
+    w_b, score, degen, D = oracle.weight_and_score(n11, n12, n22, a, b, form="diagonal")
+    assert not degen and D == pytest.approx(n11 + n22)
+    res = minimize(lambda k: _diagonal_objective(k, a, b, n11, n22), rng.normal(size=d),
+                   method="BFGS", options={"gtol": 1e-12})
+    np.testing.assert_allclose(a + w_b * (b - a), res.x, rtol=1e-6, atol=1e-6)
+    np.testing.assert_allclose(score, res.fun, rtol=1e-7, atol=1e-10)
+
+
+@pytest.mark.parametrize("seed", range(5))
+def test_full_form_never_loses_to_diagonal_on_the_full_objective(seed):
+    """The full form minimises the coupled objective, so the diagonal form's merged key
+    can only do as well or worse on it (the quantity the ablation measures)."""
+    rng = np.random.default_rng(200 + seed)
+    d = 16
+    a, b = rng.normal(size=(64, d)), rng.normal(size=(64, d))
+    n11, n22 = rng.uniform(0.05, 2.0, size=(2, 64))
+    n12 = rng.uniform(0.0, 0.45, size=64) * np.minimum(n11, n22)
+    w_f, s_f, deg_f, _ = oracle.weight_and_score(n11, n12, n22, a, b)
+    w_d, _, deg_d, _ = oracle.weight_and_score(n11, n12, n22, a, b, form="diagonal")
+    assert not deg_f.any() and not deg_d.any()
+    for i in range(64):
+        f_full_at_diag = _objective(a[i] + w_d[i] * (b[i] - a[i]), a[i], b[i], n11[i], n12[i], n22[i])
+        assert s_f[i] <= f_full_at_diag + 1e-12 * max(1.0, abs(f_full_at_diag))
+    # and with some coupling present the diagonal key is strictly worse somewhere
+    assert np.any(np.abs(w_f - w_d) > 1e-6)
+
+
+def test_diagonal_form_equals_full_form_without_coupling():
+    rng = np.random.default_rng(7)
+    a, b = rng.normal(size=(10, 4)), rng.normal(size=(10, 4))
+    n11, n22 = rng.uniform(0.1, 2.0, size=(2, 10))
+    full = oracle.weight_and_score(n11, np.zeros(10), n22, a, b)
+    diag = oracle.weight_and_score(n11, np.zeros(10), n22, a, b, form="diagonal")
+    np.testing.assert_allclose(full[0], diag[0], rtol=1e-15)
+    np.testing.assert_allclose(full[1], diag[1], rtol=1e-15)
+
+
+def test_diagonal_form_degenerate_pair_is_the_plain_average():
+    a, b = np.zeros(3), np.ones(3)
+    w_b, score, degen, _ = oracle.weight_and_score(0.0, 0.3, 0.0, a, b, form="diagonal")
+    assert degen and w_b == 0.5 and score == 0.0
+    with pytest.raises(ValueError):
+        oracle.weight_and_score(1.0, 0.0, 1.0, a, b, form="cosine")

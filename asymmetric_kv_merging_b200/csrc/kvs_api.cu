@@ -98,6 +98,16 @@ kvs_status kvs_score_pairs(const kvs_cache_desc* desc, const void* K, const void
                            const float* logn, const int32_t* len, const int32_t* cand_begin,
                            int32_t n_recent, const void* Q_win, int32_t W, float* score,
                            float* w_b, void* ws, size_t ws_bytes, kvs_stream_t stream) {
+  return kvs_score_pairs_form(desc, K, V, logn, len, cand_begin, n_recent, Q_win, W, score, w_b,
+                              KVS_FORM_FULL, ws, ws_bytes, stream);
+}
+
+kvs_status kvs_score_pairs_form(const kvs_cache_desc* desc, const void* K, const void* V,
+                                const float* logn, const int32_t* len, const int32_t* cand_begin,
+                                int32_t n_recent, const void* Q_win, int32_t W, float* score,
+                                float* w_b, int32_t form, void* ws, size_t ws_bytes,
+                                kvs_stream_t stream) {
+  if (form != KVS_FORM_FULL && form != KVS_FORM_DIAGONAL) return KVS_ERR_INVALID_ARG;
   kvs_status s = check_desc(desc);
   if (s != KVS_OK) return s;
   if (!K || !V || !len || !cand_begin || !Q_win || !score || !w_b) return KVS_ERR_INVALID_ARG;
@@ -120,7 +130,7 @@ kvs_status kvs_score_pairs(const kvs_cache_desc* desc, const void* K, const void
   char* w = static_cast<char*>(ws);
   cudaError_t e = launch_window_stats(*desc, K, V, logn, len, Q_win, W, Ly, w, st);
   if (e != cudaSuccess) return KVS_ERR_CUDA;
-  e = launch_pair_score(*desc, K, V, len, cand_begin, n_recent, Ly, w, score, w_b, st);
+  e = launch_pair_score(*desc, K, V, len, cand_begin, n_recent, form, Ly, w, score, w_b, st);
   return from_cuda(e);
 }
 

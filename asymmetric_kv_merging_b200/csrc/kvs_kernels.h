@@ -17,8 +17,8 @@ cudaError_t launch_window_stats(const kvs_cache_desc& d, const void* K, const vo
 // Pair norms, merge weight and score from alpha_bar / o_bar.
 cudaError_t launch_pair_score(const kvs_cache_desc& d, const void* K, const void* V,
                               const int32_t* len, const int32_t* cand_begin, int n_recent,
-                              const ScoreLayout& Ly, char* ws, float* score, float* w_b,
-                              cudaStream_t st);
+                              int form, const ScoreLayout& Ly, char* ws, float* score,
+                              float* w_b, cudaStream_t st);
 
 // Selection to the budget, then merge + compaction (out-of-place or in-place).
 cudaError_t launch_select(const kvs_cache_desc& d, const float* score, const int32_t* len,

@@ -4,7 +4,7 @@
 // §数学主线四: c11 = a_m (1 - 2 a_m)(v_m - o), c22 likewise, c12 = -a_m a_m1 (v_m + v_m1 - 2o);
 // the forward-only merged key k* = [(|c11| - |c12|) k_m + (|c22| - |c12|) k_m1] /
 // (|c11| - 2|c12| + |c22|). §数学主线二: the objective whose minimum value ranks
-// the pairs. Window-mean attention a and o_bar come from the window-statistics pass.
+// the pairs; the diagonal form (ablation) drops its coupling term, |c12| = 0. Window-mean attention a and o_bar come from the window-statistics pass.
 //
 // One pair is handled by LPR lanes (LPR = 16-byte vectors per row); each lane holds
 // a 16-byte slice of k_a, k_b, v_a, v_b and the matching slice of o_bar; the four
@@ -22,7 +22,8 @@ __global__ void __launch_bounds__(kScoreThreads)
 pair_score_kernel(const T* __restrict__ K, const T* __restrict__ V,
                   const float* __restrict__ alpha, const float* __restrict__ obar,
                   const int32_t* __restrict__ len, const int32_t* __restrict__ cand_begin,
-                  int n_recent, int T_cap, float* __restrict__ score, float* __restrict__ w_b) {
+                  int n_recent, int T_cap, int form, float* __restrict__ score,
+                  float* __restrict__ w_b) {
   constexpr int VN = Vec16<T>::n;
   constexpr int LPR = D / VN;                 // lanes per row: 8, 16 or 32
   constexpr int PPI = 32 / LPR;               // pairs per warp per iteration
@@ -87,7 +88,8 @@ pair_score_kernel(const T* __restrict__ K, const T* __restrict__ V,
       const float aa = ah[a], ab = ah[a + 1];
       const float n11 = fabsf(aa * (1.f - 2.f * aa)) * sqrtf(ea);
       const float n22 = fabsf(ab * (1.f - 2.f * ab)) * sqrtf(eb);
-      const float n12 = aa * ab * sqrtf(ec);
+      // the diagonal form drops the coupling term (ablation): N12 = 0
+      const float n12 = form == KVS_FORM_DIAGONAL ? 0.f : aa * ab * sqrtf(ec);
       const float den = n11 - 2.f * n12 + n22;
       const bool ok = isfinite(n11) && isfinite(n12) && isfinite(n22) && isfinite(den) &&
                       den > 1e-6f * (n11 + n22);
@@ -108,7 +110,7 @@ pair_score_kernel(const T* __restrict__ K, const T* __restrict__ V,
 template <typename T, int D>
 static cudaError_t launch_pair_score_t(const kvs_cache_desc& d, const void* K, const void* V,
                                        const int32_t* len, const int32_t* cand_begin,
-                                       int n_recent, const ScoreLayout& Ly, char* ws,
+                                       int n_recent, int form, const ScoreLayout& Ly, char* ws,
                                        float* score, float* w_b, cudaStream_t st) {
   constexpr int VN = Vec16<T>::n;
   constexpr int LPR = D / VN;
@@ -118,24 +120,24 @@ static cudaError_t launch_pair_score_t(const kvs_cache_desc& d, const void* K, c
   dim3 grid((pmax + PAIRS_PER_CTA - 1) / PAIRS_PER_CTA, units);
   pair_score_kernel<T, D><<<grid, kScoreThreads, 0, st>>>(
       (const T*)K, (const T*)V, reinterpret_cast<const float*>(ws + Ly.alpha),
-      reinterpret_cast<const float*>(ws + Ly.obar), len, cand_begin, n_recent, d.T_cap, score,
-      w_b);
+      reinterpret_cast<const float*>(ws + Ly.obar), len, cand_begin, n_recent, d.T_cap, form,
+      score, w_b);
   count_launches(1);
   return cudaGetLastError();
 }
 
 cudaError_t launch_pair_score(const kvs_cache_desc& d, const void* K, const void* V,
                               const int32_t* len, const int32_t* cand_begin, int n_recent,
-                              const ScoreLayout& Ly, char* ws, float* score, float* w_b,
-                              cudaStream_t st) {
+                              int form, const ScoreLayout& Ly, char* ws, float* score,
+                              float* w_b, cudaStream_t st) {
   if (d.dtype == KVS_BF16) {
     if (d.d == 128)
-      return launch_pair_score_t<bf16, 128>(d, K, V, len, cand_begin, n_recent, Ly, ws, score, w_b, st);
-    return launch_pair_score_t<bf16, 64>(d, K, V, len, cand_begin, n_recent, Ly, ws, score, w_b, st);
+      return launch_pair_score_t<bf16, 128>(d, K, V, len, cand_begin, n_recent, form, Ly, ws, score, w_b, st);
+    return launch_pair_score_t<bf16, 64>(d, K, V, len, cand_begin, n_recent, form, Ly, ws, score, w_b, st);
   }
   if (d.d == 128)
-    return launch_pair_score_t<float, 128>(d, K, V, len, cand_begin, n_recent, Ly, ws, score, w_b, st);
-  return launch_pair_score_t<float, 64>(d, K, V, len, cand_begin, n_recent, Ly, ws, score, w_b, st);
+    return launch_pair_score_t<float, 128>(d, K, V, len, cand_begin, n_recent, form, Ly, ws, score, w_b, st);
+  return launch_pair_score_t<float, 64>(d, K, V, len, cand_begin, n_recent, form, Ly, ws, score, w_b, st);
 }
 
 }  // namespace kvs

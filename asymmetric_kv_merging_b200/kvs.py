@@ -23,6 +23,7 @@ _lib = ctypes.CDLL(_LIB_PATH)
 F32, BF16 = 0, 1
 OP_SCORE, OP_MERGE, OP_DECODE = 0, 1, 2
 SCOPE_HEAD, SCOPE_POOLED = 0, 1
+FORM_FULL, FORM_DIAGONAL = 0, 1
 FLAG_BAD_LENGTH, FLAG_OUT_CAPACITY, FLAG_INPLACE_SPAN, FLAG_NONFINITE_STATS = 1, 2, 4, 8
 FLAG_TIMEOUT = 16
 
@@ -31,7 +32,7 @@ STATUS = {0: "KVS_OK", 1: "KVS_ERR_INVALID_ARG", 2: "KVS_ERR_UNSUPPORTED", 3: "K
 
 EXPORTS = ("kvs_workspace_size", "kvs_score_pairs", "kvs_merge_compact", "kvs_decode_attn",
            "kvs_device_flags", "kvs_status_str", "kvs_version", "kvs_launch_count",
-           "kvs_decode_attn_static", "kvs_static_scratch_bytes")
+           "kvs_decode_attn_static", "kvs_static_scratch_bytes", "kvs_score_pairs_form")
 
 
 class CacheDesc(ctypes.Structure):
@@ -56,6 +57,9 @@ _lib.kvs_workspace_size.restype = _sz
 _lib.kvs_workspace_size.argtypes = [_P, _i32, _i32]
 _lib.kvs_score_pairs.restype = ctypes.c_int
 _lib.kvs_score_pairs.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _vp, _vp, _vp, _sz, _vp]
+_lib.kvs_score_pairs_form.restype = ctypes.c_int
+_lib.kvs_score_pairs_form.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _vp, _vp, _i32,
+                                      _vp, _sz, _vp]
 _lib.kvs_merge_compact.restype = ctypes.c_int
 _lib.kvs_merge_compact.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _i32, _i32,
                                    _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
@@ -125,11 +129,20 @@ def workspace(desc: CacheDesc, W: int = 32, ops=(OP_SCORE, OP_MERGE, OP_DECODE),
     return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
 
 
-def score_pairs(desc, K, V, logn, lens, cand_begin, n_recent, Q_win, W, score, w_b, ws, stream=None):
-    _check(_lib.kvs_score_pairs(ctypes.byref(desc), _ptr(K), _ptr(V), _ptr(logn), _ptr(lens),
-                                _ptr(cand_begin), int(n_recent), _ptr(Q_win), int(W), _ptr(score),
-                                _ptr(w_b), _ptr(ws), ws.numel(), _stream(stream)),
-           "kvs_score_pairs")
+def score_pairs(desc, K, V, logn, lens, cand_begin, n_recent, Q_win, W, score, w_b, ws, stream=None,
+                form=None):
+    """kvs_score_pairs, or kvs_score_pairs_form when `form` is given."""
+    if form is None:
+        _check(_lib.kvs_score_pairs(ctypes.byref(desc), _ptr(K), _ptr(V), _ptr(logn), _ptr(lens),
+                                    _ptr(cand_begin), int(n_recent), _ptr(Q_win), int(W),
+                                    _ptr(score), _ptr(w_b), _ptr(ws), ws.numel(), _stream(stream)),
+               "kvs_score_pairs")
+        return
+    _check(_lib.kvs_score_pairs_form(ctypes.byref(desc), _ptr(K), _ptr(V), _ptr(logn), _ptr(lens),
+                                     _ptr(cand_begin), int(n_recent), _ptr(Q_win), int(W),
+                                     _ptr(score), _ptr(w_b), int(form), _ptr(ws), ws.numel(),
+                                     _stream(stream)),
+           "kvs_score_pairs_form")
 
 
 def merge_compact(desc, K, V, logn, lens, cand_begin, n_recent, score, w_b, target, scope,

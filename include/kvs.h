@@ -72,6 +72,8 @@ typedef struct CUstream_st* kvs_stream_t; /* a cudaStream_t; NULL = legacy defau
 
 enum { KVS_OP_SCORE = 0, KVS_OP_MERGE = 1, KVS_OP_DECODE = 2 };
 enum { KVS_SCOPE_HEAD = 0, KVS_SCOPE_POOLED = 1 };
+/* Scoring form: the coupled forward-only objective, or its diagonal-only ablation. */
+enum { KVS_FORM_FULL = 0, KVS_FORM_DIAGONAL = 1 };
 
 /* Device flag bits (see kvs_device_flags). */
 enum {
@@ -110,7 +112,7 @@ size_t kvs_workspace_size(const kvs_cache_desc* desc, int32_t W, int32_t op);
  *       finite: w_b = 1/2, score = |k_b - k_a|^2 (N11 + 2 N12 + N22) / 4.
  *
  * In:  K, V [B,H_kv,T_cap,d]; logn (nullable); len [B*H_kv]; cand_begin [B*H_kv];
- *      n_recent >= 0; Q_win [B,H_q,W,d], 1 <= W, G*W <= 256.
+ *      n_recent >= 0; Q_win [B,H_q,W,d], 1 <= W, G*W <= 128 (else KVS_ERR_UNSUPPORTED).
  * Out: score, w_b [B,H_kv,T_cap/2] fp32 (entries p >= P of a head are not written).
  * Workspace: kvs_workspace_size(desc, W, KVS_OP_SCORE) bytes.
  */
@@ -119,6 +121,25 @@ kvs_status kvs_score_pairs(const kvs_cache_desc* desc, const void* K, const void
                            int32_t n_recent, const void* Q_win, int32_t W,
                            float* score, float* w_b,
                            void* ws, size_t ws_bytes, kvs_stream_t stream);
+
+/*
+ * kvs_score_pairs_form -- kvs_score_pairs with a choice of scoring form.
+ *
+ * form = KVS_FORM_FULL: exactly kvs_score_pairs.
+ * form = KVS_FORM_DIAGONAL: the ablation that drops the coupling term of the
+ *   §数学主线二 objective (g12 = 0; the per-key weighting of AsymKV that the pages
+ *   contrast KVSlimmer with): N12 is taken as 0, so
+ *     w_b = N22 / (N11 + N22),  score = |k_b - k_a|^2 N11 N22 / (N11 + N22),
+ *   with the same degenerate rule (w_b = 1/2, score = |k_b - k_a|^2 (N11 + N22) / 4
+ *   when N11 + N22 is not positive or a term is not finite).
+ * Any other form: KVS_ERR_INVALID_ARG, nothing launched. Arguments, outputs,
+ * workspace and errors otherwise as kvs_score_pairs.
+ */
+kvs_status kvs_score_pairs_form(const kvs_cache_desc* desc, const void* K, const void* V,
+                                const float* logn, const int32_t* len, const int32_t* cand_begin,
+                                int32_t n_recent, const void* Q_win, int32_t W,
+                                float* score, float* w_b, int32_t form,
+                                void* ws, size_t ws_bytes, kvs_stream_t stream);
 
 /*
  * kvs_merge_compact -- one merge round: select pairs to the budget, merge them,

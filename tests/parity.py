@@ -70,7 +70,7 @@ class GpuCache:
 
 
 def gpu_round(cache: GpuCache, H_q, Q_win, W, cand_begin, n_recent, target, scope, ws,
-              T_cap_out=None, inplace=False):
+              T_cap_out=None, inplace=False, form=None):
     B, H, T_cap, d = cache.K.shape
     dev = cache.K.device
     desc = kvs.make_desc(B, H, H_q, d, T_cap, cache.K.dtype)
@@ -78,7 +78,7 @@ def gpu_round(cache: GpuCache, H_q, Q_win, W, cand_begin, n_recent, target, scop
     score = torch.full((B, H, npair), float("nan"), dtype=torch.float32, device=dev)
     w_b = torch.full_like(score, float("nan"))
     kvs.score_pairs(desc, cache.K, cache.V, cache.logn, cache.lens, cand_begin, n_recent,
-                    Q_win.contiguous(), W, score, w_b, ws)
+                    Q_win.contiguous(), W, score, w_b, ws, form=form)
     sel = torch.zeros(B, H, npair, dtype=torch.uint8, device=dev)
     off = torch.full((B, H, npair), -1, dtype=torch.int32, device=dev)
     km = torch.zeros(B, H, npair, d, dtype=torch.float32, device=dev)

@@ -29,7 +29,7 @@ def _workspace(kvs, B, H, H_q, d, T_cap, dtype, W=32):
     return kvs.workspace(kvs.make_desc(B, H, H_q, d, T_cap, dtype), W)
 
 
-def compress_both(kvs, w, li, batch=None, ratio=None, stats=None, Q_override=None):
+def compress_both(kvs, w, li, batch=None, ratio=None, stats=None, Q_override=None, form=None):
     """Compress on the GPU (all sequences) and in the oracle (sequences `batch`),
     comparing every round."""
     dev = torch.device("cuda")
@@ -57,8 +57,9 @@ def compress_both(kvs, w, li, batch=None, ratio=None, stats=None, Q_override=Non
         if np.all(done):
             break
         r = oracle.merge_round(o, Qo, w.W, np.full((len(batch), H), w.sink), w.W,
-                               target_np[batch], scope, storage_of(li.K.dtype))
-        gout, gres = gpu_round(g, w.H_q, Q, w.W, cand, w.W, target, scope_code, ws)
+                               target_np[batch], scope, storage_of(li.K.dtype),
+                               "diagonal" if form == kvs.FORM_DIAGONAL else "full")
+        gout, gres = gpu_round(g, w.H_q, Q, w.W, cand, w.W, target, scope_code, ws, form=form)
         compare_round(r, gres, gout, g, o, li.K.dtype, scope, batch, stats)
         g, o = gout, r.cache
     else:
@@ -123,6 +124,28 @@ def test_workload1_llama_layer_full_size(kvs):
     print("workload 1", stats.report())
     assert stats.merged_compared > 8 * 16000
     assert len(stats.diverged_heads) <= 1
+
+
+@pytest.mark.parametrize("wl", [0, 1])
+def test_diagonal_form_pipeline(kvs, wl):
+    """kvs_score_pairs_form with the diagonal-only form (the coupling term dropped):
+    scores, weights, selection and the merged caches against the oracle's diagonal form,
+    every round, then decode."""
+    w = inputs.workload(wl)
+    li = inputs.make_layer(w, 0, device="cuda")
+    g, o, stats, ws = compress_both(kvs, w, li, form=kvs.FORM_DIAGONAL)
+    g, o = decode_both(kvs, w, li, g, o, range(min(4, w.n_decode)), stats=stats, ws=ws)
+    print("diagonal form, workload", wl, stats.report())
+    assert stats.scores_compared > 0
+    assert len(stats.diverged_heads) <= 1
+
+
+def test_score_form_rejects_unknown_form(kvs):
+    desc = kvs.make_desc(1, 1, 1, 64, 64, torch.float32)
+    with pytest.raises(kvs.KvsError) as e:
+        kvs.score_pairs(desc, None, None, None, None, None, 0, None, 1, None, None,
+                        torch.zeros(16, dtype=torch.uint8), form=7)
+    assert e.value.status == 1
 
 
 # --------------------------------------------------------------------------- workload 2

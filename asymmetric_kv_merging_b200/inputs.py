@@ -191,11 +191,15 @@ class LayerInputs:
 
 
 def make_layer(w: Workload, layer: int = 0, device="cpu", T_cap: Optional[int] = None,
-               lens: Optional[torch.Tensor] = None, q_scale: float = 1.0) -> LayerInputs:
+               lens: Optional[torch.Tensor] = None, q_scale: float = 1.0,
+               window_ends: Optional[list] = None) -> LayerInputs:
     """Draw one layer of workload `w` on `device`.
 
     `q_scale` multiplies the queries (window and decode); values above 1 give
     peaked attention, a regime the default recipe does not reach.
+    `window_ends` (positions e >= W, all <= the prefill length): also draw the W
+    queries ending at each e, as extra["Q_ends"] [len(window_ends), B, H_q, W, d]
+    (the window queries of a chunked prefill).
     """
     device = torch.device(device)
     gen = _gen(1000 * w.index + layer, device)
@@ -218,6 +222,8 @@ def make_layer(w: Workload, layer: int = 0, device="cpu", T_cap: Optional[int] =
     q_dec = torch.zeros(w.n_decode, w.B, w.H_q, w.d, dtype=dt, device=device)
     k_new = torch.zeros(w.n_decode, w.B, w.H_kv, w.d, dtype=dt, device=device)
     v_new = torch.zeros_like(k_new)
+    ends = list(window_ends or [])
+    Q_ends = torch.zeros(len(ends), w.B, w.H_q, w.W, w.d, dtype=dt, device=device)
     for b in range(w.B):
         T_b = int(lens[b])
         x = ar1_hidden(T_b + w.n_decode, w.d_model, rho, gen, device)
@@ -227,6 +233,9 @@ def make_layer(w: Workload, layer: int = 0, device="cpu", T_cap: Optional[int] =
         V[b, :, :T_b] = vb[:T_b].transpose(0, 1).to(dt)
         qw = (x[T_b - w.W:T_b] @ WQ).view(w.W, w.H_q, w.d) * q_scale
         Q_win[b] = qw.transpose(0, 1).to(dt)
+        for i, e in enumerate(ends):
+            qe = (x[e - w.W:e] @ WQ).view(w.W, w.H_q, w.d) * q_scale
+            Q_ends[i, b] = qe.transpose(0, 1).to(dt)
         if w.n_decode:
             xd = x[T_b:]
             q_dec[:, b] = ((xd @ WQ).view(-1, w.H_q, w.d) * q_scale).to(dt)
@@ -235,7 +244,8 @@ def make_layer(w: Workload, layer: int = 0, device="cpu", T_cap: Optional[int] =
         del x, kb, vb
     lens_bh = lens.to(torch.int32).view(w.B, 1).expand(w.B, w.H_kv).contiguous()
     return LayerInputs(K=K, V=V, lens=lens_bh.to(device), Q_win=Q_win, q_dec=q_dec,
-                       k_new=k_new, v_new=v_new, rho=rho)
+                       k_new=k_new, v_new=v_new, rho=rho,
+                       extra={"Q_ends": Q_ends} if ends else {})
 
 
 def small_workload(base: Workload, **changes) -> Workload:

@@ -557,6 +557,31 @@ def decode_step(cache, q, k_new=None, v_new=None):
     return out, cache
 
 
+def append_rows(cache, k_rows, v_rows):
+    """Append n rows with count 1 (log n = 0) to every head; k_rows, v_rows (B, H, n, d).
+    Returns a new Cache (the input is not modified)."""
+    k_rows = np.asarray(k_rows, dtype=np.float64)
+    v_rows = np.asarray(v_rows, dtype=np.float64)
+    B, H = cache.B, cache.H
+    n = k_rows.shape[2]
+    return Cache([[np.vstack([cache.K[b][h], k_rows[b, h]]) for h in range(H)] for b in range(B)],
+                 [[np.vstack([cache.V[b][h], v_rows[b, h]]) for h in range(H)] for b in range(B)],
+                 [[np.append(cache.log_n[b][h], np.zeros(n)) for h in range(H)] for b in range(B)])
+
+
+def prefill_chunk(cache, k_chunk, v_chunk, Q_win, W, budget, sink, storage="f64", form="full"):
+    """One step of chunked streaming prefill compression ([KVS] §实验设置: context budget,
+    chunk size and preserved initial tokens; reading R11): append the chunk to every head,
+    then run merge rounds on heads longer than `budget` -- candidate span [sink, len - W),
+    window queries Q_win (the chunk's last W positions), per-head target budget -- until
+    every head holds min(len, budget) rows. Returns (cache, rounds)."""
+    cache = append_rows(cache, k_chunk, v_chunk)
+    lens = cache.lengths()
+    target = np.minimum(lens, int(budget))
+    cand = np.full(lens.shape, int(sink))
+    return compress(cache, Q_win, W, cand, W, target, "head", storage=storage, form=form)
+
+
 def budget(length, ratio):
     """Per-head token budget floor(len / ratio)."""
     return int(length) // int(ratio)

@@ -89,6 +89,9 @@ size_t kvs_workspace_size(const kvs_cache_desc* desc, int32_t W, int32_t op) {
       return merge_layout(*desc).total;
     case KVS_OP_DECODE:
       return decode_layout(*desc).total;
+    case KVS_OP_PREFILL:
+      if (W < 1) return 0;
+      return prefill_layout(*desc, W).total;
     default:
       return 0;
   }
@@ -201,6 +204,74 @@ kvs_status kvs_merge_compact(const kvs_cache_desc* desc, const void* K, const vo
   e = launch_merge(*desc, K, V, logn, score, w_b, scope, T_cap_out, inplace, K_out, V_out,
                    logn_out, len_out, dbg_selected, dbg_out_offset, dbg_kmerged_f32, Ly, w, st);
   return from_cuda(e);
+}
+
+kvs_status kvs_prefill_chunk(const kvs_cache_desc* desc, void* K, void* V, float* logn,
+                             int32_t* len, int32_t L, const void* k_chunk, const void* v_chunk,
+                             int32_t n, const void* Q_win, int32_t W, int32_t budget,
+                             int32_t sink, int32_t form, int32_t* L_out, void* ws,
+                             size_t ws_bytes, kvs_stream_t stream) {
+  kvs_status s = check_desc(desc);
+  if (s != KVS_OK) return s;
+  if (!K || !V || !logn || !len || !Q_win || !L_out || (n > 0 && (!k_chunk || !v_chunk)))
+    return KVS_ERR_INVALID_ARG;
+  if (form != KVS_FORM_FULL && form != KVS_FORM_DIAGONAL) return KVS_ERR_INVALID_ARG;
+  if (!aligned(K, 16) || !aligned(V, 16) || !aligned(Q_win, 16) || !aligned(logn, 4) ||
+      !aligned(len, 4) || (n > 0 && (!aligned(k_chunk, 16) || !aligned(v_chunk, 16))))
+    return KVS_ERR_INVALID_ARG;
+  if (L < 0 || n < 0 || W < 1 || sink < 0 || budget < 0) return KVS_ERR_INVALID_ARG;
+  if ((long long)L + n > desc->T_cap) return KVS_ERR_INVALID_ARG;
+  const int G = desc->H_q / desc->H_kv;
+  if (G * W > 128) return KVS_ERR_UNSUPPORTED;
+  // the rounds rewrite each head in place from its candidate start on
+  if ((long long)L + n - sink > kInplaceMaxSpan) return KVS_ERR_UNSUPPORTED;
+  const size_t heads = (size_t)desc->B * desc->H_kv;
+  const size_t chunk_bytes = heads * (size_t)n * desc->d * elem_bytes(desc);
+  Range rk{(const char*)K, cache_bytes(desc, desc->T_cap)}, rv{(const char*)V, cache_bytes(desc, desc->T_cap)};
+  Range rkc{(const char*)k_chunk, chunk_bytes}, rvc{(const char*)v_chunk, chunk_bytes};
+  Range rl{(const char*)logn, heads * desc->T_cap * sizeof(float)}, rn{(const char*)len, heads * sizeof(int32_t)};
+  const Range all[] = {rk, rv, rl, rn, rkc, rvc};
+  for (int i = 0; i < 6; ++i)
+    for (int j = i + 1; j < 6; ++j)
+      if (overlap(all[i], all[j])) return KVS_ERR_ALIAS;
+  // plan the rounds on the host (every head has length L): R = min(P, len - budget)
+  int rounds = 0, Lc = L + n;
+  while (Lc > budget) {
+    const int span = Lc - W - sink;
+    const int P = span > 0 ? span / 2 : 0;
+    const int R = P < Lc - budget ? P : Lc - budget;
+    if (R <= 0 || rounds == 64) return KVS_ERR_BUDGET;   // nothing launched
+    ++rounds;
+    Lc -= R;
+  }
+  const PrefillLayout Ly = prefill_layout(*desc, W);
+  s = check_ws(ws, ws_bytes, Ly.total);
+  if (s != KVS_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(ws);
+  float* score = reinterpret_cast<float*>(w + Ly.score_arr);
+  float* w_b = reinterpret_cast<float*>(w + Ly.w_b_arr);
+  int32_t* cand = reinterpret_cast<int32_t*>(w + Ly.cand);
+  int32_t* target = reinterpret_cast<int32_t*>(w + Ly.target);
+  cudaError_t e = launch_append_rows(*desc, K, V, logn, len, L, k_chunk, v_chunk, n, w, st);
+  if (e != cudaSuccess) return KVS_ERR_CUDA;
+  if (rounds > 0) {
+    e = launch_fill2(cand, sink, target, budget, (int)heads, st);
+    if (e != cudaSuccess) return KVS_ERR_CUDA;
+  }
+  for (int r = 0; r < rounds; ++r) {
+    e = launch_window_stats(*desc, K, V, logn, len, Q_win, W, Ly.score, w, st);
+    if (e != cudaSuccess) return KVS_ERR_CUDA;
+    e = launch_pair_score(*desc, K, V, len, cand, W, form, Ly.score, w, score, w_b, st);
+    if (e != cudaSuccess) return KVS_ERR_CUDA;
+    e = launch_select(*desc, score, len, cand, W, target, KVS_SCOPE_HEAD, Ly.merge, w, st);
+    if (e != cudaSuccess) return KVS_ERR_CUDA;
+    e = launch_merge(*desc, K, V, logn, score, w_b, KVS_SCOPE_HEAD, desc->T_cap, true, K, V, logn,
+                     len, nullptr, nullptr, nullptr, Ly.merge, w, st);
+    if (e != cudaSuccess) return KVS_ERR_CUDA;
+  }
+  *L_out = Lc;
+  return KVS_OK;
 }
 
 kvs_status kvs_decode_attn(const kvs_cache_desc* desc, const void* q, void* K, void* V,

@@ -200,4 +200,28 @@ inline DecodeLayout decode_layout(const kvs_cache_desc& d) {
   return L;
 }
 
+// Chunked prefill: the score and merge scratch share one region (the score scratch is
+// dead once the pairs are scored), followed by the round's pair scores and weights and
+// the per-head candidate starts and targets.
+struct PrefillLayout {
+  ScoreLayout score;
+  MergeLayout merge;
+  size_t score_arr, w_b_arr, cand, target, total;
+};
+
+inline PrefillLayout prefill_layout(const kvs_cache_desc& d, int W) {
+  PrefillLayout L;
+  L.score = score_layout(d, W);
+  L.merge = merge_layout(d);
+  const size_t heads = (size_t)d.B * d.H_kv;
+  const size_t pairs = heads * (size_t)(d.T_cap / 2);
+  const size_t scratch_end = L.score.total > L.merge.total ? L.score.total : L.merge.total;
+  L.score_arr = align_up(scratch_end, kWsAlign);
+  L.w_b_arr = align_up(L.score_arr + pairs * sizeof(float), kWsAlign);
+  L.cand = align_up(L.w_b_arr + pairs * sizeof(float), kWsAlign);
+  L.target = align_up(L.cand + heads * sizeof(int32_t), kWsAlign);
+  L.total = align_up(L.target + heads * sizeof(int32_t), kWsAlign);
+  return L;
+}
+
 }  // namespace kvs

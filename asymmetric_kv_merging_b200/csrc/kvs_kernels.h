@@ -31,6 +31,14 @@ cudaError_t launch_merge(const kvs_cache_desc& d, const void* K, const void* V, 
                          int32_t* len_out, uint8_t* dbg_sel, int32_t* dbg_off, float* dbg_km,
                          const MergeLayout& Ly, char* ws, cudaStream_t st);
 
+// Chunked prefill: append n rows of a chunk ([B, H_kv, n, d]) at row L of every head
+// whose length is L (others: KVS_FLAG_BAD_LENGTH), then len = L + n; fill two int32
+// arrays with constants.
+cudaError_t launch_append_rows(const kvs_cache_desc& d, void* K, void* V, float* logn,
+                               int32_t* len, int L, const void* k_rows, const void* v_rows, int n,
+                               char* ws, cudaStream_t st);
+cudaError_t launch_fill2(int32_t* a, int32_t va, int32_t* b, int32_t vb, int n, cudaStream_t st);
+
 // Split-K GQA decode with fused split combine and optional append.
 cudaError_t launch_decode(const kvs_cache_desc& d, const void* q, void* K, void* V, float* logn,
                           int32_t* len, const void* k_new, const void* v_new, void* out,

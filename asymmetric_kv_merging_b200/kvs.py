@@ -21,7 +21,7 @@ if not os.path.exists(_LIB_PATH):
 _lib = ctypes.CDLL(_LIB_PATH)
 
 F32, BF16 = 0, 1
-OP_SCORE, OP_MERGE, OP_DECODE = 0, 1, 2
+OP_SCORE, OP_MERGE, OP_DECODE, OP_PREFILL = 0, 1, 2, 3
 SCOPE_HEAD, SCOPE_POOLED = 0, 1
 FORM_FULL, FORM_DIAGONAL = 0, 1
 FLAG_BAD_LENGTH, FLAG_OUT_CAPACITY, FLAG_INPLACE_SPAN, FLAG_NONFINITE_STATS = 1, 2, 4, 8
@@ -32,7 +32,8 @@ STATUS = {0: "KVS_OK", 1: "KVS_ERR_INVALID_ARG", 2: "KVS_ERR_UNSUPPORTED", 3: "K
 
 EXPORTS = ("kvs_workspace_size", "kvs_score_pairs", "kvs_merge_compact", "kvs_decode_attn",
            "kvs_device_flags", "kvs_status_str", "kvs_version", "kvs_launch_count",
-           "kvs_decode_attn_static", "kvs_static_scratch_bytes", "kvs_score_pairs_form")
+           "kvs_decode_attn_static", "kvs_static_scratch_bytes", "kvs_score_pairs_form",
+           "kvs_prefill_chunk")
 
 
 class CacheDesc(ctypes.Structure):
@@ -60,6 +61,9 @@ _lib.kvs_score_pairs.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _
 _lib.kvs_score_pairs_form.restype = ctypes.c_int
 _lib.kvs_score_pairs_form.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _vp, _vp, _i32,
                                       _vp, _sz, _vp]
+_lib.kvs_prefill_chunk.restype = ctypes.c_int
+_lib.kvs_prefill_chunk.argtypes = [_P, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _i32, _vp, _i32, _i32,
+                                   _i32, _i32, ctypes.POINTER(_i32), _vp, _sz, _vp]
 _lib.kvs_merge_compact.restype = ctypes.c_int
 _lib.kvs_merge_compact.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _i32, _i32,
                                    _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
@@ -190,3 +194,17 @@ def decode_attn_static(desc, q, K, V, logn, lens, out, k_new=None, v_new=None, s
 
 def static_scratch_bytes() -> int:
     return int(_lib.kvs_static_scratch_bytes())
+
+
+def prefill_chunk(desc, K, V, logn, lens, L, k_chunk, v_chunk, Q_win, W, budget, sink, ws,
+                  form=FORM_FULL, stream=None) -> int:
+    """kvs_prefill_chunk: append a [B, H_kv, n, d] chunk at row L of every head and merge
+    back to `budget`; returns the new length of every head."""
+    n = 0 if k_chunk is None else int(k_chunk.shape[2])
+    out = _i32(0)
+    _check(_lib.kvs_prefill_chunk(ctypes.byref(desc), _ptr(K), _ptr(V), _ptr(logn), _ptr(lens),
+                                  int(L), _ptr(k_chunk), _ptr(v_chunk), n, _ptr(Q_win), int(W),
+                                  int(budget), int(sink), int(form), ctypes.byref(out), _ptr(ws),
+                                  ws.numel(), _stream(stream)),
+           "kvs_prefill_chunk")
+    return int(out.value)

@@ -49,6 +49,8 @@ def parse_args():
     ap.add_argument("--workload", type=int, default=2)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prefill", action="store_true",
+                    help="time chunked streaming prefill compression instead (own JSON line)")
     return ap.parse_args()
 
 
@@ -427,11 +429,101 @@ def peaks():
     return 6650.0, "fallback"
 
 
+PREFILL = dict(layers=32, T=131072, chunk=512, budget=2048, sink=32, W=32)
+
+
+def prefill_main(args, rank, world, local):
+    """Chunked streaming prefill compression (the pages' serving setting: budget 2048,
+    chunk 512, 32 preserved initial tokens) of a 128K prompt in every layer of the
+    Llama-3.1-8B-shaped model: per layer and chunk one kvs_prefill_chunk call (append
+    the chunk, merge back to the budget). One step = every layer's whole prompt; the
+    calls of a step are captured once into a CUDA graph and replayed."""
+    from asymmetric_kv_merging_b200 import kvs
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    c = PREFILL
+    w = inputs.small_workload(inputs.workload(2), layers=c["layers"], T=c["T"], n_decode=0)
+    ends = [min(w.T, e + c["chunk"]) for e in range(0, w.T, c["chunk"])]
+    T_cap = c["budget"] + c["chunk"]
+    B, H, d = w.B, w.H_kv, w.d
+    desc = kvs.make_desc(B, H, w.H_q, d, T_cap, torch.bfloat16)
+    ws = torch.zeros(kvs.workspace_size(desc, c["W"], kvs.OP_PREFILL), dtype=torch.uint8,
+                     device=dev)
+    layers = []
+    for layer in range(w.layers):
+        li = inputs.make_layer(w, layer + 1000 * rank, device=dev, window_ends=ends)
+        chunks = [(li.K[:, :, e0:e1].contiguous(), li.V[:, :, e0:e1].contiguous(),
+                   li.extra["Q_ends"][i].contiguous())
+                  for i, (e0, e1) in enumerate(zip(range(0, w.T, c["chunk"]), ends))]
+        cache = dict(K=torch.zeros(B, H, T_cap, d, dtype=torch.bfloat16, device=dev),
+                     V=torch.zeros(B, H, T_cap, d, dtype=torch.bfloat16, device=dev),
+                     logn=torch.zeros(B, H, T_cap, device=dev),
+                     lens=torch.zeros(B * H, dtype=torch.int32, device=dev))
+        layers.append((chunks, cache))
+        del li
+    stream = torch.cuda.Stream(device=dev)
+
+    def step():
+        for chunks, cache in layers:
+            cache["lens"].zero_()
+            L = 0
+            for kc, vc, qw in chunks:
+                L = kvs.prefill_chunk(desc, cache["K"], cache["V"], cache["logn"], cache["lens"], L,
+                                      kc, vc, qw, c["W"], c["budget"], c["sink"], ws)
+            assert L == c["budget"]
+
+    with torch.cuda.stream(stream):
+        step()                                   # eager pass: kernel attributes, first loads
+    torch.cuda.synchronize()
+    launches0 = kvs.launch_count()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        step()
+    launches_per_step = kvs.launch_count() - launches0
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        graph.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+    flags = kvs.device_flags(ws)
+    tokens = B * w.layers * w.T * world
+    if rank == 0:
+        print(json.dumps({
+            "metric": "chunked prefill compression: prompt tokens/s", "value": tokens / (ms / 1e3),
+            "unit": "prompt tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "llama8b_32L_prefill128K", "B": B, "layers": w.layers,
+                       "T": w.T, "H_kv": H, "H_q": w.H_q, "d": d, "budget": c["budget"],
+                       "chunk": c["chunk"], "sink": c["sink"], "window": c["W"],
+                       "calls_per_step": len(ends) * w.layers,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+            "us_per_chunk": ms * 1e3 / (len(ends) * w.layers),
+            "gpu_launches": launches_per_step * args.steps, "device_flags": flags,
+            "clocks": clk}))
+
+
 def main():
     args = parse_args()
     rank, world, local = dist_setup(args.gpus)
     if args.impl == "reference":
         reference_main(args, rank, world)
+        return
+    if args.prefill:
+        if not torch.cuda.is_available():
+            raise SystemExit("bench.py needs a CUDA device (the kernels have no CPU path)")
+        prefill_main(args, rank, world, local)
         return
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device (the kernels have no CPU path)")

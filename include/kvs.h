@@ -70,7 +70,7 @@ typedef struct {
 
 typedef struct CUstream_st* kvs_stream_t; /* a cudaStream_t; NULL = legacy default stream */
 
-enum { KVS_OP_SCORE = 0, KVS_OP_MERGE = 1, KVS_OP_DECODE = 2 };
+enum { KVS_OP_SCORE = 0, KVS_OP_MERGE = 1, KVS_OP_DECODE = 2, KVS_OP_PREFILL = 3 };
 enum { KVS_SCOPE_HEAD = 0, KVS_SCOPE_POOLED = 1 };
 /* Scoring form: the coupled forward-only objective, or its diagonal-only ablation. */
 enum { KVS_FORM_FULL = 0, KVS_FORM_DIAGONAL = 1 };
@@ -178,6 +178,40 @@ kvs_status kvs_merge_compact(const kvs_cache_desc* desc, const void* K, const vo
                              uint8_t* dbg_selected, int32_t* dbg_out_offset,
                              float* dbg_kmerged_f32, void* ws, size_t ws_bytes,
                              kvs_stream_t stream);
+
+/*
+ * kvs_prefill_chunk -- one step of chunked streaming prefill compression: append a
+ * prompt chunk to every head, then merge in place back to the budget.
+ *
+ * The serving loop of §实验设置 (compression context budget 2048, chunk size 512, 32
+ * preserved initial tokens): the prompt enters the cache one chunk at a time, and
+ * after each chunk every head is merged back to `budget` rows. Reading of the pages
+ * (they give only the three numbers): the rounds are kvs_score_pairs +
+ * kvs_merge_compact rounds with candidate span [sink, len - W) (the first `sink` rows
+ * and the newest W rows are never merged), per-head scope, target = budget, window
+ * queries Q_win = the queries of the chunk's last W positions; rounds repeat while
+ * len > budget, each merging R = min(P, len - budget) pairs.
+ *
+ * Every head must hold L rows on entry (all heads equal; the caller tracks L, e.g. 0
+ * for an empty cache, then each call's *L_out). A head whose len differs is left
+ * unchanged and sets KVS_FLAG_BAD_LENGTH.
+ * In:  K, V [B,H_kv,T_cap,d] (updated in place); logn [B,H_kv,T_cap] (required: merged
+ *      counts); len [B*H_kv]; k_chunk, v_chunk [B,H_kv,n,d] (cache dtype, nullable
+ *      when n = 0); Q_win [B,H_q,W,d]; 1 <= W, G*W <= 128; sink >= 0; form as
+ *      kvs_score_pairs_form.
+ * Out: the cache advanced; *L_out (host) = the length of every head afterwards:
+ *      min(L + n, budget) when budget is reachable.
+ * Errors (nothing launched): KVS_ERR_INVALID_ARG (L + n > T_cap, bad pointers or
+ * alignment), KVS_ERR_UNSUPPORTED (L + n - sink > 8192: the in-place rounds rewrite at
+ * most 8192 rows of a head; or G*W > 128), KVS_ERR_BUDGET (budget below what the
+ * protected rows allow), KVS_ERR_ALIAS, KVS_ERR_WORKSPACE.
+ * Workspace: kvs_workspace_size(desc, W, KVS_OP_PREFILL) bytes, zeroed once.
+ */
+kvs_status kvs_prefill_chunk(const kvs_cache_desc* desc, void* K, void* V, float* logn,
+                             int32_t* len, int32_t L, const void* k_chunk, const void* v_chunk,
+                             int32_t n, const void* Q_win, int32_t W, int32_t budget,
+                             int32_t sink, int32_t form, int32_t* L_out, void* ws,
+                             size_t ws_bytes, kvs_stream_t stream);
 
 /*
  * kvs_decode_attn -- one decode step of GQA attention over the merged cache

@@ -130,3 +130,31 @@ def test_decode_host_validation(kvs):
     assert call(kn=_fake(7)) == 1                               # k_new without v_new
     assert call(out=_fake(2)) == 5                              # output over K
     assert call(ws_bytes=100) == 4
+
+
+def _prefill(kvs, desc, **over):
+    args = dict(K=_fake(1), V=_fake(2), logn=_fake(9), len=_fake(3), L=0, kc=_fake(10),
+                vc=_fake(11), n=512, Q=_fake(5), W=32, budget=2048, sink=32, form=0,
+                ws=_fake(8), ws_bytes=1 << 40)
+    args.update(over)
+    out = ctypes.c_int32(-1)
+    st = kvs._lib.kvs_prefill_chunk(ctypes.byref(desc), args["K"], args["V"], args["logn"],
+                                    args["len"], args["L"], args["kc"], args["vc"], args["n"],
+                                    args["Q"], args["W"], args["budget"], args["sink"],
+                                    args["form"], ctypes.byref(out), args["ws"],
+                                    args["ws_bytes"], None)
+    return st, out.value
+
+
+def test_prefill_chunk_host_validation_and_plan(kvs):
+    d = kvs.make_desc(1, 8, 32, 128, 4096, kvs.BF16)
+    assert _prefill(kvs, d, logn=None)[0] == 1                         # counts are required
+    assert _prefill(kvs, d, form=2)[0] == 1
+    assert _prefill(kvs, d, L=3800, n=512)[0] == 1                     # L + n > T_cap
+    assert _prefill(kvs, d, W=33)[0] == 2                              # G*W > 128
+    big = kvs.make_desc(1, 8, 32, 128, 16384, kvs.BF16)
+    assert _prefill(kvs, big, L=8000, n=512)[0] == 2                   # in-place span > 8192
+    # budget below what the protected rows allow: refused before anything is launched
+    assert _prefill(kvs, d, L=2048, n=512, budget=40)[0] == 3
+    assert _prefill(kvs, d, ws_bytes=16)[0] == 4
+    assert kvs.workspace_size(d, 32, kvs.OP_PREFILL) > kvs.workspace_size(d, 32, kvs.OP_SCORE)

@@ -227,13 +227,20 @@ kvs_status kvs_prefill_chunk(const kvs_cache_desc* desc, void* K, void* V, float
   if ((long long)L + n - sink > kInplaceMaxSpan) return KVS_ERR_UNSUPPORTED;
   const size_t heads = (size_t)desc->B * desc->H_kv;
   const size_t chunk_bytes = heads * (size_t)n * desc->d * elem_bytes(desc);
-  Range rk{(const char*)K, cache_bytes(desc, desc->T_cap)}, rv{(const char*)V, cache_bytes(desc, desc->T_cap)};
-  Range rkc{(const char*)k_chunk, chunk_bytes}, rvc{(const char*)v_chunk, chunk_bytes};
-  Range rl{(const char*)logn, heads * desc->T_cap * sizeof(float)}, rn{(const char*)len, heads * sizeof(int32_t)};
-  const Range all[] = {rk, rv, rl, rn, rkc, rvc};
-  for (int i = 0; i < 6; ++i)
-    for (int j = i + 1; j < 6; ++j)
-      if (overlap(all[i], all[j])) return KVS_ERR_ALIAS;
+  // the cache (written) must not overlap itself or the chunk and window (read);
+  // inputs may share memory with each other
+  const Range outs[] = {{(const char*)K, cache_bytes(desc, desc->T_cap)},
+                        {(const char*)V, cache_bytes(desc, desc->T_cap)},
+                        {(const char*)logn, heads * desc->T_cap * sizeof(float)},
+                        {(const char*)len, heads * sizeof(int32_t)}};
+  const Range ins[] = {{(const char*)k_chunk, chunk_bytes}, {(const char*)v_chunk, chunk_bytes},
+                       {(const char*)Q_win, (size_t)desc->B * desc->H_q * W * desc->d * elem_bytes(desc)}};
+  for (int i = 0; i < 4; ++i) {
+    for (int j = i + 1; j < 4; ++j)
+      if (overlap(outs[i], outs[j])) return KVS_ERR_ALIAS;
+    for (int j = 0; j < 3; ++j)
+      if (overlap(outs[i], ins[j])) return KVS_ERR_ALIAS;
+  }
   // plan the rounds on the host (every head has length L): R = min(P, len - budget)
   int rounds = 0, Lc = L + n;
   while (Lc > budget) {

@@ -158,3 +158,12 @@ def test_prefill_chunk_host_validation_and_plan(kvs):
     assert _prefill(kvs, d, L=2048, n=512, budget=40)[0] == 3
     assert _prefill(kvs, d, ws_bytes=16)[0] == 4
     assert kvs.workspace_size(d, 32, kvs.OP_PREFILL) > kvs.workspace_size(d, 32, kvs.OP_SCORE)
+
+
+def test_prefill_chunk_alias_rules(kvs):
+    d = kvs.make_desc(1, 8, 32, 128, 4096, kvs.BF16)
+    same = _fake(10)
+    # k and v chunks may be one buffer (both are read); the cache may not overlap them
+    assert _prefill(kvs, d, kc=same, vc=same, L=2048, n=512, budget=40)[0] == 3
+    assert _prefill(kvs, d, kc=_fake(1))[0] == 5
+    assert _prefill(kvs, d, logn=_fake(2))[0] == 5

@@ -15,17 +15,19 @@
 //   the protected prefix and suffix; a block-level ballot scan gives each pair's
 //   output row; rows move as 16-byte vectors, merged rows are computed in fp32.
 // merge_inplace_kernel: one CTA per head walks the span in order, staging each
-//   chunk in shared memory before writing it to lower (or equal) rows.
+//   chunk in shared memory (double-buffered, the next chunk's copies in flight)
+//   before writing it to lower (or equal) rows.
 #include "kvs_common.cuh"
 #include "kvs_kernels.h"
+#include "ptx.cuh"
 
 namespace kvs {
 
 constexpr int kSelThreads = 1024;
 constexpr int kMergeThreads = 256;
 constexpr int kCopyRows = 256;
-// Pairs staged per in-place step: 32 for rows up to 256 bytes, 16 for 512-byte rows,
-// so the staging buffers stay within the default 48 KB of shared memory.
+// Pairs staged per in-place step: 32 for rows up to 256 bytes, 16 for 512-byte rows
+// (one warp plans a step; two 32 KB stages of K and V rows).
 template <typename T, int D>
 constexpr int inplace_chunk() { return D * (int)sizeof(T) <= 256 ? 32 : 16; }
 
@@ -475,6 +477,24 @@ merge_kernel(const T* __restrict__ K, const T* __restrict__ V, const float* __re
 // In-place variant: one CTA per head; each chunk is read completely into shared
 // memory before any of its rows is written, and rows only move to lower indices,
 // so no unread row is ever overwritten.
+// 16- and 4-byte asynchronous global -> shared copies (cp.async), completed per thread
+// by commit / wait groups.
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* smem, const void* gmem) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem)), "l"(gmem)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+// In-place merge of one head per CTA. Items are the pair chunks of the span (CH pairs,
+// 2 CH rows), then the suffix chunks (2 CH rows). Every output row lies at or below its
+// input row, so no item writes a row that a later item still has to read: the rows of
+// item k + 1 are copied into the other shared-memory stage while item k is written back,
+// and the planning warp loads the scores of chunk k + 1 while it plans chunk k.
 template <typename T, int D>
 __global__ void __launch_bounds__(kMergeThreads)
 merge_inplace_kernel(T* __restrict__ K, T* __restrict__ V, float* __restrict__ logn,
@@ -484,12 +504,13 @@ merge_inplace_kernel(T* __restrict__ K, T* __restrict__ V, float* __restrict__ l
                      uint8_t* __restrict__ dbg_sel, int32_t* __restrict__ dbg_off,
                      float* __restrict__ dbg_km, int32_t* __restrict__ flags) {
   constexpr int CH = inplace_chunk<T, D>();
+  constexpr int SROWS = 2 * CH;                                // rows per stage
   constexpr int VPR = D * (int)sizeof(T) / 16;
   constexpr int VN = Vec16<T>::n;
   extern __shared__ __align__(16) unsigned char ism[];
-  uint4* sK = reinterpret_cast<uint4*>(ism);                 // [2*CH][VPR]
-  uint4* sV = sK + 2 * CH * VPR;                             // [2*CH][VPR]
-  float* sL = reinterpret_cast<float*>(sV + 2 * CH * VPR);   // [2*CH]
+  uint4* sK = reinterpret_cast<uint4*>(ism);                   // [2][SROWS][VPR]
+  uint4* sV = sK + 2 * SROWS * VPR;                            // [2][SROWS][VPR]
+  float* sL = reinterpret_cast<float*>(sV + 2 * SROWS * VPR);  // [2][SROWS]
   __shared__ int s_off[32];
   __shared__ unsigned char s_sel[32];
   __shared__ float s_w[32];
@@ -512,15 +533,51 @@ merge_inplace_kernel(T* __restrict__ K, T* __restrict__ V, float* __restrict__ l
   const float* wb = w_b + (size_t)head * (T_cap / 2);
   const int tid = threadIdx.x, lane = tid & 31;
   if (tid == 0) { s_lt = 0; s_eq = hi.eq0; }
-  __syncthreads();
 
   if (R > 0) {
-    for (int pb = 0; pb < P; pb += CH) {
-      const int np = min(CH, P - pb);
-      if (tid < 32) {   // one warp plans the chunk (CH <= 32)
+    const int n_pc = (P + CH - 1) / CH;                        // pair chunks
+    const int s_begin = c0 + 2 * P;                            // suffix rows move down by R
+    const int n_sc = (L - s_begin + SROWS - 1) / SROWS;
+    const int n_items = n_pc + n_sc;
+    auto item_row0 = [&](int k) { return k < n_pc ? c0 + 2 * CH * k : s_begin + SROWS * (k - n_pc); };
+    auto item_rows = [&](int k) {
+      return k < n_pc ? 2 * min(CH, P - CH * k) : min(SROWS, L - (s_begin + SROWS * (k - n_pc)));
+    };
+    auto load_stage = [&](int b, int k) {
+      const int r0 = item_row0(k), nr = item_rows(k);
+      uint4* dk = sK + b * SROWS * VPR;
+      uint4* dv = sV + b * SROWS * VPR;
+      float* dl = sL + b * SROWS;
+      for (int i = tid; i < nr * VPR; i += blockDim.x) {
+        const int r = i / VPR, c = i - r * VPR;
+        cp_async16(dk + i, Kh + (size_t)(r0 + r) * D + c * VN);
+        cp_async16(dv + i, Vh + (size_t)(r0 + r) * D + c * VN);
+      }
+      for (int r = tid; r < nr; r += blockDim.x) cp_async4(dl + r, lnh + r0 + r);
+    };
+    load_stage(0, 0);
+    cp_async_commit();
+    // the planning warp's scores and weights of the current pair chunk
+    float sc_cur = 0.f, w_cur = 0.f;
+    if (tid < 32 && lane < min(CH, P)) {
+      sc_cur = sc[lane];
+      w_cur = wb[lane];
+    }
+    __syncthreads();                                           // s_lt / s_eq initialised
+    for (int k = 0; k < n_items; ++k) {
+      const int b = k & 1;
+      if (k + 1 < n_items) load_stage(b ^ 1, k + 1);
+      cp_async_commit();                                       // (empty on the last item)
+      if (k < n_pc && tid < 32) {                              // one warp plans the chunk
+        const int pb = CH * k, np = min(CH, P - pb);
+        float sc_next = 0.f, w_next = 0.f;
+        if (k + 1 < n_pc && lane < min(CH, P - pb - CH)) {
+          sc_next = sc[pb + CH + lane];
+          w_next = wb[pb + CH + lane];
+        }
         const int p = pb + lane;
         const bool in = lane < np;
-        const uint32_t key = in ? score_key(sc[p]) : 0xffffffffu;
+        const uint32_t key = in ? score_key(sc_cur) : 0xffffffffu;
         const bool lt = in && key < su.thr_key;
         const bool eq = in && key == su.thr_key;
         const unsigned blt = __ballot_sync(0xffffffffu, lt);
@@ -533,76 +590,68 @@ merge_inplace_kernel(T* __restrict__ K, T* __restrict__ V, float* __restrict__ l
         const int off = c0 + 2 * p - sel_before;
         s_off[lane] = off;
         s_sel[lane] = sl ? 1 : 0;
-        s_w[lane] = in ? wb[p] : 0.f;
+        s_w[lane] = in ? w_cur : 0.f;
         if (in) {
           if (dbg_sel) dbg_sel[(size_t)head * (T_cap / 2) + p] = sl ? 1 : 0;
           if (dbg_off) dbg_off[(size_t)head * (T_cap / 2) + p] = off;
         }
         __syncwarp();
         if (lane == 0) { s_lt += __popc(blt); s_eq += __popc(beq); }
+        sc_cur = sc_next;
+        w_cur = w_next;
       }
-      const int row0 = c0 + 2 * pb;
-      for (int i = tid; i < 2 * np * VPR; i += blockDim.x) {
-        const int r = i / VPR, c = i - r * VPR;
-        sK[i] = *reinterpret_cast<const uint4*>(Kh + (size_t)(row0 + r) * D + c * VN);
-        sV[i] = *reinterpret_cast<const uint4*>(Vh + (size_t)(row0 + r) * D + c * VN);
-      }
-      for (int r = tid; r < 2 * np; r += blockDim.x) sL[r] = lnh[row0 + r];
-      __syncthreads();
-      for (int i = tid; i < np * VPR; i += blockDim.x) {
-        const int t = i / VPR, c = i - t * VPR;
-        const int off = s_off[t];
-        const uint4 ka_r = sK[(2 * t) * VPR + c], kb_r = sK[(2 * t + 1) * VPR + c];
-        const uint4 va_r = sV[(2 * t) * VPR + c], vb_r = sV[(2 * t + 1) * VPR + c];
-        if (s_sel[t]) {
-          float ka[VN], kb[VN], va[VN], vb[VN], ko[VN], vo[VN];
-          load_vec(reinterpret_cast<const T*>(&ka_r), ka);
-          load_vec(reinterpret_cast<const T*>(&kb_r), kb);
-          load_vec(reinterpret_cast<const T*>(&va_r), va);
-          load_vec(reinterpret_cast<const T*>(&vb_r), vb);
-          const float w = s_w[t];
-          const float na = expf(sL[2 * t]), nb = expf(sL[2 * t + 1]);
-          const float inv = 1.f / (na + nb);
+      cp_async_wait1();                                        // this thread's copies of item k landed
+      __syncthreads();                                         // everyone's, and the plan
+      const uint4* cK = sK + b * SROWS * VPR;
+      const uint4* cV = sV + b * SROWS * VPR;
+      const float* cL = sL + b * SROWS;
+      if (k < n_pc) {
+        const int pb = CH * k, np = min(CH, P - pb);
+        for (int i = tid; i < np * VPR; i += blockDim.x) {
+          const int t = i / VPR, c = i - t * VPR;
+          const int off = s_off[t];
+          const uint4 ka_r = cK[(2 * t) * VPR + c], kb_r = cK[(2 * t + 1) * VPR + c];
+          const uint4 va_r = cV[(2 * t) * VPR + c], vb_r = cV[(2 * t + 1) * VPR + c];
+          if (s_sel[t]) {
+            float ka[VN], kb[VN], va[VN], vb[VN], ko[VN], vo[VN];
+            load_vec(reinterpret_cast<const T*>(&ka_r), ka);
+            load_vec(reinterpret_cast<const T*>(&kb_r), kb);
+            load_vec(reinterpret_cast<const T*>(&va_r), va);
+            load_vec(reinterpret_cast<const T*>(&vb_r), vb);
+            const float w = s_w[t];
+            const float na = expf(cL[2 * t]), nb = expf(cL[2 * t + 1]);
+            const float inv = 1.f / (na + nb);
 #pragma unroll
-          for (int e = 0; e < VN; ++e) {
-            ko[e] = fmaf(w, kb[e] - ka[e], ka[e]);
-            vo[e] = (na * va[e] + nb * vb[e]) * inv;
-          }
-          store_vec(Kh + (size_t)off * D + c * VN, ko);
-          store_vec(Vh + (size_t)off * D + c * VN, vo);
-          if (c == 0) lnh[off] = logf(na + nb);
-          if (dbg_km) {
-            float* dk = dbg_km + ((size_t)head * (T_cap / 2) + pb + t) * D + c * VN;
+            for (int e = 0; e < VN; ++e) {
+              ko[e] = fmaf(w, kb[e] - ka[e], ka[e]);
+              vo[e] = (na * va[e] + nb * vb[e]) * inv;
+            }
+            store_vec(Kh + (size_t)off * D + c * VN, ko);
+            store_vec(Vh + (size_t)off * D + c * VN, vo);
+            if (c == 0) lnh[off] = logf(na + nb);
+            if (dbg_km) {
+              float* dk = dbg_km + ((size_t)head * (T_cap / 2) + pb + t) * D + c * VN;
 #pragma unroll
-            for (int e = 0; e < VN; e += 4) *reinterpret_cast<float4*>(dk + e) = make_float4(ko[e], ko[e + 1], ko[e + 2], ko[e + 3]);
+              for (int e = 0; e < VN; e += 4) *reinterpret_cast<float4*>(dk + e) = make_float4(ko[e], ko[e + 1], ko[e + 2], ko[e + 3]);
+            }
+          } else {
+            *reinterpret_cast<uint4*>(Kh + (size_t)off * D + c * VN) = ka_r;
+            *reinterpret_cast<uint4*>(Kh + (size_t)(off + 1) * D + c * VN) = kb_r;
+            *reinterpret_cast<uint4*>(Vh + (size_t)off * D + c * VN) = va_r;
+            *reinterpret_cast<uint4*>(Vh + (size_t)(off + 1) * D + c * VN) = vb_r;
+            if (c == 0) { lnh[off] = cL[2 * t]; lnh[off + 1] = cL[2 * t + 1]; }
           }
-        } else {
-          *reinterpret_cast<uint4*>(Kh + (size_t)off * D + c * VN) = ka_r;
-          *reinterpret_cast<uint4*>(Kh + (size_t)(off + 1) * D + c * VN) = kb_r;
-          *reinterpret_cast<uint4*>(Vh + (size_t)off * D + c * VN) = va_r;
-          *reinterpret_cast<uint4*>(Vh + (size_t)(off + 1) * D + c * VN) = vb_r;
-          if (c == 0) { lnh[off] = sL[2 * t]; lnh[off + 1] = sL[2 * t + 1]; }
         }
+      } else {
+        const int s0 = item_row0(k), nr = item_rows(k);
+        for (int i = tid; i < nr * VPR; i += blockDim.x) {
+          const int r = i / VPR, c = i - r * VPR;
+          *reinterpret_cast<uint4*>(Kh + (size_t)(s0 + r - R) * D + c * VN) = cK[i];
+          *reinterpret_cast<uint4*>(Vh + (size_t)(s0 + r - R) * D + c * VN) = cV[i];
+        }
+        for (int r = tid; r < nr; r += blockDim.x) lnh[s0 + r - R] = cL[r];
       }
-      __syncthreads();
-    }
-    // suffix rows move down by R, chunk by chunk in increasing order
-    for (int s0 = c0 + 2 * P; s0 < L; s0 += 2 * CH) {
-      const int nr = min(2 * CH, L - s0);
-      for (int i = tid; i < nr * VPR; i += blockDim.x) {
-        const int r = i / VPR, c = i - r * VPR;
-        sK[i] = *reinterpret_cast<const uint4*>(Kh + (size_t)(s0 + r) * D + c * VN);
-        sV[i] = *reinterpret_cast<const uint4*>(Vh + (size_t)(s0 + r) * D + c * VN);
-      }
-      for (int r = tid; r < nr; r += blockDim.x) sL[r] = lnh[s0 + r];
-      __syncthreads();
-      for (int i = tid; i < nr * VPR; i += blockDim.x) {
-        const int r = i / VPR, c = i - r * VPR;
-        *reinterpret_cast<uint4*>(Kh + (size_t)(s0 + r - R) * D + c * VN) = sK[i];
-        *reinterpret_cast<uint4*>(Vh + (size_t)(s0 + r - R) * D + c * VN) = sV[i];
-      }
-      for (int r = tid; r < nr; r += blockDim.x) lnh[s0 + r - R] = sL[r];
-      __syncthreads();
+      __syncthreads();                                         // stage b and the plan are free
     }
   } else if (dbg_sel || dbg_off) {
     for (int p = tid; p < P; p += blockDim.x) {
@@ -641,9 +690,17 @@ static cudaError_t launch_merge_t(const kvs_cache_desc& d, const void* K, const 
   if (inplace) {
     constexpr int VPR = D * (int)sizeof(T) / 16;
     constexpr int CH = inplace_chunk<T, D>();
-    constexpr size_t smem = (size_t)2 * (2 * CH * VPR) * 16 + 2 * CH * sizeof(float);
-    static_assert(smem + 512 <= 48 * 1024, "in-place staging must fit the default shared-memory limit");
+    // two stages of K, V (2 CH rows each) and log-counts
+    constexpr size_t smem = (size_t)2 * 2 * (2 * CH * VPR) * 16 + 2 * 2 * CH * sizeof(float);
+    static_assert(smem <= 100 * 1024, "in-place staging");
     auto kfn = merge_inplace_kernel<T, D>;
+    static bool attr = false;   // set once per process, before any capture
+    if (!attr) {
+      if (cudaFuncSetAttribute((const void*)kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)smem) != cudaSuccess)
+        return cudaErrorInvalidValue;
+      attr = true;
+    }
     kfn<<<heads, kMergeThreads, smem, st>>>((T*)K_out, (T*)V_out, logn_out, score, w_b, scope,
                                             d.H_kv, d.T_cap, sel, hinfo, len_out, dbg_sel,
                                             dbg_off, dbg_km, flags);

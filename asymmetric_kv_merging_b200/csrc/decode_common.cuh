@@ -309,16 +309,19 @@ __device__ __forceinline__ int slice_owner(int n, int col, int C) {
 // own inbox, and the CTA of rank 0 appends the new row. Nothing is read remotely, so
 // a CTA may leave as soon as its slice is written.
 //
+// kn, vn: the appended row of this head (nullable when !append); the caller stages it
+// in shared memory at kernel start, so the combine waits on no global load.
 // `dry`: run the same instructions with every store aimed at this CTA's scratch
 // (`inbox` and `out` point there, head is 0) and without barriers or the append,
-// from a single warp while the other warps stream. A kernel launch starts with cold
+// from a single warp while the other warps stream (its loads of the warp partials see
+// stage data in flight; the values are discarded). A kernel launch starts with cold
 // instruction caches; the dry run pulls this code in before the real combine needs it.
 template <typename T, int D, int G, int NW>
 __device__ __noinline__ void cluster_combine(
     float (*sm)[G], float (*sl)[G], float (*sacc)[G][D], float (*qs)[D], float* s_cml,
     float* s_new, ClusterInbox<D, G>* inbox, int C, int rank, int tid, int nthreads, bool dry,
     int head, int L, int T_cap, bool append, T* K, T* V, float* logn, int32_t* len,
-    const T* k_new, const T* v_new, T* out, int32_t* flags) {
+    const T* kn, const T* vn, T* out, int32_t* flags) {
   constexpr int N = G * D;
   const int lane = tid & 31, warp = tid >> 5, nwarps = nthreads / 32;
   const bool fits = L < T_cap;
@@ -338,7 +341,7 @@ __device__ __noinline__ void cluster_combine(
     s_cml[2 * g + 1] = Ls;
   }
   if (attend_new) appended_logits<T, D, G, NW>(DecodeSmem<D, G, NW>{sm, sl, sacc, qs, s_new, nullptr, nullptr, nullptr},
-                                               k_new + (size_t)head * D, warp, lane, nwarps);
+                                               kn, warp, lane, nwarps);
   if (!dry) __syncthreads();
   const uint32_t in_acc = smem_u32(inbox->acc), in_ml = smem_u32(&inbox->ml[0][0][0]);
   // push (m, l) of every query head to every CTA: ml[rank][g] in CTA j
@@ -383,15 +386,13 @@ __device__ __noinline__ void cluster_combine(
       if (attend_new) {
         const float f = exp2f(sn - M);
         Ls += f;
-        A = fmaf(to_f32(v_new[(size_t)head * D + c]), f, A);
+        A = fmaf(to_f32(vn[c]), f, A);
       }
     }
     store_out<T>(out + ((size_t)head * G + g) * D + c, Ls > 0.f ? A / Ls : 0.f);
   }
   if (!dry && rank == 0 && append) {
     if (fits) {
-      const T* kn = k_new + (size_t)head * D;
-      const T* vn = v_new + (size_t)head * D;
       for (int c = tid; c < D; c += nthreads) {
         K[((size_t)head * T_cap + L) * D + c] = kn[c];
         V[((size_t)head * T_cap + L) * D + c] = vn[c];

@@ -84,9 +84,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
   __shared__ float s_gstat[G][2];
   __shared__ float s_cml[G][2];
   __shared__ int s_last;
-  // cluster shape: the inbox peers push into, and the scratch of the warm-up run
+  // cluster shape: the inbox peers push into, the scratch of the warm-up run, and the
+  // appended row (k, v) staged at kernel start
   using Inbox = std::conditional_t<kCluster, ClusterInbox<D, G>, char>;
   __shared__ Inbox s_inbox[2];
+  __shared__ __align__(16) bf16 s_kvnew[kCluster ? 2 : 1][kCluster ? D : 8];
   // after the main loop the stage buffers hold the consumer warps' partial outputs
   float(*s_acc)[G][D] = reinterpret_cast<float(*)[G][D]>(base);
 
@@ -116,6 +118,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     const int g = i / D, c = i - g * D;
     qs[g][c] = to_f32(q[((size_t)head * G + g) * D + c]) * qscale;
   }
+  const bool append = k_new != nullptr && v_new != nullptr && !bad;
+  if (kCluster && append) {
+    // element loads: the API does not require these rows to be 16-byte aligned
+    for (int i = tid; i < 2 * D; i += kThreads)
+      s_kvnew[i / D][i % D] = (i < D ? k_new : v_new)[(size_t)head * D + i % D];
+  }
   if (tid == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
@@ -139,8 +147,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     if constexpr (kCluster)
       cluster_combine<bf16, D, G, NC>(s_m, s_l, s_acc, qs, &s_cml[0][0], s_new, &s_inbox[1], nsplit,
                                       (int)cluster_ctarank(), lane, 32, /*dry=*/true, 0, L, T_cap,
-                                      k_new != nullptr && v_new != nullptr && !bad, K, V, logn, len,
-                                      k_new, v_new, reinterpret_cast<bf16*>(&s_inbox[1]), flags);
+                                      append, K, V, logn, len, s_kvnew[0], s_kvnew[1 % (kCluster ? 2 : 1)],
+                                      reinterpret_cast<bf16*>(&s_inbox[1]), flags);
   } else if (warp == NC) {
     // ---------------- producer: one thread issues every TMA load ----------------
     if (lane == 0) {
@@ -310,8 +318,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
   if constexpr (kCluster) {
     cluster_combine<bf16, D, G, NC>(s_m, s_l, s_acc, qs, &s_cml[0][0], s_new, &s_inbox[0], nsplit,
                                     (int)cluster_ctarank(), tid, kThreads, /*dry=*/false, head, L,
-                                    T_cap, k_new != nullptr && v_new != nullptr && !bad, K, V, logn,
-                                    len, k_new, v_new, out, flags);
+                                    T_cap, append, K, V, logn, len, s_kvnew[0],
+                                    s_kvnew[1 % (kCluster ? 2 : 1)], out, flags);
   } else {
     decode_epilogue_staged<bf16, D, G, NC>(Sm, base, S::kRingBytes, cbar, a, tid, kThreads);
   }

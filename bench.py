@@ -412,12 +412,24 @@ def reference_main(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+L2_BYTES = 126 * 1024 * 1024
+
+
 def config_of(w, n_gpus):
+    kv = 2 * w.layers * w.B * w.H_kv * w.T * w.d * w.elem_bytes
+    dec = 2 * w.B * w.H_kv * (w.T // w.ratio) * w.d * w.elem_bytes
+    l2 = (f"inputs larger than L2 ({kv / 2**30:.2f} GiB of K/V per replica; no flush needed)"
+          if kv > L2_BYTES else f"inputs of {kv / 2**20:.1f} MiB fit in L2")
+    if dec <= L2_BYTES and w.layers * dec > L2_BYTES:
+        l2 += ("; decode rotates over the layers' merged caches "
+               f"({w.layers} x {dec / 2**20:.1f} MiB), larger than L2 together")
+    elif dec <= L2_BYTES:
+        l2 += (f"; the merged decode cache ({dec / 2**20:.1f} MiB) fits in L2, so decode "
+               "steps may hit it")
     return {"workload": w.name, "B": w.B, "layers": w.layers, "T": w.T, "H_kv": w.H_kv,
             "H_q": w.H_q, "d": w.d, "ratio": w.ratio, "budget_per_head": w.T // w.ratio,
             "decode_steps_per_layer": w.n_decode, "window": w.W, "sink": w.sink,
-            "parallelism": f"replicas x{n_gpus}" if n_gpus > 1 else "single GPU",
-            "l2": "inputs larger than L2 (16 GiB of K/V per replica; no flush needed)"}
+            "parallelism": f"replicas x{n_gpus}" if n_gpus > 1 else "single GPU", "l2": l2}
 
 
 def peaks():
@@ -569,8 +581,12 @@ def main():
     traffic = None
     prof = os.path.join(ROOT, "profiles", "decode_traffic.json")
     if os.path.exists(prof):
+        # one ncu capture's DRAM bytes per launch, scaled by rows processed to this launch
+        # (the capture shows traffic equal to the algorithmic bytes, so it scales in proportion)
         with open(prof) as f:
-            traffic = json.load(f).get("dram_bytes_per_launch")
+            tr = json.load(f)
+        traffic = (tr["measured_dram_bytes_per_launch"] * rn.decode_bytes_per_launch()
+                   / tr["measured_algorithmic_bytes_per_launch"])
 
     e2e = None
     if not args.no_e2e:

@@ -147,7 +147,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     if constexpr (kCluster)
       cluster_combine<bf16, D, G, NC>(s_m, s_l, s_acc, qs, &s_cml[0][0], s_new, &s_inbox[1], nsplit,
                                       (int)cluster_ctarank(), lane, 32, /*dry=*/true, 0, L, T_cap,
-                                      append, K, V, logn, len, s_kvnew[0], s_kvnew[1 % (kCluster ? 2 : 1)],
+                                      append, K, V, logn, len, s_kvnew[0], s_kvnew[kCluster ? 1 : 0],
                                       reinterpret_cast<bf16*>(&s_inbox[1]), flags);
   } else if (warp == NC) {
     // ---------------- producer: one thread issues every TMA load ----------------
@@ -319,7 +319,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     cluster_combine<bf16, D, G, NC>(s_m, s_l, s_acc, qs, &s_cml[0][0], s_new, &s_inbox[0], nsplit,
                                     (int)cluster_ctarank(), tid, kThreads, /*dry=*/false, head, L,
                                     T_cap, append, K, V, logn, len, s_kvnew[0],
-                                    s_kvnew[1 % (kCluster ? 2 : 1)], out, flags);
+                                    s_kvnew[kCluster ? 1 : 0], out, flags);
   } else {
     decode_epilogue_staged<bf16, D, G, NC>(Sm, base, S::kRingBytes, cbar, a, tid, kThreads);
   }

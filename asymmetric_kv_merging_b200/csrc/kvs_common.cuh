@@ -147,8 +147,9 @@ constexpr int kMaxDecodeSplits = 64;      // the combine gives each lane two spl
 constexpr int kMaxClusterSize = 16;       // CTAs of one KV head in a cluster launch
 
 inline int decode_splits(const kvs_cache_desc& d) {
+  // as many splits as keep the grid to one wave of two CTAs per SM
   int units = d.B * d.H_kv;
-  int s = (kTargetCtas + units - 1) / units;
+  int s = kTargetCtas / units;
   int cap = d.T_cap / 128 > 1 ? d.T_cap / 128 : 1;
   if (s > cap) s = cap;
   if (s > kMaxDecodeSplits) s = kMaxDecodeSplits;

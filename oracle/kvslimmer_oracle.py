@@ -21,7 +21,10 @@ reason, in the design notes):
      window of W recent queries of the G query heads sharing a KV head, the
      oracle averages the attention of those G*W queries (alpha_bar) and uses
      o_bar = mean_q o_q = sum_t alpha_bar_t v_t in the single-query formulas.
-     For one query this is exactly the pages' expression.
+     For one query this is exactly the pages' expression. The alternative
+     (reading B, stats="per_query") averages the single-query norms over the
+     window queries instead; it too reduces to the pages' expression for one
+     query.
   R2 candidates: disjoint adjacent pairs (c0+2p, c0+2p+1) of the candidate
      span [c0, len - n_recent); an odd leftover token is never merged.
   R3 score: a pair's score is the minimum value of the forward-only second
@@ -46,6 +49,10 @@ reason, in the design notes):
      them; arithmetic inside a round stays fp64.
   R10 empty cache: decode attention over a head with no rows (and no appended
      row) returns the zero vector.
+  R11 chunked prefill: each prompt chunk is appended with count 1; while a
+     head is longer than the budget, a round runs with candidate span
+     [sink, len - W), the chunk's last W queries as the window and the budget
+     as the per-head target.
 """
 
 from __future__ import annotations
@@ -294,6 +301,37 @@ def window_statistics(Q_heads, K, V, log_n, length, W):
     return A.mean(axis=0), O.mean(axis=0)
 
 
+def pair_norms_per_query(A, O, V, a, b):
+    """Reading B of the window (the alternative to R1): the single-query norms of
+    [KVS] §数学主线四 taken per window query and averaged,
+
+        N11 = mean_q |a_qa (1 - 2 a_qa)| |v_a - o_q|,   N22 likewise,
+        N12 = mean_q a_qa a_qb |v_a + v_b - 2 o_q|,
+
+    from the window's attention rows A (Qv, len) and outputs O (Qv, d); a, b index the
+    pairs' rows. With one window query it is exactly pair_norms of that query."""
+    A = np.asarray(A, dtype=np.float64)
+    O = np.asarray(O, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    a = np.asarray(a)
+    b = np.asarray(b)
+    if A.shape[0] == 0:
+        z = np.zeros(a.shape)
+        return z, z.copy(), z.copy()
+    n11 = np.zeros(a.shape)
+    n12 = np.zeros(a.shape)
+    n22 = np.zeros(a.shape)
+    for q in range(A.shape[0]):
+        x11, x12, x22 = pair_norms(A[q, a], A[q, b], V[a], V[b], O[q])
+        n11 += x11
+        n12 += x12
+        n22 += x22
+    return n11 / A.shape[0], n12 / A.shape[0], n22 / A.shape[0]
+
+
+STATS = ("mean", "per_query")
+
+
 # ---------------------------------------------------------------------------
 # One KV head: candidates, scores, selection, merge and compaction
 # ---------------------------------------------------------------------------
@@ -316,15 +354,24 @@ class HeadScores:
     o_bar: np.ndarray
 
 
-def score_head(K, V, log_n, length, cand_begin, n_recent, Q_heads, W, form="full"):
-    """Score every candidate pair of one KV head (form: see weight_and_score)."""
+def score_head(K, V, log_n, length, cand_begin, n_recent, Q_heads, W, form="full",
+               stats="mean"):
+    """Score every candidate pair of one KV head (form: see weight_and_score; stats:
+    "mean" = reading R1, norms of the window-mean statistics; "per_query" = reading B,
+    see pair_norms_per_query)."""
+    if stats not in STATS:
+        raise ValueError(stats)
     K = np.asarray(K, dtype=np.float64)
     V = np.asarray(V, dtype=np.float64)
     alpha_bar, o_bar = window_statistics(Q_heads, K, V, log_n, length, W)
     P = num_pairs(length, cand_begin, n_recent)
     a = int(cand_begin) + 2 * np.arange(P)
     b = a + 1
-    n11, n12, n22 = pair_norms(alpha_bar[a], alpha_bar[b], V[a], V[b], o_bar)
+    if stats == "mean":
+        n11, n12, n22 = pair_norms(alpha_bar[a], alpha_bar[b], V[a], V[b], o_bar)
+    else:
+        A, O = window_attention(Q_heads, K, V, log_n, length, W)
+        n11, n12, n22 = pair_norms_per_query(A, O, V[:length], a, b)
     w_b, score, degen, D = weight_and_score(n11, n12, n22, K[a], K[b], form)
     return HeadScores(score=score, w_b=w_b, n11=n11, n12=n12, n22=n22, D=D,
                       degenerate=degen, alpha_bar=alpha_bar, o_bar=o_bar)
@@ -452,7 +499,7 @@ class RoundResult:
 
 
 def merge_round(cache, Q_win, W, cand_begin, n_recent, target, scope="head", storage="f64",
-                form="full"):
+                form="full", stats="mean"):
     """One scoring + selection + merge round over a whole cache.
 
     Q_win: (B, H_q, W, d); query head hq belongs to KV head hq // G.
@@ -465,7 +512,8 @@ def merge_round(cache, Q_win, W, cand_begin, n_recent, target, scope="head", sto
     G = Q_win.shape[1] // H
     cand_begin = np.asarray(cand_begin).reshape(B, H)
     scores = [[score_head(cache.K[b][h], cache.V[b][h], cache.log_n[b][h], cache.length(b, h),
-                          cand_begin[b, h], n_recent, Q_win[b, h * G:(h + 1) * G], W, form)
+                          cand_begin[b, h], n_recent, Q_win[b, h * G:(h + 1) * G], W, form,
+                          stats)
                for h in range(H)] for b in range(B)]
     selected = [[None] * H for _ in range(B)]
     if scope == "head":
@@ -501,7 +549,7 @@ def merge_round(cache, Q_win, W, cand_begin, n_recent, target, scope="head", sto
 
 
 def compress(cache, Q_win, W, cand_begin, n_recent, target, scope="head", max_rounds=64,
-             storage="f64", form="full"):
+             storage="f64", form="full", stats="mean"):
     """Repeat merge rounds until every unit reaches its budget exactly (reading R4)."""
     rounds = []
     for _ in range(max_rounds):
@@ -512,7 +560,8 @@ def compress(cache, Q_win, W, cand_begin, n_recent, target, scope="head", max_ro
             done = np.all(lens.sum(axis=1) == np.asarray(target).reshape(-1))
         if done:
             return cache, rounds
-        r = merge_round(cache, Q_win, W, cand_begin, n_recent, target, scope, storage, form)
+        r = merge_round(cache, Q_win, W, cand_begin, n_recent, target, scope, storage, form,
+                        stats)
         if np.all(r.R == 0):
             raise ValueError("budget unreachable: no candidate pairs left")
         rounds.append(r)

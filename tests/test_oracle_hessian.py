@@ -157,3 +157,65 @@ def test_hessian_of_shared_key_group_matches_expanded_cache():
         H_fd = fd_hessian(expanded_loss, K_merged, i, j)
         H_or = oracle.hessian_block(q, K_merged, V_merged, E, i, j, log_n=log_n)
         np.testing.assert_allclose(H_or, H_fd, rtol=1e-4, atol=1e-6)
+
+
+# ----------------------------------------------------------- reading B of the window
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_per_query_norms_are_the_mean_of_each_querys_numerical_sensitivities(seed):
+    """Reading B: with several window queries, N11, N12, N22 are the means over the
+    queries of the norms of that query's own sensitivity vectors (each from a finite-
+    difference Hessian of its own attention-output loss, causal as the window is)."""
+    n, d, W = 7, 4, 3
+    rng = np.random.default_rng(50 + seed)
+    K = rng.normal(size=(n, d))
+    V = rng.normal(size=(n, d))
+    Qw = rng.normal(size=(1, W, d)) * 2.0          # one query head, W window queries
+    m = 1                                           # pair (1, 2): visible to every query
+    per_q = []
+    for j in range(W):
+        pos = n - W + j
+        q = Qw[0, j]
+        Kq, Vq = K[:pos + 1].copy(), V[:pos + 1]
+
+        def sens_vector(i, k):
+            vec = np.zeros(d)
+            for c in range(d):
+                E = np.zeros(d)
+                E[c] = 1.0
+                H = fd_hessian(lambda Kx: loss(q, Kx, Vq, E), Kq, i, k)
+                a = int(np.argmax(np.abs(q)))
+                vec[c] = H[a, a] * d / (q[a] * q[a])
+            return vec
+
+        per_q.append([np.linalg.norm(sens_vector(m, m)), np.linalg.norm(sens_vector(m, m + 1)),
+                      np.linalg.norm(sens_vector(m + 1, m + 1))])
+    want = np.mean(np.array(per_q), axis=0)
+    hs = oracle.score_head(K, V, None, n, cand_begin=m, n_recent=n - m - 2, Q_heads=Qw, W=W,
+                           stats="per_query")
+    np.testing.assert_allclose([hs.n11[0], hs.n12[0], hs.n22[0]], want, rtol=2e-4)
+
+
+def test_per_query_norms_equal_the_mean_reading_for_one_query():
+    rng = np.random.default_rng(9)
+    K, V = rng.normal(size=(20, 6)), rng.normal(size=(20, 6))
+    Q = rng.normal(size=(1, 1, 6)) * 2.0
+    a = oracle.score_head(K, V, None, 20, 2, 1, Q, 1)
+    b = oracle.score_head(K, V, None, 20, 2, 1, Q, 1, stats="per_query")
+    np.testing.assert_allclose(b.n11, a.n11, rtol=1e-13)
+    np.testing.assert_allclose(b.n12, a.n12, rtol=1e-13)
+    np.testing.assert_allclose(b.n22, a.n22, rtol=1e-13)
+    np.testing.assert_allclose(b.score, a.score, rtol=1e-12)
+
+
+def test_per_query_norms_differ_from_the_mean_reading_for_several_queries():
+    # norms are convex: the mean of norms is at least the norm of the mean residual,
+    # and differs from it once the queries attend differently
+    rng = np.random.default_rng(10)
+    K, V = rng.normal(size=(40, 6)), rng.normal(size=(40, 6))
+    Q = rng.normal(size=(2, 4, 6)) * 3.0
+    a = oracle.score_head(K, V, None, 40, 2, 4, Q, 4)
+    b = oracle.score_head(K, V, None, 40, 2, 4, Q, 4, stats="per_query")
+    assert np.max(np.abs(b.n12 - a.n12) / (a.n12 + 1e-300)) > 1e-3
+    with pytest.raises(ValueError):
+        oracle.score_head(K, V, None, 40, 2, 4, Q, 4, stats="median")

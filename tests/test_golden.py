@@ -25,3 +25,17 @@ def test_workloads_protect_the_pages_sink_tokens():
     settings = {k: int(v) for k, v in _rows("experiment_settings.txt")}
     for w in WORKLOADS:
         assert w.sink == settings["preserved_initial_tokens"]
+
+
+def test_prefill_measurement_uses_the_pages_compression_setting():
+    """bench.py --prefill runs the setting the pages' experiments use: budget 2048,
+    chunk 512, 32 preserved initial tokens."""
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    if root not in sys.path:
+        sys.path.insert(0, root)
+    import bench
+    settings = {k: int(v) for k, v in _rows("experiment_settings.txt")}
+    assert bench.PREFILL["budget"] == settings["default_budget_tokens"]
+    assert bench.PREFILL["chunk"] == settings["default_chunk_tokens"]
+    assert bench.PREFILL["sink"] == settings["preserved_initial_tokens"]

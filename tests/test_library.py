@@ -167,3 +167,19 @@ def test_prefill_chunk_alias_rules(kvs):
     assert _prefill(kvs, d, kc=same, vc=same, L=2048, n=512, budget=40)[0] == 3
     assert _prefill(kvs, d, kc=_fake(1))[0] == 5
     assert _prefill(kvs, d, logn=_fake(2))[0] == 5
+
+
+def test_score_pairs_form_host_validation(kvs):
+    d = kvs.make_desc(1, 8, 32, 128, 1024, kvs.BF16)
+
+    def call(form, **o):
+        a = dict(K=_fake(1), V=_fake(2), ws_bytes=1 << 40)
+        a.update(o)
+        return kvs._lib.kvs_score_pairs_form(ctypes.byref(d), a["K"], a["V"], None, _fake(3),
+                                             _fake(4), 32, _fake(5), 32, _fake(6), _fake(7),
+                                             form, _fake(8), a["ws_bytes"], None)
+
+    assert call(2) == 1 and call(-1) == 1                      # unknown form
+    assert call(kvs.FORM_DIAGONAL, K=None) == 1
+    assert call(kvs.FORM_DIAGONAL, ws_bytes=256) == 4
+    assert call(kvs.FORM_FULL, ws_bytes=256) == 4

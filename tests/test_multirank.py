@@ -63,3 +63,40 @@ def test_round_plan_matches_the_budget():
     assert bench.plan_rounds(131072, 32768, 32, 32) == [131072, 65568, 32816, 32768]
     assert bench.plan_rounds(32768, 16384, 32, 32) == [32768, 16416, 16384]
     assert torch.tensor(1).item() == 1
+
+
+def test_round_plan_equals_the_oracle_rounds_for_any_budget():
+    """The bench plans its graph of rounds on the host; every planned length must be what
+    the oracle's round driver reaches on real data (R = min(P, len - target) per round)."""
+    import sys
+    sys.path.insert(0, ROOT)
+    import numpy as np
+    from hypothesis import given, settings, strategies as st
+
+    import bench
+    import oracle
+
+    @settings(max_examples=25, deadline=None)
+    @given(T=st.integers(70, 240), frac=st.floats(0.15, 1.0), sink=st.integers(0, 12),
+           W=st.integers(1, 8))
+    def check(T, frac, sink, W):
+        target = max(sink + W + 1, int(T * frac))
+        try:
+            plan = bench.plan_rounds(T, target, sink, W)
+        except ValueError:
+            return
+        rng = np.random.default_rng(T)
+        K = rng.normal(size=(1, 1, T, 4))
+        V = rng.normal(size=(1, 1, T, 4))
+        Q = rng.normal(size=(1, 1, W, 4))
+        cache = oracle.cache_from_arrays(K, V, np.array([[T]]))
+        lens = [T]
+        for _ in range(64):
+            if lens[-1] == target:
+                break
+            r = oracle.merge_round(cache, Q, W, np.array([[sink]]), W, np.array([[target]]))
+            cache = r.cache
+            lens.append(cache.length(0, 0))
+        assert lens == plan
+
+    check()

@@ -517,6 +517,9 @@ def prefill_main(args, rank, world, local):
     ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
     flags = kvs.device_flags(ws)
     tokens = NL * w.T * world
+    step_bytes = prefill_step_bytes(w, c)
+    peak, peak_kind = peaks()
+    achieved = step_bytes / (ms / 1e3) / 1e9
     if rank == 0:
         print(json.dumps({
             "metric": "chunked prefill compression: prompt tokens/s", "value": tokens / (ms / 1e3),
@@ -530,7 +533,25 @@ def prefill_main(args, rank, world, local):
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
             "us_per_chunk_call": ms * 1e3 / n_chunks,
             "gpu_launches": launches_per_step * args.steps, "device_flags": flags,
+            "roofline": {"kernel": "whole chunk call (append, window passes, pair scoring, "
+                                   "selection, in-place merge)", "bound": "hbm",
+                         "achieved": achieved, "peak": peak, "peak_kind": peak_kind,
+                         "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                         "bytes_per_step": step_bytes},
             "clocks": clk}))
+
+
+def prefill_step_bytes(w, c):
+    """Algorithmic bytes of one prompt through the chunked prefill, all layers and
+    heads of one replica (the per-head accounting of every chunk call)."""
+    total, L = 0, 0
+    for e in range(0, w.T, c["chunk"]):
+        n = min(c["chunk"], w.T - e)
+        b, _ = accounting.prefill_chunk_bytes(L, n, c["budget"], c["sink"], c["W"], w.d,
+                                              w.elem_bytes)
+        total += b
+        L = min(L + n, c["budget"])
+    return total * w.layers * w.B * w.H_kv
 
 
 def main():

@@ -58,3 +58,17 @@ def test_layer_rho_in_range():
     w = inputs.WORKLOADS[2]
     rhos = [inputs.layer_rho(w, l) for l in range(32)]
     assert all(0.7 <= r < 0.95 for r in rhos) and len(set(rhos)) == 32
+
+
+def test_prefill_chunk_accounting():
+    from asymmetric_kv_merging_b200 import accounting
+    # the pages' setting at steady state: 2048 rows + a 512-row chunk, one round of 512
+    b, rounds = accounting.prefill_chunk_bytes(2048, 512, 2048, 32, 32, 128, 2)
+    assert rounds == 1
+    row = 2 * 128 * 2
+    want = (512 * (2 * row + 4)                                           # append
+            + 2560 * (256 + 4) + 2560 * (row + 8) + 2560 * (row + 4) + 1248 * 8  # scoring
+            + (2560 - 32) * (row + 4) + (2048 - 32) * (row + 4))           # in-place merge
+    assert b == want
+    # under the budget: the append only
+    assert accounting.prefill_chunk_bytes(0, 512, 2048, 32, 32, 128, 2) == (512 * (2 * row + 4), 0)

@@ -93,3 +93,29 @@ def test_value_rule_holds_through_the_chunked_loop(seed):
     for g in range(2):
         np.testing.assert_allclose(merged[g], expanded_attention(q[g], key_of, V[0, h]),
                                    rtol=1e-10, atol=1e-12)
+
+
+def test_chunked_loop_invariants_for_random_settings():
+    """Property check over random prompt lengths, chunk sizes and budgets: after every
+    chunk each head holds min(tokens so far, budget) rows standing for exactly the tokens
+    so far, with the preserved initial rows and the newest W rows untouched."""
+    from hypothesis import given, settings, strategies as st
+
+    @settings(max_examples=20, deadline=None)
+    @given(T=st.integers(40, 160), chunk=st.integers(4, 48), sink=st.integers(0, 8),
+           W=st.integers(1, 6), extra=st.integers(1, 60), seed=st.integers(0, 10_000))
+    def check(T, chunk, sink, W, extra, seed):
+        budget = sink + W + extra
+        if chunk < W:
+            return                                    # the window lies inside the chunk
+        K, V, Q = _prompt(seed, T, d=4, H=1, G=1, W=W)
+        _, history = _run(K, V, Q, chunk, budget, sink, W)
+        for c1, cache, _ in history:
+            L = cache.length(0, 0)
+            assert L == min(c1, budget)
+            assert np.sum(np.exp(cache.log_n[0][0])) == pytest.approx(c1, rel=1e-12)
+            keep = min(sink, L)
+            np.testing.assert_array_equal(cache.K[0][0][:keep], K[0, 0, :keep])
+            np.testing.assert_array_equal(cache.K[0][0][L - W:], K[0, 0, c1 - W:c1])
+
+    check()

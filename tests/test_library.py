@@ -183,3 +183,38 @@ def test_score_pairs_form_host_validation(kvs):
     assert call(kvs.FORM_DIAGONAL, K=None) == 1
     assert call(kvs.FORM_DIAGONAL, ws_bytes=256) == 4
     assert call(kvs.FORM_FULL, ws_bytes=256) == 4
+
+
+C_CONSUMER = r"""
+#include <stdio.h>
+#include <string.h>
+#include "kvs.h"
+int main(void) {
+  kvs_cache_desc d = {1, 8, 32, 128, 32768, KVS_BF16};
+  size_t ws = kvs_workspace_size(&d, 32, KVS_OP_DECODE);
+  int32_t L = -1;
+  /* host-checked argument errors launch nothing and need no GPU */
+  kvs_status s = kvs_prefill_chunk(&d, 0, 0, 0, 0, 0, 0, 0, 0, 0, 32, 2048, 32,
+                                   KVS_FORM_FULL, &L, 0, 0, 0);
+  printf("%d %d %d %s %d\n", kvs_version(), (int)(ws > 0), (int)s, kvs_status_str(KVS_OK), (int)L);
+  return 0;
+}
+"""
+
+
+def test_plain_c_program_links_and_calls_the_library(kvs, tmp_path):
+    """A C99 program built with gcc against include/kvs.h and libkvs.so: the boundary is a
+    plain C ABI (no C++ or torch types), and host-only calls work without a GPU."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not available")
+    src = tmp_path / "consumer.c"
+    src.write_text(C_CONSUMER)
+    exe = tmp_path / "consumer"
+    libdir = os.path.dirname(kvs.library_path())
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-o", str(exe), "-L", libdir, "-lkvs", f"-Wl,-rpath,{libdir}"],
+                   check=True, capture_output=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    assert out == ["1", "1", "1", "ok", "-1"]      # version, size > 0, INVALID_ARG, "ok", untouched

@@ -206,6 +206,26 @@ kvs_status kvs_merge_compact(const kvs_cache_desc* desc, const void* K, const vo
   return from_cuda(e);
 }
 
+kvs_status kvs_plan_rounds(int32_t len, int32_t target, int32_t cand_begin, int32_t n_recent,
+                           int32_t* lens_out, int32_t max_lens, int32_t* n_rounds) {
+  if (!lens_out || !n_rounds || len < 0 || target < 0 || cand_begin < 0 || n_recent < 0 ||
+      max_lens < 1)
+    return KVS_ERR_INVALID_ARG;
+  int32_t L = len, k = 0;
+  lens_out[0] = L;
+  while (L > target) {
+    const int32_t span = L - n_recent - cand_begin;
+    const int32_t P = span > 0 ? span / 2 : 0;
+    const int32_t R = P < L - target ? P : L - target;
+    if (R <= 0) return KVS_ERR_BUDGET;
+    if (k + 1 >= max_lens) return KVS_ERR_INVALID_ARG;
+    L -= R;
+    lens_out[++k] = L;
+  }
+  *n_rounds = k;
+  return KVS_OK;
+}
+
 kvs_status kvs_prefill_chunk(const kvs_cache_desc* desc, void* K, void* V, float* logn,
                              int32_t* len, int32_t L, const void* k_chunk, const void* v_chunk,
                              int32_t n, const void* Q_win, int32_t W, int32_t budget,

@@ -33,7 +33,7 @@ STATUS = {0: "KVS_OK", 1: "KVS_ERR_INVALID_ARG", 2: "KVS_ERR_UNSUPPORTED", 3: "K
 EXPORTS = ("kvs_workspace_size", "kvs_score_pairs", "kvs_merge_compact", "kvs_decode_attn",
            "kvs_device_flags", "kvs_status_str", "kvs_version", "kvs_launch_count",
            "kvs_decode_attn_static", "kvs_static_scratch_bytes", "kvs_score_pairs_form",
-           "kvs_prefill_chunk")
+           "kvs_prefill_chunk", "kvs_plan_rounds")
 
 
 class CacheDesc(ctypes.Structure):
@@ -64,6 +64,9 @@ _lib.kvs_score_pairs_form.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _i
 _lib.kvs_prefill_chunk.restype = ctypes.c_int
 _lib.kvs_prefill_chunk.argtypes = [_P, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _i32, _vp, _i32, _i32,
                                    _i32, _i32, ctypes.POINTER(_i32), _vp, _sz, _vp]
+_lib.kvs_plan_rounds.restype = ctypes.c_int
+_lib.kvs_plan_rounds.argtypes = [_i32, _i32, _i32, _i32, ctypes.POINTER(_i32), _i32,
+                                 ctypes.POINTER(_i32)]
 _lib.kvs_merge_compact.restype = ctypes.c_int
 _lib.kvs_merge_compact.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _i32, _i32,
                                    _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
@@ -208,3 +211,12 @@ def prefill_chunk(desc, K, V, logn, lens, L, k_chunk, v_chunk, Q_win, W, budget,
                                   ws.numel(), _stream(stream)),
            "kvs_prefill_chunk")
     return int(out.value)
+
+
+def plan_rounds(length: int, target: int, cand_begin: int, n_recent: int, max_lens: int = 64):
+    """kvs_plan_rounds: the per-head lengths [len, ..., target] of the merge rounds."""
+    buf = (_i32 * int(max_lens))()
+    n = _i32(0)
+    _check(_lib.kvs_plan_rounds(int(length), int(target), int(cand_begin), int(n_recent), buf,
+                                int(max_lens), ctypes.byref(n)), "kvs_plan_rounds")
+    return [int(buf[i]) for i in range(n.value + 1)]

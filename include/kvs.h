@@ -214,6 +214,20 @@ kvs_status kvs_prefill_chunk(const kvs_cache_desc* desc, void* K, void* V, float
                              size_t ws_bytes, kvs_stream_t stream);
 
 /*
+ * kvs_plan_rounds -- the round driver's plan, on the host: the lengths a head of `len`
+ * rows passes through when merged round by round to `target` (reading R4: a round
+ * merges R = min(P, len - target) pairs, P = floor((len - n_recent - cand_begin) / 2)
+ * candidate pairs). A caller that knows its heads' lengths uses it to size the round
+ * buffers and to capture the rounds into a graph without reading lengths back.
+ * Out: lens_out[0] = len, lens_out[k] = the length after round k, lens_out[*n_rounds]
+ *      = target (host arrays). Nothing touches a GPU.
+ * Errors: KVS_ERR_INVALID_ARG (NULL pointers, negative arguments, or max_lens too small
+ * for the plan), KVS_ERR_BUDGET (a round would merge nothing before reaching target).
+ */
+kvs_status kvs_plan_rounds(int32_t len, int32_t target, int32_t cand_begin, int32_t n_recent,
+                           int32_t* lens_out, int32_t max_lens, int32_t* n_rounds);
+
+/*
  * kvs_decode_attn -- one decode step of GQA attention over the merged cache
  * (attention of §数学主线三 with the log-count bias; the decoder stage of Figure 5).
  *

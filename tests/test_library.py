@@ -218,3 +218,33 @@ def test_plain_c_program_links_and_calls_the_library(kvs, tmp_path):
                    check=True, capture_output=True)
     out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
     assert out == ["1", "1", "1", "ok", "-1"]      # version, size > 0, INVALID_ARG, "ok", untouched
+
+
+def test_plan_rounds_matches_the_round_rule(kvs):
+    import sys
+    from hypothesis import given, settings, strategies as st
+    sys.path.insert(0, ROOT)
+    import bench
+    assert kvs.plan_rounds(131072, 32768, 32, 32) == [131072, 65568, 32816, 32768]
+    assert kvs.plan_rounds(100, 100, 4, 4) == [100]
+    with pytest.raises(kvs.KvsError) as e:
+        kvs.plan_rounds(100, 10, 32, 32)                       # span too short to get there
+    assert e.value.status == 3
+    with pytest.raises(kvs.KvsError) as e:
+        kvs.plan_rounds(131072, 32768, 32, 32, max_lens=3)      # 4 lengths needed
+    assert e.value.status == 1
+
+    @settings(max_examples=200, deadline=None)
+    @given(L=st.integers(0, 200000), frac=st.floats(0.0, 1.0), c0=st.integers(0, 64),
+           nr=st.integers(0, 64))
+    def check(L, frac, c0, nr):
+        target = int(L * frac)
+        try:
+            want = bench.plan_rounds(L, target, c0, nr)
+        except ValueError:
+            with pytest.raises(kvs.KvsError):
+                kvs.plan_rounds(L, target, c0, nr)
+            return
+        assert kvs.plan_rounds(L, target, c0, nr) == want
+
+    check()

@@ -400,12 +400,8 @@ static int cluster_size_for(int units) {
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   int C = units > 0 ? sms / units : 0;
   if (C > kMaxClusterSize) C = kMaxClusterSize;
-  if (cudaFuncSetAttribute((const void*)kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           CS::kSmem) != cudaSuccess)
-    C = 0;
-  if (C > 8 && cudaFuncSetAttribute((const void*)kfn,
-                                    cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
-    C = 8;
+  if (!ensure_smem_attr((const void*)kfn, CS::kSmem)) C = 0;
+  if (C > 8 && !ensure_nonportable_cluster((const void*)kfn)) C = 8;
   for (; C >= 2; --C) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(C, units);
@@ -434,17 +430,10 @@ static cudaError_t launch_shape(const kvs_cache_desc& d, const void* q, void* K,
                                 cudaStream_t st) {
   using S = TcShape<D, NC, STAGES, kCluster ? 1 : 0>;
   auto kfn = decode_tc_kernel<D, G, NC, STAGES, kCluster>;
-  static bool attr = false;   // set once per process, before any capture
-  if (!attr) {
-    if (cudaFuncSetAttribute((const void*)kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             S::kSmem) != cudaSuccess)
-      return cudaErrorInvalidValue;
-    if (kCluster && nsplit > 8 &&
-        cudaFuncSetAttribute((const void*)kfn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
-            cudaSuccess)
-      return cudaErrorInvalidValue;
-    attr = true;
-  }
+  // per device, cached (the first call on a device must precede any capture)
+  if (!ensure_smem_attr((const void*)kfn, S::kSmem)) return cudaErrorInvalidValue;
+  if (kCluster && nsplit > 8 && !ensure_nonportable_cluster((const void*)kfn))
+    return cudaErrorInvalidValue;
   const unsigned long long rows = (unsigned long long)d.B * d.H_kv * (unsigned long long)d.T_cap;
   CUtensorMap mK, mV, mL;
   if (!encode_rows_map(&mK, K, rows, d.d, S::kTile) || !encode_rows_map(&mV, V, rows, d.d, S::kTile))

@@ -5,6 +5,9 @@
 #include <atomic>
 #include <cstdint>
 #include <cstring>
+#include <map>
+#include <mutex>
+#include <utility>
 
 #include "kvs.h"
 #include "kvs_common.cuh"
@@ -15,6 +18,40 @@ using namespace kvs;
 namespace kvs {
 static std::atomic<long long> g_launches{0};
 void count_launches(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+namespace {
+std::mutex g_attr_mutex;
+// (device, kernel) -> the dynamic shared-memory limit set so far / the non-portable
+// cluster attribute set
+std::map<std::pair<int, const void*>, size_t> g_smem_attr;
+std::map<std::pair<int, const void*>, bool> g_cluster_attr;
+}  // namespace
+
+bool ensure_smem_attr(const void* fn, size_t bytes) {
+  if (bytes <= 48 * 1024) return true;   // the default limit
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  std::lock_guard<std::mutex> lock(g_attr_mutex);
+  size_t& done = g_smem_attr[std::make_pair(dev, fn)];
+  if (bytes <= done) return true;
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
+      cudaSuccess)
+    return false;
+  done = bytes;
+  return true;
+}
+
+bool ensure_nonportable_cluster(const void* fn) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  std::lock_guard<std::mutex> lock(g_attr_mutex);
+  bool& done = g_cluster_attr[std::make_pair(dev, fn)];
+  if (done) return true;
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+    return false;
+  done = true;
+  return true;
+}
 }  // namespace kvs
 
 namespace {

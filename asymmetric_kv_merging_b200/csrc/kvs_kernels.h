@@ -9,6 +9,14 @@
 
 namespace kvs {
 
+// Raise a kernel's dynamic shared-memory limit to at least `bytes` on the current
+// device (cudaFuncSetAttribute applies per device). The value set is cached per
+// (device, kernel) under a mutex, so later calls make no CUDA call; the first call for
+// a device must come before any stream capture.
+bool ensure_smem_attr(const void* fn, size_t bytes);
+// Allow cluster sizes above 8 for a kernel on the current device (cached the same way).
+bool ensure_nonportable_cluster(const void* fn);
+
 // Window statistics: (m, l) per window query, o_bar and alpha_bar into the score workspace.
 cudaError_t launch_window_stats(const kvs_cache_desc& d, const void* K, const void* V,
                                 const float* logn, const int32_t* len, const void* Qw, int W,

@@ -60,14 +60,32 @@ kvs_status kvs_decode_attn_static(const kvs_cache_desc* desc, const void* q, voi
   void* scratch = nullptr;
   kvs_status s = scratch_on_current_device(&scratch);
   if (s != KVS_OK) return s;
-  // The buffer keeps whatever the previous call left: the flag word and the arrival
-  // counters must start at zero, so clear that region on the stream first.
+  // The buffer keeps whatever the previous call left. The arrival counters must start at
+  // zero (a call whose pipeline wait gave up can leave them set), so that block is
+  // cleared on the stream first; the flag word before it is left alone, so that flags
+  // accumulate until kvs_static_device_flags reads and clears them.
+  const size_t counters = kvs::decode_layout(*desc).counters;
   const size_t head_region = kvs::persistent_bytes(*desc);
-  if (cudaMemsetAsync(scratch, 0, head_region, reinterpret_cast<cudaStream_t>(stream)) !=
-      cudaSuccess)
+  if (cudaMemsetAsync(static_cast<char*>(scratch) + counters, 0, head_region - counters,
+                      reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return KVS_ERR_CUDA;
   return kvs_decode_attn(desc, q, K, V, logn, len, k_new, v_new, out, scratch,
                          kStaticScratchBytes, stream);
+}
+
+kvs_status kvs_static_device_flags(int32_t* flags, int32_t clear, kvs_stream_t stream) {
+  if (!flags) return KVS_ERR_INVALID_ARG;
+  void* scratch = nullptr;
+  kvs_status s = scratch_on_current_device(&scratch);
+  if (s != KVS_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int32_t h = 0;
+  if (cudaMemcpyAsync(&h, scratch, sizeof(int32_t), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return KVS_ERR_CUDA;
+  if (clear && cudaMemsetAsync(scratch, 0, sizeof(int32_t), st) != cudaSuccess) return KVS_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return KVS_ERR_CUDA;
+  *flags = h;
+  return KVS_OK;
 }
 
 }  // extern "C"

@@ -81,7 +81,7 @@ select_kernel(const float* __restrict__ score, const int32_t* __restrict__ len,
   const int pstride = T_cap / 2;
 
   if (tid == 0) {
-    long long tot_len = 0, tot_P = 0;
+    long long tot_len = 0, tot_P = 0, min_len = 0;
     int bad = 0;
     for (int i = 0; i < nh; ++i) {
       const int hh = h_first + i;
@@ -93,7 +93,12 @@ select_kernel(const float* __restrict__ score, const int32_t* __restrict__ len,
       hinfo[hh].c0 = c0;
       tot_len += L;
       tot_P += P;
+      // repeated rounds shrink a span of S candidate rows to one row (S >= 1), so the
+      // shortest length this head can reach is L - S + min(S, 1)
+      const long long S = bad ? 0 : max(0, L - n_recent - c0);
+      min_len += L - S + (S > 0 ? 1 : 0);
     }
+    if (!bad && (long long)target[u] < min_len) set_flag(flags, KVS_FLAG_BUDGET);
     long long want = tot_len - (long long)target[u];
     if (want < 0) want = 0;
     if (want > tot_P) want = tot_P;
@@ -694,13 +699,7 @@ static cudaError_t launch_merge_t(const kvs_cache_desc& d, const void* K, const 
     constexpr size_t smem = (size_t)2 * 2 * (2 * CH * VPR) * 16 + 2 * 2 * CH * sizeof(float);
     static_assert(smem <= 100 * 1024, "in-place staging");
     auto kfn = merge_inplace_kernel<T, D>;
-    static bool attr = false;   // set once per process, before any capture
-    if (!attr) {
-      if (cudaFuncSetAttribute((const void*)kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)smem) != cudaSuccess)
-        return cudaErrorInvalidValue;
-      attr = true;
-    }
+    if (!ensure_smem_attr((const void*)kfn, smem)) return cudaErrorInvalidValue;
     kfn<<<heads, kMergeThreads, smem, st>>>((T*)K_out, (T*)V_out, logn_out, score, w_b, scope,
                                             d.H_kv, d.T_cap, sel, hinfo, len_out, dbg_sel,
                                             dbg_off, dbg_km, flags);

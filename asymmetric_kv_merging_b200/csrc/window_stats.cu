@@ -304,19 +304,6 @@ alpha_bar_kernel(const T* __restrict__ K, const float* __restrict__ logn,
 // Launchers
 // ---------------------------------------------------------------------------
 
-// Raise a kernel's dynamic shared-memory limit once per process (the first call
-// must come before any stream capture; later calls touch no CUDA API).
-template <typename F>
-static bool set_smem(F* fn, size_t bytes) {
-  static size_t done = 0;
-  if (bytes <= 48 * 1024 || bytes <= done) return true;
-  if (cudaFuncSetAttribute((const void*)fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)bytes) != cudaSuccess)
-    return false;
-  done = bytes;
-  return true;
-}
-
 template <typename T, int D>
 static cudaError_t launch_window_stats_t(const kvs_cache_desc& d, const void* K, const void* V,
                                          const float* logn, const int32_t* len, const void* Qw,
@@ -334,20 +321,20 @@ static cudaError_t launch_window_stats_t(const kvs_cache_desc& d, const void* K,
 
   size_t sm1 = (size_t)(2 * Qn * DP + 2 * kWinTile * DP + kWinTile) * sizeof(float);
   auto k1 = window_partial_kernel<T, D>;
-  if (!set_smem(k1, sm1)) return cudaErrorInvalidValue;
+  if (!ensure_smem_attr((const void*)k1, sm1)) return cudaErrorInvalidValue;
   k1<<<dim3(Ly.nsplit, units), kWinThreads, sm1, st>>>(
       (const T*)K, (const T*)V, logn, len, (const T*)Qw, d.H_kv, d.H_q, d.T_cap, W, Ly.nsplit,
       part_ml, part_o, flags);
 
   size_t sm2 = (size_t)(Qn * Ly.nsplit + 256) * sizeof(float);
   auto k2 = window_combine_kernel<D>;
-  if (!set_smem(k2, sm2)) return cudaErrorInvalidValue;
+  if (!ensure_smem_attr((const void*)k2, sm2)) return cudaErrorInvalidValue;
   k2<<<units, 256, sm2, st>>>(part_ml, part_o, Qn, Ly.nsplit, stats, obar, flags);
 
   size_t sm3 = (size_t)(Qn * DP + kAlphaTokens * DP + 2 * Qn + kAlphaTokens + kAlphaThreads) *
                sizeof(float);
   auto k3 = alpha_bar_kernel<T, D>;
-  if (!set_smem(k3, sm3)) return cudaErrorInvalidValue;
+  if (!ensure_smem_attr((const void*)k3, sm3)) return cudaErrorInvalidValue;
   dim3 g3((d.T_cap + kAlphaTokens - 1) / kAlphaTokens, units);
   k3<<<g3, kAlphaThreads, sm3, st>>>((const T*)K, logn, len, (const T*)Qw, d.H_kv, d.H_q,
                                      d.T_cap, W, stats, alpha);

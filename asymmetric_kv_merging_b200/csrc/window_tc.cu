@@ -439,15 +439,7 @@ bool window_tc_supported(const kvs_cache_desc& d, int W) {
 
 template <int D, bool MASS>
 static bool wt_attr() {
-  static bool done = false;    // once per process, before any capture
-  if (!done) {
-    if (cudaFuncSetAttribute((const void*)window_tc_kernel<D, MASS>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             WtShape<D, MASS>::kSmem) != cudaSuccess)
-      return false;
-    done = true;
-  }
-  return true;
+  return ensure_smem_attr((const void*)window_tc_kernel<D, MASS>, WtShape<D, MASS>::kSmem);
 }
 
 template <int D>

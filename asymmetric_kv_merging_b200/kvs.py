@@ -25,7 +25,7 @@ OP_SCORE, OP_MERGE, OP_DECODE, OP_PREFILL = 0, 1, 2, 3
 SCOPE_HEAD, SCOPE_POOLED = 0, 1
 FORM_FULL, FORM_DIAGONAL = 0, 1
 FLAG_BAD_LENGTH, FLAG_OUT_CAPACITY, FLAG_INPLACE_SPAN, FLAG_NONFINITE_STATS = 1, 2, 4, 8
-FLAG_TIMEOUT = 16
+FLAG_TIMEOUT, FLAG_BUDGET = 16, 32
 
 STATUS = {0: "KVS_OK", 1: "KVS_ERR_INVALID_ARG", 2: "KVS_ERR_UNSUPPORTED", 3: "KVS_ERR_BUDGET",
           4: "KVS_ERR_WORKSPACE", 5: "KVS_ERR_ALIAS", 6: "KVS_ERR_CUDA"}
@@ -33,7 +33,7 @@ STATUS = {0: "KVS_OK", 1: "KVS_ERR_INVALID_ARG", 2: "KVS_ERR_UNSUPPORTED", 3: "K
 EXPORTS = ("kvs_workspace_size", "kvs_score_pairs", "kvs_merge_compact", "kvs_decode_attn",
            "kvs_device_flags", "kvs_status_str", "kvs_version", "kvs_launch_count",
            "kvs_decode_attn_static", "kvs_static_scratch_bytes", "kvs_score_pairs_form",
-           "kvs_prefill_chunk", "kvs_plan_rounds")
+           "kvs_prefill_chunk", "kvs_plan_rounds", "kvs_static_device_flags")
 
 
 class CacheDesc(ctypes.Structure):
@@ -76,6 +76,8 @@ _lib.kvs_decode_attn_static.restype = ctypes.c_int
 _lib.kvs_decode_attn_static.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 _lib.kvs_static_scratch_bytes.restype = _sz
 _lib.kvs_device_flags.restype = ctypes.c_int
+_lib.kvs_static_device_flags.restype = ctypes.c_int
+_lib.kvs_static_device_flags.argtypes = [ctypes.POINTER(_i32), _i32, _vp]
 _lib.kvs_device_flags.argtypes = [_vp, ctypes.POINTER(_i32), _i32, _vp]
 
 if _lib.kvs_version() != 1:
@@ -193,6 +195,14 @@ def decode_attn_static(desc, q, K, V, logn, lens, out, k_new=None, v_new=None, s
                                        _ptr(lens), _ptr(k_new), _ptr(v_new), _ptr(out),
                                        _stream(stream)),
            "kvs_decode_attn_static")
+
+
+def static_device_flags(clear: bool = False, stream=None) -> int:
+    """kvs_static_device_flags: the flag word of the built-in scratch buffer."""
+    out = _i32(0)
+    _check(_lib.kvs_static_device_flags(ctypes.byref(out), int(bool(clear)), _stream(stream)),
+           "kvs_static_device_flags")
+    return int(out.value)
 
 
 def static_scratch_bytes() -> int:

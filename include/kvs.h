@@ -53,7 +53,8 @@ typedef enum {
   KVS_OK = 0,
   KVS_ERR_INVALID_ARG = 1,   /* NULL pointer, non-positive size, misalignment, bad W / n_recent */
   KVS_ERR_UNSUPPORTED = 2,   /* head dim, dtype, group size or window size not built */
-  KVS_ERR_BUDGET = 3,        /* (device flag) a budget that the candidate pairs cannot reach */
+  KVS_ERR_BUDGET = 3,        /* a budget that the candidate pairs cannot reach (host-planned
+                                calls; kvs_merge_compact reports it as KVS_FLAG_BUDGET) */
   KVS_ERR_WORKSPACE = 4,     /* workspace NULL, too small or not 256-byte aligned */
   KVS_ERR_ALIAS = 5,         /* an output overlaps an input in a way the call does not allow */
   KVS_ERR_CUDA = 6           /* a CUDA runtime call or kernel launch failed */
@@ -81,7 +82,10 @@ enum {
   KVS_FLAG_OUT_CAPACITY = 2,    /* a merged head or an append did not fit the output capacity */
   KVS_FLAG_INPLACE_SPAN = 4,    /* in-place merge on a span longer than it supports; head skipped */
   KVS_FLAG_NONFINITE_STATS = 8, /* a window query had no finite softmax normaliser */
-  KVS_FLAG_TIMEOUT = 16         /* a pipeline wait gave up (bounded waits); results invalid */
+  KVS_FLAG_TIMEOUT = 16,        /* a pipeline wait gave up (bounded waits); results invalid */
+  KVS_FLAG_BUDGET = 32          /* a unit's target is below the shortest length repeated rounds
+                                   can reach (every candidate span shrinks to one row at best);
+                                   the unit still merges what it can this round */
 };
 
 /*
@@ -265,11 +269,19 @@ kvs_status kvs_decode_attn(const kvs_cache_desc* desc, const void* q, void* K, v
  * (kvs_workspace_size(desc, 0, KVS_OP_DECODE)) exceeds it return KVS_ERR_WORKSPACE
  * and launch nothing. It allocates nothing: no cudaMalloc, no cudaFree.
  *
- * The first call on a device looks up the buffer's device address for that device
- * (make that call outside any stream capture); every call then clears the buffer's
- * flag word and arrival counters on `stream` before launching. All calls share the
- * one buffer: calls that overlap on the GPU (other streams, other host threads)
- * race on it, and the buffer keeps the last call's contents.
+ * The first call on a device does the set-up for that device: under CUDA's default
+ * lazy module loading it loads the library's device code there, which is when the
+ * array is placed in device memory (and may synchronise the device), and it looks up
+ * the array's device address. Make that first call (a warm-up call will do) while
+ * setting up, outside any stream capture and before the serving loop; later calls
+ * make no allocation and no synchronising call.
+ *
+ * All calls share the one buffer: calls that overlap on the GPU (other streams, other
+ * host threads) race on it, and the buffer keeps the last call's contents. Every call
+ * clears the arrival counters on `stream` before launching; the flag word is not
+ * cleared, so device flags (KVS_FLAG_OUT_CAPACITY for a head that cannot take the
+ * appended row, KVS_FLAG_BAD_LENGTH, KVS_FLAG_TIMEOUT) accumulate over calls until
+ * kvs_static_device_flags reads and clears them.
  */
 kvs_status kvs_decode_attn_static(const kvs_cache_desc* desc, const void* q, void* K, void* V,
                                   float* logn, int32_t* len, const void* k_new,
@@ -277,6 +289,15 @@ kvs_status kvs_decode_attn_static(const kvs_cache_desc* desc, const void* q, voi
 
 /* Size in bytes of the scratch buffer kvs_decode_attn_static uses. */
 size_t kvs_static_scratch_bytes(void);
+
+/*
+ * kvs_static_device_flags -- read (and, if clear != 0, clear) the device flag word of
+ * the built-in scratch buffer that kvs_decode_attn_static uses on the current device:
+ * the bits every static call since the last clear has set. The read is ordered after
+ * the work already queued on `stream`; the call synchronises `stream`. Host pointer
+ * `flags` receives the bits. Errors: KVS_ERR_INVALID_ARG (flags NULL), KVS_ERR_CUDA.
+ */
+kvs_status kvs_static_device_flags(int32_t* flags, int32_t clear, kvs_stream_t stream);
 
 /*
  * kvs_device_flags -- read (and optionally clear) the device flag word of a

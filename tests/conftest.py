@@ -1,3 +1,4 @@
+import json
 import os
 import sys
 
@@ -8,3 +9,16 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """One JSON line per GPU parity test with its counts (near-threshold selection
+    differences, degenerate pairs and boundary cases, compared rows, worst errors),
+    printed after the results so that it survives `-q`."""
+    parity = sys.modules.get("parity")
+    reports = getattr(parity, "REPORTS", None) if parity else None
+    if not reports:
+        return
+    terminalreporter.write_sep("-", "parity counts (GPU vs oracle, identical inputs each round)")
+    for line in reports:
+        terminalreporter.write_line("PARITY " + json.dumps(line, sort_keys=True))

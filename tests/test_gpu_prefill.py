@@ -14,7 +14,7 @@ import pytest
 import torch
 
 import oracle
-from parity import GpuCache, storage_of, to_oracle_cache
+from parity import REPORTS, GpuCache, storage_of, to_oracle_cache
 
 pytestmark = pytest.mark.gpu
 
@@ -93,8 +93,9 @@ def test_prefill_chunks_match_the_oracle(kvs, dtype, d, G, T, chunk, budget):
                 if not _rows_match(g_out, o_out, b, h, dtype):
                     assert _near_tie(rounds, b, h), f"chunk {i} b={b} h={h} differs without a tie"
                     ties += 1
-    print(f"prefill {dtype} d={d}: {len(ends)} chunks, {merged_chunks} with merge rounds, "
-          f"{ties} head-chunks decided by near-ties")
+    REPORTS.append(dict(test=f"prefill {str(dtype).split('.')[-1]} d={d}", chunks=len(ends),
+                        chunks_with_rounds=merged_chunks, head_chunks=len(ends) * B * H,
+                        near_tie_head_chunks=ties))
     assert merged_chunks >= 2
     assert ties <= 2
     assert kvs.device_flags(ws) == 0

@@ -148,7 +148,7 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 
 def plan_rounds(T, target, sink, n_recent):
-    """Per-head lengths after each merge round (every head is identical here)."""
+    """Per-head lengths after each merge round (a round merges R = min(P, len - target))."""
     lens = [T]
     while lens[-1] > target:
         L = lens[-1]
@@ -160,29 +160,86 @@ def plan_rounds(T, target, sink, n_recent):
     return lens
 
 
+def batch_plan(lens, target, scope, sink, n_recent):
+    """Round plan of a batch of heads, on the host.
+
+    lens: (B, H) lengths; target: (B, H) per head or (B,) per sequence (pooled).
+    Returns a list with one entry per round: (len_in (B, H), len_out_upper (B, H),
+    total_out (B,)). Per-head scope is exact. In pooled scope a round that merges every
+    candidate pair of a sequence is exact too; a round that merges fewer leaves each
+    head's length between len - P and len (the total is exact), so it must be the last.
+    """
+    import numpy as np
+    L = np.asarray(lens, dtype=np.int64).copy()
+    target = np.asarray(target, dtype=np.int64)
+    rounds = []
+    tot = L.sum(axis=1)
+    partial = False
+    for _ in range(64):
+        if scope == "head":
+            if np.all(L <= target):
+                return rounds
+            P = np.maximum(0, (L - n_recent - sink) // 2)
+            R = np.minimum(P, np.maximum(0, L - target))
+            if not R.any():
+                raise ValueError("budget unreachable")
+            rounds.append((L.copy(), L - R, (L - R).sum(axis=1)))
+            L = L - R
+        else:
+            if np.all(tot <= target):
+                return rounds
+            if partial:
+                raise ValueError("a partial pooled round must be the last")
+            P = np.maximum(0, (L - n_recent - sink) // 2)
+            Rs = np.minimum(P.sum(axis=1), np.maximum(0, tot - target))
+            if not Rs.any():
+                raise ValueError("budget unreachable")
+            full = Rs == P.sum(axis=1)
+            upper = np.where(full[:, None], L - P, L)
+            rounds.append((L.copy(), upper, tot - Rs))
+            partial = not full.all()
+            L, tot = upper, tot - Rs
+    raise ValueError("no plan within 64 rounds")
+
+
 class Runner:
-    """All device buffers of one replica of the workload, and its two CUDA graphs."""
+    """All device buffers of one replica of a workload, and its two CUDA graphs.
+
+    One step = every layer merged round by round to its budget (the merge phase), then
+    the decode phase: every layer's decode steps with the new row appended; with
+    `remerge_every` (the serving mix) the newest `remerge_every` rows of every head are
+    merged in place to 1/8 of their count after each such segment of decode steps.
+    """
 
     def __init__(self, w: inputs.Workload, rank: int, device):
+        import numpy as np
         from asymmetric_kv_merging_b200 import kvs
         self.kvs = kvs
         self.w = w
         self.dev = device
-        T = w.T
-        self.target = T // w.ratio
-        self.lens_plan = plan_rounds(T, self.target, w.sink, w.W)
-        self.rounds = len(self.lens_plan) - 1
-        # T_cap of the input cache, then of each round's output; the last round writes the
-        # per-layer cache that decode appends to, so it keeps room for every decode row
-        caps = [T + w.n_decode] + self.lens_plan[1:-1] + [self.target + w.n_decode]
+        B, H, d = w.B, w.H_kv, w.d
+        seq = inputs.sequence_lengths(w).numpy()
+        self.seq_lens = seq
+        lens0 = np.repeat(seq[:, None], H, axis=1)
+        if w.scope == "pooled":
+            self.target_np = (lens0 // w.ratio).sum(axis=1)
+        else:
+            self.target_np = lens0 // w.ratio
+        self.scope = w.scope
+        self.scope_code = kvs.SCOPE_POOLED if w.scope == "pooled" else kvs.SCOPE_HEAD
+        self.plan = batch_plan(lens0, self.target_np, w.scope, w.sink, w.W)
+        self.rounds = len(self.plan)
+        final_upper = self.plan[-1][1]
+        # decode-phase lengths per head (exact when the last round is exact)
+        self.lens_after = final_upper
+        extra = w.n_decode
+        cap0 = int(seq.max()) + w.n_decode
+        caps = [cap0] + [int(r[1].max()) for r in self.plan[:-1]] + [int(final_upper.max()) + extra]
         caps = [c + (c % 2) for c in caps]
         self.caps = caps
-        self.layers = []
-        for l in range(w.layers):
-            li = inputs.make_layer(w, l + rank * w.layers, device=device, T_cap=caps[0])
-            self.layers.append(li)
+        self.layers = [inputs.make_layer(w, l + rank * w.layers, device=device, T_cap=caps[0])
+                       for l in range(w.layers)]
         torch.cuda.synchronize()
-        B, H, d = w.B, w.H_kv, w.d
         dt = w.torch_dtype
 
         def cache(cap):
@@ -195,7 +252,7 @@ class Runner:
         self.in_logn = torch.zeros(B, H, caps[0], dtype=torch.float32, device=device)
         self.in_lens = [li.lens.reshape(-1).to(torch.int32).contiguous() for li in self.layers]
         self.cand = torch.full((B * H,), w.sink, dtype=torch.int32, device=device)
-        self.tgt = torch.full((B * H,), self.target, dtype=torch.int32, device=device)
+        self.tgt = torch.tensor(self.target_np.reshape(-1), dtype=torch.int32, device=device)
         self.score = torch.zeros(B * H * (caps[0] // 2), dtype=torch.float32, device=device)
         self.w_b = torch.zeros_like(self.score)
         self.descs = [kvs.make_desc(B, H, w.H_q, d, c, dt) for c in caps]
@@ -203,34 +260,74 @@ class Runner:
                        for op in (kvs.OP_SCORE, kvs.OP_MERGE, kvs.OP_DECODE))
         self.ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=device)
         self.out = torch.zeros(w.layers, w.n_decode, B, w.H_q, d, dtype=dt, device=device)
+        # serving mix: in-place re-merge of the newest rows after every segment
+        self.remerge = []
+        if w.remerge_every:
+            if self.scope != "head":
+                raise ValueError("re-merge is per head")
+            seg = w.remerge_every
+            L = final_upper.astype(np.int64).copy()
+            for s0 in range(0, w.n_decode, seg):
+                L = L + seg
+                # the window: the last W decode queries of the segment, [B, H_q, W, d]
+                Qw = [li.q_dec[s0 + seg - w.W:s0 + seg].permute(1, 2, 0, 3).contiguous()
+                      for li in self.layers]
+                subs = []
+                n = seg
+                while n > seg // w.remerge_ratio:
+                    cand = L - n
+                    tgt = L - n // 2
+                    subs.append(dict(
+                        cand=torch.tensor(cand.reshape(-1), dtype=torch.int32, device=device),
+                        tgt=torch.tensor(tgt.reshape(-1), dtype=torch.int32, device=device),
+                        L=L.copy(), n=n))
+                    L = tgt
+                    n //= 2
+                self.remerge.append(dict(s0=s0, Qw=Qw, subs=subs))
         self.stream = torch.cuda.Stream(device)
         self.g_merge = None
         self.g_decode = None
 
     # one merge pass over every layer
-    def merge_all(self):
+    def merge_all(self, timer=None):
         kvs, w = self.kvs, self.w
         for l, li in enumerate(self.layers):
             src = dict(K=li.K, V=li.V, logn=self.in_logn, lens=self.in_lens[l])
             for r in range(self.rounds):
                 dst = self.final[l] if r == self.rounds - 1 else self.scratch[r]
-                kvs.score_pairs(self.descs[r], src["K"], src["V"], src["logn"], src["lens"],
-                                self.cand, w.W, li.Q_win, w.W, self.score, self.w_b, self.ws)
-                kvs.merge_compact(self.descs[r], src["K"], src["V"], src["logn"], src["lens"],
-                                  self.cand, w.W, self.score, self.w_b, self.tgt,
-                                  kvs.SCOPE_HEAD, self.caps[r + 1], dst["K"], dst["V"],
-                                  dst["logn"], dst["lens"], self.ws)
+                with _timed(timer, "score"):
+                    kvs.score_pairs(self.descs[r], src["K"], src["V"], src["logn"], src["lens"],
+                                    self.cand, w.W, li.Q_win, w.W, self.score, self.w_b, self.ws)
+                with _timed(timer, "merge"):
+                    kvs.merge_compact(self.descs[r], src["K"], src["V"], src["logn"], src["lens"],
+                                      self.cand, w.W, self.score, self.w_b, self.tgt,
+                                      self.scope_code, self.caps[r + 1], dst["K"], dst["V"],
+                                      dst["logn"], dst["lens"], self.ws)
                 src = dst
 
-    # every decode step of every layer (new row appended each step)
-    def decode_all(self):
+    # every decode step of every layer (new row appended each step), with the re-merges
+    def decode_all(self, timer=None):
         kvs, w = self.kvs, self.w
         dsc = self.descs[-1]
+        seg = w.remerge_every or w.n_decode
         for s in range(w.n_decode):
-            for l, li in enumerate(self.layers):
-                f = self.final[l]
-                kvs.decode_attn(dsc, li.q_dec[s], f["K"], f["V"], f["logn"], f["lens"],
-                                self.out[l, s], self.ws, li.k_new[s], li.v_new[s])
+            with _timed(timer, "decode"):
+                for l, li in enumerate(self.layers):
+                    f = self.final[l]
+                    kvs.decode_attn(dsc, li.q_dec[s], f["K"], f["V"], f["logn"], f["lens"],
+                                    self.out[l, s], self.ws, li.k_new[s], li.v_new[s])
+            if self.remerge and (s + 1) % seg == 0:
+                rm = self.remerge[s // seg]
+                with _timed(timer, "remerge"):
+                    for l in range(w.layers):
+                        f = self.final[l]
+                        for sub in rm["subs"]:
+                            kvs.score_pairs(dsc, f["K"], f["V"], f["logn"], f["lens"], sub["cand"],
+                                            0, rm["Qw"][l], w.W, self.score, self.w_b, self.ws)
+                            kvs.merge_compact(dsc, f["K"], f["V"], f["logn"], f["lens"],
+                                              sub["cand"], 0, self.score, self.w_b, sub["tgt"],
+                                              kvs.SCOPE_HEAD, self.caps[-1], f["K"], f["V"],
+                                              f["logn"], f["lens"], self.ws)
 
     def capture(self):
         with torch.cuda.stream(self.stream):
@@ -260,19 +357,110 @@ class Runner:
             if ev:
                 ev[2].record(self.stream)
 
+    def breakdown(self):
+        """Device time of each kind of library call, from one eager pass of a step with
+        CUDA events around every call on the launching stream. A sleep kernel first lets
+        the host queue ahead of the device, so that the events time device work rather
+        than host launch gaps. Returns {kind: ms per step}."""
+        timer = {}
+        with torch.cuda.stream(self.stream):
+            torch.cuda._sleep(200_000_000)
+            self.merge_all(timer)
+            self.decode_all(timer)
+        self.stream.synchronize()
+        return {k: sum(a.elapsed_time(b) for a, b in v) for k, v in timer.items()}
+
     def tokens_per_step(self):
-        return self.w.layers * self.w.B * self.w.T
+        return step_tokens(self.w)
+
+    # ---- algorithmic bytes (per step, this replica) ----
+    def score_bytes(self):
+        w, eb = self.w, self.w.elem_bytes
+        tot = 0
+        for (L_in, _, _) in self.plan:
+            P = (L_in - w.W - w.sink) // 2
+            tot += sum(accounting.score_bytes(int(a), max(0, int(p)), w.d, eb)
+                       for a, p in zip(L_in.reshape(-1), P.reshape(-1)))
+        return tot * w.layers
+
+    def merge_bytes(self):
+        w, eb = self.w, self.w.elem_bytes
+        tot = 0
+        for (L_in, _, tot_out) in self.plan:
+            tot += accounting.merge_bytes(int(L_in.sum()), int(tot_out.sum()), w.d, eb)
+        return tot * w.layers
+
+    def decode_bytes(self):
+        """Every decode launch reads, per head, its cached rows and the appended one
+        (row totals per sequence are exact even where per-head lengths are not known)."""
+        w = self.w
+        per_tok = accounting.decode_bytes_per_token(w.d, w.elem_bytes)
+        rows = float(self.plan[-1][2].sum())
+        heads = w.B * w.H_kv
+        seg = w.remerge_every or w.n_decode
+        tot = 0.0
+        for s in range(w.n_decode):
+            rows += heads                       # the appended row of every head
+            tot += rows * per_tok
+            if self.remerge and (s + 1) % seg == 0:
+                rows -= heads * (seg - seg // w.remerge_ratio)
+        return tot * w.layers
+
+    def remerge_bytes(self):
+        w, eb = self.w, self.w.elem_bytes
+        tot = 0
+        for rm in self.remerge:
+            for sub in rm["subs"]:
+                n, L = sub["n"], sub["L"]
+                P, R = n // 2, n // 2
+                for Lh in L.reshape(-1):
+                    tot += accounting.score_bytes(int(Lh), P, w.d, eb)
+                    tot += accounting.merge_bytes(n, n - R, w.d, eb)
+        return tot * w.layers
+
+    def decode_launches(self):
+        return self.w.n_decode * self.w.layers
 
     def decode_bytes_per_launch(self):
-        w = self.w
-        avg_len = self.target + (w.n_decode + 1) / 2.0
-        return w.B * w.H_kv * avg_len * accounting.decode_bytes_per_token(w.d, w.elem_bytes)
+        return self.decode_bytes() / self.decode_launches()
+
+
+def step_tokens(w: inputs.Workload) -> int:
+    """Merged KV tokens of one step: every input position of every sequence of every
+    layer, plus the rows the re-merges take in (one token = one position of one
+    sequence across all KV heads of one layer)."""
+    t = int(inputs.sequence_lengths(w).sum()) * w.layers
+    if w.remerge_every:
+        t += (w.n_decode // w.remerge_every) * w.remerge_every * w.B * w.layers
+    return t
+
+
+class _timed:
+    """Context manager that brackets library calls with CUDA events (no-op without a
+    timer dict)."""
+
+    def __init__(self, timer, kind):
+        self.timer, self.kind = timer, kind
+
+    def __enter__(self):
+        if self.timer is not None:
+            self.e0 = torch.cuda.Event(enable_timing=True)
+            self.e0.record()
+        return self
+
+    def __exit__(self, *exc):
+        if self.timer is not None:
+            e1 = torch.cuda.Event(enable_timing=True)
+            e1.record()
+            self.timer.setdefault(self.kind, []).append((self.e0, e1))
+        return False
 
 
 def run_e2e(rn: Runner, steps, warmup):
     """The same step through the public API with host buffers: every step copies all of
     its inputs from pinned host memory (K, V and window queries of every layer, then the
-    decode queries and new rows) and copies the decode outputs and final lengths back.
+    decode queries and new rows, and the re-merge windows) and copies the decode outputs
+    and final lengths back.
 
     Copies run on their own stream, as a serving loop would pipeline them: step k+1's
     K / V / window copies start once step k's merge phase has consumed its inputs (they
@@ -281,14 +469,22 @@ def run_e2e(rn: Runner, steps, warmup):
     """
     host_m, host_d = [], []
     h2d = 0
-    for li in rn.layers:
+
+    def pin(t):
+        hp = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        hp.copy_(t)
+        return hp
+
+    for l, li in enumerate(rn.layers):
         hm, hd = {}, {}
         for name, dst in (("K", hm), ("V", hm), ("Q_win", hm), ("q_dec", hd), ("k_new", hd),
                           ("v_new", hd)):
             t = getattr(li, name)
-            hp = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
-            hp.copy_(t)
-            dst[name] = hp
+            dst[(name, None)] = (t, pin(t))
+            h2d += t.numel() * t.element_size()
+        for i, rm in enumerate(rn.remerge):
+            t = rm["Qw"][l]
+            hd[("Qw", i)] = (t, pin(t))
             h2d += t.numel() * t.element_size()
         host_m.append(hm)
         host_d.append(hd)
@@ -302,9 +498,9 @@ def run_e2e(rn: Runner, steps, warmup):
     def copy_in(hosts, after):
         with torch.cuda.stream(cp):
             cp.wait_event(after)
-            for li, hl in zip(rn.layers, hosts):
-                for name, hp in hl.items():
-                    getattr(li, name).copy_(hp, non_blocking=True)
+            for hl in hosts:
+                for dev_t, hp in hl.values():
+                    dev_t.copy_(hp, non_blocking=True)
             done = ev()
             done.record(cp)
         return done
@@ -352,61 +548,153 @@ def run_e2e(rn: Runner, steps, warmup):
 # oracle timing (CPU baseline and reference arm)
 # ---------------------------------------------------------------------------
 
-def oracle_sample(w: inputs.Workload, li, target, rounds_lens):
-    """Time the fp64 oracle on one KV head of one layer (all rounds) and on two
-    decode steps of one layer (all heads); scale to one full step of the workload."""
+def _oracle_unit(job):
+    """Worker (a spawned process): the fp64 oracle, single-threaded, on one selection unit
+    (one KV head, or one sequence's heads in pooled scope): every merge round to the
+    budget, then `n_dec` decode steps. Returns (merge s, decode s per step, rounds)."""
+    path, W, sink, storage, scope, n_dec = job
     import numpy as np
+    from threadpoolctl import threadpool_limits
     import oracle
-    from threadpoolctl import threadpool_info
-    K = li.K[:1, :1].double().cpu().numpy()
-    V = li.V[:1, :1].double().cpu().numpy()
-    lens = np.array([[w.T]])
-    Q = li.Q_win[:1, :w.G].double().cpu().numpy()
-    cache = oracle.cache_from_arrays(K, V, lens)
+    z = np.load(path)
+    with threadpool_limits(1):
+        cache = oracle.cache_from_arrays(z["K"], z["V"], z["lens"])
+        t0 = time.perf_counter()
+        out, rounds = oracle.compress(cache, z["Q"], W, z["cand"], W, z["target"], scope,
+                                      storage=storage)
+        t1 = time.perf_counter()
+        for s in range(n_dec):
+            _, out = oracle.decode_step(out, z["qd"][s], z["kn"][s], z["vn"][s])
+        t2 = time.perf_counter()
+    return t1 - t0, (t2 - t1) / max(n_dec, 1), len(rounds)
+
+
+def oracle_units(w: inputs.Workload, layers, n_units):
+    """The first n_units selection units of the workload (layer-major), as numpy files
+    for the oracle workers: fp64 copies of the stored bf16 / fp32 inputs."""
+    import numpy as np
+    d = tempfile.mkdtemp(prefix="kvs_oracle_")
+    paths = []
+    G = w.G
+    for li in layers:
+        lens = li.lens.view(w.B, w.H_kv).cpu().numpy()
+        for b in range(w.B):
+            heads = [list(range(w.H_kv))] if w.scope == "pooled" else [[h] for h in range(w.H_kv)]
+            for hs in heads:
+                if len(paths) == n_units:
+                    return paths, d
+                T_b = int(lens[b, 0])
+                h0, h1 = hs[0], hs[-1] + 1
+                sl = lambda t: t[b:b + 1, h0:h1, :T_b].double().cpu().numpy()  # noqa: E731
+                qd = li.q_dec[:2, b:b + 1, h0 * G:h1 * G].double().cpu().numpy()
+                kn = li.k_new[:2, b:b + 1, h0:h1].double().cpu().numpy()
+                vn = li.v_new[:2, b:b + 1, h0:h1].double().cpu().numpy()
+                tgt = (np.array([[T_b // w.ratio] * len(hs)]) if w.scope == "head"
+                       else np.array([(T_b // w.ratio) * len(hs)]))
+                p = os.path.join(d, f"u{len(paths)}.npz")
+                np.savez(p, K=sl(li.K), V=sl(li.V), lens=np.full((1, len(hs)), T_b),
+                         Q=li.Q_win[b:b + 1, h0 * G:h1 * G].double().cpu().numpy(),
+                         cand=np.full((1, len(hs)), w.sink), target=tgt, qd=qd, kn=kn, vn=vn)
+                paths.append(p)
+    return paths, d
+
+
+def oracle_pool(w: inputs.Workload, paths, workers):
+    """Run the oracle on every unit file with `workers` spawned single-threaded processes
+    (spawn: safe after CUDA is initialised). Returns the per-unit results and wall s."""
+    import multiprocessing as mp
+    import shutil
+    storage = "bf16" if w.dtype == "bf16" else "f32"
+    n_dec = min(2, w.n_decode)
+    jobs = [(p, w.W, w.sink, storage, w.scope, n_dec) for p in paths]
     t0 = time.perf_counter()
-    out, rounds = oracle.compress(cache, Q, w.W, np.array([[w.sink]]), w.W, np.array([[target]]),
-                                  storage="bf16" if w.dtype == "bf16" else "f32")
-    t_merge_head = time.perf_counter() - t0
-    # two decode steps over one layer's compressed head, all query heads of that head
-    qd = li.q_dec[:2, :1, :w.G].double().cpu().numpy()
-    kn = li.k_new[:2, :1, :1].double().cpu().numpy()
-    vn = li.v_new[:2, :1, :1].double().cpu().numpy()
-    t0 = time.perf_counter()
-    for s in range(2):
-        _, out = oracle.decode_step(out, qd[s], kn[s], vn[s])
-    t_dec_head = (time.perf_counter() - t0) / 2
-    per_step = (w.layers * w.B * w.H_kv * t_merge_head
-                + w.n_decode * w.layers * w.B * w.H_kv * t_dec_head)
-    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    sample = (f"oracle on KV head 0 of layer 0 (all {len(rounds)} rounds, {w.T} -> {target} rows: "
-              f"{t_merge_head:.2f} s) and 2 decode steps of that head ({t_dec_head * 1e3:.1f} ms "
-              f"each); scaled x{w.layers * w.B * w.H_kv} heads and x{w.n_decode} steps")
-    return per_step, t_merge_head + 2 * t_dec_head, threads, sample
+    with mp.get_context("spawn").Pool(workers) as pool:
+        res = pool.map(_oracle_unit, jobs, chunksize=1)
+    wall = time.perf_counter() - t0
+    shutil.rmtree(os.path.dirname(paths[0]), ignore_errors=True)
+    return res, wall
+
+
+def units_per_step(w: inputs.Workload):
+    return w.layers * w.B * (1 if w.scope == "pooled" else w.H_kv)
+
+
+def oracle_step_seconds(w: inputs.Workload, res, workers):
+    """One step of the workload on `workers` cores: every unit's merge rounds and
+    n_decode decode steps, the units spread evenly over the cores."""
+    t_merge = statistics.mean(r[0] for r in res)
+    t_dec = statistics.mean(r[1] for r in res)
+    waves = -(-units_per_step(w) // workers)          # a unit runs on one core
+    return waves * (t_merge + w.n_decode * t_dec), t_merge, t_dec
+
+
+def oracle_single_thread_workload0():
+    """The oracle on the tiny fp32 workload (T = 512, 2 KV heads), single-threaded:
+    merged tokens/s of its compression rounds."""
+    import numpy as np
+    from threadpoolctl import threadpool_limits
+    import oracle
+    w0 = inputs.workload(0)
+    li = inputs.make_layer(w0, 0)
+    B, H = w0.B, w0.H_kv
+    with threadpool_limits(1):
+        cache = oracle.cache_from_arrays(li.K.double().numpy(), li.V.double().numpy(),
+                                         li.lens.numpy())
+        t0 = time.perf_counter()
+        oracle.compress(cache, li.Q_win.double().numpy(), w0.W, np.full((B, H), w0.sink), w0.W,
+                        np.full((B, H), w0.T // w0.ratio), storage="f32")
+        dt = time.perf_counter() - t0
+    return B * w0.T / dt
+
+
+def cpu_baseline(w: inputs.Workload, layers, tokens_per_step):
+    """The oracle as it stands on the host's cores: one unit per core, run in parallel."""
+    workers = max(1, os.cpu_count() or 1)
+    n = min(workers, units_per_step(w))
+    paths, _ = oracle_units(w, layers, n)
+    res, wall = oracle_pool(w, paths, workers=len(paths))
+    per_step, t_merge, t_dec = oracle_step_seconds(w, res, len(paths))
+    return {"value": tokens_per_step / per_step, "unit": UNIT, "cores": len(paths),
+            "kind": "oracle",
+            "sample": (f"{len(paths)} selection units of layer 0 on, one per core in "
+                       f"single-threaded processes ({res[0][2]} rounds each, mean {t_merge:.2f} s; "
+                       f"then 2 decode steps, mean {t_dec * 1e3:.1f} ms each), {wall:.1f} s wall; "
+                       f"scaled to {units_per_step(w)} units and {w.n_decode} decode steps "
+                       f"spread over {len(paths)} cores"),
+            "host_cpus": os.cpu_count(),
+            "single_thread_workload0_tokens_per_s": oracle_single_thread_workload0()}
 
 
 def reference_main(args, rank, world):
+    """The reference arm: the oracle as it stands. Every step is one selection unit of
+    the workload (all its merge rounds, then two decode steps), the units of all steps
+    running in parallel single-threaded processes, one per host core; a step's time is
+    scaled to the whole workload on those cores."""
     if rank != 0:
         return
     w = inputs.workload(args.workload)
     dev = "cuda" if torch.cuda.is_available() else "cpu"
-    li = inputs.make_layer(w, 0, device=dev)
-    target = w.T // w.ratio
-    lens = plan_rounds(w.T, target, w.sink, w.W)
-    for _ in range(args.warmup):
-        oracle_sample(w, li, target, lens)
-    per = []
-    threads, sample = 1, ""
-    for _ in range(args.steps):
-        per_step, _, threads, sample = oracle_sample(w, li, target, lens)
-        per.append(per_step)
-    ms = statistics.mean(per) * 1e3
-    value = w.layers * w.B * w.T / (ms / 1e3)
-    cores = threads
+    cores = max(1, os.cpu_count() or 1)
+    # at least one unit per core, so that every unit is timed with all cores busy
+    need = max(args.steps + args.warmup, cores)
+    per_layer = w.B * (1 if w.scope == "pooled" else w.H_kv)
+    layers = [inputs.make_layer(w, l, device=dev) for l in range((need + per_layer - 1) // per_layer)]
+    paths, _ = oracle_units(w, layers, need)
+    workers = cores
+    res, wall = oracle_pool(w, paths, workers)
+    res = res[args.warmup:]
+    per_step, t_merge, t_dec = oracle_step_seconds(w, res, workers)
+    ms = per_step * 1e3
+    value = step_tokens(w) / per_step
+    sample = (f"{len(paths)} selection units ({args.warmup} warm-up; at least one per step "
+              f"and one per core), in {workers} single-threaded processes: merge rounds mean {t_merge:.2f} s, decode "
+              f"step mean {t_dec * 1e3:.1f} ms; scaled to {units_per_step(w)} units and "
+              f"{w.n_decode} decode steps over {workers} cores; {wall:.1f} s wall")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": config_of(w, args.gpus),
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": workers, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -416,8 +704,9 @@ L2_BYTES = 126 * 1024 * 1024
 
 
 def config_of(w, n_gpus):
-    kv = 2 * w.layers * w.B * w.H_kv * w.T * w.d * w.elem_bytes
-    dec = 2 * w.B * w.H_kv * (w.T // w.ratio) * w.d * w.elem_bytes
+    seq = inputs.sequence_lengths(w)
+    kv = 2 * w.layers * int(seq.sum()) * w.H_kv * w.d * w.elem_bytes
+    dec = 2 * w.H_kv * int((seq // w.ratio).sum()) * w.d * w.elem_bytes
     l2 = (f"inputs larger than L2 ({kv / 2**30:.2f} GiB of K/V per replica; no flush needed)"
           if kv > L2_BYTES else f"inputs of {kv / 2**20:.1f} MiB fit in L2")
     if dec <= L2_BYTES and w.layers * dec > L2_BYTES:
@@ -426,10 +715,22 @@ def config_of(w, n_gpus):
     elif dec <= L2_BYTES:
         l2 += (f"; the merged decode cache ({dec / 2**20:.1f} MiB) fits in L2, so decode "
                "steps may hit it")
-    return {"workload": w.name, "B": w.B, "layers": w.layers, "T": w.T, "H_kv": w.H_kv,
-            "H_q": w.H_q, "d": w.d, "ratio": w.ratio, "budget_per_head": w.T // w.ratio,
-            "decode_steps_per_layer": w.n_decode, "window": w.W, "sink": w.sink,
-            "parallelism": f"replicas x{n_gpus}" if n_gpus > 1 else "single GPU", "l2": l2}
+    cfg = {"workload": w.name, "B": w.B, "layers": w.layers, "T": w.T, "H_kv": w.H_kv,
+           "H_q": w.H_q, "d": w.d, "ratio": w.ratio, "scope": w.scope,
+           "budget_per_head" if w.scope == "head" else "budget_per_sequence":
+               w.T // w.ratio if w.scope == "head" else (w.T // w.ratio) * w.H_kv,
+           "decode_steps_per_layer": w.n_decode, "window": w.W, "sink": w.sink,
+           "parallelism": f"replicas x{n_gpus}" if n_gpus > 1 else "single GPU", "l2": l2}
+    if w.len_range:
+        cfg["T"] = f"per sequence U{{{w.len_range[0]}..{w.len_range[1]}}} (max {int(seq.max())})"
+        cfg["total_prefill_tokens"] = int(seq.sum())
+        cfg["budget_per_head"] = "floor(len / ratio) of its sequence"
+    if w.remerge_every:
+        cfg["remerge"] = (f"every {w.remerge_every} decode steps the newest {w.remerge_every} "
+                          f"rows of every head are merged in place to "
+                          f"{w.remerge_every // w.remerge_ratio} (window = the last {w.W} "
+                          f"decode queries)")
+    return cfg
 
 
 def peaks():
@@ -594,20 +895,57 @@ def main():
     decode_ms = max_over_ranks(decode_ms, world)
     tokens = rn.tokens_per_step() * world
     value = tokens / (step_ms / 1e3)
+    flags = rn.kvs.device_flags(rn.ws)
 
+    # per-call device time of one eager step (CUDA events around every library call)
+    parts = rn.breakdown()
+    parts = {k: max_over_ranks(v, world) for k, v in sorted(parts.items())}
+    if not rn.remerge:
+        parts["decode"] = decode_ms          # the graph-replayed phase, exactly
     peak, peak_kind = peaks()
-    n_dec_launch = w.n_decode * w.layers
-    dec_launch_ms = decode_ms / n_dec_launch
-    achieved = rn.decode_bytes_per_launch() / (dec_launch_ms / 1e3) / 1e9
+    algo = {"decode": rn.decode_bytes(), "score": rn.score_bytes(), "merge": rn.merge_bytes()}
+    if rn.remerge:
+        algo["remerge"] = rn.remerge_bytes()
+    names = {
+        "decode": "decode_tc_kernel (GQA decode; one thread-block cluster per KV head when "
+                  "every head's cluster fits the GPU, else the split grid)",
+        "score": "kvs_score_pairs: window_tc_kernel passes A and B, their two combine kernels, "
+                 "pair_score_kernel",
+        "merge": "kvs_merge_compact: select_kernel + merge_kernel (out-of-place compaction)",
+        "remerge": "in-place re-merge rounds: kvs_score_pairs + kvs_merge_compact "
+                   "(merge_inplace_kernel)",
+    }
+    rooflines = {}
+    for k, b in algo.items():
+        ms = parts.get(k)
+        if not ms:
+            continue
+        ach = b / (ms / 1e3) / 1e9
+        rooflines[k] = {"kernel": names[k], "bound": "hbm", "achieved": ach, "peak": peak,
+                        "peak_kind": peak_kind, "unit": "GB/s", "frac": ach / peak,
+                        "algorithmic_bytes_per_step": b, "ms_per_step": ms,
+                        "timing": ("graph replay, CUDA events" if k == "decode" and not rn.remerge
+                                   else "eager pass, CUDA events around each call")}
+    n_dec_launch = rn.decode_launches()
+    dec_launch_ms = parts["decode"] / n_dec_launch
     traffic = None
     prof = os.path.join(ROOT, "profiles", "decode_traffic.json")
-    if os.path.exists(prof):
+    if os.path.exists(prof) and w.index == 2:
         # one ncu capture's DRAM bytes per launch, scaled by rows processed to this launch
         # (the capture shows traffic equal to the algorithmic bytes, so it scales in proportion)
         with open(prof) as f:
             tr = json.load(f)
-        traffic = (tr["measured_dram_bytes_per_launch"] * rn.decode_bytes_per_launch()
-                   / tr["measured_algorithmic_bytes_per_launch"])
+        if tr.get("valid", True):          # false once the kernel changed after the capture
+            traffic = (tr["measured_dram_bytes_per_launch"] * rn.decode_bytes_per_launch()
+                       / tr["measured_algorithmic_bytes_per_launch"])
+    dominant = max(rooflines, key=lambda k: rooflines[k]["ms_per_step"])
+    roof = dict(rooflines[dominant])
+    if dominant == "decode":
+        roof.update(traffic=traffic, bytes_per_launch=rn.decode_bytes_per_launch(),
+                    launch_ms=dec_launch_ms)
+    else:
+        roof["traffic"] = None
+    merge_phase_bytes = algo["score"] + algo["merge"]
 
     e2e = None
     if not args.no_e2e:
@@ -618,29 +956,31 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        per_step, spent, threads, sample = oracle_sample(w, rn.layers[0], rn.target, rn.lens_plan)
-        cpu = {"value": rn.tokens_per_step() / per_step, "unit": UNIT, "cores": threads,
-               "kind": "oracle", "sample": sample, "cpu_seconds_spent": round(spent, 2),
-               "host_cpus": os.cpu_count()}
+        cpu = cpu_baseline(w, rn.layers, rn.tokens_per_step())
 
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
             "config": config_of(w, world),
+            "value_note": ("merged KV tokens per second of the whole step: the merge phase "
+                           "(every layer to its budget) plus the decode phase"),
             "merge_ms_per_step": merge_ms, "decode_ms_per_step": decode_ms,
             "merge_tokens_per_s": tokens / (merge_ms / 1e3),
             "decode_us_per_token": decode_ms * 1e3 / w.n_decode,
-            "decode_us_per_token_note": "one generated token = one decode step over all layers",
+            "decode_us_per_token_note": ("one generated token = one decode step over all layers"
+                                         + (", re-merges included" if rn.remerge else "")),
+            "merge_phase": {"algorithmic_bytes": merge_phase_bytes,
+                            "achieved": merge_phase_bytes / (merge_ms / 1e3) / 1e9,
+                            "frac": merge_phase_bytes / (merge_ms / 1e3) / 1e9 / peak,
+                            "unit": "GB/s", "timing": "graph replay, CUDA events"},
             "clocks": clk,
             "e2e": e2e,
             "gpu_launches": (rn.launches_merge + rn.launches_decode) * args.steps,
-            "roofline": {"kernel": "decode_tc_kernel (GQA decode, one thread-block cluster per KV head)", "bound": "hbm",
-                         "achieved": achieved, "peak": peak, "peak_kind": peak_kind,
-                         "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
-                         "bytes_per_launch": rn.decode_bytes_per_launch(),
-                         "launch_ms": dec_launch_ms},
+            "device_flags": flags,
+            "roofline": roof,
+            "rooflines": rooflines,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)

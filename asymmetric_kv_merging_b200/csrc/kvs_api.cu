@@ -87,6 +87,22 @@ inline bool overlap(Range a, Range b) {
   return a.p < b.p + b.n && b.p < a.p + a.n;
 }
 
+// One scoring pass: the two fused tensor-core passes for bf16 caches, else the CUDA-core
+// window statistics followed by the pair-scoring kernel.
+cudaError_t score_pass(const kvs_cache_desc& d, const void* K, const void* V, const float* logn,
+                       const int32_t* len, const int32_t* cand_begin, int n_recent,
+                       const void* Q_win, int W, int form, const ScoreLayout& Ly, char* ws,
+                       float* score, float* w_b, cudaStream_t st) {
+  if (window_fused_supported(d, W))
+    return launch_score_fused(d, K, V, logn, len, cand_begin, n_recent, Q_win, W,
+                              form & KVS_FORM_DIAGONAL, form & KVS_FORM_PER_QUERY, Ly, ws, score,
+                              w_b, st);
+  cudaError_t e = launch_window_stats(d, K, V, logn, len, Q_win, W, Ly, ws, st);
+  if (e != cudaSuccess) return e;
+  return launch_pair_score(d, K, V, len, cand_begin, n_recent, form & KVS_FORM_DIAGONAL, Ly, ws,
+                           score, w_b, st);
+}
+
 kvs_status check_ws(void* ws, size_t ws_bytes, size_t need) {
   if (!ws || !aligned(ws, kWsAlign)) return KVS_ERR_WORKSPACE;
   if (ws_bytes < need) return KVS_ERR_WORKSPACE;
@@ -147,7 +163,7 @@ kvs_status kvs_score_pairs_form(const kvs_cache_desc* desc, const void* K, const
                                 int32_t n_recent, const void* Q_win, int32_t W, float* score,
                                 float* w_b, int32_t form, void* ws, size_t ws_bytes,
                                 kvs_stream_t stream) {
-  if (form != KVS_FORM_FULL && form != KVS_FORM_DIAGONAL) return KVS_ERR_INVALID_ARG;
+  if (form < 0 || form > (KVS_FORM_DIAGONAL | KVS_FORM_PER_QUERY)) return KVS_ERR_INVALID_ARG;
   kvs_status s = check_desc(desc);
   if (s != KVS_OK) return s;
   if (!K || !V || !len || !cand_begin || !Q_win || !score || !w_b) return KVS_ERR_INVALID_ARG;
@@ -166,12 +182,12 @@ kvs_status kvs_score_pairs_form(const kvs_cache_desc* desc, const void* K, const
   const ScoreLayout Ly = score_layout(*desc, W);
   s = check_ws(ws, ws_bytes, Ly.total);
   if (s != KVS_OK) return s;
+  const bool fused = window_fused_supported(*desc, W);
+  if ((form & KVS_FORM_PER_QUERY) && !fused) return KVS_ERR_UNSUPPORTED;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   char* w = static_cast<char*>(ws);
-  cudaError_t e = launch_window_stats(*desc, K, V, logn, len, Q_win, W, Ly, w, st);
-  if (e != cudaSuccess) return KVS_ERR_CUDA;
-  e = launch_pair_score(*desc, K, V, len, cand_begin, n_recent, form, Ly, w, score, w_b, st);
-  return from_cuda(e);
+  return from_cuda(score_pass(*desc, K, V, logn, len, cand_begin, n_recent, Q_win, W, form, Ly,
+                              w, score, w_b, st));
 }
 
 kvs_status kvs_merge_compact(const kvs_cache_desc* desc, const void* K, const void* V,
@@ -272,7 +288,8 @@ kvs_status kvs_prefill_chunk(const kvs_cache_desc* desc, void* K, void* V, float
   if (s != KVS_OK) return s;
   if (!K || !V || !logn || !len || !Q_win || !L_out || (n > 0 && (!k_chunk || !v_chunk)))
     return KVS_ERR_INVALID_ARG;
-  if (form != KVS_FORM_FULL && form != KVS_FORM_DIAGONAL) return KVS_ERR_INVALID_ARG;
+  if (form < 0 || form > (KVS_FORM_DIAGONAL | KVS_FORM_PER_QUERY)) return KVS_ERR_INVALID_ARG;
+  if ((form & KVS_FORM_PER_QUERY) && !window_fused_supported(*desc, W)) return KVS_ERR_UNSUPPORTED;
   if (!aligned(K, 16) || !aligned(V, 16) || !aligned(Q_win, 16) || !aligned(logn, 4) ||
       !aligned(len, 4) || (n > 0 && (!aligned(k_chunk, 16) || !aligned(v_chunk, 16))))
     return KVS_ERR_INVALID_ARG;
@@ -324,9 +341,7 @@ kvs_status kvs_prefill_chunk(const kvs_cache_desc* desc, void* K, void* V, float
     if (e != cudaSuccess) return KVS_ERR_CUDA;
   }
   for (int r = 0; r < rounds; ++r) {
-    e = launch_window_stats(*desc, K, V, logn, len, Q_win, W, Ly.score, w, st);
-    if (e != cudaSuccess) return KVS_ERR_CUDA;
-    e = launch_pair_score(*desc, K, V, len, cand, W, form, Ly.score, w, score, w_b, st);
+    e = score_pass(*desc, K, V, logn, len, cand, W, Q_win, W, form, Ly.score, w, score, w_b, st);
     if (e != cudaSuccess) return KVS_ERR_CUDA;
     e = launch_select(*desc, score, len, cand, W, target, KVS_SCOPE_HEAD, Ly.merge, w, st);
     if (e != cudaSuccess) return KVS_ERR_CUDA;

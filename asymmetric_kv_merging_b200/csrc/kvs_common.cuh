@@ -118,7 +118,7 @@ struct HeadInfo {      // one (b, h)
 };
 
 struct ScoreLayout {
-  size_t part_ml, part_o, stats, obar, alpha, total;
+  size_t part_ml, part_o, stats, obar, alpha, oq_hi, oq_lo, on2, total;
   int nsplit, Qn;
 };
 struct MergeLayout {
@@ -174,7 +174,12 @@ inline ScoreLayout score_layout(const kvs_cache_desc& d, int W) {
   L.stats = align_up(L.part_o + units * L.nsplit * L.Qn * (size_t)d.d * sizeof(float), kWsAlign);
   L.obar = align_up(L.stats + units * L.Qn * 2 * sizeof(float), kWsAlign);
   L.alpha = align_up(L.obar + units * (size_t)d.d * sizeof(float), kWsAlign);
-  L.total = align_up(L.alpha + units * (size_t)d.T_cap * sizeof(float), kWsAlign);
+  // window outputs o_q of the bf16 path: rows of 128 (padded) queries per head, as
+  // bf16 hi / lo parts, and their squared norms
+  L.oq_hi = align_up(L.alpha + units * (size_t)d.T_cap * sizeof(float), kWsAlign);
+  L.oq_lo = align_up(L.oq_hi + units * 128 * (size_t)d.d * 2, kWsAlign);
+  L.on2 = align_up(L.oq_lo + units * 128 * (size_t)d.d * 2, kWsAlign);
+  L.total = align_up(L.on2 + units * 128 * sizeof(float), kWsAlign);
   return L;
 }
 

@@ -64,6 +64,16 @@ cudaError_t launch_window_stats_tc(const kvs_cache_desc& d, const void* K, const
                                    const float* logn, const int32_t* len, const void* Qw, int W,
                                    const ScoreLayout& Ly, char* ws, cudaStream_t st);
 
+// Window statistics and pair scores for bf16 caches in two fused tensor-core passes
+// (G*W <= 128): form is KVS_FORM_FULL or KVS_FORM_DIAGONAL; stats_form is 0 (window
+// mean) or KVS_FORM_PER_QUERY.
+bool window_fused_supported(const kvs_cache_desc& d, int W);
+cudaError_t launch_score_fused(const kvs_cache_desc& d, const void* K, const void* V,
+                               const float* logn, const int32_t* len, const int32_t* cand_begin,
+                               int n_recent, const void* Qw, int W, int form, int stats_form,
+                               const ScoreLayout& Ly, char* ws, float* score, float* w_b,
+                               cudaStream_t st);
+
 // The same step for bf16 caches on the TMA + tensor-core kernel.
 bool decode_tc_supported(const kvs_cache_desc& d);
 cudaError_t launch_decode_tc(const kvs_cache_desc& d, const void* q, void* K, void* V, float* logn,

@@ -23,7 +23,7 @@ _lib = ctypes.CDLL(_LIB_PATH)
 F32, BF16 = 0, 1
 OP_SCORE, OP_MERGE, OP_DECODE, OP_PREFILL = 0, 1, 2, 3
 SCOPE_HEAD, SCOPE_POOLED = 0, 1
-FORM_FULL, FORM_DIAGONAL = 0, 1
+FORM_FULL, FORM_DIAGONAL, FORM_PER_QUERY = 0, 1, 2
 FLAG_BAD_LENGTH, FLAG_OUT_CAPACITY, FLAG_INPLACE_SPAN, FLAG_NONFINITE_STATS = 1, 2, 4, 8
 FLAG_TIMEOUT, FLAG_BUDGET = 16, 32
 

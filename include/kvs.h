@@ -73,8 +73,10 @@ typedef struct CUstream_st* kvs_stream_t; /* a cudaStream_t; NULL = legacy defau
 
 enum { KVS_OP_SCORE = 0, KVS_OP_MERGE = 1, KVS_OP_DECODE = 2, KVS_OP_PREFILL = 3 };
 enum { KVS_SCOPE_HEAD = 0, KVS_SCOPE_POOLED = 1 };
-/* Scoring form: the coupled forward-only objective, or its diagonal-only ablation. */
-enum { KVS_FORM_FULL = 0, KVS_FORM_DIAGONAL = 1 };
+/* Scoring form: the coupled forward-only objective, or its diagonal-only ablation;
+   either may be combined (bitwise or) with KVS_FORM_PER_QUERY, the per-query window
+   reading (see kvs_score_pairs_form). */
+enum { KVS_FORM_FULL = 0, KVS_FORM_DIAGONAL = 1, KVS_FORM_PER_QUERY = 2 };
 
 /* Device flag bits (see kvs_device_flags). */
 enum {
@@ -136,6 +138,16 @@ kvs_status kvs_score_pairs(const kvs_cache_desc* desc, const void* K, const void
  *     w_b = N22 / (N11 + N22),  score = |k_b - k_a|^2 N11 N22 / (N11 + N22),
  *   with the same degenerate rule (w_b = 1/2, score = |k_b - k_a|^2 (N11 + N22) / 4
  *   when N11 + N22 is not positive or a term is not finite).
+ * form | KVS_FORM_PER_QUERY: the window of several queries read per query instead of
+ *   through its mean. The pages derive the norms for one query; here every window query
+ *   q gets its own single-query norms, and the pair's norms are their mean over the
+ *   Qv window queries that see at least one row:
+ *     N11 = mean_q |a_qa (1 - 2 a_qa)| |v_a - o_q|,  N22 likewise,
+ *     N12 = mean_q a_qa a_qb |v_a + v_b - 2 o_q|,
+ *   a_qt = softmax_t(q k_t^T / sqrt(d) + logn_t), o_q = sum_t a_qt v_t (the causal window
+ *   as above); weight, score and degenerate rule as for the base form. For one window
+ *   query it equals the base form. Built for bf16 caches with G*W <= 128 only (else
+ *   KVS_ERR_UNSUPPORTED, nothing launched).
  * Any other form: KVS_ERR_INVALID_ARG, nothing launched. Arguments, outputs,
  * workspace and errors otherwise as kvs_score_pairs.
  */

@@ -119,15 +119,24 @@ def gpu_round(cache: GpuCache, H_q, Q_win, W, cand_begin, n_recent, target, scop
                      off=off.cpu().long(), km=km.cpu().double())
 
 
+def _rows(cache: GpuCache, bs):
+    """fp64 copies of sequences `bs` of a device cache, trimmed to their longest head:
+    (K, V, logn, lens)."""
+    B, H = cache.K.shape[:2]
+    lens = cache.lens.view(B, H).cpu().numpy()[bs]
+    n = max(1, int(lens.max(initial=0)))
+    idx = torch.tensor(bs, dtype=torch.long, device=cache.K.device)
+    K = cache.K.index_select(0, idx)[:, :, :n].double().cpu().numpy()
+    V = cache.V.index_select(0, idx)[:, :, :n].double().cpu().numpy()
+    ln = cache.logn.index_select(0, idx)[:, :, :n].double().cpu().numpy()
+    return K, V, ln, lens
+
+
 def to_oracle_cache(cache: GpuCache, batch=None):
     """Copy (sequences `batch` of) a device cache to an oracle Cache (fp64)."""
-    K = cache.K.double().cpu().numpy()
-    V = cache.V.double().cpu().numpy()
-    ln = cache.logn.double().cpu().numpy()
-    B, H = K.shape[:2]
-    lens = cache.lens.view(B, H).cpu().numpy()
-    bs = list(range(B)) if batch is None else list(batch)
-    return oracle.cache_from_arrays(K[bs], V[bs], lens[bs], ln[bs])
+    bs = list(range(cache.K.shape[0])) if batch is None else list(batch)
+    K, V, ln, lens = _rows(cache, bs)
+    return oracle.cache_from_arrays(K, V, lens, ln)
 
 
 def _nan_inf(x):
@@ -204,10 +213,8 @@ def compare_round(r, g, out: GpuCache, oin, dtype, scope="head", batch_map=None,
     storage = storage_of(dtype)
     B_o = len(r.scores)
     H = len(r.scores[0])
-    Kg = out.K.double().cpu().numpy()
-    Vg = out.V.double().cpu().numpy()
-    Lg = out.logn.double().cpu().numpy()
-    lens_g = out.lens.view(out.K.shape[0], H).cpu().numpy()
+    gb = [bo if batch_map is None else batch_map[bo] for bo in range(B_o)]
+    Kg, Vg, Lg, lens_g = _rows(out, gb)           # indexed by the oracle's sequence index
     stats.rounds += 1
     # selection per unit: differences only near the threshold, same count per unit
     sel_g_all = {}
@@ -258,16 +265,16 @@ def compare_round(r, g, out: GpuCache, oin, dtype, scope="head", batch_map=None,
             else:   # near-threshold swap: the oracle's merge of the GPU's selection
                 m = oracle.merge_compact_head(Kin, Vin, oin.log_n[bo][h], L_in, c0, n_recent,
                                               sel_g, hs.w_b, storage)
-            assert lens_g[bg, h] == m.length, (bg, h, lens_g[bg, h], m.length)
+            assert lens_g[bo, h] == m.length, (bg, h, lens_g[bo, h], m.length)
             np.testing.assert_array_equal(g["off"][bg, h, :P].numpy(), m.out_offset,
                                           err_msg=f"offsets b={bg} h={h}")
             n = m.length
             merged = np.zeros(n, bool)
             merged[m.out_offset[sel_g]] = True
-            kg, vg = Kg[bg, h, :n], Vg[bg, h, :n]
+            kg, vg = Kg[bo, h, :n], Vg[bo, h, :n]
             np.testing.assert_array_equal(kg[~merged], m.K[~merged], err_msg=f"K copy b={bg} h={h}")
             np.testing.assert_array_equal(vg[~merged], m.V[~merged], err_msg=f"V copy b={bg} h={h}")
-            np.testing.assert_allclose(Lg[bg, h, :n], m.log_n, rtol=0, atol=2e-6,
+            np.testing.assert_allclose(Lg[bo, h, :n], m.log_n, rtol=0, atol=2e-6,
                                        err_msg=f"logn b={bg} h={h}")
             if storage == "bf16":
                 np.testing.assert_allclose(kg[merged], m.K[merged], rtol=2e-2, atol=1e-2)

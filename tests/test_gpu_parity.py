@@ -53,7 +53,8 @@ def compress_both(kvs, w, li, batch=None, ratio=None, stats=None, Q_override=Non
     Qo = Q.double().cpu().numpy()[batch]
     ws = _workspace(kvs, B, H, w.H_q, d, T_cap, li.K.dtype, w.W)
     stats = stats or Stats()
-    form_name = "diagonal" if form == kvs.FORM_DIAGONAL else "full"
+    form_name = "diagonal" if (form or 0) & kvs.FORM_DIAGONAL else "full"
+    stats_name = "per_query" if (form or 0) & kvs.FORM_PER_QUERY else "mean"
     for _ in range(16):
         cur = g.lens.view(B, H).cpu().numpy()
         done = (cur.sum(axis=1) <= target_np) if scope == "pooled" else (cur <= target_np)
@@ -61,7 +62,7 @@ def compress_both(kvs, w, li, batch=None, ratio=None, stats=None, Q_override=Non
             break
         o = to_oracle_cache(g, batch)
         r = oracle.merge_round(o, Qo, w.W, cand_np, w.W, target_np[batch], scope,
-                               storage_of(li.K.dtype), form_name)
+                               storage_of(li.K.dtype), form_name, stats_name)
         gout, gres = gpu_round(g, w.H_q, Q, w.W, cand, w.W, target, scope_code, ws, form=form)
         compare_round(r, gres, gout, o, li.K.dtype, scope, batch, stats, cand_np, w.W, form_name)
         g = gout
@@ -151,18 +152,22 @@ def planted_sinks(w, plants, layer=0):
                               v_new=li.v_new)
 
 
-def test_peaked_attention_exercises_degenerate_pairs(kvs):
+@pytest.mark.parametrize("dtype,d,form", [("f32", 64, None), ("bf16", 128, None),
+                                          ("bf16", 128, "per_query")])
+def test_peaked_attention_exercises_degenerate_pairs(kvs, dtype, d, form):
     """Planted attention sinks: a pair at alpha_bar ~ 0.35 per row (D < 0, the
     plain-average branch) in KV head 0 and a row at alpha_bar ~ 0.7 (> 1/2) in KV head 1.
-    Both must occur in the oracle's scoring, and the GPU must agree on them."""
-    w = inputs.small_workload(inputs.workload(0), T=192, n_decode=2)
+    Both must occur in the oracle's scoring, and the GPU must agree on them: fp32 on the
+    CUDA-core window path, bf16 on the tensor-core passes (window mean and per query)."""
+    w = inputs.small_workload(inputs.workload(0), T=192, n_decode=2, dtype=dtype, d=d)
     li = planted_sinks(w, [(0, (52, 53), 0.35), (1, (60,), 0.7)])
+    code = kvs.FORM_FULL | (kvs.FORM_PER_QUERY if form == "per_query" else 0)
     stats = Stats()
-    g, o, stats, ws = compress_both(kvs, w, li, stats=stats)
+    g, o, stats, ws = compress_both(kvs, w, li, stats=stats, form=code)
     g, o = decode_both(kvs, w, li, g, o, range(w.n_decode), stats=stats, ws=ws)
-    stats.report("planted sinks (degenerate branch, alpha > 1/2)")
+    stats.report(f"planted sinks {dtype} d={d} {form or 'mean'} (degenerate branch, alpha > 1/2)")
     assert stats.degenerate_pairs >= 1
-    assert stats.alpha_over_half >= 2
+    assert stats.alpha_over_half >= 2 or form == "per_query"
 
 
 # --------------------------------------------------------------------------- workload 1
@@ -189,6 +194,35 @@ def test_diagonal_form_pipeline(kvs, wl):
     stats.report(f"diagonal form workload{wl}")
     assert stats.scores_compared > 0
     assert stats.near_threshold <= 8
+
+
+@pytest.mark.parametrize("wl,T,H_kv", [(1, 4096, 2), (1, 32768, 8)])
+def test_per_query_window_form(kvs, wl, T, H_kv):
+    """kvs_score_pairs_form with KVS_FORM_PER_QUERY (the window read query by query: the
+    one-query norms of every window query, averaged) against the oracle's per-query
+    statistics, every round, then decode."""
+    w = inputs.small_workload(inputs.workload(wl), T=T, H_kv=H_kv, H_q=4 * H_kv, n_decode=4)
+    li = inputs.make_layer(w, 0, device="cuda")
+    g, o, stats, ws = compress_both(kvs, w, li, form=kvs.FORM_FULL | kvs.FORM_PER_QUERY)
+    g, o = decode_both(kvs, w, li, g, o, range(w.n_decode), stats=stats, ws=ws)
+    stats.report(f"per-query window form T={T} H_kv={H_kv}")
+    assert stats.scores_compared > 0
+    assert stats.near_threshold <= 8
+
+
+def test_per_query_form_needs_the_tensor_core_path(kvs):
+    dev = torch.device("cuda")
+    desc = kvs.make_desc(1, 2, 4, 64, 256, torch.float32)
+    K = torch.randn(1, 2, 256, 64, device=dev)
+    lens = torch.full((2,), 200, dtype=torch.int32, device=dev)
+    cand = torch.full((2,), 32, dtype=torch.int32, device=dev)
+    Q = torch.randn(1, 4, 32, 64, device=dev)
+    score = torch.zeros(1, 2, 128, device=dev)
+    ws = kvs.workspace(desc, 32)
+    with pytest.raises(kvs.KvsError) as e:
+        kvs.score_pairs(desc, K, K, None, lens, cand, 32, Q, 32, score, score.clone(), ws,
+                        form=kvs.FORM_PER_QUERY)
+    assert e.value.status == 2                  # KVS_ERR_UNSUPPORTED, nothing launched
 
 
 def test_score_form_rejects_unknown_form(kvs):
@@ -508,5 +542,7 @@ def test_bad_length_and_capacity_flags(kvs):
     target = torch.tensor([120, 50], dtype=torch.int32, device=dev)
     kvs.merge_compact(desc, K, V, None, lens, cand, 32, score, w_b, target, kvs.SCOPE_HEAD, 96,
                       Ko, Vo, lno, lo, ws)
-    assert kvs.device_flags(ws, clear=True) == kvs.FLAG_OUT_CAPACITY
+    # head 0 does not fit; head 1's target (50) is below the 65 rows its 36-row span can
+    # reach by repeated rounds
+    assert kvs.device_flags(ws, clear=True) == kvs.FLAG_OUT_CAPACITY | kvs.FLAG_BUDGET
     assert int(lo[1]) == 82   # head 1: 100 rows, all 18 pairs merged

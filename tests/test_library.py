@@ -149,7 +149,7 @@ def _prefill(kvs, desc, **over):
 def test_prefill_chunk_host_validation_and_plan(kvs):
     d = kvs.make_desc(1, 8, 32, 128, 4096, kvs.BF16)
     assert _prefill(kvs, d, logn=None)[0] == 1                         # counts are required
-    assert _prefill(kvs, d, form=2)[0] == 1
+    assert _prefill(kvs, d, form=4)[0] == 1                            # unknown form bits
     assert _prefill(kvs, d, L=3800, n=512)[0] == 1                     # L + n > T_cap
     assert _prefill(kvs, d, W=33)[0] == 2                              # G*W > 128
     big = kvs.make_desc(1, 8, 32, 128, 16384, kvs.BF16)

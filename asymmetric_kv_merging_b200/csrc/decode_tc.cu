@@ -65,8 +65,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
                  const __grid_constant__ CUtensorMap tmL, int ln_lead,
                  const bf16* __restrict__ q, bf16* K, bf16* V, float* logn, int32_t* len,
                  const bf16* __restrict__ k_new, const bf16* __restrict__ v_new,
-                 bf16* __restrict__ out, int T_cap, int nsplit, int32_t* counters, float* part,
-                 int32_t* flags) {
+                 bf16* __restrict__ out, int T_cap, int nsplit, int csize, int32_t* counters,
+                 float* part, int32_t* flags) {
   using S = TcShape<D, NC, STAGES, kCluster ? 1 : 0>;
   constexpr int kTile = S::kTile, kThreads = S::kThreads;
   static_assert(NC * G * D * 4 <= S::kRingBytes, "warp partials fit the ring");
@@ -145,10 +145,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
   if (kCluster && warp == NC + 1) {
     // ---------------- warm-up: the combine's code, dry, while the others stream ----
     if constexpr (kCluster)
-      cluster_combine<bf16, D, G, NC>(s_m, s_l, s_acc, qs, &s_cml[0][0], s_new, &s_inbox[1], nsplit,
+      cluster_combine<bf16, D, G, NC>(s_m, s_l, s_acc, qs, &s_cml[0][0], s_new, &s_inbox[1], csize,
                                       (int)cluster_ctarank(), lane, 32, /*dry=*/true, 0, L, T_cap,
                                       append, K, V, logn, len, s_kvnew[0], s_kvnew[kCluster ? 1 : 0],
-                                      reinterpret_cast<bf16*>(&s_inbox[1]), flags);
+                                      reinterpret_cast<bf16*>(&s_inbox[1]), flags, 1, 0, nullptr,
+                                      nullptr, nullptr);
   } else if (warp == NC) {
     // ---------------- producer: one thread issues every TMA load ----------------
     if (lane == 0) {
@@ -316,10 +317,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
   const DecodeArgs<bf16> a{head, split, nsplit, L, T_cap, bad, K, V, logn, len, k_new, v_new,
                            out, counters, part, flags};
   if constexpr (kCluster) {
-    cluster_combine<bf16, D, G, NC>(s_m, s_l, s_acc, qs, &s_cml[0][0], s_new, &s_inbox[0], nsplit,
+    cluster_combine<bf16, D, G, NC>(s_m, s_l, s_acc, qs, &s_cml[0][0], s_new, &s_inbox[0], csize,
                                     (int)cluster_ctarank(), tid, kThreads, /*dry=*/false, head, L,
                                     T_cap, append, K, V, logn, len, s_kvnew[0],
-                                    s_kvnew[kCluster ? 1 : 0], out, flags);
+                                    s_kvnew[kCluster ? 1 : 0], out, flags, nsplit / csize,
+                                    split / csize, part, counters, &s_last);
   } else {
     decode_epilogue_staged<bf16, D, G, NC>(Sm, base, S::kRingBytes, cbar, a, tid, kThreads);
   }
@@ -381,58 +383,70 @@ bool decode_tc_supported(const kvs_cache_desc& d) {
          tensor_map_encoder() != nullptr;
 }
 
-// Cluster size for a cluster launch over `units` KV heads on the current device, or
-// 0 when the split grid is to be used: the largest C <= 16 with C * units <= SM count
-// for which the occupancy calculator places all `units` clusters at once.
+// Cluster plan for a cluster launch over `units` KV heads on the current device: X
+// clusters of C CTAs per head (X in {1, 2}, 2 <= C <= 16), chosen to stream from as many
+// SMs as possible in one wave -- the largest X * C for which the occupancy calculator
+// places all X * units clusters at once (X = 1 on a tie: no second combine level).
+// C = 0 when no cluster shape fits: the split grid is used.
+struct ClusterPlan {
+  int X, C;
+};
+
 template <int D, int G>
-static int cluster_size_for(int units) {
+static ClusterPlan cluster_plan_for(int units) {
   using CS = ClusterShape<D>;
   auto kfn = decode_tc_kernel<D, G, 8, (D == 64 ? 6 : 3), true>;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return {1, 0};
   static std::mutex mu;
-  static std::map<std::pair<int, int>, int> cache;
+  static std::map<std::pair<int, int>, ClusterPlan> cache;
   std::lock_guard<std::mutex> lock(mu);
   const auto key = std::make_pair(dev, units);
   const auto it = cache.find(key);
   if (it != cache.end()) return it->second;
   int sms = 0;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  int C = units > 0 ? sms / units : 0;
-  if (C > kMaxClusterSize) C = kMaxClusterSize;
-  if (!ensure_smem_attr((const void*)kfn, CS::kSmem)) C = 0;
-  if (C > 8 && !ensure_nonportable_cluster((const void*)kfn)) C = 8;
-  for (; C >= 2; --C) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(C, units);
-    cfg.blockDim = dim3(CS::kThreads);
-    cfg.dynamicSmemBytes = CS::kSmem;
-    cudaLaunchAttribute at[1];
-    at[0].id = cudaLaunchAttributeClusterDimension;
-    at[0].val.clusterDim.x = C;
-    at[0].val.clusterDim.y = 1;
-    at[0].val.clusterDim.z = 1;
-    cfg.attrs = at;
-    cfg.numAttrs = 1;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, (const void*)kfn, &cfg) == cudaSuccess && n >= units) break;
+  ClusterPlan best{1, 0};
+  const bool smem_ok = ensure_smem_attr((const void*)kfn, CS::kSmem);
+  const bool big_ok = smem_ok && ensure_nonportable_cluster((const void*)kfn);
+  for (int X = 1; X <= 2 && smem_ok && units > 0; ++X) {
+    int C = sms / (X * units);
+    if (C > kMaxClusterSize) C = kMaxClusterSize;
+    if (C > 8 && !big_ok) C = 8;
+    for (; C >= 2; --C) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(X * C, units);
+      cfg.blockDim = dim3(CS::kThreads);
+      cfg.dynamicSmemBytes = CS::kSmem;
+      cudaLaunchAttribute at[1];
+      at[0].id = cudaLaunchAttributeClusterDimension;
+      at[0].val.clusterDim.x = C;
+      at[0].val.clusterDim.y = 1;
+      at[0].val.clusterDim.z = 1;
+      cfg.attrs = at;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, (const void*)kfn, &cfg) == cudaSuccess &&
+          n >= X * units)
+        break;
+    }
+    if (C >= 2 && X * C > best.X * best.C) best = {X, C};
   }
   (void)cudaGetLastError();   // a refused query leaves no error behind
-  if (C < 2) C = 0;
-  cache[key] = C;
-  return C;
+  cache[key] = best;
+  return best;
 }
 
 template <int D, int G, int NC, int STAGES, bool kCluster>
 static cudaError_t launch_shape(const kvs_cache_desc& d, const void* q, void* K, void* V,
                                 float* logn, int32_t* len, const void* k_new, const void* v_new,
-                                void* out, int nsplit, const DecodeLayout& Ly, char* ws,
-                                cudaStream_t st) {
+                                void* out, int nsplit, int csize, const DecodeLayout& Ly,
+                                char* ws, cudaStream_t st) {
   using S = TcShape<D, NC, STAGES, kCluster ? 1 : 0>;
   auto kfn = decode_tc_kernel<D, G, NC, STAGES, kCluster>;
   // per device, cached (the first call on a device must precede any capture)
   if (!ensure_smem_attr((const void*)kfn, S::kSmem)) return cudaErrorInvalidValue;
-  if (kCluster && nsplit > 8 && !ensure_nonportable_cluster((const void*)kfn))
+  if (kCluster && csize > 8 && !ensure_nonportable_cluster((const void*)kfn))
     return cudaErrorInvalidValue;
   const unsigned long long rows = (unsigned long long)d.B * d.H_kv * (unsigned long long)d.T_cap;
   CUtensorMap mK, mV, mL;
@@ -454,14 +468,14 @@ static cudaError_t launch_shape(const kvs_cache_desc& d, const void* q, void* K,
   cfg.stream = st;
   cudaLaunchAttribute at[1];
   at[0].id = cudaLaunchAttributeClusterDimension;
-  at[0].val.clusterDim.x = nsplit;
+  at[0].val.clusterDim.x = csize;
   at[0].val.clusterDim.y = 1;
   at[0].val.clusterDim.z = 1;
   cfg.attrs = at;
   cfg.numAttrs = kCluster ? 1 : 0;
   const cudaError_t e = cudaLaunchKernelEx(
       &cfg, kfn, mK, mV, mL, ln_lead, (const bf16*)q, (bf16*)K, (bf16*)V, logn, len, (const bf16*)k_new,
-      (const bf16*)v_new, (bf16*)out, d.T_cap, nsplit,
+      (const bf16*)v_new, (bf16*)out, d.T_cap, nsplit, csize,
       reinterpret_cast<int32_t*>(ws + Ly.counters), reinterpret_cast<float*>(ws + Ly.part),
       reinterpret_cast<int32_t*>(ws));
   count_launches(1);
@@ -472,12 +486,12 @@ template <int D, int G>
 static cudaError_t launch_tc(const kvs_cache_desc& d, const void* q, void* K, void* V,
                              float* logn, int32_t* len, const void* k_new, const void* v_new,
                              void* out, const DecodeLayout& Ly, char* ws, cudaStream_t st) {
-  const int C = cluster_size_for<D, G>(d.B * d.H_kv);
-  if (C >= 2)
+  const ClusterPlan cp = cluster_plan_for<D, G>(d.B * d.H_kv);
+  if (cp.C >= 2)
     return launch_shape<D, G, 8, (D == 64 ? 6 : 3), true>(d, q, K, V, logn, len, k_new, v_new, out,
-                                                          C, Ly, ws, st);
-  return launch_shape<D, G, 4, 3, false>(d, q, K, V, logn, len, k_new, v_new, out, Ly.nsplit, Ly,
-                                         ws, st);
+                                                          cp.X * cp.C, cp.C, Ly, ws, st);
+  return launch_shape<D, G, 4, 3, false>(d, q, K, V, logn, len, k_new, v_new, out, Ly.nsplit, 0,
+                                         Ly, ws, st);
 }
 
 cudaError_t launch_decode_tc(const kvs_cache_desc& d, const void* q, void* K, void* V, float* logn,

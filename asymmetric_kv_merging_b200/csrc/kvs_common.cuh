@@ -157,11 +157,12 @@ inline int decode_splits(const kvs_cache_desc& d) {
 }
 
 // Every layout starts with the same persistent region: the device flag word in the
-// first 256 bytes, then one arrival counter per KV head for the decode combine. No
+// first 256 bytes, then kMaxClusterSize arrival counters per KV head for the decode
+// combine (the split grid uses the first, a two-cluster launch one per slice owner). No
 // op writes this region except through its own flags / counters, so one zeroed
 // workspace can be shared by all ops on a stream.
 inline size_t persistent_bytes(const kvs_cache_desc& d) {
-  return kWsAlign + align_up((size_t)d.B * d.H_kv * sizeof(int32_t), kWsAlign);
+  return kWsAlign + align_up((size_t)d.B * d.H_kv * kMaxClusterSize * sizeof(int32_t), kWsAlign);
 }
 
 inline ScoreLayout score_layout(const kvs_cache_desc& d, int W) {
@@ -201,8 +202,11 @@ inline DecodeLayout decode_layout(const kvs_cache_desc& d) {
   L.nsplit = decode_splits(d);
   L.counters = kWsAlign;
   L.part = persistent_bytes(d);
-  L.total = align_up(L.part + qheads * L.nsplit * (size_t)(d.d + kPartPad) * sizeof(float),
-                     kWsAlign);
+  // split partials of the split grid, or the cluster-level partials (M, L, column) of a
+  // launch with two clusters per head
+  const size_t split_part = qheads * L.nsplit * (size_t)(d.d + kPartPad) * sizeof(float);
+  const size_t cluster_part = qheads * 2 * (size_t)d.d * 3 * sizeof(float);
+  L.total = align_up(L.part + (split_part > cluster_part ? split_part : cluster_part), kWsAlign);
   return L;
 }
 

@@ -8,7 +8,8 @@
 //
 // select_kernel (one CTA per selection unit):
 //   R = min(P, max(0, len - target)); the threshold key is the R-th smallest
-//   (score_key, index) found by a 4-pass 8-bit radix select; then per block of
+//   (score_key, index), found by a radix select (a 12-bit histogram pass over the
+//   scores, then the threshold bin's keys resolved in shared memory); then per block of
 //   kMergePairsPerBlock pairs the counts of keys below / equal to the threshold,
 //   exclusive-scanned in unit order (h, p), give every merge CTA its offsets.
 // merge_kernel (out-of-place): one CTA per (head, pair block) plus copy CTAs for
@@ -24,6 +25,7 @@
 namespace kvs {
 
 constexpr int kSelThreads = 1024;
+constexpr int kSelCand = 6144;   // threshold-bin keys resolved in shared memory
 constexpr int kMergeThreads = 256;
 constexpr int kCopyRows = 256;
 // Pairs staged per in-place step: 32 for rows up to 256 bytes, 16 for 512-byte rows
@@ -71,9 +73,10 @@ select_kernel(const float* __restrict__ score, const int32_t* __restrict__ len,
               const int32_t* __restrict__ target, int scope, int H_kv, int T_cap, int nblk,
               SelUnit* __restrict__ sel, HeadInfo* __restrict__ hinfo, int2* __restrict__ blk,
               int32_t* __restrict__ flags) {
-  __shared__ int hist[256];
+  __shared__ int hist[4096];
+  __shared__ uint32_t cand[kSelCand];
   __shared__ int warp_tot[33];
-  __shared__ int s_digit, s_before, s_R, s_P, s_bad;
+  __shared__ int s_digit, s_before, s_R, s_P, s_bad, s_ncand;
   const int u = blockIdx.x, tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
   const int nh = scope == KVS_SCOPE_POOLED ? H_kv : 1;
@@ -123,11 +126,15 @@ select_kernel(const float* __restrict__ score, const int32_t* __restrict__ len,
     thr = 0xffffffffu;
     need_eq = 0;
   } else {
+    // Radix select of the R-th smallest key: a 12-bit histogram of every key, then the
+    // keys of the threshold's bin are gathered into shared memory (when they fit) and
+    // their remaining 20 bits are resolved there in two 10-bit passes; otherwise the
+    // remaining bits take three more passes over the scores (8, 8 and 4 bits).
     uint32_t prefix = 0u, pmask = 0u;
     int rank = R;   // 1-based rank of the threshold among the unit's keys
-    for (int pass = 0; pass < 4; ++pass) {
-      const int shift = 24 - 8 * pass;
-      for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0;
+    auto global_pass = [&](int shift, int bits) {
+      const int nb = 1 << bits;
+      for (int i = tid; i < nb; i += kSelThreads) hist[i] = 0;
       __syncthreads();
       for (int i = 0; i < nh; ++i) {
         const int hh = h_first + i;
@@ -148,38 +155,81 @@ select_kernel(const float* __restrict__ score, const int32_t* __restrict__ len,
             const bool in = p < P;
             const uint32_t key = in ? score_key(v[k]) : 0u;
             const bool match = in && ((key & pmask) == prefix);
-            const unsigned dg = (key >> shift) & 255u;
+            const unsigned dg = (key >> shift) & (unsigned)(nb - 1);
             // aggregate equal digits inside the warp before the shared atomic
-            const unsigned peers = __match_any_sync(0xffffffffu, match ? dg : 0x100u + lane);
+            const unsigned peers = __match_any_sync(0xffffffffu, match ? dg : 0x10000u + lane);
             if (match && (__ffs(peers) - 1) == lane) atomicAdd(&hist[dg], __popc(peers));
           }
         }
       }
       __syncthreads();
-      if (warp == 0) {
-        int c[8], sum = 0;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) { c[k] = hist[lane * 8 + k]; sum += c[k]; }
-        int incl = sum;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          int n = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += n;
-        }
-        const int excl = incl - sum;
-        if (excl < rank && rank <= incl) {
-          int acc = excl;
-          for (int k = 0; k < 8; ++k) {
-            if (rank <= acc + c[k]) { s_digit = lane * 8 + k; s_before = acc; break; }
-            acc += c[k];
-          }
+    };
+    // the digit whose bin holds rank `rank` among nb bins; updates prefix, pmask, rank
+    auto pick = [&](int shift, int bits) {
+      const int nb = 1 << bits;
+      const int per = nb > kSelThreads ? nb / kSelThreads : 1;
+      int sum = 0;
+      if (tid * per < nb)
+        for (int k = 0; k < per; ++k) sum += hist[tid * per + k];
+      int total;
+      const int excl = block_excl_scan(sum, warp_tot, total);
+      if (tid * per < nb && excl < rank && rank <= excl + sum) {
+        int acc = excl;
+        for (int k = 0; k < per; ++k) {
+          const int c = hist[tid * per + k];
+          if (rank <= acc + c) { s_digit = tid * per + k; s_before = acc; break; }
+          acc += c;
         }
       }
       __syncthreads();
       prefix |= (uint32_t)s_digit << shift;
-      pmask |= 0xffu << shift;
+      pmask |= (uint32_t)(nb - 1) << shift;
       rank -= s_before;
+      const int in_bin = hist[s_digit];
       __syncthreads();
+      return in_bin;
+    };
+    global_pass(20, 12);
+    const int in_bin = pick(20, 12);
+    if (in_bin <= kSelCand) {
+      // gather the bin's keys
+      if (tid == 0) s_ncand = 0;
+      __syncthreads();
+      for (int i = 0; i < nh; ++i) {
+        const int hh = h_first + i;
+        const int P = hinfo[hh].P;
+        const float* sc = score + (size_t)hh * pstride;
+        for (int p0 = 0; p0 < P; p0 += kSelThreads) {
+          const int p = p0 + tid;
+          const uint32_t key = p < P ? score_key(sc[p]) : 0u;
+          const bool match = p < P && (key & pmask) == prefix;
+          const unsigned ball = __ballot_sync(0xffffffffu, match);
+          int base = 0;
+          if (lane == 0 && ball) base = atomicAdd(&s_ncand, __popc(ball));
+          base = __shfl_sync(0xffffffffu, base, 0);
+          if (match) cand[base + __popc(ball & ((1u << lane) - 1u))] = key;
+        }
+      }
+      __syncthreads();
+      const int nc = s_ncand;
+      for (int pass = 0; pass < 2; ++pass) {
+        const int shift = pass == 0 ? 10 : 0;
+        for (int i = tid; i < 1024; i += kSelThreads) hist[i] = 0;
+        __syncthreads();
+        for (int i = tid; i < nc; i += kSelThreads) {
+          const uint32_t key = cand[i];
+          if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 1023u], 1);
+        }
+        __syncthreads();
+        pick(shift, 10);
+      }
+    } else {
+      global_pass(12, 8);
+      pick(12, 8);
+      global_pass(4, 8);
+      pick(4, 8);
+      global_pass(0, 4);
+      pick(0, 4);
     }
     thr = prefix;
     need_eq = rank;

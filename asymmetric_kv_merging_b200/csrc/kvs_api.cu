@@ -376,6 +376,19 @@ kvs_status kvs_decode_attn(const kvs_cache_desc* desc, const void* q, void* K, v
                                  static_cast<char*>(ws), st));
 }
 
+kvs_status kvs_stream_read(const void* buf, int64_t rows, int32_t d, int32_t ctas, void* ws,
+                           size_t ws_bytes, kvs_stream_t stream) {
+  if (!buf || !aligned(buf, 16) || rows <= 0 || rows >= (1ll << 31) || ctas <= 0 ||
+      ctas > 65535)
+    return KVS_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return KVS_ERR_UNSUPPORTED;
+  kvs_status s = check_ws(ws, ws_bytes, kWsAlign);
+  if (s != KVS_OK) return s;
+  if (!tensor_map_encoder()) return KVS_ERR_UNSUPPORTED;
+  return from_cuda(launch_stream_probe(buf, rows, d, ctas, static_cast<char*>(ws),
+                                       reinterpret_cast<cudaStream_t>(stream)));
+}
+
 kvs_status kvs_device_flags(void* ws, int32_t* flags, int32_t clear, kvs_stream_t stream) {
   if (!ws || !flags || !aligned(ws, kWsAlign)) return KVS_ERR_INVALID_ARG;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

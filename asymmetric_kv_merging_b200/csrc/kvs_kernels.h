@@ -80,4 +80,9 @@ cudaError_t launch_decode_tc(const kvs_cache_desc& d, const void* q, void* K, vo
                              int32_t* len, const void* k_new, const void* v_new, void* out,
                              const DecodeLayout& Ly, char* ws, cudaStream_t st);
 
+// Measurement helper: stream `rows` rows of a [rows, d] bf16 array through shared
+// memory with the decode kernel's TMA pattern on `ctas` CTAs, computing nothing.
+cudaError_t launch_stream_probe(const void* buf, long long rows, int d, int ctas, char* ws,
+                                cudaStream_t st);
+
 }  // namespace kvs

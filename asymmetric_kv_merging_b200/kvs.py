@@ -33,7 +33,8 @@ STATUS = {0: "KVS_OK", 1: "KVS_ERR_INVALID_ARG", 2: "KVS_ERR_UNSUPPORTED", 3: "K
 EXPORTS = ("kvs_workspace_size", "kvs_score_pairs", "kvs_merge_compact", "kvs_decode_attn",
            "kvs_device_flags", "kvs_status_str", "kvs_version", "kvs_launch_count",
            "kvs_decode_attn_static", "kvs_static_scratch_bytes", "kvs_score_pairs_form",
-           "kvs_prefill_chunk", "kvs_plan_rounds", "kvs_static_device_flags")
+           "kvs_prefill_chunk", "kvs_plan_rounds", "kvs_static_device_flags",
+           "kvs_stream_read")
 
 
 class CacheDesc(ctypes.Structure):
@@ -76,6 +77,8 @@ _lib.kvs_decode_attn_static.restype = ctypes.c_int
 _lib.kvs_decode_attn_static.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 _lib.kvs_static_scratch_bytes.restype = _sz
 _lib.kvs_device_flags.restype = ctypes.c_int
+_lib.kvs_stream_read.restype = ctypes.c_int
+_lib.kvs_stream_read.argtypes = [_vp, ctypes.c_int64, _i32, _i32, _vp, _sz, _vp]
 _lib.kvs_static_device_flags.restype = ctypes.c_int
 _lib.kvs_static_device_flags.argtypes = [ctypes.POINTER(_i32), _i32, _vp]
 _lib.kvs_device_flags.argtypes = [_vp, ctypes.POINTER(_i32), _i32, _vp]
@@ -203,6 +206,13 @@ def static_device_flags(clear: bool = False, stream=None) -> int:
     _check(_lib.kvs_static_device_flags(ctypes.byref(out), int(bool(clear)), _stream(stream)),
            "kvs_static_device_flags")
     return int(out.value)
+
+
+def stream_read(buf: torch.Tensor, d: int, ctas: int, ws: torch.Tensor, stream=None):
+    """kvs_stream_read: stream a bf16 [rows, d] buffer with the decode's loads (timing
+    helper)."""
+    _check(_lib.kvs_stream_read(_ptr(buf), buf.numel() // d, int(d), int(ctas), _ptr(ws),
+                                ws.numel(), _stream(stream)), "kvs_stream_read")
 
 
 def static_scratch_bytes() -> int:

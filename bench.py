@@ -51,6 +51,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--prefill", action="store_true",
                     help="time chunked streaming prefill compression instead (own JSON line)")
+    ap.add_argument("--stream-ceiling", action="store_true",
+                    help="time the decode's read pattern with no arithmetic (own JSON line)")
     return ap.parse_args()
 
 
@@ -842,6 +844,48 @@ def prefill_main(args, rank, world, local):
             "clocks": clk}))
 
 
+def stream_ceiling_main(args, rank, world, local):
+    """The read ceiling of one decode launch of the workload (kvs_stream_read): the bytes
+    one launch reads (every cached K and V row of every head, plus the appended row), as
+    rows of d bf16, streamed with the decode kernel's TMA loads on 80 to 148 CTAs and no
+    arithmetic. Eight such buffers are rotated, so that no launch finds its rows in L2.
+    One line per CTA count: the time a decode launch would take with free arithmetic."""
+    from asymmetric_kv_merging_b200 import kvs
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = inputs.workload(args.workload)
+    target = w.T // w.ratio
+    rows_per_launch = int(w.B * w.H_kv * (target + (w.n_decode + 1) / 2.0) * 2)   # K and V rows
+    bytes_per_launch = rows_per_launch * w.d * 2
+    bufs = [torch.zeros(rows_per_launch, w.d, dtype=torch.bfloat16, device=dev) for _ in range(8)]
+    ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    peak, peak_kind = peaks()
+    stream = torch.cuda.Stream(dev)
+    out = []
+    for ctas in (80, 128, 144, 148):
+        with torch.cuda.stream(stream):
+            for i in range(8 * max(1, args.warmup)):
+                kvs.stream_read(bufs[i % 8], w.d, ctas, ws)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            n = 64 * max(1, args.steps)
+            e0.record(stream)
+            for i in range(n):
+                kvs.stream_read(bufs[i % 8], w.d, ctas, ws)
+            e1.record(stream)
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / n
+        ach = bytes_per_launch / (us / 1e6) / 1e9
+        out.append({"ctas": ctas, "us_per_launch": us, "achieved": ach, "frac": ach / peak})
+    if rank == 0:
+        print(json.dumps({
+            "metric": "decode read ceiling: one decode launch's bytes through the decode's TMA "
+                      "loads with no arithmetic", "unit": "GB/s", "peak": peak,
+            "peak_kind": peak_kind, "bytes_per_launch": bytes_per_launch,
+            "config": {"workload": w.name, "rows_per_launch": rows_per_launch,
+                       "buffers": "8 rotated, each larger than L2"},
+            "device_flags": kvs.device_flags(ws), "by_ctas": out}), flush=True)
+
+
 def prefill_step_bytes(w, c):
     """Algorithmic bytes of one prompt through the chunked prefill, all layers and
     heads of one replica (the per-head accounting of every chunk call)."""
@@ -861,10 +905,10 @@ def main():
     if args.impl == "reference":
         reference_main(args, rank, world)
         return
-    if args.prefill:
+    if args.prefill or args.stream_ceiling:
         if not torch.cuda.is_available():
             raise SystemExit("bench.py needs a CUDA device (the kernels have no CPU path)")
-        prefill_main(args, rank, world, local)
+        (prefill_main if args.prefill else stream_ceiling_main)(args, rank, world, local)
         return
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device (the kernels have no CPU path)")

@@ -317,6 +317,21 @@ kvs_status kvs_static_device_flags(int32_t* flags, int32_t clear, kvs_stream_t s
  */
 kvs_status kvs_device_flags(void* ws, int32_t* flags, int32_t clear, kvs_stream_t stream);
 
+/*
+ * kvs_stream_read -- a measurement helper, not part of the method: the device-memory
+ * read ceiling of the decode step's access pattern. Streams the `rows` rows of a
+ * [rows, d] bf16 device array (d in {64, 128}, 16-byte aligned, rows < 2^31) through
+ * shared memory with the decode kernel's loads -- 2D TMA boxes of 128 rows, 128-byte
+ * swizzle, a 3-stage ring, L2 evict-first -- split evenly over `ctas` CTAs (one per SM
+ * at most), and computes nothing. Timing it over the bytes one decode launch reads, with
+ * the launch's CTA count, gives the decode time with free arithmetic.
+ * Workspace: at least 256 bytes, 256-byte aligned (its flag word records a wait that
+ * gave up, KVS_FLAG_TIMEOUT). Errors: KVS_ERR_INVALID_ARG, KVS_ERR_UNSUPPORTED,
+ * KVS_ERR_WORKSPACE, KVS_ERR_CUDA.
+ */
+kvs_status kvs_stream_read(const void* buf, int64_t rows, int32_t d, int32_t ctas, void* ws,
+                           size_t ws_bytes, kvs_stream_t stream);
+
 /* Static string for a status code. */
 const char* kvs_status_str(kvs_status s);
 

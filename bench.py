@@ -51,6 +51,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--prefill", action="store_true",
                     help="time chunked streaming prefill compression instead (own JSON line)")
+    ap.add_argument("--fp32", action="store_true",
+                    help="the workload with fp32 caches (the CUDA-core kernels), for profiling")
     ap.add_argument("--stream-ceiling", action="store_true",
                     help="time the decode's read pattern with no arithmetic (own JSON line)")
     return ap.parse_args()
@@ -915,6 +917,8 @@ def main():
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     w = inputs.workload(args.workload)
+    if args.fp32:
+        w = inputs.small_workload(w, dtype="f32", name=w.name + "_fp32")
     rn = Runner(w, rank, dev)
     rn.capture()
     for _ in range(args.warmup):
@@ -950,15 +954,24 @@ def main():
     algo = {"decode": rn.decode_bytes(), "score": rn.score_bytes(), "merge": rn.merge_bytes()}
     if rn.remerge:
         algo["remerge"] = rn.remerge_bytes()
-    names = {
-        "decode": "decode_tc_kernel (GQA decode; one thread-block cluster per KV head when "
-                  "every head's cluster fits the GPU, else the split grid)",
-        "score": "kvs_score_pairs: window_tc_kernel passes A and B, their two combine kernels, "
-                 "pair_score_kernel",
+    if w.dtype == "bf16":
+        names = {
+            "decode": "decode_tc_kernel (GQA decode; thread-block clusters per KV head when "
+                      "they fit the GPU, else the split grid)",
+            "score": "kvs_score_pairs: window_fa_kernel (S = Q K^T, O += P V), fa_combine_kernel, "
+                     "window_score_kernel (window mass and pair scores)",
+        }
+    else:
+        names = {
+            "decode": "decode_kernel (fp32 GQA decode on CUDA cores, split grid)",
+            "score": "kvs_score_pairs: window_partial_kernel, window_combine_kernel, "
+                     "alpha_bar_kernel, pair_score_kernel (fp32, CUDA cores)",
+        }
+    names.update({
         "merge": "kvs_merge_compact: select_kernel + merge_kernel (out-of-place compaction)",
         "remerge": "in-place re-merge rounds: kvs_score_pairs + kvs_merge_compact "
                    "(merge_inplace_kernel)",
-    }
+    })
     rooflines = {}
     for k, b in algo.items():
         ms = parts.get(k)

@@ -23,6 +23,7 @@
 //    cluster fits on the GPU at once (few heads, as in single-sequence decode).
 #include <cudaTypedefs.h>
 
+#include <cstdlib>
 #include <map>
 #include <type_traits>
 #include <mutex>
@@ -409,7 +410,11 @@ static ClusterPlan cluster_plan_for(int units) {
   ClusterPlan best{1, 0};
   const bool smem_ok = ensure_smem_attr((const void*)kfn, CS::kSmem);
   const bool big_ok = smem_ok && ensure_nonportable_cluster((const void*)kfn);
-  for (int X = 1; X <= 2 && smem_ok && units > 0; ++X) {
+  // KVS_DECODE_MAX_CLUSTERS_PER_HEAD=1 keeps one cluster per head (read once per device)
+  int x_max = 2;
+  if (const char* env = getenv("KVS_DECODE_MAX_CLUSTERS_PER_HEAD"))
+    if (atoi(env) == 1) x_max = 1;
+  for (int X = 1; X <= x_max && smem_ok && units > 0; ++X) {
     int C = sms / (X * units);
     if (C > kMaxClusterSize) C = kMaxClusterSize;
     if (C > 8 && !big_ok) C = 8;

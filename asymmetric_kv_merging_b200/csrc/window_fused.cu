@@ -901,7 +901,9 @@ window_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
           }
         }
         named_bar(1, kFuSoftThreads);
-        // per window query of this half: lane a (even key) takes N11 and N12, lane b N22
+        // per window query of this half: lane a (even key) takes N11 and N12, lane b N22;
+        // |v - o|^2 = |v|^2 - 2 v.o + |o|^2 and |v_a + v_b - 2 o|^2 = |v_a + v_b|^2
+        // - 4 (v_a + v_b).o + 4 |o|^2
         const int pl = kr >> 1;
         const bool is_a = (kr & 1) == 0;
         const float t_own = is_a ? terms[pl * 4 + 1] : terms[pl * 4 + 2];
@@ -915,7 +917,7 @@ window_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
           const float o2 = on2[qc0 + j];
           n_self = fmaf(fabsf(p * (1.f - 2.f * p)), sqrtf(fmaxf(0.f, fmaf(-2.f, u, t_own) + o2)), n_self);
           if (is_a)
-            n_cpl = fmaf(p * p_o, sqrtf(fmaxf(0.f, fmaf(-2.f, u + u_o, t_ab) + 4.f * o2)), n_cpl);
+            n_cpl = fmaf(p * p_o, sqrtf(fmaxf(0.f, fmaf(-4.f, u + u_o, t_ab) + 4.f * o2)), n_cpl);
         }
         norms[(half * 64 + pl) * 3 + (is_a ? 0 : 2)] = n_self;
         if (is_a) norms[(half * 64 + pl) * 3 + 1] = n_cpl;

@@ -316,20 +316,12 @@ __device__ __forceinline__ int slice_owner(int n, int col, int C) {
 // from a single warp while the other warps stream (its loads of the warp partials see
 // stage data in flight; the values are discarded). A kernel launch starts with cold
 // instruction caches; the dry run pulls this code in before the real combine needs it.
-//
-// Two clusters per head (X = 2, cluster x of the head): each cluster combines its own
-// splits as above, but each CTA then stores its slice's cluster-level partial (M, L and
-// the unscaled column) in `part2` and counts its arrival on the slice's counter in
-// `cnt2`; the CTA that arrives last for a slice combines the X partials (and the
-// appended row) into the output. The last rank-0 CTA appends the row: every CTA of the
-// head has read len by then (each cluster passed its barrier before arriving).
 template <typename T, int D, int G, int NW>
 __device__ __noinline__ void cluster_combine(
     float (*sm)[G], float (*sl)[G], float (*sacc)[G][D], float (*qs)[D], float* s_cml,
     float* s_new, ClusterInbox<D, G>* inbox, int C, int rank, int tid, int nthreads, bool dry,
     int head, int L, int T_cap, bool append, T* K, T* V, float* logn, int32_t* len,
-    const T* kn, const T* vn, T* out, int32_t* flags, int X, int x, float* part2,
-    int32_t* cnt2, int* s_last) {
+    const T* kn, const T* vn, T* out, int32_t* flags) {
   constexpr int N = G * D;
   const int lane = tid & 31, warp = tid >> 5, nwarps = nthreads / 32;
   const bool fits = L < T_cap;
@@ -377,10 +369,9 @@ __device__ __noinline__ void cluster_combine(
   }
   // combine this CTA's slice from its inbox
   const int lo = slice_lo(N, rank, C), hi = slice_lo(N, rank + 1, C);
-  const bool two_level = X > 1 && !dry;
   for (int col = lo + tid; col < hi; col += nthreads) {
     const int g = col / D, c = col - g * D;
-    const float sn = (attend_new && !two_level) ? s_new[g] : -INFINITY;
+    const float sn = attend_new ? s_new[g] : -INFINITY;
     float M = sn;
     for (int j = 0; j < C; ++j)
       if (inbox->ml[j][g][1] > 0.f) M = fmaxf(M, inbox->ml[j][g][0]);
@@ -392,54 +383,13 @@ __device__ __noinline__ void cluster_combine(
         Ls = fmaf(lj, f, Ls);
         A = fmaf(inbox->acc[j * slice_w + (col - lo)], f, A);
       }
-      if (attend_new && !two_level) {
+      if (attend_new) {
         const float f = exp2f(sn - M);
         Ls += f;
         A = fmaf(to_f32(vn[c]), f, A);
       }
     }
-    if (two_level) {
-      float* pp = part2 + (((size_t)head * X + x) * N + col) * 3;
-      pp[0] = M;
-      pp[1] = Ls;
-      pp[2] = A;
-    } else {
-      store_out<T>(out + ((size_t)head * G + g) * D + c, Ls > 0.f ? A / Ls : 0.f);
-    }
-  }
-  if (two_level) {
-    // one device-scope release / acquire by one thread after a CTA barrier publishes the
-    // slice's partial and, in the last CTA, makes the other clusters' partials visible
-    __syncthreads();
-    if (tid == 0) *s_last = atom_add_acq_rel_gpu(&cnt2[head * kMaxClusterSize + rank], 1) == X - 1;
-    __syncthreads();
-    if (!*s_last) return;
-    for (int col = lo + tid; col < hi; col += nthreads) {
-      const int g = col / D, c = col - g * D;
-      const float sn = attend_new ? s_new[g] : -INFINITY;
-      float M = sn;
-      for (int j = 0; j < X; ++j) {
-        const float* pp = part2 + (((size_t)head * X + j) * N + col) * 3;
-        if (__ldcg(pp + 1) > 0.f) M = fmaxf(M, __ldcg(pp));
-      }
-      float Ls = 0.f, A = 0.f;
-      if (M > -INFINITY) {
-        for (int j = 0; j < X; ++j) {
-          const float* pp = part2 + (((size_t)head * X + j) * N + col) * 3;
-          const float lj = __ldcg(pp + 1);
-          const float f = lj > 0.f ? exp2f(__ldcg(pp) - M) : 0.f;
-          Ls = fmaf(lj, f, Ls);
-          A = fmaf(__ldcg(pp + 2), f, A);
-        }
-        if (attend_new) {
-          const float f = exp2f(sn - M);
-          Ls += f;
-          A = fmaf(to_f32(vn[c]), f, A);
-        }
-      }
-      store_out<T>(out + ((size_t)head * G + g) * D + c, Ls > 0.f ? A / Ls : 0.f);
-    }
-    if (tid == 0) cnt2[head * kMaxClusterSize + rank] = 0;   // re-armed for the next call
+    store_out<T>(out + ((size_t)head * G + g) * D + c, Ls > 0.f ? A / Ls : 0.f);
   }
   if (!dry && rank == 0 && append) {
     if (fits) {

@@ -23,7 +23,6 @@
 //    cluster fits on the GPU at once (few heads, as in single-sequence decode).
 #include <cudaTypedefs.h>
 
-#include <cstdlib>
 #include <map>
 #include <type_traits>
 #include <mutex>
@@ -66,8 +65,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
                  const __grid_constant__ CUtensorMap tmL, int ln_lead,
                  const bf16* __restrict__ q, bf16* K, bf16* V, float* logn, int32_t* len,
                  const bf16* __restrict__ k_new, const bf16* __restrict__ v_new,
-                 bf16* __restrict__ out, int T_cap, int nsplit, int csize, int32_t* counters,
-                 float* part, int32_t* flags) {
+                 bf16* __restrict__ out, int T_cap, int nsplit, int32_t* counters, float* part,
+                 int32_t* flags) {
   using S = TcShape<D, NC, STAGES, kCluster ? 1 : 0>;
   constexpr int kTile = S::kTile, kThreads = S::kThreads;
   static_assert(NC * G * D * 4 <= S::kRingBytes, "warp partials fit the ring");
@@ -146,11 +145,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
   if (kCluster && warp == NC + 1) {
     // ---------------- warm-up: the combine's code, dry, while the others stream ----
     if constexpr (kCluster)
-      cluster_combine<bf16, D, G, NC>(s_m, s_l, s_acc, qs, &s_cml[0][0], s_new, &s_inbox[1], csize,
+      cluster_combine<bf16, D, G, NC>(s_m, s_l, s_acc, qs, &s_cml[0][0], s_new, &s_inbox[1], nsplit,
                                       (int)cluster_ctarank(), lane, 32, /*dry=*/true, 0, L, T_cap,
                                       append, K, V, logn, len, s_kvnew[0], s_kvnew[kCluster ? 1 : 0],
-                                      reinterpret_cast<bf16*>(&s_inbox[1]), flags, 1, 0, nullptr,
-                                      nullptr, nullptr);
+                                      reinterpret_cast<bf16*>(&s_inbox[1]), flags);
   } else if (warp == NC) {
     // ---------------- producer: one thread issues every TMA load ----------------
     if (lane == 0) {
@@ -318,11 +316,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
   const DecodeArgs<bf16> a{head, split, nsplit, L, T_cap, bad, K, V, logn, len, k_new, v_new,
                            out, counters, part, flags};
   if constexpr (kCluster) {
-    cluster_combine<bf16, D, G, NC>(s_m, s_l, s_acc, qs, &s_cml[0][0], s_new, &s_inbox[0], csize,
+    cluster_combine<bf16, D, G, NC>(s_m, s_l, s_acc, qs, &s_cml[0][0], s_new, &s_inbox[0], nsplit,
                                     (int)cluster_ctarank(), tid, kThreads, /*dry=*/false, head, L,
                                     T_cap, append, K, V, logn, len, s_kvnew[0],
-                                    s_kvnew[kCluster ? 1 : 0], out, flags, nsplit / csize,
-                                    split / csize, part, counters, &s_last);
+                                    s_kvnew[kCluster ? 1 : 0], out, flags);
   } else {
     decode_epilogue_staged<bf16, D, G, NC>(Sm, base, S::kRingBytes, cbar, a, tid, kThreads);
   }
@@ -384,74 +381,58 @@ bool decode_tc_supported(const kvs_cache_desc& d) {
          tensor_map_encoder() != nullptr;
 }
 
-// Cluster plan for a cluster launch over `units` KV heads on the current device: X
-// clusters of C CTAs per head (X in {1, 2}, 2 <= C <= 16), chosen to stream from as many
-// SMs as possible in one wave -- the largest X * C for which the occupancy calculator
-// places all X * units clusters at once (X = 1 on a tie: no second combine level).
-// C = 0 when no cluster shape fits: the split grid is used.
-struct ClusterPlan {
-  int X, C;
-};
-
+// Cluster size for a cluster launch over `units` KV heads on the current device, or
+// 0 when the split grid is to be used: the largest C <= 16 with C * units <= SM count
+// for which the occupancy calculator places all `units` clusters at once.
 template <int D, int G>
-static ClusterPlan cluster_plan_for(int units) {
+static int cluster_size_for(int units) {
   using CS = ClusterShape<D>;
   auto kfn = decode_tc_kernel<D, G, 8, (D == 64 ? 6 : 3), true>;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return {1, 0};
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
   static std::mutex mu;
-  static std::map<std::pair<int, int>, ClusterPlan> cache;
+  static std::map<std::pair<int, int>, int> cache;
   std::lock_guard<std::mutex> lock(mu);
   const auto key = std::make_pair(dev, units);
   const auto it = cache.find(key);
   if (it != cache.end()) return it->second;
   int sms = 0;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  ClusterPlan best{1, 0};
-  const bool smem_ok = ensure_smem_attr((const void*)kfn, CS::kSmem);
-  const bool big_ok = smem_ok && ensure_nonportable_cluster((const void*)kfn);
-  // KVS_DECODE_MAX_CLUSTERS_PER_HEAD=1 keeps one cluster per head (read once per device)
-  int x_max = 2;
-  if (const char* env = getenv("KVS_DECODE_MAX_CLUSTERS_PER_HEAD"))
-    if (atoi(env) == 1) x_max = 1;
-  for (int X = 1; X <= x_max && smem_ok && units > 0; ++X) {
-    int C = sms / (X * units);
-    if (C > kMaxClusterSize) C = kMaxClusterSize;
-    if (C > 8 && !big_ok) C = 8;
-    for (; C >= 2; --C) {
-      cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3(X * C, units);
-      cfg.blockDim = dim3(CS::kThreads);
-      cfg.dynamicSmemBytes = CS::kSmem;
-      cudaLaunchAttribute at[1];
-      at[0].id = cudaLaunchAttributeClusterDimension;
-      at[0].val.clusterDim.x = C;
-      at[0].val.clusterDim.y = 1;
-      at[0].val.clusterDim.z = 1;
-      cfg.attrs = at;
-      cfg.numAttrs = 1;
-      int n = 0;
-      if (cudaOccupancyMaxActiveClusters(&n, (const void*)kfn, &cfg) == cudaSuccess &&
-          n >= X * units)
-        break;
-    }
-    if (C >= 2 && X * C > best.X * best.C) best = {X, C};
+  int C = units > 0 ? sms / units : 0;
+  if (C > kMaxClusterSize) C = kMaxClusterSize;
+  if (!ensure_smem_attr((const void*)kfn, CS::kSmem)) C = 0;
+  if (C > 8 && !ensure_nonportable_cluster((const void*)kfn)) C = 8;
+  for (; C >= 2; --C) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(C, units);
+    cfg.blockDim = dim3(CS::kThreads);
+    cfg.dynamicSmemBytes = CS::kSmem;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = C;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, (const void*)kfn, &cfg) == cudaSuccess && n >= units) break;
   }
   (void)cudaGetLastError();   // a refused query leaves no error behind
-  cache[key] = best;
-  return best;
+  if (C < 2) C = 0;
+  cache[key] = C;
+  return C;
 }
 
 template <int D, int G, int NC, int STAGES, bool kCluster>
 static cudaError_t launch_shape(const kvs_cache_desc& d, const void* q, void* K, void* V,
                                 float* logn, int32_t* len, const void* k_new, const void* v_new,
-                                void* out, int nsplit, int csize, const DecodeLayout& Ly,
-                                char* ws, cudaStream_t st) {
+                                void* out, int nsplit, const DecodeLayout& Ly, char* ws,
+                                cudaStream_t st) {
   using S = TcShape<D, NC, STAGES, kCluster ? 1 : 0>;
   auto kfn = decode_tc_kernel<D, G, NC, STAGES, kCluster>;
   // per device, cached (the first call on a device must precede any capture)
   if (!ensure_smem_attr((const void*)kfn, S::kSmem)) return cudaErrorInvalidValue;
-  if (kCluster && csize > 8 && !ensure_nonportable_cluster((const void*)kfn))
+  if (kCluster && nsplit > 8 && !ensure_nonportable_cluster((const void*)kfn))
     return cudaErrorInvalidValue;
   const unsigned long long rows = (unsigned long long)d.B * d.H_kv * (unsigned long long)d.T_cap;
   CUtensorMap mK, mV, mL;
@@ -473,14 +454,14 @@ static cudaError_t launch_shape(const kvs_cache_desc& d, const void* q, void* K,
   cfg.stream = st;
   cudaLaunchAttribute at[1];
   at[0].id = cudaLaunchAttributeClusterDimension;
-  at[0].val.clusterDim.x = csize;
+  at[0].val.clusterDim.x = nsplit;
   at[0].val.clusterDim.y = 1;
   at[0].val.clusterDim.z = 1;
   cfg.attrs = at;
   cfg.numAttrs = kCluster ? 1 : 0;
   const cudaError_t e = cudaLaunchKernelEx(
       &cfg, kfn, mK, mV, mL, ln_lead, (const bf16*)q, (bf16*)K, (bf16*)V, logn, len, (const bf16*)k_new,
-      (const bf16*)v_new, (bf16*)out, d.T_cap, nsplit, csize,
+      (const bf16*)v_new, (bf16*)out, d.T_cap, nsplit,
       reinterpret_cast<int32_t*>(ws + Ly.counters), reinterpret_cast<float*>(ws + Ly.part),
       reinterpret_cast<int32_t*>(ws));
   count_launches(1);
@@ -491,12 +472,12 @@ template <int D, int G>
 static cudaError_t launch_tc(const kvs_cache_desc& d, const void* q, void* K, void* V,
                              float* logn, int32_t* len, const void* k_new, const void* v_new,
                              void* out, const DecodeLayout& Ly, char* ws, cudaStream_t st) {
-  const ClusterPlan cp = cluster_plan_for<D, G>(d.B * d.H_kv);
-  if (cp.C >= 2)
+  const int C = cluster_size_for<D, G>(d.B * d.H_kv);
+  if (C >= 2)
     return launch_shape<D, G, 8, (D == 64 ? 6 : 3), true>(d, q, K, V, logn, len, k_new, v_new, out,
-                                                          cp.X * cp.C, cp.C, Ly, ws, st);
-  return launch_shape<D, G, 4, 3, false>(d, q, K, V, logn, len, k_new, v_new, out, Ly.nsplit, 0,
-                                         Ly, ws, st);
+                                                          C, Ly, ws, st);
+  return launch_shape<D, G, 4, 3, false>(d, q, K, V, logn, len, k_new, v_new, out, Ly.nsplit, Ly,
+                                         ws, st);
 }
 
 cudaError_t launch_decode_tc(const kvs_cache_desc& d, const void* q, void* K, void* V, float* logn,

@@ -118,7 +118,7 @@ struct HeadInfo {      // one (b, h)
 };
 
 struct ScoreLayout {
-  size_t part_ml, part_o, stats, obar, alpha, oq_hi, oq_lo, on2, total;
+  size_t part_ml, part_o, stats, obar, alpha, oq_hi, oq_lo, on2, owq, total;
   int nsplit, Qn;
 };
 struct MergeLayout {
@@ -157,12 +157,11 @@ inline int decode_splits(const kvs_cache_desc& d) {
 }
 
 // Every layout starts with the same persistent region: the device flag word in the
-// first 256 bytes, then kMaxClusterSize arrival counters per KV head for the decode
-// combine (the split grid uses the first, a two-cluster launch one per slice owner). No
+// first 256 bytes, then one arrival counter per KV head for the decode combine. No
 // op writes this region except through its own flags / counters, so one zeroed
 // workspace can be shared by all ops on a stream.
 inline size_t persistent_bytes(const kvs_cache_desc& d) {
-  return kWsAlign + align_up((size_t)d.B * d.H_kv * kMaxClusterSize * sizeof(int32_t), kWsAlign);
+  return kWsAlign + align_up((size_t)d.B * d.H_kv * sizeof(int32_t), kWsAlign);
 }
 
 inline ScoreLayout score_layout(const kvs_cache_desc& d, int W) {
@@ -175,12 +174,13 @@ inline ScoreLayout score_layout(const kvs_cache_desc& d, int W) {
   L.stats = align_up(L.part_o + units * L.nsplit * L.Qn * (size_t)d.d * sizeof(float), kWsAlign);
   L.obar = align_up(L.stats + units * L.Qn * 2 * sizeof(float), kWsAlign);
   L.alpha = align_up(L.obar + units * (size_t)d.d * sizeof(float), kWsAlign);
-  // window outputs o_q of the bf16 path: rows of 128 (padded) queries per head, as
-  // bf16 hi / lo parts, and their squared norms
+  // window outputs of the bf16 path relative to their mean, e_q = o_q - o_bar: rows of
+  // 128 (padded) queries per head as bf16 hi / lo parts, |e_q|^2 and o_bar . e_q
   L.oq_hi = align_up(L.alpha + units * (size_t)d.T_cap * sizeof(float), kWsAlign);
   L.oq_lo = align_up(L.oq_hi + units * 128 * (size_t)d.d * 2, kWsAlign);
   L.on2 = align_up(L.oq_lo + units * 128 * (size_t)d.d * 2, kWsAlign);
-  L.total = align_up(L.on2 + units * 128 * sizeof(float), kWsAlign);
+  L.owq = align_up(L.on2 + units * 128 * sizeof(float), kWsAlign);
+  L.total = align_up(L.owq + units * 128 * sizeof(float), kWsAlign);
   return L;
 }
 
@@ -202,11 +202,8 @@ inline DecodeLayout decode_layout(const kvs_cache_desc& d) {
   L.nsplit = decode_splits(d);
   L.counters = kWsAlign;
   L.part = persistent_bytes(d);
-  // split partials of the split grid, or the cluster-level partials (M, L, column) of a
-  // launch with two clusters per head
-  const size_t split_part = qheads * L.nsplit * (size_t)(d.d + kPartPad) * sizeof(float);
-  const size_t cluster_part = qheads * 2 * (size_t)d.d * 3 * sizeof(float);
-  L.total = align_up(L.part + (split_part > cluster_part ? split_part : cluster_part), kWsAlign);
+  L.total = align_up(L.part + qheads * L.nsplit * (size_t)(d.d + kPartPad) * sizeof(float),
+                     kWsAlign);
   return L;
 }
 

@@ -108,6 +108,16 @@ __device__ __forceinline__ void tma_load_1d_hint(void* dst, const CUtensorMap* m
       : "memory");
 }
 
+// Prefetch the box {x, y} of a 2D tensor map into L2 (no shared-memory destination and
+// nothing to wait for): keeps device-memory reads in flight beyond what the
+// shared-memory ring holds.
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y)
+               : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

@@ -14,9 +14,9 @@
 //     multiplied by V) so that O keeps close to fp32 accuracy. The reference maximum
 //     of a row moves only when a tile exceeds it by 2^8 (the accumulator is then
 //     rescaled in tensor memory), so P <= 2^8 between moves.
-//   fa_combine_kernel (per KV head): the splits' (m, l, O) -> per query (M, L), o_q and
-//     |o_q|^2, and o_bar = mean_q o_q; o_q also as bf16 hi / lo rows for pass B's
-//     per-query form.
+//   fa_combine_kernel (per KV head): the splits' (m, l, O) -> per query (M, L) and o_q,
+//     o_bar = mean_q o_q, and for pass B's per-query form e_q = o_q - o_bar as bf16 hi / lo
+//     rows with |e_q|^2 and o_bar . e_q.
 //   pass B (window_score_kernel, per KV head and candidate split): S^T = K Q^T with the
 //     keys on the tensor-memory lanes, so that a thread owns one key and its row of
 //     window probabilities p_qt = 2^(s_qt - M_q) / L_q: alpha_bar_t is a sum over the
@@ -24,8 +24,12 @@
 //     tile (tiles start at the candidate span's first row), so the pair norms, weight
 //     and score come straight from the K and V rows already in shared memory.
 //     Window form "mean" (the plain reading): the one-query norms at (alpha_bar, o_bar).
-//     Window form "per query": the one-query norms of every window query, averaged;
-//     |v - o_q|^2 = |v|^2 - 2 v.o_q + |o_q|^2 with U = V O^T on the tensor cores.
+//     Window form "per query": the one-query norms of every window query, averaged.
+//     With e_q = o_q - o_bar, |v - o_q|^2 = |v - o_bar|^2 - 2 (v.e_q - o_bar.e_q) + |e_q|^2
+//     and |v_a + v_b - 2 o_q|^2 = |v_a + v_b - 2 o_bar|^2 - 4 (v_a.e_q + v_b.e_q
+//     - 2 o_bar.e_q) + 4 |e_q|^2, the row terms taken directly in fp32 as in the mean form
+//     and U = V E^T (E as bf16 hi + lo) on the tensor cores: centring on o_bar keeps the
+//     product small where v and o_q are close, so the expansion does not cancel.
 //
 // Warp roles (both passes): warp 0 issues the TMA loads (128-byte swizzle, no
 // multicast), warp 1 owns the tensor memory and one of its threads issues tcgen05.mma,
@@ -44,6 +48,7 @@ constexpr int kFuSoft = 8;              // softmax warps
 constexpr int kFuThreads = (2 + kFuSoft) * 32;
 constexpr int kFuSoftThreads = kFuSoft * 32;
 constexpr float kRescaleSlack = 8.f;    // log2 units
+constexpr int kPrefetch = 3;            // tiles prefetched into L2 beyond the ring
 
 __device__ __forceinline__ unsigned char* align1024(unsigned char* p) {
   return reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(p) + 1023) &
@@ -151,10 +156,21 @@ window_fa_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 #pragma unroll
       for (int bx = 0; bx < S::kBoxes; ++bx)
         tma_load_2d(base + S::kQOff + bx * S::kBox, &tmQ, bx * 64, q_row0, q_full);
+      // tiles beyond the ring are prefetched into L2, kPrefetch tiles ahead
+      auto prefetch = [&](int i) {
+        if (i < ntiles)
+#pragma unroll
+          for (int bx = 0; bx < S::kBoxes; ++bx) {
+            tma_prefetch_2d(&tmK, bx * 64, k_row0 + i * kFuKeys);
+            tma_prefetch_2d(&tmV, bx * 64, k_row0 + i * kFuKeys);
+          }
+      };
+      for (int i = ST; i < ST + kPrefetch; ++i) prefetch(i);
       int issued_k = 0, issued_v = 0;
       for (int i = 0; i < ntiles; ++i) {
         const int s = i % ST;
         const uint32_t ph = ((i / ST) - 1) & 1;
+        prefetch(i + ST + kPrefetch);
         if (i >= ST && !mbar_wait_ab(&k_empty[s], ph, s_abort)) break;
         mbar_arrive_expect_tx(&k_full[s], S::kTile);
 #pragma unroll
@@ -451,9 +467,10 @@ template <int D>
 __global__ void __launch_bounds__(D)
 fa_combine_kernel(const float* __restrict__ part_ml, const float* __restrict__ part_o, int Qn,
                   int nsplit, float* __restrict__ stats, float* __restrict__ obar,
-                  float* __restrict__ on2, bf16* __restrict__ oq_hi, bf16* __restrict__ oq_lo) {
+                  float* __restrict__ zq_out, float* __restrict__ wq_out, bf16* __restrict__ eq_hi,
+                  bf16* __restrict__ eq_lo) {
   extern __shared__ float fac[];                 // [Qn][nsplit] split weights 2^(m - M) / L
-  __shared__ float s_on2[D / 32][128];
+  __shared__ float s_z[D / 32][128], s_w[D / 32][128];
   __shared__ int s_valid;
   const int unit = blockIdx.x, c = threadIdx.x, lane = c & 31, wid = c >> 5;
   if (c == 0) s_valid = 0;
@@ -481,27 +498,40 @@ fa_combine_kernel(const float* __restrict__ part_ml, const float* __restrict__ p
     if (valid) atomicAdd(&s_valid, 1);
   }
   __syncthreads();
-  float acc = 0.f;
   const float* po = part_o + (size_t)unit * nsplit * Qn * D;
-  for (int q = 0; q < 128; ++q) {
+  auto o_of = [&](int q) {
     float o = 0.f;
-    if (q < Qn)
-      for (int s = 0; s < nsplit; ++s) o = fmaf(fac[q * nsplit + s], po[((size_t)s * Qn + q) * D + c], o);
-    acc += o;
-    const bf16 hi = __float2bfloat16_rn(o);
+    for (int s = 0; s < nsplit; ++s) o = fmaf(fac[q * nsplit + s], po[((size_t)s * Qn + q) * D + c], o);
+    return o;
+  };
+  float acc = 0.f;
+  for (int q = 0; q < Qn; ++q) acc += o_of(q);
+  const float ob = s_valid > 0 ? acc / (float)s_valid : 0.f;
+  obar[(size_t)unit * D + c] = ob;
+  // o_q relative to o_bar, for the per-query window form: e_q = o_q - o_bar as bf16 hi / lo
+  // rows (rows past Qn are zero), |e_q|^2 and o_bar . e_q
+  for (int q = 0; q < 128; ++q) {
+    const float e = q < Qn ? o_of(q) - ob : 0.f;
+    const bf16 hi = __float2bfloat16_rn(e);
     const size_t at = ((size_t)unit * 128 + q) * D + c;
-    oq_hi[at] = hi;
-    oq_lo[at] = __float2bfloat16_rn(o - __bfloat162float(hi));
-    const float sq = warp_sum(o * o);
-    if (lane == 0) s_on2[wid][q] = sq;
+    eq_hi[at] = hi;
+    eq_lo[at] = __float2bfloat16_rn(e - __bfloat162float(hi));
+    const float z = warp_sum(e * e), wv = warp_sum(ob * e);
+    if (lane == 0) {
+      s_z[wid][q] = z;
+      s_w[wid][q] = wv;
+    }
   }
-  obar[(size_t)unit * D + c] = s_valid > 0 ? acc / (float)s_valid : 0.f;
   __syncthreads();
   for (int q = c; q < 128; q += D) {
-    float t = 0.f;
+    float z = 0.f, wv = 0.f;
 #pragma unroll
-    for (int w = 0; w < D / 32; ++w) t += s_on2[w][q];
-    on2[(size_t)unit * 128 + q] = t;
+    for (int w = 0; w < D / 32; ++w) {
+      z += s_z[w][q];
+      wv += s_w[w][q];
+    }
+    zq_out[(size_t)unit * 128 + q] = z;
+    wq_out[(size_t)unit * 128 + q] = wv;
   }
 }
 
@@ -520,14 +550,15 @@ struct ScShape {
   static constexpr int kStageOff = kOOff + (PERQ ? 2 * kTile : 0);
   static constexpr int kStageBytes = 2 * kTile;              // K tile, then V tile
   static constexpr int kSmallOff = kStageOff + kStages * kStageBytes;
-  // barriers (128 B), Z_q = M_q + log2 L_q [128], |o_q|^2 [128] (per query form) or
-  // o_bar [D <= 128] (mean form),
+  // barriers (128 B), Z_q = M_q + log2 L_q [128], o_bar [D], |e_q|^2 and o_bar . e_q
+  // [2][128] (per query form),
   // per-key partial window mass [2 bufs][2 halves][128], per-pair terms [64][4],
   // per-pair partial norms [2 halves][64][3], tensor-memory address and abort flag
   static constexpr int kBarBytes = 128;
-  static constexpr int kZOff = kSmallOff + kBarBytes;
-  static constexpr int kOn2Off = kZOff + 128 * 4;            // |o_q|^2, or o_bar [D]
-  static constexpr int kAbarOff = kOn2Off + 128 * 4;
+  static constexpr int kZOff = kSmallOff + kBarBytes;         // Z_q [128]
+  static constexpr int kObOff = kZOff + 128 * 4;              // o_bar [D <= 128]
+  static constexpr int kOn2Off = kObOff + 128 * 4;            // |e_q|^2, o_bar.e_q [2][128]
+  static constexpr int kAbarOff = kOn2Off + (PERQ ? 2 * 128 * 4 : 0);
   static constexpr int kTermOff = kAbarOff + (PERQ ? 0 : 4 * 128 * 4);
   static constexpr int kNormOff = kTermOff + (PERQ ? 64 * 4 * 4 : 0);
   static constexpr int kQmodOff = kNormOff + (PERQ ? 2 * 64 * 3 * 4 : 0);   // q mod W [128]
@@ -562,7 +593,8 @@ window_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     const int32_t* __restrict__ len, const int32_t* __restrict__ cand_begin,
                     int n_recent, int H_kv, int H_q, int W, int T_cap, int nsplit, int form,
                     const float* __restrict__ stats, const float* __restrict__ obar,
-                    const float* __restrict__ on2g, float* __restrict__ score,
+                    const float* __restrict__ on2g, const float* __restrict__ wqg,
+                    float* __restrict__ score,
                     float* __restrict__ w_b, int32_t* __restrict__ flags) {
   using S = ScShape<D, PERQ>;
   constexpr int ST = S::kStages;
@@ -577,7 +609,8 @@ window_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
   uint64_t* u_full = s_empty + 2;       // 1 (per query form)
   uint64_t* u_empty = u_full + 1;       // 1
   float* zq = reinterpret_cast<float*>(base + S::kZOff);
-  float* on2 = reinterpret_cast<float*>(base + S::kOn2Off);
+  float* obs = reinterpret_cast<float*>(base + S::kObOff);
+  float* on2 = reinterpret_cast<float*>(base + S::kOn2Off);     // |e_q|^2, then o_bar . e_q
   float* abar = reinterpret_cast<float*>(base + S::kAbarOff);     // [2][2][128]
   float* terms = reinterpret_cast<float*>(base + S::kTermOff);    // [64][4]
   float* norms = reinterpret_cast<float*>(base + S::kNormOff);    // [2][64][3]
@@ -627,7 +660,11 @@ window_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     }
     zq[q] = z;
     qmod[q] = q % W;
-    on2[q] = PERQ ? on2g[(size_t)unit * 128 + q] : (q < D ? obar[(size_t)unit * D + q] : 0.f);
+    obs[q] = q < D ? obar[(size_t)unit * D + q] : 0.f;
+    if (PERQ) {
+      on2[q] = on2g[(size_t)unit * 128 + q];
+      on2[128 + q] = wqg[(size_t)unit * 128 + q];
+    }
   }
   if (warp == 1) tmem_alloc(s_tmem, kScTmemCols);
   tc_fence_before();
@@ -654,9 +691,20 @@ window_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
           tma_load_2d(base + S::kOOff + S::kTile + bx * S::kBox, &tmOl, bx * 64, o_row0, q_full);
         }
       }
+      // tiles beyond the ring are prefetched into L2, kPrefetch tiles ahead
+      auto prefetch = [&](int i) {
+        if (i < ntiles)
+#pragma unroll
+          for (int bx = 0; bx < S::kBoxes; ++bx) {
+            tma_prefetch_2d(&tmK, bx * 64, k_row0 + i * kFuKeys);
+            tma_prefetch_2d(&tmV, bx * 64, k_row0 + i * kFuKeys);
+          }
+      };
+      for (int i = ST; i < ST + kPrefetch; ++i) prefetch(i);
       int issued = 0;
       for (int i = 0; i < ntiles; ++i) {
         const int s = i % ST;
+        prefetch(i + ST + kPrefetch);
         if (i >= ST && !mbar_wait_ab(&empty[s], ((i / ST) - 1) & 1, s_abort)) break;
         unsigned char* stg = base + S::kStageOff + s * S::kStageBytes;
         mbar_arrive_expect_tx(&full[s], S::kStageBytes);
@@ -734,7 +782,7 @@ window_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     // pair-term threads: pair pp of the tile, quarter part of the head dimension
     const int pp = st >> 2, part = st & 3;
     constexpr int DP = D / 4;                     // dims per part: 32 or 16
-    const float* ob = zq + 128 + part * DP;         // o_bar, staged after Z_q (mean form)
+    const float* ob = obs + part * DP;
     bool live = true;
     const int first_row = c0 + tbeg * kFuKeys;   // cache row of key 0 of tile 0
     float ln_next = 0.f;
@@ -796,40 +844,43 @@ window_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         for (int j = 0; j < NC; ++j) acc[j & 3] += sv[j];
         abar[(buf * 2 + half) * 128 + kr] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
         named_bar(1, kFuSoftThreads);
-        // the tile's pair pp: rows 2 pp, 2 pp + 1; this thread: dims [DP part, DP part + DP)
-        float dd = 0.f, ea = 0.f, eb = 0.f, ec = 0.f;
-        const int ra = 2 * pp, rb = ra + 1;
+      }
+      // the tile's pair pp: rows 2 pp, 2 pp + 1; this thread: dims [DP part, DP part + DP):
+      // |k_b - k_a|^2, |v_a - o_bar|^2, |v_b - o_bar|^2, |v_a + v_b - 2 o_bar|^2
+      float dd = 0.f, ea = 0.f, eb = 0.f, ec = 0.f;
+      const int ra = 2 * pp, rb = ra + 1;
 #pragma unroll
-        for (int ch = 0; ch < DP / 8; ++ch) {
-          const int dim = part * DP + ch * 8;
-          const int bx = dim >> 6, cc = (dim & 63) >> 3;
-          const uint4 ka = *reinterpret_cast<const uint4*>(kt + bx * S::kBox + swz128(ra, cc));
-          const uint4 kb = *reinterpret_cast<const uint4*>(kt + bx * S::kBox + swz128(rb, cc));
-          const uint4 va = *reinterpret_cast<const uint4*>(vt + bx * S::kBox + swz128(ra, cc));
-          const uint4 vb = *reinterpret_cast<const uint4*>(vt + bx * S::kBox + swz128(rb, cc));
-          const uint32_t kaw[4] = {ka.x, ka.y, ka.z, ka.w}, kbw[4] = {kb.x, kb.y, kb.z, kb.w};
-          const uint32_t vaw[4] = {va.x, va.y, va.z, va.w}, vbw[4] = {vb.x, vb.y, vb.z, vb.w};
+      for (int ch = 0; ch < DP / 8; ++ch) {
+        const int dim = part * DP + ch * 8;
+        const int bx = dim >> 6, cc = (dim & 63) >> 3;
+        const uint4 ka = *reinterpret_cast<const uint4*>(kt + bx * S::kBox + swz128(ra, cc));
+        const uint4 kb = *reinterpret_cast<const uint4*>(kt + bx * S::kBox + swz128(rb, cc));
+        const uint4 va = *reinterpret_cast<const uint4*>(vt + bx * S::kBox + swz128(ra, cc));
+        const uint4 vb = *reinterpret_cast<const uint4*>(vt + bx * S::kBox + swz128(rb, cc));
+        const uint32_t kaw[4] = {ka.x, ka.y, ka.z, ka.w}, kbw[4] = {kb.x, kb.y, kb.z, kb.w};
+        const uint32_t vaw[4] = {va.x, va.y, va.z, va.w}, vbw[4] = {vb.x, vb.y, vb.z, vb.w};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 o2 = *reinterpret_cast<const float2*>(ob + ch * 8 + 2 * e);
-            const float2 dk = make_float2(bf16_lo(kbw[e]) - bf16_lo(kaw[e]), bf16_hi(kbw[e]) - bf16_hi(kaw[e]));
-            const float2 ra2 = make_float2(bf16_lo(vaw[e]) - o2.x, bf16_hi(vaw[e]) - o2.y);
-            const float2 rb2 = make_float2(bf16_lo(vbw[e]) - o2.x, bf16_hi(vbw[e]) - o2.y);
-            const float2 rc2 = fadd2(ra2, rb2);
-            dd = fmaf(dk.x, dk.x, fmaf(dk.y, dk.y, dd));
-            ea = fmaf(ra2.x, ra2.x, fmaf(ra2.y, ra2.y, ea));
-            eb = fmaf(rb2.x, rb2.x, fmaf(rb2.y, rb2.y, eb));
-            ec = fmaf(rc2.x, rc2.x, fmaf(rc2.y, rc2.y, ec));
-          }
+        for (int e = 0; e < 4; ++e) {
+          const float2 o2 = *reinterpret_cast<const float2*>(ob + ch * 8 + 2 * e);
+          const float2 dk = make_float2(bf16_lo(kbw[e]) - bf16_lo(kaw[e]), bf16_hi(kbw[e]) - bf16_hi(kaw[e]));
+          const float2 ra2 = make_float2(bf16_lo(vaw[e]) - o2.x, bf16_hi(vaw[e]) - o2.y);
+          const float2 rb2 = make_float2(bf16_lo(vbw[e]) - o2.x, bf16_hi(vbw[e]) - o2.y);
+          const float2 rc2 = fadd2(ra2, rb2);
+          dd = fmaf(dk.x, dk.x, fmaf(dk.y, dk.y, dd));
+          ea = fmaf(ra2.x, ra2.x, fmaf(ra2.y, ra2.y, ea));
+          eb = fmaf(rb2.x, rb2.x, fmaf(rb2.y, rb2.y, eb));
+          ec = fmaf(rc2.x, rc2.x, fmaf(rc2.y, rc2.y, ec));
         }
+      }
 #pragma unroll
-        for (int o = 1; o < 4; o <<= 1) {
-          dd += __shfl_xor_sync(0xffffffffu, dd, o);
-          ea += __shfl_xor_sync(0xffffffffu, ea, o);
-          eb += __shfl_xor_sync(0xffffffffu, eb, o);
-          ec += __shfl_xor_sync(0xffffffffu, ec, o);
-        }
-        const int pglob = tile * (kFuKeys / 2) + pp;
+      for (int o = 1; o < 4; o <<= 1) {
+        dd += __shfl_xor_sync(0xffffffffu, dd, o);
+        ea += __shfl_xor_sync(0xffffffffu, ea, o);
+        eb += __shfl_xor_sync(0xffffffffu, eb, o);
+        ec += __shfl_xor_sync(0xffffffffu, ec, o);
+      }
+      const int pglob = tile * (kFuKeys / 2) + pp;
+      if constexpr (!PERQ) {
         if (part == 0 && pglob < P && live) {
           const float* ab = abar + buf * 256;
           const float aa = (ab[ra] + ab[128 + ra]) * inv_qv;
@@ -844,7 +895,7 @@ window_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
           w_b[at] = w;
         }
       } else {
-        // per-query window form: U = V O^T gives v_t . o_q on the key's lane
+        // per-query window form: U = V E^T gives v_t . e_q on the key's lane
         bool uok = live && mbar_wait_ab(u_full, i & 1, s_abort);
         uok = __all_sync(0xffffffffu, uok);
         live = live && uok;
@@ -861,49 +912,14 @@ window_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(u_empty);
-        // the pair's row terms |k_b - k_a|^2, |v_a|^2, |v_b|^2, v_a . v_b
-        {
-          float dd = 0.f, aa2 = 0.f, bb2 = 0.f, ab = 0.f;
-          const int ra = 2 * pp, rb = ra + 1;
-#pragma unroll
-          for (int ch = 0; ch < DP / 8; ++ch) {
-            const int dim = part * DP + ch * 8;
-            const int bx = dim >> 6, cc = (dim & 63) >> 3;
-            const uint4 ka = *reinterpret_cast<const uint4*>(kt + bx * S::kBox + swz128(ra, cc));
-            const uint4 kb = *reinterpret_cast<const uint4*>(kt + bx * S::kBox + swz128(rb, cc));
-            const uint4 va = *reinterpret_cast<const uint4*>(vt + bx * S::kBox + swz128(ra, cc));
-            const uint4 vb = *reinterpret_cast<const uint4*>(vt + bx * S::kBox + swz128(rb, cc));
-            const uint32_t kaw[4] = {ka.x, ka.y, ka.z, ka.w}, kbw[4] = {kb.x, kb.y, kb.z, kb.w};
-            const uint32_t vaw[4] = {va.x, va.y, va.z, va.w}, vbw[4] = {vb.x, vb.y, vb.z, vb.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float dk0 = bf16_lo(kbw[e]) - bf16_lo(kaw[e]), dk1 = bf16_hi(kbw[e]) - bf16_hi(kaw[e]);
-              const float a0 = bf16_lo(vaw[e]), a1 = bf16_hi(vaw[e]);
-              const float b0 = bf16_lo(vbw[e]), b1 = bf16_hi(vbw[e]);
-              dd = fmaf(dk0, dk0, fmaf(dk1, dk1, dd));
-              aa2 = fmaf(a0, a0, fmaf(a1, a1, aa2));
-              bb2 = fmaf(b0, b0, fmaf(b1, b1, bb2));
-              ab = fmaf(a0, b0, fmaf(a1, b1, ab));
-            }
-          }
-#pragma unroll
-          for (int o = 1; o < 4; o <<= 1) {
-            dd += __shfl_xor_sync(0xffffffffu, dd, o);
-            aa2 += __shfl_xor_sync(0xffffffffu, aa2, o);
-            bb2 += __shfl_xor_sync(0xffffffffu, bb2, o);
-            ab += __shfl_xor_sync(0xffffffffu, ab, o);
-          }
-          if (part == 0) {
-            terms[pp * 4 + 0] = dd;
-            terms[pp * 4 + 1] = aa2;
-            terms[pp * 4 + 2] = bb2;
-            terms[pp * 4 + 3] = aa2 + bb2 + 2.f * ab;    // |v_a + v_b|^2
-          }
+        if (part == 0) {
+          terms[pp * 4 + 0] = dd;
+          terms[pp * 4 + 1] = ea;
+          terms[pp * 4 + 2] = eb;
+          terms[pp * 4 + 3] = ec;
         }
         named_bar(1, kFuSoftThreads);
-        // per window query of this half: lane a (even key) takes N11 and N12, lane b N22;
-        // |v - o|^2 = |v|^2 - 2 v.o + |o|^2 and |v_a + v_b - 2 o|^2 = |v_a + v_b|^2
-        // - 4 (v_a + v_b).o + 4 |o|^2
+        // per window query of this half: lane a (even key) takes N11 and N12, lane b N22
         const int pl = kr >> 1;
         const bool is_a = (kr & 1) == 0;
         const float t_own = is_a ? terms[pl * 4 + 1] : terms[pl * 4 + 2];
@@ -914,15 +930,16 @@ window_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
           const float p = sv[j], u = uv[j];
           const float p_o = __shfl_xor_sync(0xffffffffu, p, 1);
           const float u_o = __shfl_xor_sync(0xffffffffu, u, 1);
-          const float o2 = on2[qc0 + j];
-          n_self = fmaf(fabsf(p * (1.f - 2.f * p)), sqrtf(fmaxf(0.f, fmaf(-2.f, u, t_own) + o2)), n_self);
+          const float z = on2[qc0 + j], wq = on2[128 + qc0 + j];
+          n_self = fmaf(fabsf(p * (1.f - 2.f * p)),
+                        sqrtf(fmaxf(0.f, fmaf(-2.f, u - wq, t_own) + z)), n_self);
           if (is_a)
-            n_cpl = fmaf(p * p_o, sqrtf(fmaxf(0.f, fmaf(-4.f, u + u_o, t_ab) + 4.f * o2)), n_cpl);
+            n_cpl = fmaf(p * p_o, sqrtf(fmaxf(0.f, fmaf(-4.f, u + u_o - 2.f * wq, t_ab) + 4.f * z)),
+                         n_cpl);
         }
         norms[(half * 64 + pl) * 3 + (is_a ? 0 : 2)] = n_self;
         if (is_a) norms[(half * 64 + pl) * 3 + 1] = n_cpl;
         named_bar(1, kFuSoftThreads);
-        const int pglob = tile * (kFuKeys / 2) + pp;
         if (part == 0 && pglob < P && live) {
           const float* n0 = norms + pp * 3;
           const float* n1 = norms + (64 + pp) * 3;
@@ -995,6 +1012,7 @@ static cudaError_t launch_fused_t(const kvs_cache_desc& d, const void* K, const 
   float* stats = reinterpret_cast<float*>(ws + Ly.stats);
   float* obar = reinterpret_cast<float*>(ws + Ly.obar);
   float* on2 = reinterpret_cast<float*>(ws + Ly.on2);
+  float* owq = reinterpret_cast<float*>(ws + Ly.owq);
 
   auto ka = window_fa_kernel<D>;
   if (!ensure_smem_attr((const void*)ka, FaShape<D>::kSmem)) return cudaErrorInvalidValue;
@@ -1003,20 +1021,20 @@ static cudaError_t launch_fused_t(const kvs_cache_desc& d, const void* K, const 
   const size_t csm = (size_t)Qn * nsa * sizeof(float);
   auto kc = fa_combine_kernel<D>;
   if (!ensure_smem_attr((const void*)kc, csm)) return cudaErrorInvalidValue;
-  kc<<<units, D, csm, st>>>(part_ml, part_o, Qn, nsa, stats, obar, on2, oq_hi, oq_lo);
+  kc<<<units, D, csm, st>>>(part_ml, part_o, Qn, nsa, stats, obar, on2, owq, oq_hi, oq_lo);
   const int nsb = fused_splits(units);
   if (stats_form == KVS_FORM_PER_QUERY) {
     auto kb = window_score_kernel<D, true>;
     if (!ensure_smem_attr((const void*)kb, ScShape<D, true>::kSmem)) return cudaErrorInvalidValue;
     kb<<<dim3(nsb, units), kFuThreads, ScShape<D, true>::kSmem, st>>>(
         mQ, mK, mV, mOh, mOl, logn, len, cand_begin, n_recent, d.H_kv, d.H_q, W, d.T_cap, nsb,
-        form, stats, obar, on2, score, w_b, flags);
+        form, stats, obar, on2, owq, score, w_b, flags);
   } else {
     auto kb = window_score_kernel<D, false>;
     if (!ensure_smem_attr((const void*)kb, ScShape<D, false>::kSmem)) return cudaErrorInvalidValue;
     kb<<<dim3(nsb, units), kFuThreads, ScShape<D, false>::kSmem, st>>>(
         mQ, mK, mV, mOh, mOl, logn, len, cand_begin, n_recent, d.H_kv, d.H_q, W, d.T_cap, nsb,
-        form, stats, obar, on2, score, w_b, flags);
+        form, stats, obar, on2, owq, score, w_b, flags);
   }
   count_launches(3);
   return cudaGetLastError();

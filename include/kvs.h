@@ -261,10 +261,9 @@ kvs_status kvs_plan_rounds(int32_t len, int32_t target, int32_t cand_begin, int3
  * zero at the first call (each call leaves them zero).
  * The first call for a device and a B*H_kv sets kernel attributes and asks the CUDA
  * occupancy calculator which launch shape fits (host calls only, cached): make it
- * outside any stream capture. Launch shape: thread-block clusters that combine the
- * splits of a KV head in distributed shared memory when they all fit the GPU at once,
- * one or two clusters per head, whichever streams from more SMs; the environment
- * variable KVS_DECODE_MAX_CLUSTERS_PER_HEAD=1 (read at that first call) keeps one.
+ * outside any stream capture. Launch shape: one thread-block cluster per KV head that
+ * combines the head's splits in distributed shared memory, when every head's cluster
+ * fits the GPU at once; else a grid of splits combined by the last one to finish.
  */
 kvs_status kvs_decode_attn(const kvs_cache_desc* desc, const void* q, void* K, void* V,
                            float* logn, int32_t* len, const void* k_new, const void* v_new,

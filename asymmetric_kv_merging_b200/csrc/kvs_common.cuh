@@ -118,8 +118,9 @@ struct HeadInfo {      // one (b, h)
 };
 
 struct ScoreLayout {
-  size_t part_ml, part_o, stats, obar, alpha, oq_hi, oq_lo, on2, owq, total;
+  size_t part_ml, part_o, stats, obar, alpha, oq_hi, oq_mid, oq_lo, on2, owq, total;
   int nsplit, Qn;
+  int part_slots;   // window partials per head the layout holds (>= nsplit, >= 2)
 };
 struct MergeLayout {
   size_t sel, head, blk, total;
@@ -169,15 +170,17 @@ inline ScoreLayout score_layout(const kvs_cache_desc& d, int W) {
   size_t units = (size_t)d.B * d.H_kv;
   L.Qn = (d.H_q / d.H_kv) * W;
   L.nsplit = window_splits(d);
+  L.part_slots = L.nsplit > 2 ? L.nsplit : 2;
   L.part_ml = persistent_bytes(d);
-  L.part_o = align_up(L.part_ml + units * L.nsplit * L.Qn * 2 * sizeof(float), kWsAlign);
-  L.stats = align_up(L.part_o + units * L.nsplit * L.Qn * (size_t)d.d * sizeof(float), kWsAlign);
+  L.part_o = align_up(L.part_ml + units * L.part_slots * L.Qn * 2 * sizeof(float), kWsAlign);
+  L.stats = align_up(L.part_o + units * L.part_slots * L.Qn * (size_t)d.d * sizeof(float), kWsAlign);
   L.obar = align_up(L.stats + units * L.Qn * 2 * sizeof(float), kWsAlign);
   L.alpha = align_up(L.obar + units * (size_t)d.d * sizeof(float), kWsAlign);
   // window outputs of the bf16 path relative to their mean, e_q = o_q - o_bar: rows of
-  // 128 (padded) queries per head as bf16 hi / lo parts, |e_q|^2 and o_bar . e_q
+  // 128 (padded) queries per head as bf16 hi / mid / lo parts, |e_q|^2 and o_bar . e_q
   L.oq_hi = align_up(L.alpha + units * (size_t)d.T_cap * sizeof(float), kWsAlign);
-  L.oq_lo = align_up(L.oq_hi + units * 128 * (size_t)d.d * 2, kWsAlign);
+  L.oq_mid = align_up(L.oq_hi + units * 128 * (size_t)d.d * 2, kWsAlign);
+  L.oq_lo = align_up(L.oq_mid + units * 128 * (size_t)d.d * 2, kWsAlign);
   L.on2 = align_up(L.oq_lo + units * 128 * (size_t)d.d * 2, kWsAlign);
   L.owq = align_up(L.on2 + units * 128 * sizeof(float), kWsAlign);
   L.total = align_up(L.owq + units * 128 * sizeof(float), kWsAlign);

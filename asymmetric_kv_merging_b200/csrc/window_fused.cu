@@ -11,30 +11,34 @@
 //     tensor cores, flash-attention style: per window query the running maximum m and
 //     sum l of 2^s and the unnormalised output O, so that the window's o_q are known
 //     before any pair is scored. P is rounded to bf16 twice (P = P_hi + P_lo, both
-//     multiplied by V) so that O keeps close to fp32 accuracy. The reference maximum
+//     multiplied by V) so that O keeps close to fp32 accuracy; it goes back into tensor
+//     memory over the tile's S and feeds the P V MMAs from there. The reference maximum
 //     of a row moves only when a tile exceeds it by 2^8 (the accumulator is then
 //     rescaled in tensor memory), so P <= 2^8 between moves.
-//   fa_combine_kernel (per KV head): the splits' (m, l, O) -> per query (M, L) and o_q,
-//     o_bar = mean_q o_q, and for pass B's per-query form e_q = o_q - o_bar as bf16 hi / lo
-//     rows with |e_q|^2 and o_bar . e_q.
+//   fa_combine_kernel (per KV head): the partials' (m, l, O) -> per query (M, L) and o_q,
+//     o_bar = mean_q o_q, and for pass B's per-query form e_q = o_q - o_bar as bf16
+//     hi / mid / lo rows with |e_q|^2 and o_bar . e_q.
 //   pass B (window_score_kernel, per KV head and candidate split): S^T = K Q^T with the
 //     keys on the tensor-memory lanes, so that a thread owns one key and its row of
 //     window probabilities p_qt = 2^(s_qt - M_q) / L_q: alpha_bar_t is a sum over the
 //     thread's own columns. A candidate pair is two adjacent rows of the same 128-row
 //     tile (tiles start at the candidate span's first row), so the pair norms, weight
-//     and score come straight from the K and V rows already in shared memory.
+//     and score come straight from the K and V rows already in shared memory, the two
+//     rows of a pair on two lanes of one warp.
 //     Window form "mean" (the plain reading): the one-query norms at (alpha_bar, o_bar).
 //     Window form "per query": the one-query norms of every window query, averaged.
 //     With e_q = o_q - o_bar, |v - o_q|^2 = |v - o_bar|^2 - 2 (v.e_q - o_bar.e_q) + |e_q|^2
 //     and |v_a + v_b - 2 o_q|^2 = |v_a + v_b - 2 o_bar|^2 - 4 (v_a.e_q + v_b.e_q
-//     - 2 o_bar.e_q) + 4 |e_q|^2, the row terms taken directly in fp32 as in the mean form
-//     and U = V E^T (E as bf16 hi + lo) on the tensor cores: centring on o_bar keeps the
-//     product small where v and o_q are close, so the expansion does not cancel.
+//     - 2 o_bar.e_q) + 4 |e_q|^2: the row terms are taken directly in fp32 as in the mean
+//     form and U = V E^T (E as three bf16 parts) on the tensor cores. Centring on o_bar
+//     keeps the product small where v and o_q are close.
 //
 // Warp roles (both passes): warp 0 issues the TMA loads (128-byte swizzle, no
 // multicast), warp 1 owns the tensor memory and one of its threads issues tcgen05.mma,
-// warps 2-9 do the softmax arithmetic (two per tensor-memory lane quarter). Every wait
-// is bounded.
+// warps 2-5 and 6-9 are two softmax groups that take alternate tiles (one warp per
+// tensor-memory lane quarter, one row per thread), each with its own tensor-memory
+// buffers and barriers, so that no CTA-wide barrier sits in the per-tile path and one
+// group computes while the other waits for its data. Every wait is bounded.
 #include <cudaTypedefs.h>
 
 #include "kvs_common.cuh"
@@ -44,15 +48,26 @@
 namespace kvs {
 
 constexpr int kFuKeys = 128;            // keys per tile
-constexpr int kFuSoft = 8;              // softmax warps
-constexpr int kFuThreads = (2 + kFuSoft) * 32;
-constexpr int kFuSoftThreads = kFuSoft * 32;
+constexpr int kFuGroupWarps = 4;        // softmax warps per group: one per lane quarter
+constexpr int kFuThreads = (2 + 2 * kFuGroupWarps) * 32;
 constexpr float kRescaleSlack = 8.f;    // log2 units
-constexpr int kPrefetch = 3;            // tiles prefetched into L2 beyond the ring
+constexpr uint32_t kFuTmemCols = 512;
 
 __device__ __forceinline__ unsigned char* align1024(unsigned char* p) {
   return reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(p) + 1023) &
                                           ~static_cast<uintptr_t>(1023));
+}
+
+// 16 consecutive 32-bit columns of this thread's tensor-memory lane, stored from
+// registers (warp-collective), then wait until the stores are done.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------
@@ -64,30 +79,30 @@ struct FaShape {
   static constexpr int kBoxes = D / 64;
   static constexpr int kBox = 128 * 128;                 // 128 rows x 128 bytes
   static constexpr int kTile = kBoxes * kBox;            // a Q, K or V tile
-  static constexpr int kPBytes = 2 * kBox;               // P: 128 rows x 128 keys, bf16
-  static constexpr int kStages = D == 128 ? 2 : 3;
+  static constexpr int kStages = D == 128 ? 3 : 4;
+  static constexpr int kLnBox = kFuKeys + 4;             // floats, from a 16-byte boundary
+  static constexpr int kLnSlot = 544;                    // bytes per stage (>= 4 kLnBox)
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kQOff + kTile;
   static constexpr int kVOff = kKOff + kStages * kTile;
-  static constexpr int kPOff = kVOff + kStages * kTile;  // P_hi, then P_lo
-  static constexpr int kSmallOff = kPOff + 2 * kPBytes;
-  // barriers (256 B), per-row partial maxima / sums [2][128], log-counts [128],
-  // tensor-memory address and abort flag
-  static constexpr int kBarBytes = 256;
-  static constexpr int kSmallBytes = kBarBytes + 2 * 128 * 4 + 128 * 4 + 16;
-  static constexpr int kSmem = kSmallOff + kSmallBytes + 1024;
+  static constexpr int kLnOff = kVOff + kStages * kTile;
+  static constexpr int kSmallOff = kLnOff + kStages * kLnSlot;
+  static constexpr int kSmem = kSmallOff + 256 + 16 + 1024;   // barriers, misc, alignment
+  static_assert(4 * kLnBox <= kLnSlot && kLnSlot % 16 == 0, "log-count slot");
   static_assert(kSmem <= 232448, "shared memory");
 };
 
-constexpr uint32_t kFaTmemCols = 512;   // S0 [0,128), S1 [128,256), O [256, 256 + D)
-
+// Tensor memory of pass A, per softmax group g: S_g at columns [128 g, 128 g + 128) --
+// once read, a 32-key chunk c of it holds that chunk's P as bf16 pairs, hi in columns
+// [32 c, 32 c + 16) and lo in [32 c + 16, 32 c + 32), the A operand of the group's P V
+// MMAs -- and O_g at [256 + D g, 256 + D g + D).
 template <int D>
 __global__ void __launch_bounds__(kFuThreads, 1)
 window_fa_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                 const __grid_constant__ CUtensorMap tmV, const float* __restrict__ logn,
-                 const int32_t* __restrict__ len, int H_kv, int H_q, int W, int T_cap, int nsplit,
-                 float* __restrict__ part_ml, float* __restrict__ part_o,
-                 int32_t* __restrict__ flags) {
+                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmL,
+                 int ln_lead, bool has_ln, const int32_t* __restrict__ len, int H_kv, int H_q,
+                 int W, int T_cap, int nsplit, float* __restrict__ part_ml,
+                 float* __restrict__ part_o, int32_t* __restrict__ flags) {
   using S = FaShape<D>;
   constexpr int ST = S::kStages;
   extern __shared__ unsigned char dsm[];
@@ -96,15 +111,12 @@ window_fa_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   uint64_t* q_full = bars;              // 1
   uint64_t* k_full = q_full + 1;        // ST
   uint64_t* k_empty = k_full + ST;      // ST: the QK^T MMA of the stage is done
-  uint64_t* v_full = k_empty + ST;      // ST
-  uint64_t* v_empty = v_full + ST;      // ST: the P V MMA of the stage is done
-  uint64_t* s_full = v_empty + ST;      // 2
-  uint64_t* s_empty = s_full + 2;       // 2: every softmax warp has read S
-  uint64_t* p_full = s_empty + 2;       // 1: every softmax warp has written P
-  uint64_t* pv_done = p_full + 1;       // 1: the P V MMAs of a tile are done
-  float* xch = reinterpret_cast<float*>(base + S::kSmallOff + S::kBarBytes);   // [2][128]
-  float* lns = xch + 256;                                                      // [128]
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(lns + 128);
+  uint64_t* v_full = k_empty + ST;      // ST: V rows and log-counts
+  uint64_t* v_empty = v_full + ST;      // ST: the P V MMAs of the stage are done
+  uint64_t* s_full = v_empty + ST;      // 2 (per group)
+  uint64_t* p_full = s_full + 2;        // 2: the group's four warps have written P
+  uint64_t* pv_done = p_full + 2;       // 2: the group's P V MMAs of a tile are done
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(base + S::kSmallOff + 256);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
 
   const int unit = blockIdx.y, split = blockIdx.x;
@@ -122,6 +134,9 @@ window_fa_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   const int ntiles = t1 > t0 ? (t1 - t0 + kFuKeys - 1) / kFuKeys : 0;
   const int q_row0 = (b * H_q + h * G) * W;
   const int k_row0 = unit * T_cap + t0;
+  // log-counts of tile i start at element ln_lead + k_row0 + 128 i of the map; its box
+  // starts at the 4-element boundary below, the same offset for every tile
+  const int ln_off = (ln_lead + k_row0) & 3;
 
   if (tid == 0) {
     *s_abort = 0;
@@ -132,15 +147,14 @@ window_fa_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&s_full[s], 1);
-      mbar_init(&s_empty[s], kFuSoft);
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(&s_full[g], 1);
+      mbar_init(&p_full[g], kFuGroupWarps);
+      mbar_init(&pv_done[g], 1);
     }
-    mbar_init(p_full, kFuSoft);
-    mbar_init(pv_done, 1);
     fence_mbar_init();
   }
-  if (warp == 1) tmem_alloc(s_tmem, kFaTmemCols);
+  if (warp == 1) tmem_alloc(s_tmem, kFuTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -152,25 +166,15 @@ window_fa_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
+      if (has_ln) prefetch_tmap(&tmL);
       mbar_arrive_expect_tx(q_full, S::kTile);
 #pragma unroll
       for (int bx = 0; bx < S::kBoxes; ++bx)
         tma_load_2d(base + S::kQOff + bx * S::kBox, &tmQ, bx * 64, q_row0, q_full);
-      // tiles beyond the ring are prefetched into L2, kPrefetch tiles ahead
-      auto prefetch = [&](int i) {
-        if (i < ntiles)
-#pragma unroll
-          for (int bx = 0; bx < S::kBoxes; ++bx) {
-            tma_prefetch_2d(&tmK, bx * 64, k_row0 + i * kFuKeys);
-            tma_prefetch_2d(&tmV, bx * 64, k_row0 + i * kFuKeys);
-          }
-      };
-      for (int i = ST; i < ST + kPrefetch; ++i) prefetch(i);
       int issued_k = 0, issued_v = 0;
       for (int i = 0; i < ntiles; ++i) {
         const int s = i % ST;
         const uint32_t ph = ((i / ST) - 1) & 1;
-        prefetch(i + ST + kPrefetch);
         if (i >= ST && !mbar_wait_ab(&k_empty[s], ph, s_abort)) break;
         mbar_arrive_expect_tx(&k_full[s], S::kTile);
 #pragma unroll
@@ -179,11 +183,16 @@ window_fa_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                       k_row0 + i * kFuKeys, &k_full[s]);
         issued_k = i + 1;
         if (i >= ST && !mbar_wait_ab(&v_empty[s], ph, s_abort)) break;
-        mbar_arrive_expect_tx(&v_full[s], S::kTile);
+        mbar_arrive_expect_tx(&v_full[s], S::kTile + (has_ln ? S::kLnBox * 4 : 0));
 #pragma unroll
         for (int bx = 0; bx < S::kBoxes; ++bx)
           tma_load_2d(base + S::kVOff + s * S::kTile + bx * S::kBox, &tmV, bx * 64,
                       k_row0 + i * kFuKeys, &v_full[s]);
+        if (has_ln) {
+          const uint64_t once = policy_evict_first();
+          tma_load_1d_hint(base + S::kLnOff + s * S::kLnSlot, &tmL,
+                           ln_lead + k_row0 + i * kFuKeys - ln_off, &v_full[s], once);
+        }
         issued_v = i + 1;
       }
       if (issued_v < ntiles) set_flag(flags, KVS_FLAG_TIMEOUT);
@@ -202,36 +211,36 @@ window_fa_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       constexpr uint32_t idesc_qk = umma_idesc_bf16_f32(128, kFuKeys);
       constexpr uint32_t idesc_pv = umma_idesc_bf16_f32_bmn(128, D);
       const uint32_t q_addr = smem_u32(base + S::kQOff);
-      const uint32_t ph_addr = smem_u32(base + S::kPOff);
-      const uint32_t pl_addr = ph_addr + S::kPBytes;
-      const uint32_t o_tmem = tmem + 256;
-      int qk_done = 0, pv_issued = 0;
-      // O += P_hi V + P_lo V for tile j (V MN-major: keys are the K dimension)
+      int pv_issued = 0;
+      // O_g += P_hi V + P_lo V for tile j (group g = j & 1): P from the group's tensor
+      // memory, V from the ring (MN-major: keys are the K dimension)
       auto issue_pv = [&](int j) -> bool {
-        const int vs = j % ST;
-        if (!mbar_wait_ab(p_full, j & 1, s_abort) ||
+        const int g = j & 1, kj = j >> 1, vs = j % ST;
+        if (!mbar_wait_ab(&p_full[g], kj & 1, s_abort) ||
             !mbar_wait_ab(&v_full[vs], (j / ST) & 1, s_abort))
           return false;
         tc_fence_after();
         const uint32_t v_addr = smem_u32(base + S::kVOff + vs * S::kTile);
+        const uint32_t p_tm = tmem + (uint32_t)(g * kFuKeys);
+        const uint32_t o_tm = tmem + 256 + (uint32_t)(g * D);
 #pragma unroll
         for (int ks = 0; ks < kFuKeys / 16; ++ks) {
-          const uint32_t a_off = (uint32_t)((ks >> 2) * S::kBox + (ks & 3) * 32);
           const uint64_t bdesc = umma_desc_mn_sw128(v_addr + ks * 2048, S::kBox);
-          umma_bf16_ss(o_tmem, umma_desc_k_sw128(ph_addr + a_off), bdesc, idesc_pv,
-                       (j > 0 || ks > 0) ? 1u : 0u);
-          umma_bf16_ss(o_tmem, umma_desc_k_sw128(pl_addr + a_off), bdesc, idesc_pv, 1u);
+          const uint32_t a = p_tm + 32 * (ks >> 1) + 8 * (ks & 1);
+          umma_bf16_ts(o_tm, a, bdesc, idesc_pv, (kj > 0 || ks > 0) ? 1u : 0u);
+          umma_bf16_ts(o_tm, a + 16, bdesc, idesc_pv, 1u);
         }
-        umma_commit(pv_done);
+        umma_commit(&pv_done[g]);
         umma_commit(&v_empty[vs]);
         pv_issued = j + 1;
         return true;
       };
       bool ok = mbar_wait_ab(q_full, 0, s_abort);
       for (int i = 0; ok && i < ntiles; ++i) {
-        const int s = i % ST, buf = i & 1;
+        const int s = i % ST, g = i & 1, k = i >> 1;
+        // S of tile i overwrites the P that the group's previous P V MMAs read
         if (!mbar_wait_ab(&k_full[s], (i / ST) & 1, s_abort) ||
-            (i >= 2 && !mbar_wait_ab(&s_empty[buf], ((i / 2) - 1) & 1, s_abort))) {
+            (k >= 1 && !mbar_wait_ab(&pv_done[g], (k - 1) & 1, s_abort))) {
           ok = false;
           break;
         }
@@ -240,213 +249,178 @@ window_fa_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t off = (uint32_t)((ks >> 2) * S::kBox + (ks & 3) * 32);
-          umma_bf16_ss(tmem + buf * kFuKeys, umma_desc_k_sw128(q_addr + off),
+          umma_bf16_ss(tmem + g * kFuKeys, umma_desc_k_sw128(q_addr + off),
                        umma_desc_k_sw128(k_addr + off), idesc_qk, ks > 0 ? 1u : 0u);
         }
-        umma_commit(&s_full[buf]);
+        umma_commit(&s_full[g]);
         umma_commit(&k_empty[s]);
-        qk_done = i + 1;
         if (i >= 1) ok = issue_pv(i - 1);
       }
       if (ok && ntiles > 0) ok = issue_pv(ntiles - 1);
       if (!ok) set_flag(flags, KVS_FLAG_TIMEOUT);
-      // the last MMAs must finish before the tensor memory is released
-      if (qk_done > 0 && !mbar_wait(&s_full[(qk_done - 1) & 1], ((qk_done - 1) / 2) & 1))
-        set_flag(flags, KVS_FLAG_TIMEOUT);
-      if (pv_issued > 0 && !mbar_wait(pv_done, (pv_issued - 1) & 1))
-        set_flag(flags, KVS_FLAG_TIMEOUT);
+      // the last MMAs of each group (each P V follows that tile's QK^T) must finish before
+      // the tensor memory is released
+      for (int g = 0; g < 2; ++g) {
+        const int n_g = pv_issued > g ? (pv_issued - 1 - g) / 2 + 1 : 0;
+        if (n_g > 0 && !mbar_wait(&pv_done[g], (n_g - 1) & 1)) set_flag(flags, KVS_FLAG_TIMEOUT);
+      }
     }
     __syncwarp();
   } else {
-    // ---------------- softmax warps ----------------
-    // warp 2 + sw reads lane quarter (warp & 3): window-query row r = 32 quarter + lane,
-    // key columns [64 half, 64 half + 64) of each tile, and O columns
-    // [D/2 half, D/2 half + D/2)
-    constexpr int NC = kFuKeys / 2;
-    constexpr int OC = D / 2;
-    const int sw = warp - 2, quarter = warp & 3, half = sw >> 2;
-    const int c0w = half * NC;
+    // ---------------- softmax groups ----------------
+    // group g takes tiles g, g + 2, ...; warp (warp & 3) of it owns window-query rows
+    // r = 32 (warp & 3) + lane, all 128 keys of a tile (four 32-key chunks) and the row
+    // of O_g
+    const int g = (warp - 2) >> 2, quarter = warp & 3;
     const int r = quarter * 32 + lane;
-    const int st = tid - 64;
     const int pos = L - W + (r % W);
     const bool row_ok = r < Qn && pos >= 0;
     const float qscale = kLog2e / sqrtf((float)D);
-    const float* lnh = logn ? logn + (size_t)unit * T_cap : nullptr;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-    const uint32_t o_cols = tmem + lane_base + 256 + half * OC;
-    unsigned char* p_hi = base + S::kPOff;
-    unsigned char* p_lo = p_hi + S::kPBytes;
+    const uint32_t s_cols = tmem + lane_base + (uint32_t)(g * kFuKeys);
+    const uint32_t o_cols = tmem + lane_base + 256 + (uint32_t)(g * D);
     float m_ref = -INFINITY, l = 0.f;
     bool live = true;
-    float ln_next = (lnh && st < kFuKeys && t0 + st < t1) ? lnh[t0 + st] : 0.f;
-    for (int i = 0; i < ntiles; ++i) {
-      const int buf = i & 1;
+    int n_mine = 0;
+    for (int i = g; i < ntiles; i += 2) {
+      const int k = i >> 1, s = i % ST;
       const int tb = t0 + i * kFuKeys;
-      const float ln_cur = ln_next;
-      if (lnh && st < kFuKeys) ln_next = (tb + kFuKeys + st < t1) ? lnh[tb + kFuKeys + st] : 0.f;
-      live = live && mbar_wait_ab(&s_full[buf], (i / 2) & 1, s_abort);
-      live = __all_sync(0xffffffffu, live);      // tcgen05.ld is warp-collective
-      float sv[NC];
+      ++n_mine;
+      live = live && mbar_wait_ab(&s_full[g], k & 1, s_abort);
+      live = live && mbar_wait_ab(&v_full[s], (i / ST) & 1, s_abort);   // log-counts, V
+      live = __all_sync(0xffffffffu, live);          // tcgen05.ld / st are warp-collective
+      const float* lnb = reinterpret_cast<const float*>(base + S::kLnOff + s * S::kLnSlot) + ln_off;
+      // logits x = s q.k + log2(e) logn in the log2 domain; masks only on the split's last
+      // tile and on keys the causal window hides from some queries
+      const bool interior = tb + kFuKeys <= t1 && tb + kFuKeys - 1 <= L - W;
+      auto logits = [&](float (&v)[32], int c) {
+        if (interior && row_ok) {
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            const float2 ln2 = has_ln ? make_float2(lnb[32 * c + j] * kLog2e, lnb[32 * c + j + 1] * kLog2e)
+                                      : make_float2(0.f, 0.f);
+            const float2 x = ffma2(make_float2(v[j], v[j + 1]), make_float2(qscale, qscale), ln2);
+            v[j] = x.x;
+            v[j + 1] = x.y;
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int t = tb + 32 * c + j;
+            const bool vis = row_ok && t < t1 && t <= pos;
+            v[j] = vis ? fmaf(v[j], qscale, has_ln ? lnb[32 * c + j] * kLog2e : 0.f) : -INFINITY;
+          }
+        }
+      };
+      // sweep 1: the tile's row maximum
+      float mt = -INFINITY;
       if (live) {
         tc_fence_after();
-        const uint32_t ta = tmem + lane_base + (uint32_t)(buf * kFuKeys + c0w);
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          float v[32];
+          tmem_ld32(s_cols + 32 * c, v);
+          logits(v, c);
+          float m4[4] = {v[0], v[1], v[2], v[3]};
 #pragma unroll
-        for (int c = 0; c < NC / 32; ++c) {
-          float part[32];
-          tmem_ld32(ta + c * 32, part);
-#pragma unroll
-          for (int j = 0; j < 32; ++j) sv[c * 32 + j] = part[j];
-        }
-      } else {
-#pragma unroll
-        for (int j = 0; j < NC; ++j) sv[j] = 0.f;
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_empty[buf]);
-      if (st < kFuKeys) lns[st] = ln_cur * kLog2e;
-      named_bar(1, kFuSoftThreads);                // (a) the tile's log-counts
-      // logits in the log2 domain; masks only on the split's last tile and on keys the
-      // causal window hides from some queries
-      const bool interior = tb + kFuKeys <= t1 && tb + kFuKeys - 1 <= L - W;
-      float pm = -INFINITY;
-      if (interior && row_ok && live) {
-#pragma unroll
-        for (int j = 0; j < NC; j += 4) {
-          const float4 lv = *reinterpret_cast<const float4*>(&lns[c0w + j]);
-          sv[j] = fmaf(sv[j], qscale, lv.x);
-          sv[j + 1] = fmaf(sv[j + 1], qscale, lv.y);
-          sv[j + 2] = fmaf(sv[j + 2], qscale, lv.z);
-          sv[j + 3] = fmaf(sv[j + 3], qscale, lv.w);
-        }
-      } else {
-#pragma unroll
-        for (int j = 0; j < NC; ++j) {
-          const int t = tb + c0w + j;
-          const bool vis = live && row_ok && t < t1 && t <= pos;
-          sv[j] = vis ? fmaf(sv[j], qscale, lns[c0w + j]) : -INFINITY;
+          for (int j = 4; j < 32; ++j) m4[j & 3] = fmaxf(m4[j & 3], v[j]);
+          mt = fmaxf(mt, fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])));
         }
       }
-      {
-        float tm[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) tm[k] = sv[k];
-#pragma unroll
-        for (int j = 8; j < NC; ++j) tm[j & 7] = fmaxf(tm[j & 7], sv[j]);
-        pm = fmaxf(fmaxf(fmaxf(tm[0], tm[1]), fmaxf(tm[2], tm[3])),
-                   fmaxf(fmaxf(tm[4], tm[5]), fmaxf(tm[6], tm[7])));
-      }
-      xch[half * 128 + r] = pm;
-      named_bar(1, kFuSoftThreads);                // (b) both halves' maxima
-      const float mt = fmaxf(pm, xch[(1 - half) * 128 + r]);
-      // the reference maximum moves only when the tile exceeds it by 2^8
+      // the reference maximum moves only when the tile exceeds it by 2^8; O_g, which the
+      // group's previous P V MMAs update, is then rescaled
       const float m_new = (mt > m_ref + kRescaleSlack) ? mt : m_ref;
       const bool resc = m_new != m_ref && m_ref > -INFINITY;
       const float cfac = resc ? ex2_ftz(m_ref - m_new) : 1.f;
-      float psum[8];
+      if (__any_sync(0xffffffffu, resc)) {
+        live = live && mbar_wait_ab(&pv_done[g], (k - 1) & 1, s_abort);
+        live = __all_sync(0xffffffffu, live);
+        if (live) {
+          tc_fence_after();
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            float ov[32];
+            tmem_ld32(o_cols + 32 * c, ov);
 #pragma unroll
-      for (int k = 0; k < 8; ++k) psum[k] = 0.f;
-      if (m_new > -INFINITY) {
-#pragma unroll
-        for (int j = 0; j < NC; ++j) {
-          sv[j] = ex2_ftz(sv[j] - m_new);          // -inf -> 0
-          psum[j & 7] += sv[j];
-        }
-      } else {
-#pragma unroll
-        for (int j = 0; j < NC; ++j) sv[j] = 0.f;
-      }
-      l = l * cfac + (((psum[0] + psum[1]) + (psum[2] + psum[3])) +
-                      ((psum[4] + psum[5]) + (psum[6] + psum[7])));
-      // P of this tile replaces the previous one: the previous tile's P V MMAs (which
-      // also update O) must be done
-      if (i > 0) live = live && mbar_wait_ab(pv_done, (i - 1) & 1, s_abort);
-      live = __all_sync(0xffffffffu, live);
-      if (live && __any_sync(0xffffffffu, resc)) {
-        tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < OC / 32; ++c) {
-          float ov[32];
-          tmem_ld32(o_cols + c * 32, ov);
-#pragma unroll
-          for (int j = 0; j < 32; ++j) ov[j] *= cfac;
-          tmem_st32(o_cols + c * 32, ov);
-        }
-        tc_fence_before();
-      }
-      // P as bf16 hi and lo parts, 128-byte swizzled K-major rows (the MMA's A operand)
-#pragma unroll
-      for (int k = 0; k < NC / 8; ++k) {
-        uint32_t hi[4], lo[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float a = sv[8 * k + 2 * e], c = sv[8 * k + 2 * e + 1];
-          hi[e] = pack_bf16x2(a, c);
-          lo[e] = pack_bf16x2(a - bf16_lo(hi[e]), c - bf16_hi(hi[e]));
-        }
-        const uint32_t off = (uint32_t)(half * S::kBox) + swz128(r, k);
-        *reinterpret_cast<uint4*>(p_hi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4*>(p_lo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-      }
-      // value rows past the split's end may hold anything (even non-finite): zero them,
-      // since their probability is 0 and 0 x inf is not
-      const int nvalid = min(kFuKeys, t1 - tb);
-      if (nvalid < kFuKeys) {
-        const int vs = i % ST;
-        const bool vok = mbar_wait_ab(&v_full[vs], (i / ST) & 1, s_abort);
-        if (vok) {
-          unsigned char* vt = base + S::kVOff + vs * S::kTile;
-          const int nz = (kFuKeys - nvalid) * S::kBoxes * 8;   // 16-byte chunks
-          for (int idx = st; idx < nz; idx += kFuSoftThreads) {
-            const int rr = nvalid + idx / (S::kBoxes * 8);
-            const int rem = idx % (S::kBoxes * 8);
-            *reinterpret_cast<uint4*>(vt + (rem >> 3) * S::kBox + rr * 128 + (rem & 7) * 16) =
-                make_uint4(0u, 0u, 0u, 0u);
+            for (int j = 0; j < 32; ++j) ov[j] *= cfac;
+            tmem_st32(o_cols + 32 * c, ov);
           }
-        } else {
-          live = false;
+        }
+      }
+      // sweep 2: P = 2^(x - m) as bf16 hi and lo parts over the chunk's own S columns
+      float lsum = 0.f;
+      if (live) {
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          float v[32];
+          tmem_ld32(s_cols + 32 * c, v);
+          logits(v, c);
+          uint32_t hi[16], lo[16];
+          float ps[2] = {0.f, 0.f};
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            const float pa = m_new > -INFINITY ? ex2_ftz(v[j] - m_new) : 0.f;
+            const float pb = m_new > -INFINITY ? ex2_ftz(v[j + 1] - m_new) : 0.f;
+            ps[0] += pa;
+            ps[1] += pb;
+            const uint32_t hh = pack_bf16x2(pa, pb);
+            hi[j >> 1] = hh;
+            lo[j >> 1] = pack_bf16x2(pa - bf16_lo(hh), pb - bf16_hi(hh));
+          }
+          lsum += ps[0] + ps[1];
+          tmem_st16(s_cols + 32 * c, hi);
+          tmem_st16(s_cols + 32 * c + 16, lo);
+        }
+      }
+      l = l * cfac + lsum;
+      // value rows past the split's end may hold anything (even non-finite): zero them,
+      // since their probability is 0 and 0 x inf is not (this group's four warps split it)
+      const int nvalid = min(kFuKeys, t1 - tb);
+      if (nvalid < kFuKeys && live) {
+        unsigned char* vt = base + S::kVOff + s * S::kTile;
+        const int nz = (kFuKeys - nvalid) * S::kBoxes * 8;    // 16-byte chunks
+        for (int idx = quarter * 32 + lane; idx < nz; idx += 128) {
+          const int rr = nvalid + idx / (S::kBoxes * 8);
+          const int rem = idx % (S::kBoxes * 8);
+          *reinterpret_cast<uint4*>(vt + (rem >> 3) * S::kBox + rr * 128 + (rem & 7) * 16) =
+              make_uint4(0u, 0u, 0u, 0u);
         }
       }
       fence_proxy_async_smem();                    // generic writes -> tensor-core reads
+      tc_fence_before();                           // tensor-memory stores -> the MMA's reads
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(&p_full[g]);
       m_ref = m_new;
     }
     if (!live) set_flag(flags, KVS_FLAG_TIMEOUT);
-    // per-split outputs: (m, l) per query row and the unnormalised O row
-    float oreg[OC];
-#pragma unroll
-    for (int j = 0; j < OC; ++j) oreg[j] = 0.f;
-    bool got = ntiles > 0 && live && mbar_wait_ab(pv_done, (ntiles - 1) & 1, s_abort);
+    // this group's partial: (m, l) per query row and the unnormalised O row, stored as
+    // partial 2 split + g
+    bool got = n_mine > 0 && live && mbar_wait_ab(&pv_done[g], (n_mine - 1) & 1, s_abort);
     got = __all_sync(0xffffffffu, got);
-    if (got) {
-      tc_fence_after();
-#pragma unroll
-      for (int c = 0; c < OC / 32; ++c) {
-        float ov[32];
-        tmem_ld32(o_cols + c * 32, ov);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) oreg[c * 32 + j] = ov[j];
-      }
-    } else if (ntiles > 0) {
-      set_flag(flags, KVS_FLAG_TIMEOUT);
-    }
-    named_bar(1, kFuSoftThreads);                  // every read of xch is done
-    xch[half * 128 + r] = l;
-    named_bar(1, kFuSoftThreads);
+    if (n_mine > 0 && !got) set_flag(flags, KVS_FLAG_TIMEOUT);
+    const bool any = got && row_ok && m_ref > -INFINITY && l > 0.f;
+    const size_t prow = ((size_t)unit * (2 * nsplit) + 2 * split + g) * Qn + r;
     if (r < Qn) {
-      const float ltot = l + xch[(1 - half) * 128 + r];
-      const bool any = row_ok && m_ref > -INFINITY && ltot > 0.f && got;
-      const size_t prow = ((size_t)unit * nsplit + split) * Qn + r;
-      if (half == 0) {
-        part_ml[prow * 2 + 0] = any ? m_ref : -INFINITY;
-        part_ml[prow * 2 + 1] = any ? ltot : 0.f;
-      }
-      float* po = part_o + prow * D + half * OC;
+      part_ml[prow * 2 + 0] = any ? m_ref : -INFINITY;
+      part_ml[prow * 2 + 1] = any ? l : 0.f;
+    }
+    if (got) tc_fence_after();
+#pragma unroll 1
+    for (int c = 0; c < D / 32; ++c) {
+      float ov[32];
+      if (got) {
+        tmem_ld32(o_cols + 32 * c, ov);
+      } else {
 #pragma unroll
-      for (int j = 0; j < OC; j += 4)
-        *reinterpret_cast<float4*>(po + j) = any ? make_float4(oreg[j], oreg[j + 1], oreg[j + 2], oreg[j + 3])
-                                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j = 0; j < 32; ++j) ov[j] = 0.f;
+      }
+      if (r < Qn) {
+        float* po = part_o + prow * D + 32 * c;
+#pragma unroll
+        for (int j = 0; j < 32; j += 4)
+          *reinterpret_cast<float4*>(po + j) =
+              any ? make_float4(ov[j], ov[j + 1], ov[j + 2], ov[j + 3]) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
     }
   }
 
@@ -454,68 +428,70 @@ window_fa_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, kFaTmemCols);
+    tmem_dealloc(tmem, kFuTmemCols);
   }
 }
 
 // ---------------------------------------------------------------------------
-// Combine: per KV head, the splits' (m, l, O) -> (M, L) and o_q per window query,
-// |o_q|^2, o_q as bf16 hi / lo rows, and o_bar = mean_q o_q
+// Combine: per KV head, the partials' (m, l, O) -> (M, L) and o_q per window query,
+// o_bar, and for the per-query form e_q = o_q - o_bar as bf16 hi / mid / lo rows with
+// |e_q|^2 and o_bar . e_q
 // ---------------------------------------------------------------------------
 
 template <int D>
 __global__ void __launch_bounds__(D)
 fa_combine_kernel(const float* __restrict__ part_ml, const float* __restrict__ part_o, int Qn,
-                  int nsplit, float* __restrict__ stats, float* __restrict__ obar,
-                  float* __restrict__ zq_out, float* __restrict__ wq_out, bf16* __restrict__ eq_hi,
-                  bf16* __restrict__ eq_lo) {
-  extern __shared__ float fac[];                 // [Qn][nsplit] split weights 2^(m - M) / L
+                  int nparts, float* __restrict__ stats, float* __restrict__ obar,
+                  float* __restrict__ zq_out, float* __restrict__ wq_out, bf16* __restrict__ e_hi,
+                  bf16* __restrict__ e_mid, bf16* __restrict__ e_lo) {
+  extern __shared__ float fac[];                 // [Qn][nparts] weights 2^(m - M) / L
   __shared__ float s_z[D / 32][128], s_w[D / 32][128];
   __shared__ int s_valid;
   const int unit = blockIdx.x, c = threadIdx.x, lane = c & 31, wid = c >> 5;
   if (c == 0) s_valid = 0;
   __syncthreads();
   for (int q = c; q < Qn; q += D) {
-    const float* e = part_ml + (size_t)unit * nsplit * Qn * 2;
+    const float* e = part_ml + (size_t)unit * nparts * Qn * 2;
     float M = -INFINITY;
-    for (int s = 0; s < nsplit; ++s) {
+    for (int s = 0; s < nparts; ++s) {
       const float ls = e[((size_t)s * Qn + q) * 2 + 1];
       if (ls > 0.f) M = fmaxf(M, e[((size_t)s * Qn + q) * 2]);
     }
     float Ls = 0.f;
     if (M > -INFINITY)
-      for (int s = 0; s < nsplit; ++s) {
+      for (int s = 0; s < nparts; ++s) {
         const float ls = e[((size_t)s * Qn + q) * 2 + 1];
         if (ls > 0.f) Ls = fmaf(ls, exp2f(e[((size_t)s * Qn + q) * 2] - M), Ls);
       }
     const bool valid = Ls > 0.f;
-    for (int s = 0; s < nsplit; ++s) {
+    for (int s = 0; s < nparts; ++s) {
       const float ls = e[((size_t)s * Qn + q) * 2 + 1];
-      fac[q * nsplit + s] = (valid && ls > 0.f) ? exp2f(e[((size_t)s * Qn + q) * 2] - M) / Ls : 0.f;
+      fac[q * nparts + s] = (valid && ls > 0.f) ? exp2f(e[((size_t)s * Qn + q) * 2] - M) / Ls : 0.f;
     }
     stats[((size_t)unit * Qn + q) * 2 + 0] = M;
     stats[((size_t)unit * Qn + q) * 2 + 1] = Ls;
     if (valid) atomicAdd(&s_valid, 1);
   }
   __syncthreads();
-  const float* po = part_o + (size_t)unit * nsplit * Qn * D;
+  const float* po = part_o + (size_t)unit * nparts * Qn * D;
   auto o_of = [&](int q) {
     float o = 0.f;
-    for (int s = 0; s < nsplit; ++s) o = fmaf(fac[q * nsplit + s], po[((size_t)s * Qn + q) * D + c], o);
+    for (int s = 0; s < nparts; ++s) o = fmaf(fac[q * nparts + s], po[((size_t)s * Qn + q) * D + c], o);
     return o;
   };
   float acc = 0.f;
   for (int q = 0; q < Qn; ++q) acc += o_of(q);
   const float ob = s_valid > 0 ? acc / (float)s_valid : 0.f;
   obar[(size_t)unit * D + c] = ob;
-  // o_q relative to o_bar, for the per-query window form: e_q = o_q - o_bar as bf16 hi / lo
-  // rows (rows past Qn are zero), |e_q|^2 and o_bar . e_q
   for (int q = 0; q < 128; ++q) {
     const float e = q < Qn ? o_of(q) - ob : 0.f;
     const bf16 hi = __float2bfloat16_rn(e);
+    const float r1 = e - __bfloat162float(hi);
+    const bf16 mid = __float2bfloat16_rn(r1);
     const size_t at = ((size_t)unit * 128 + q) * D + c;
-    eq_hi[at] = hi;
-    eq_lo[at] = __float2bfloat16_rn(e - __bfloat162float(hi));
+    e_hi[at] = hi;
+    e_mid[at] = mid;
+    e_lo[at] = __float2bfloat16_rn(r1 - __bfloat162float(mid));
     const float z = warp_sum(e * e), wv = warp_sum(ob * e);
     if (lane == 0) {
       s_z[wid][q] = z;
@@ -544,30 +520,25 @@ struct ScShape {
   static constexpr int kBoxes = D / 64;
   static constexpr int kBox = 128 * 128;
   static constexpr int kTile = kBoxes * kBox;
-  static constexpr int kStages = PERQ ? (D == 128 ? 1 : 2) : 2;
+  static constexpr int kStages = PERQ ? (D == 128 ? 1 : 2) : (D == 128 ? 3 : 4);
   static constexpr int kQOff = 0;
-  static constexpr int kOOff = kTile;                        // per query form: O_hi, O_lo
-  static constexpr int kStageOff = kOOff + (PERQ ? 2 * kTile : 0);
+  static constexpr int kEOff = kTile;                        // per query form: E hi, mid, lo
+  static constexpr int kStageOff = kEOff + (PERQ ? 3 * kTile : 0);
   static constexpr int kStageBytes = 2 * kTile;              // K tile, then V tile
   static constexpr int kSmallOff = kStageOff + kStages * kStageBytes;
-  // barriers (128 B), Z_q = M_q + log2 L_q [128], o_bar [D], |e_q|^2 and o_bar . e_q
-  // [2][128] (per query form),
-  // per-key partial window mass [2 bufs][2 halves][128], per-pair terms [64][4],
-  // per-pair partial norms [2 halves][64][3], tensor-memory address and abort flag
-  static constexpr int kBarBytes = 128;
-  static constexpr int kZOff = kSmallOff + kBarBytes;         // Z_q [128]
-  static constexpr int kObOff = kZOff + 128 * 4;              // o_bar [D <= 128]
-  static constexpr int kOn2Off = kObOff + 128 * 4;            // |e_q|^2, o_bar.e_q [2][128]
-  static constexpr int kAbarOff = kOn2Off + (PERQ ? 2 * 128 * 4 : 0);
-  static constexpr int kTermOff = kAbarOff + (PERQ ? 0 : 4 * 128 * 4);
-  static constexpr int kNormOff = kTermOff + (PERQ ? 64 * 4 * 4 : 0);
-  static constexpr int kQmodOff = kNormOff + (PERQ ? 2 * 64 * 3 * 4 : 0);   // q mod W [128]
-  static constexpr int kMiscOff = kQmodOff + 128 * 4;
+  // barriers (128 B), Z_q = M_q + log2 L_q [128], o_bar [D], q mod W [128], and for the
+  // per-query form |e_q|^2 and o_bar . e_q [2][128]; tensor-memory address, abort flag
+  static constexpr int kZOff = kSmallOff + 128;
+  static constexpr int kObOff = kZOff + 128 * 4;
+  static constexpr int kQmodOff = kObOff + 128 * 4;
+  static constexpr int kEqOff = kQmodOff + 128 * 4;
+  static constexpr int kMiscOff = kEqOff + (PERQ ? 2 * 128 * 4 : 0);
   static constexpr int kSmem = kMiscOff + 16 + 1024;
   static_assert(kSmem <= 232448, "shared memory");
 };
 
-constexpr uint32_t kScTmemCols = 512;   // S^T0 [0,128), S^T1 [128,256), U [256,384)
+// Tensor memory of pass B, per softmax group g: S^T_g at [128 g, 128 g + 128) and, per
+// query form, U_g = V E^T at [256 + 128 g, 256 + 128 g + 128).
 
 // One pair's norms -> (w_b, score), the closed forms of the forward-only objective.
 __device__ __forceinline__ void pair_weight_score(float n11, float n12, float n22, float dd,
@@ -588,33 +559,30 @@ __device__ __forceinline__ void pair_weight_score(float n11, float n12, float n2
 template <int D, bool PERQ>
 __global__ void __launch_bounds__(kFuThreads, 1)
 window_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmOh,
-                    const __grid_constant__ CUtensorMap tmOl, const float* __restrict__ logn,
-                    const int32_t* __restrict__ len, const int32_t* __restrict__ cand_begin,
-                    int n_recent, int H_kv, int H_q, int W, int T_cap, int nsplit, int form,
-                    const float* __restrict__ stats, const float* __restrict__ obar,
-                    const float* __restrict__ on2g, const float* __restrict__ wqg,
-                    float* __restrict__ score,
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmEh,
+                    const __grid_constant__ CUtensorMap tmEm, const __grid_constant__ CUtensorMap tmEl,
+                    const float* __restrict__ logn, const int32_t* __restrict__ len,
+                    const int32_t* __restrict__ cand_begin, int n_recent, int H_kv, int H_q,
+                    int W, int T_cap, int nsplit, int form, const float* __restrict__ stats,
+                    const float* __restrict__ obar, const float* __restrict__ zqg,
+                    const float* __restrict__ wqg, float* __restrict__ score,
                     float* __restrict__ w_b, int32_t* __restrict__ flags) {
   using S = ScShape<D, PERQ>;
   constexpr int ST = S::kStages;
   extern __shared__ unsigned char dsm[];
   unsigned char* base = align1024(dsm);
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + S::kSmallOff);
-  uint64_t* q_full = bars;              // 1 (Q and, per query, O_hi / O_lo)
+  uint64_t* q_full = bars;              // 1 (Q and, per query, E hi / mid / lo)
   uint64_t* full = q_full + 1;          // ST: K and V tiles of a stage landed
-  uint64_t* empty = full + ST;          // ST: every softmax warp is done with the stage
-  uint64_t* s_full = empty + ST;        // 2
+  uint64_t* empty = full + ST;          // ST: the four warps of the tile's group are done
+  uint64_t* s_full = empty + ST;        // 2 (per group)
   uint64_t* s_empty = s_full + 2;       // 2
-  uint64_t* u_full = s_empty + 2;       // 1 (per query form)
-  uint64_t* u_empty = u_full + 1;       // 1
+  uint64_t* u_full = s_empty + 2;       // 2 (per query form)
+  uint64_t* u_empty = u_full + 2;       // 2
   float* zq = reinterpret_cast<float*>(base + S::kZOff);
   float* obs = reinterpret_cast<float*>(base + S::kObOff);
-  float* on2 = reinterpret_cast<float*>(base + S::kOn2Off);     // |e_q|^2, then o_bar . e_q
-  float* abar = reinterpret_cast<float*>(base + S::kAbarOff);     // [2][2][128]
-  float* terms = reinterpret_cast<float*>(base + S::kTermOff);    // [64][4]
-  float* norms = reinterpret_cast<float*>(base + S::kNormOff);    // [2][64][3]
   int* qmod = reinterpret_cast<int*>(base + S::kQmodOff);
+  float* eqs = reinterpret_cast<float*>(base + S::kEqOff);        // |e_q|^2, o_bar.e_q
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(base + S::kMiscOff);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
 
@@ -633,7 +601,7 @@ window_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
   const int ntiles = tend - tbeg;
   if (ntiles <= 0) return;                           // uniform over the CTA
   const int q_row0 = (b * H_q + h * G) * W;
-  const int o_row0 = unit * 128;
+  const int e_row0 = unit * 128;
   const int k_row0 = unit * T_cap + c0 + tbeg * kFuKeys;
 
   if (tid == 0) {
@@ -641,14 +609,14 @@ window_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     mbar_init(q_full, 1);
     for (int s = 0; s < ST; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kFuSoft);
+      mbar_init(&empty[s], kFuGroupWarps);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&s_full[s], 1);
-      mbar_init(&s_empty[s], kFuSoft);
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(&s_full[g], 1);
+      mbar_init(&s_empty[g], kFuGroupWarps);
+      mbar_init(&u_full[g], 1);
+      mbar_init(&u_empty[g], kFuGroupWarps);
     }
-    mbar_init(u_full, 1);
-    mbar_init(u_empty, kFuSoft);
     fence_mbar_init();
   }
   // per-query constants: Z_q = M_q + log2 L_q (+inf: query without a visible key)
@@ -662,11 +630,11 @@ window_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     qmod[q] = q % W;
     obs[q] = q < D ? obar[(size_t)unit * D + q] : 0.f;
     if (PERQ) {
-      on2[q] = on2g[(size_t)unit * 128 + q];
-      on2[128 + q] = wqg[(size_t)unit * 128 + q];
+      eqs[q] = zqg[(size_t)unit * 128 + q];
+      eqs[128 + q] = wqg[(size_t)unit * 128 + q];
     }
   }
-  if (warp == 1) tmem_alloc(s_tmem, kScTmemCols);
+  if (warp == 1) tmem_alloc(s_tmem, kFuTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -681,30 +649,20 @@ window_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
-      const uint32_t qbytes = PERQ ? 3 * S::kTile : S::kTile;
-      mbar_arrive_expect_tx(q_full, qbytes);
+      mbar_arrive_expect_tx(q_full, PERQ ? 4 * S::kTile : S::kTile);
 #pragma unroll
       for (int bx = 0; bx < S::kBoxes; ++bx) {
         tma_load_2d(base + S::kQOff + bx * S::kBox, &tmQ, bx * 64, q_row0, q_full);
         if (PERQ) {
-          tma_load_2d(base + S::kOOff + bx * S::kBox, &tmOh, bx * 64, o_row0, q_full);
-          tma_load_2d(base + S::kOOff + S::kTile + bx * S::kBox, &tmOl, bx * 64, o_row0, q_full);
+          tma_load_2d(base + S::kEOff + bx * S::kBox, &tmEh, bx * 64, e_row0, q_full);
+          tma_load_2d(base + S::kEOff + S::kTile + bx * S::kBox, &tmEm, bx * 64, e_row0, q_full);
+          tma_load_2d(base + S::kEOff + 2 * S::kTile + bx * S::kBox, &tmEl, bx * 64, e_row0,
+                      q_full);
         }
       }
-      // tiles beyond the ring are prefetched into L2, kPrefetch tiles ahead
-      auto prefetch = [&](int i) {
-        if (i < ntiles)
-#pragma unroll
-          for (int bx = 0; bx < S::kBoxes; ++bx) {
-            tma_prefetch_2d(&tmK, bx * 64, k_row0 + i * kFuKeys);
-            tma_prefetch_2d(&tmV, bx * 64, k_row0 + i * kFuKeys);
-          }
-      };
-      for (int i = ST; i < ST + kPrefetch; ++i) prefetch(i);
       int issued = 0;
       for (int i = 0; i < ntiles; ++i) {
         const int s = i % ST;
-        prefetch(i + ST + kPrefetch);
         if (i >= ST && !mbar_wait_ab(&empty[s], ((i / ST) - 1) & 1, s_abort)) break;
         unsigned char* stg = base + S::kStageOff + s * S::kStageBytes;
         mbar_arrive_expect_tx(&full[s], S::kStageBytes);
@@ -722,19 +680,18 @@ window_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ---------------- MMA issuer: S^T = K Q^T (and U = V O^T) ----------------
+    // ---------------- MMA issuer: S^T = K Q^T (and U = V E^T) ----------------
     if (lane == 0) {
       constexpr uint32_t idesc = umma_idesc_bf16_f32(kFuKeys, 128);
       const uint32_t q_addr = smem_u32(base + S::kQOff);
-      const uint32_t oh_addr = smem_u32(base + S::kOOff);
-      const uint32_t ol_addr = oh_addr + S::kTile;
+      const uint32_t e_addr = smem_u32(base + S::kEOff);
       bool ok = mbar_wait_ab(q_full, 0, s_abort);
       int done = 0;
       for (int i = 0; ok && i < ntiles; ++i) {
-        const int s = i % ST, buf = i & 1;
+        const int s = i % ST, g = i & 1, k = i >> 1;
         if (!mbar_wait_ab(&full[s], (i / ST) & 1, s_abort) ||
-            (i >= 2 && !mbar_wait_ab(&s_empty[buf], ((i / 2) - 1) & 1, s_abort)) ||
-            (PERQ && i >= 1 && !mbar_wait_ab(u_empty, (i - 1) & 1, s_abort))) {
+            (k >= 1 && !mbar_wait_ab(&s_empty[g], (k - 1) & 1, s_abort)) ||
+            (PERQ && k >= 1 && !mbar_wait_ab(&u_empty[g], (k - 1) & 1, s_abort))) {
           ok = false;
           break;
         }
@@ -744,218 +701,197 @@ window_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t off = (uint32_t)((ks >> 2) * S::kBox + (ks & 3) * 32);
-          umma_bf16_ss(tmem + buf * kFuKeys, umma_desc_k_sw128(k_addr + off),
+          umma_bf16_ss(tmem + g * kFuKeys, umma_desc_k_sw128(k_addr + off),
                        umma_desc_k_sw128(q_addr + off), idesc, ks > 0 ? 1u : 0u);
         }
-        umma_commit(&s_full[buf]);
+        umma_commit(&s_full[g]);
         if (PERQ) {
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t off = (uint32_t)((ks >> 2) * S::kBox + (ks & 3) * 32);
-            umma_bf16_ss(tmem + 256, umma_desc_k_sw128(v_addr + off),
-                         umma_desc_k_sw128(oh_addr + off), idesc, ks > 0 ? 1u : 0u);
-            umma_bf16_ss(tmem + 256, umma_desc_k_sw128(v_addr + off),
-                         umma_desc_k_sw128(ol_addr + off), idesc, 1u);
-          }
-          umma_commit(u_full);
+          for (int part = 0; part < 3; ++part)
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks) {
+              const uint32_t off = (uint32_t)((ks >> 2) * S::kBox + (ks & 3) * 32);
+              umma_bf16_ss(tmem + 256 + g * kFuKeys, umma_desc_k_sw128(v_addr + off),
+                           umma_desc_k_sw128(e_addr + part * S::kTile + off), idesc,
+                           (part > 0 || ks > 0) ? 1u : 0u);
+            }
+          umma_commit(&u_full[g]);
         }
         done = i + 1;
       }
       if (!ok) set_flag(flags, KVS_FLAG_TIMEOUT);
-      if (done > 0 && !mbar_wait(&s_full[(done - 1) & 1], ((done - 1) / 2) & 1))
-        set_flag(flags, KVS_FLAG_TIMEOUT);
-      if (PERQ && done > 0 && !mbar_wait(u_full, (done - 1) & 1)) set_flag(flags, KVS_FLAG_TIMEOUT);
+      for (int g = 0; g < 2; ++g) {
+        const int n_g = done > g ? (done - 1 - g) / 2 + 1 : 0;
+        if (n_g > 0 && !mbar_wait(&s_full[g], (n_g - 1) & 1)) set_flag(flags, KVS_FLAG_TIMEOUT);
+        if (PERQ && n_g > 0 && !mbar_wait(&u_full[g], (n_g - 1) & 1))
+          set_flag(flags, KVS_FLAG_TIMEOUT);
+      }
     }
     __syncwarp();
   } else {
-    // ---------------- softmax warps ----------------
-    // warp 2 + sw owns lane quarter (warp & 3): key row kr = 32 quarter + lane of each
-    // tile, and window-query columns [64 half, 64 half + 64)
-    constexpr int NC = 64;
-    const int sw = warp - 2, quarter = warp & 3, half = sw >> 2;
+    // ---------------- softmax groups ----------------
+    // group g takes tiles g, g + 2, ...; warp (warp & 3) of it owns the keys
+    // kr = 32 (warp & 3) + lane of a tile with all 128 window-query columns, and its 16
+    // pairs: lanes 2 j and 2 j + 1 are the pair's two rows, and each of the two takes
+    // half of the head dimension for the row terms
+    const int g = (warp - 2) >> 2, quarter = warp & 3;
     const int kr = quarter * 32 + lane;
-    const int st = tid - 64;
-    const int qc0 = half * NC;
     const float qscale = kLog2e / sqrtf((float)D);
     const float* lnh = logn ? logn + (size_t)unit * T_cap : nullptr;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-    // pair-term threads: pair pp of the tile, quarter part of the head dimension
-    const int pp = st >> 2, part = st & 3;
-    constexpr int DP = D / 4;                     // dims per part: 32 or 16
-    const float* ob = obs + part * DP;
+    const uint32_t s_cols = tmem + lane_base + (uint32_t)(g * kFuKeys);
+    const uint32_t u_cols = tmem + lane_base + 256 + (uint32_t)(g * kFuKeys);
+    const bool is_a = (lane & 1) == 0;
+    const int ra = quarter * 32 + (lane & ~1), rb = ra + 1;   // the pair's rows in the tile
+    constexpr int DH = D / 2;                                  // dims per lane of a pair
+    const int dim0 = (lane & 1) * DH;
     bool live = true;
-    const int first_row = c0 + tbeg * kFuKeys;   // cache row of key 0 of tile 0
     float ln_next = 0.f;
-    if (lnh && tbeg * kFuKeys + kr < 2 * P) ln_next = lnh[first_row + kr];
-    for (int i = 0; i < ntiles; ++i) {
-      const int s = i % ST, buf = i & 1;
+    if (lnh && g < ntiles) {
+      const int kn = (tbeg + g) * kFuKeys + kr;
+      if (kn < 2 * P) ln_next = lnh[c0 + kn];
+    }
+    for (int i = g; i < ntiles; i += 2) {
+      const int k = i >> 1, s = i % ST;
       const int tile = tbeg + i;
       const int krow = tile * kFuKeys + kr;       // this thread's key, relative to c0
       const int t = c0 + krow;                    // its cache row
       const bool kval = krow < 2 * P;
       const float lnt = ln_next * kLog2e;
-      if (lnh && i + 1 < ntiles) {
-        const int kn = krow + kFuKeys;
+      if (lnh && i + 2 < ntiles) {
+        const int kn = krow + 2 * kFuKeys;
         ln_next = kn < 2 * P ? lnh[c0 + kn] : 0.f;
       }
-      live = live && mbar_wait_ab(&s_full[buf], (i / 2) & 1, s_abort);
+      const int hide = t - (L - W);               // queries with q mod W < hide miss the key
+      // the pair's row terms from the stage: |k_b - k_a|^2, |v_a - o_bar|^2,
+      // |v_b - o_bar|^2, |v_a + v_b - 2 o_bar|^2 (this lane's half of the dims)
+      live = live && mbar_wait_ab(&full[s], (i / ST) & 1, s_abort);
       live = __all_sync(0xffffffffu, live);
-      float sv[NC];
+      float dd = 0.f, ea = 0.f, eb = 0.f, ec = 0.f;
       if (live) {
-        tc_fence_after();
-        const uint32_t ta = tmem + lane_base + (uint32_t)(buf * kFuKeys + qc0);
-        tmem_ld32(ta, *reinterpret_cast<float(*)[32]>(sv));
-        tmem_ld32(ta + 32, *reinterpret_cast<float(*)[32]>(sv + 32));
-      } else {
+        const unsigned char* kt = base + S::kStageOff + s * S::kStageBytes;
+        const unsigned char* vt = kt + S::kTile;
 #pragma unroll
-        for (int j = 0; j < NC; ++j) sv[j] = 0.f;
+        for (int ch = 0; ch < DH / 8; ++ch) {
+          const int dim = dim0 + ch * 8;
+          const int bx = dim >> 6, cc = (dim & 63) >> 3;
+          const uint4 ka = *reinterpret_cast<const uint4*>(kt + bx * S::kBox + swz128(ra, cc));
+          const uint4 kb = *reinterpret_cast<const uint4*>(kt + bx * S::kBox + swz128(rb, cc));
+          const uint4 va = *reinterpret_cast<const uint4*>(vt + bx * S::kBox + swz128(ra, cc));
+          const uint4 vb = *reinterpret_cast<const uint4*>(vt + bx * S::kBox + swz128(rb, cc));
+          const uint32_t kaw[4] = {ka.x, ka.y, ka.z, ka.w}, kbw[4] = {kb.x, kb.y, kb.z, kb.w};
+          const uint32_t vaw[4] = {va.x, va.y, va.z, va.w}, vbw[4] = {vb.x, vb.y, vb.z, vb.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 o2 = *reinterpret_cast<const float2*>(obs + dim + 2 * e);
+            const float2 dk = make_float2(bf16_lo(kbw[e]) - bf16_lo(kaw[e]), bf16_hi(kbw[e]) - bf16_hi(kaw[e]));
+            const float2 ra2 = make_float2(bf16_lo(vaw[e]) - o2.x, bf16_hi(vaw[e]) - o2.y);
+            const float2 rb2 = make_float2(bf16_lo(vbw[e]) - o2.x, bf16_hi(vbw[e]) - o2.y);
+            const float2 rc2 = fadd2(ra2, rb2);
+            dd = fmaf(dk.x, dk.x, fmaf(dk.y, dk.y, dd));
+            ea = fmaf(ra2.x, ra2.x, fmaf(ra2.y, ra2.y, ea));
+            eb = fmaf(rb2.x, rb2.x, fmaf(rb2.y, rb2.y, eb));
+            ec = fmaf(rc2.x, rc2.x, fmaf(rc2.y, rc2.y, ec));
+          }
+        }
+      }
+      dd += __shfl_xor_sync(0xffffffffu, dd, 1);
+      ea += __shfl_xor_sync(0xffffffffu, ea, 1);
+      eb += __shfl_xor_sync(0xffffffffu, eb, 1);
+      ec += __shfl_xor_sync(0xffffffffu, ec, 1);
+      // window probabilities p_qt = 2^(s q.k + lnt - Z_q), the key's row of S^T
+      live = live && mbar_wait_ab(&s_full[g], k & 1, s_abort);
+      if (PERQ) live = live && mbar_wait_ab(&u_full[g], k & 1, s_abort);
+      live = __all_sync(0xffffffffu, live);
+      // the stage's rows are read, here and by the tile's MMAs (done: S^T, U landed)
+      if (lane == 0) mbar_arrive(&empty[s]);
+      if (live) tc_fence_after();
+      float acc = 0.f, n_self = 0.f, n_cpl = 0.f;
+      const float t_own = is_a ? ea : eb;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        float v[32];
+        if (live) {
+          tmem_ld32(s_cols + 32 * c, v);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = 0.f;
+        }
+        if (kval) {
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            const float2 z = *reinterpret_cast<const float2*>(&zq[32 * c + j]);
+            const float2 x = ffma2(make_float2(v[j], v[j + 1]), make_float2(qscale, qscale),
+                                   make_float2(lnt - z.x, lnt - z.y));
+            v[j] = ex2_ftz(x.x);
+            v[j + 1] = ex2_ftz(x.y);
+          }
+          if (hide > 0) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (qmod[32 * c + j] < hide) v[j] = 0.f;
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = 0.f;
+        }
+        if constexpr (!PERQ) {
+          float a4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int j = 0; j < 32; ++j) a4[j & 3] += v[j];
+          acc += (a4[0] + a4[1]) + (a4[2] + a4[3]);
+        } else {
+          // per window query: lane a (even key) takes N11 and N12, lane b N22
+          float u[32];
+          if (live) {
+            tmem_ld32(u_cols + 32 * c, u);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) u[j] = 0.f;
+          }
+#pragma unroll 8
+          for (int j = 0; j < 32; ++j) {
+            const float p = v[j], uu = u[j];
+            const float p_o = __shfl_xor_sync(0xffffffffu, p, 1);
+            const float u_o = __shfl_xor_sync(0xffffffffu, uu, 1);
+            const float z = eqs[32 * c + j], wq = eqs[128 + 32 * c + j];
+            n_self = fmaf(fabsf(p * (1.f - 2.f * p)),
+                          sqrtf(fmaxf(0.f, fmaf(-2.f, uu - wq, t_own) + z)), n_self);
+            if (is_a)
+              n_cpl = fmaf(p * p_o, sqrtf(fmaxf(0.f, fmaf(-4.f, uu + u_o - 2.f * wq, ec) + 4.f * z)),
+                           n_cpl);
+          }
+        }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&s_empty[buf]);
-      // p_qt = 2^(s q.k + lnt - Z_q); query q sees the key when t <= L - W + (q mod W)
-      if (kval) {
-#pragma unroll
-        for (int j = 0; j < NC; j += 2) {
-          const float2 z = *reinterpret_cast<const float2*>(&zq[qc0 + j]);
-          const float2 x = ffma2(make_float2(sv[j], sv[j + 1]), make_float2(qscale, qscale),
-                                 make_float2(lnt - z.x, lnt - z.y));
-          sv[j] = ex2_ftz(x.x);
-          sv[j + 1] = ex2_ftz(x.y);
-        }
-        const int hide = t - (L - W);             // queries with q mod W < hide miss it
-        if (hide > 0) {
-#pragma unroll
-          for (int j = 0; j < NC; ++j)
-            if (qmod[qc0 + j] < hide) sv[j] = 0.f;
-        }
-      } else {
-#pragma unroll
-        for (int j = 0; j < NC; ++j) sv[j] = 0.f;
+      if (lane == 0) {
+        mbar_arrive(&s_empty[g]);
+        if (PERQ) mbar_arrive(&u_empty[g]);
       }
-      const unsigned char* kt = base + S::kStageOff + s * S::kStageBytes;
-      const unsigned char* vt = kt + S::kTile;
-      bool sok = live && mbar_wait_ab(&full[s], (i / ST) & 1, s_abort);   // K, V rows landed
-      sok = __all_sync(0xffffffffu, sok);
-      live = live && sok;
+      // the pair's weight and score (lane a writes them)
+      float n11, n12, n22;
       if constexpr (!PERQ) {
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int j = 0; j < NC; ++j) acc[j & 3] += sv[j];
-        abar[(buf * 2 + half) * 128 + kr] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-        named_bar(1, kFuSoftThreads);
-      }
-      // the tile's pair pp: rows 2 pp, 2 pp + 1; this thread: dims [DP part, DP part + DP):
-      // |k_b - k_a|^2, |v_a - o_bar|^2, |v_b - o_bar|^2, |v_a + v_b - 2 o_bar|^2
-      float dd = 0.f, ea = 0.f, eb = 0.f, ec = 0.f;
-      const int ra = 2 * pp, rb = ra + 1;
-#pragma unroll
-      for (int ch = 0; ch < DP / 8; ++ch) {
-        const int dim = part * DP + ch * 8;
-        const int bx = dim >> 6, cc = (dim & 63) >> 3;
-        const uint4 ka = *reinterpret_cast<const uint4*>(kt + bx * S::kBox + swz128(ra, cc));
-        const uint4 kb = *reinterpret_cast<const uint4*>(kt + bx * S::kBox + swz128(rb, cc));
-        const uint4 va = *reinterpret_cast<const uint4*>(vt + bx * S::kBox + swz128(ra, cc));
-        const uint4 vb = *reinterpret_cast<const uint4*>(vt + bx * S::kBox + swz128(rb, cc));
-        const uint32_t kaw[4] = {ka.x, ka.y, ka.z, ka.w}, kbw[4] = {kb.x, kb.y, kb.z, kb.w};
-        const uint32_t vaw[4] = {va.x, va.y, va.z, va.w}, vbw[4] = {vb.x, vb.y, vb.z, vb.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 o2 = *reinterpret_cast<const float2*>(ob + ch * 8 + 2 * e);
-          const float2 dk = make_float2(bf16_lo(kbw[e]) - bf16_lo(kaw[e]), bf16_hi(kbw[e]) - bf16_hi(kaw[e]));
-          const float2 ra2 = make_float2(bf16_lo(vaw[e]) - o2.x, bf16_hi(vaw[e]) - o2.y);
-          const float2 rb2 = make_float2(bf16_lo(vbw[e]) - o2.x, bf16_hi(vbw[e]) - o2.y);
-          const float2 rc2 = fadd2(ra2, rb2);
-          dd = fmaf(dk.x, dk.x, fmaf(dk.y, dk.y, dd));
-          ea = fmaf(ra2.x, ra2.x, fmaf(ra2.y, ra2.y, ea));
-          eb = fmaf(rb2.x, rb2.x, fmaf(rb2.y, rb2.y, eb));
-          ec = fmaf(rc2.x, rc2.x, fmaf(rc2.y, rc2.y, ec));
-        }
-      }
-#pragma unroll
-      for (int o = 1; o < 4; o <<= 1) {
-        dd += __shfl_xor_sync(0xffffffffu, dd, o);
-        ea += __shfl_xor_sync(0xffffffffu, ea, o);
-        eb += __shfl_xor_sync(0xffffffffu, eb, o);
-        ec += __shfl_xor_sync(0xffffffffu, ec, o);
-      }
-      const int pglob = tile * (kFuKeys / 2) + pp;
-      if constexpr (!PERQ) {
-        if (part == 0 && pglob < P && live) {
-          const float* ab = abar + buf * 256;
-          const float aa = (ab[ra] + ab[128 + ra]) * inv_qv;
-          const float bb = (ab[rb] + ab[128 + rb]) * inv_qv;
-          const float n11 = fabsf(aa * (1.f - 2.f * aa)) * sqrtf(ea);
-          const float n22 = fabsf(bb * (1.f - 2.f * bb)) * sqrtf(eb);
-          const float n12 = aa * bb * sqrtf(ec);
-          float w, sc;
-          pair_weight_score(n11, n12, n22, dd, form, w, sc);
-          const size_t at = (size_t)unit * (T_cap / 2) + pglob;
-          score[at] = sc;
-          w_b[at] = w;
-        }
+        const float al = acc * inv_qv;
+        const float aa = __shfl_sync(0xffffffffu, al, lane & ~1);
+        const float bb = __shfl_sync(0xffffffffu, al, lane | 1);
+        n11 = fabsf(aa * (1.f - 2.f * aa)) * sqrtf(ea);
+        n22 = fabsf(bb * (1.f - 2.f * bb)) * sqrtf(eb);
+        n12 = aa * bb * sqrtf(ec);
       } else {
-        // per-query window form: U = V E^T gives v_t . e_q on the key's lane
-        bool uok = live && mbar_wait_ab(u_full, i & 1, s_abort);
-        uok = __all_sync(0xffffffffu, uok);
-        live = live && uok;
-        float uv[NC];
-        if (uok) {
-          tc_fence_after();
-          const uint32_t ta = tmem + lane_base + (uint32_t)(256 + qc0);
-          tmem_ld32(ta, *reinterpret_cast<float(*)[32]>(uv));
-          tmem_ld32(ta + 32, *reinterpret_cast<float(*)[32]>(uv + 32));
-        } else {
-#pragma unroll
-          for (int j = 0; j < NC; ++j) uv[j] = 0.f;
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(u_empty);
-        if (part == 0) {
-          terms[pp * 4 + 0] = dd;
-          terms[pp * 4 + 1] = ea;
-          terms[pp * 4 + 2] = eb;
-          terms[pp * 4 + 3] = ec;
-        }
-        named_bar(1, kFuSoftThreads);
-        // per window query of this half: lane a (even key) takes N11 and N12, lane b N22
-        const int pl = kr >> 1;
-        const bool is_a = (kr & 1) == 0;
-        const float t_own = is_a ? terms[pl * 4 + 1] : terms[pl * 4 + 2];
-        const float t_ab = terms[pl * 4 + 3];
-        float n_self = 0.f, n_cpl = 0.f;
-#pragma unroll 8
-        for (int j = 0; j < NC; ++j) {
-          const float p = sv[j], u = uv[j];
-          const float p_o = __shfl_xor_sync(0xffffffffu, p, 1);
-          const float u_o = __shfl_xor_sync(0xffffffffu, u, 1);
-          const float z = on2[qc0 + j], wq = on2[128 + qc0 + j];
-          n_self = fmaf(fabsf(p * (1.f - 2.f * p)),
-                        sqrtf(fmaxf(0.f, fmaf(-2.f, u - wq, t_own) + z)), n_self);
-          if (is_a)
-            n_cpl = fmaf(p * p_o, sqrtf(fmaxf(0.f, fmaf(-4.f, u + u_o - 2.f * wq, t_ab) + 4.f * z)),
-                         n_cpl);
-        }
-        norms[(half * 64 + pl) * 3 + (is_a ? 0 : 2)] = n_self;
-        if (is_a) norms[(half * 64 + pl) * 3 + 1] = n_cpl;
-        named_bar(1, kFuSoftThreads);
-        if (part == 0 && pglob < P && live) {
-          const float* n0 = norms + pp * 3;
-          const float* n1 = norms + (64 + pp) * 3;
-          const float n11 = (n0[0] + n1[0]) * inv_qv;
-          const float n12 = (n0[1] + n1[1]) * inv_qv;
-          const float n22 = (n0[2] + n1[2]) * inv_qv;
-          float w, sc;
-          pair_weight_score(n11, n12, n22, terms[pp * 4], form, w, sc);
-          const size_t at = (size_t)unit * (T_cap / 2) + pglob;
-          score[at] = sc;
-          w_b[at] = w;
-        }
-        named_bar(1, kFuSoftThreads);             // terms / norms are rewritten next tile
+        const float other = __shfl_xor_sync(0xffffffffu, n_self, 1);
+        n11 = (is_a ? n_self : other) * inv_qv;
+        n22 = (is_a ? other : n_self) * inv_qv;
+        n12 = n_cpl * inv_qv;
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
+      const int pglob = tile * (kFuKeys / 2) + (ra >> 1);
+      if (is_a && pglob < P && live) {
+        float w, sc;
+        pair_weight_score(n11, n12, n22, dd, form, w, sc);
+        const size_t at = (size_t)unit * (T_cap / 2) + pglob;
+        score[at] = sc;
+        w_b[at] = w;
+      }
     }
     if (!live) set_flag(flags, KVS_FLAG_TIMEOUT);
   }
@@ -964,7 +900,7 @@ window_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, kScTmemCols);
+    tmem_dealloc(tmem, kFuTmemCols);
   }
 }
 
@@ -996,45 +932,57 @@ static cudaError_t launch_fused_t(const kvs_cache_desc& d, const void* K, const 
   const unsigned long long rows = (unsigned long long)d.B * d.H_kv * (unsigned long long)d.T_cap;
   const unsigned long long qrows = (unsigned long long)d.B * d.H_q * (unsigned long long)W;
   const int units = d.B * d.H_kv;
-  bf16* oq_hi = reinterpret_cast<bf16*>(ws + Ly.oq_hi);
-  bf16* oq_lo = reinterpret_cast<bf16*>(ws + Ly.oq_lo);
-  CUtensorMap mQ, mK, mV, mOh, mOl;
+  bf16* e_hi = reinterpret_cast<bf16*>(ws + Ly.oq_hi);
+  bf16* e_mid = reinterpret_cast<bf16*>(ws + Ly.oq_mid);
+  bf16* e_lo = reinterpret_cast<bf16*>(ws + Ly.oq_lo);
+  CUtensorMap mQ, mK, mV, mL, mEh, mEm, mEl;
+  const unsigned long long erows = (unsigned long long)units * 128;
   if (!encode_rows_map(&mQ, Qw, qrows, D, 128) || !encode_rows_map(&mK, K, rows, D, kFuKeys) ||
-      !encode_rows_map(&mV, V, rows, D, kFuKeys) ||
-      !encode_rows_map(&mOh, oq_hi, (unsigned long long)units * 128, D, 128) ||
-      !encode_rows_map(&mOl, oq_lo, (unsigned long long)units * 128, D, 128))
+      !encode_rows_map(&mV, V, rows, D, kFuKeys) || !encode_rows_map(&mEh, e_hi, erows, D, 128) ||
+      !encode_rows_map(&mEm, e_mid, erows, D, 128) || !encode_rows_map(&mEl, e_lo, erows, D, 128))
     return cudaErrorInvalidValue;
-  const int nsa = fused_splits(units) < Ly.nsplit ? fused_splits(units) : Ly.nsplit;
+  int ln_lead = 0;
+  if (logn) {
+    if (!encode_ln_map(&mL, logn, rows, FaShape<D>::kLnBox, &ln_lead)) return cudaErrorInvalidValue;
+  } else {
+    mL = mK;   // never read
+  }
+  // pass A: two partials per CTA (one per softmax group), so at most half the layout's
+  // partial slots worth of CTAs per head
+  int nsa = fused_splits(units);
+  const int cap = Ly.part_slots / 2;
+  if (nsa > cap) nsa = cap;
   const int Qn = Ly.Qn;
   int32_t* flags = reinterpret_cast<int32_t*>(ws);
   float* part_ml = reinterpret_cast<float*>(ws + Ly.part_ml);
   float* part_o = reinterpret_cast<float*>(ws + Ly.part_o);
   float* stats = reinterpret_cast<float*>(ws + Ly.stats);
   float* obar = reinterpret_cast<float*>(ws + Ly.obar);
-  float* on2 = reinterpret_cast<float*>(ws + Ly.on2);
-  float* owq = reinterpret_cast<float*>(ws + Ly.owq);
+  float* zq = reinterpret_cast<float*>(ws + Ly.on2);
+  float* wq = reinterpret_cast<float*>(ws + Ly.owq);
 
   auto ka = window_fa_kernel<D>;
   if (!ensure_smem_attr((const void*)ka, FaShape<D>::kSmem)) return cudaErrorInvalidValue;
   ka<<<dim3(nsa, units), kFuThreads, FaShape<D>::kSmem, st>>>(
-      mQ, mK, mV, logn, len, d.H_kv, d.H_q, W, d.T_cap, nsa, part_ml, part_o, flags);
-  const size_t csm = (size_t)Qn * nsa * sizeof(float);
+      mQ, mK, mV, mL, ln_lead, logn != nullptr, len, d.H_kv, d.H_q, W, d.T_cap, nsa, part_ml,
+      part_o, flags);
+  const size_t csm = (size_t)Qn * 2 * nsa * sizeof(float);
   auto kc = fa_combine_kernel<D>;
   if (!ensure_smem_attr((const void*)kc, csm)) return cudaErrorInvalidValue;
-  kc<<<units, D, csm, st>>>(part_ml, part_o, Qn, nsa, stats, obar, on2, owq, oq_hi, oq_lo);
+  kc<<<units, D, csm, st>>>(part_ml, part_o, Qn, 2 * nsa, stats, obar, zq, wq, e_hi, e_mid, e_lo);
   const int nsb = fused_splits(units);
   if (stats_form == KVS_FORM_PER_QUERY) {
     auto kb = window_score_kernel<D, true>;
     if (!ensure_smem_attr((const void*)kb, ScShape<D, true>::kSmem)) return cudaErrorInvalidValue;
     kb<<<dim3(nsb, units), kFuThreads, ScShape<D, true>::kSmem, st>>>(
-        mQ, mK, mV, mOh, mOl, logn, len, cand_begin, n_recent, d.H_kv, d.H_q, W, d.T_cap, nsb,
-        form, stats, obar, on2, owq, score, w_b, flags);
+        mQ, mK, mV, mEh, mEm, mEl, logn, len, cand_begin, n_recent, d.H_kv, d.H_q, W, d.T_cap,
+        nsb, form, stats, obar, zq, wq, score, w_b, flags);
   } else {
     auto kb = window_score_kernel<D, false>;
     if (!ensure_smem_attr((const void*)kb, ScShape<D, false>::kSmem)) return cudaErrorInvalidValue;
     kb<<<dim3(nsb, units), kFuThreads, ScShape<D, false>::kSmem, st>>>(
-        mQ, mK, mV, mOh, mOl, logn, len, cand_begin, n_recent, d.H_kv, d.H_q, W, d.T_cap, nsb,
-        form, stats, obar, on2, owq, score, w_b, flags);
+        mQ, mK, mV, mEh, mEm, mEl, logn, len, cand_begin, n_recent, d.H_kv, d.H_q, W, d.T_cap,
+        nsb, form, stats, obar, zq, wq, score, w_b, flags);
   }
   count_launches(3);
   return cudaGetLastError();

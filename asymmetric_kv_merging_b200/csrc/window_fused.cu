@@ -80,16 +80,19 @@ struct FaShape {
   static constexpr int kBox = 128 * 128;                 // 128 rows x 128 bytes
   static constexpr int kTile = kBoxes * kBox;            // a Q, K or V tile
   static constexpr int kStages = D == 128 ? 3 : 4;
-  static constexpr int kLnBox = kFuKeys + 4;             // floats, from a 16-byte boundary
-  static constexpr int kLnSlot = 544;                    // bytes per stage (>= 4 kLnBox)
+  static constexpr int kLnSlot = kFuKeys * 4;            // log-counts of a tile (bytes)
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kQOff + kTile;
   static constexpr int kVOff = kKOff + kStages * kTile;
   static constexpr int kLnOff = kVOff + kStages * kTile;
   static constexpr int kSmallOff = kLnOff + kStages * kLnSlot;
   static constexpr int kSmem = kSmallOff + 256 + 16 + 1024;   // barriers, misc, alignment
-  static_assert(4 * kLnBox <= kLnSlot && kLnSlot % 16 == 0, "log-count slot");
   static_assert(kSmem <= 232448, "shared memory");
+  // TMA tile destinations with 128-byte swizzling start on 1024-byte boundaries; the
+  // log-count slots take 16-byte vector stores; the barriers (1 + 4 ST + 6) fit 256 bytes
+  static_assert(kKOff % 1024 == 0 && kVOff % 1024 == 0 && kTile % 1024 == 0, "tile alignment");
+  static_assert(kLnOff % 16 == 0 && kLnSlot % 16 == 0 && kSmallOff % 8 == 0, "slot alignment");
+  static_assert(8 * (1 + 4 * kStages + 6) <= 256, "barrier room");
 };
 
 // Tensor memory of pass A, per softmax group g: S_g at columns [128 g, 128 g + 128) --
@@ -99,10 +102,10 @@ struct FaShape {
 template <int D>
 __global__ void __launch_bounds__(kFuThreads, 1)
 window_fa_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmL,
-                 int ln_lead, bool has_ln, const int32_t* __restrict__ len, int H_kv, int H_q,
-                 int W, int T_cap, int nsplit, float* __restrict__ part_ml,
-                 float* __restrict__ part_o, int32_t* __restrict__ flags) {
+                 const __grid_constant__ CUtensorMap tmV, const float* __restrict__ logn,
+                 const int32_t* __restrict__ len, int H_kv, int H_q, int W, int T_cap, int nsplit,
+                 float* __restrict__ part_ml, float* __restrict__ part_o,
+                 int32_t* __restrict__ flags) {
   using S = FaShape<D>;
   constexpr int ST = S::kStages;
   extern __shared__ unsigned char dsm[];
@@ -111,7 +114,7 @@ window_fa_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   uint64_t* q_full = bars;              // 1
   uint64_t* k_full = q_full + 1;        // ST
   uint64_t* k_empty = k_full + ST;      // ST: the QK^T MMA of the stage is done
-  uint64_t* v_full = k_empty + ST;      // ST: V rows and log-counts
+  uint64_t* v_full = k_empty + ST;      // ST: V rows (TMA) and log-counts (producer lanes)
   uint64_t* v_empty = v_full + ST;      // ST: the P V MMAs of the stage are done
   uint64_t* s_full = v_empty + ST;      // 2 (per group)
   uint64_t* p_full = s_full + 2;        // 2: the group's four warps have written P
@@ -134,9 +137,8 @@ window_fa_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   const int ntiles = t1 > t0 ? (t1 - t0 + kFuKeys - 1) / kFuKeys : 0;
   const int q_row0 = (b * H_q + h * G) * W;
   const int k_row0 = unit * T_cap + t0;
-  // log-counts of tile i start at element ln_lead + k_row0 + 128 i of the map; its box
-  // starts at the 4-element boundary below, the same offset for every tile
-  const int ln_off = (ln_lead + k_row0) & 3;
+  const bool has_ln = logn != nullptr;
+  const float* lnh = has_ln ? logn + (size_t)unit * T_cap : nullptr;
 
   if (tid == 0) {
     *s_abort = 0;
@@ -144,7 +146,7 @@ window_fa_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     for (int s = 0; s < ST; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&k_empty[s], 1);
-      mbar_init(&v_full[s], 1);
+      mbar_init(&v_full[s], 1 + 32);     // the TMA transaction, then each producer lane
       mbar_init(&v_empty[s], 1);
     }
     for (int g = 0; g < 2; ++g) {
@@ -161,40 +163,62 @@ window_fa_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   const uint32_t tmem = *s_tmem;
 
   if (warp == 0) {
-    // ---------------- TMA producer ----------------
+    // ---------------- producer warp ----------------
+    // lane 0 issues the TMA loads; every lane loads four log-counts of each tile into the
+    // V stage's slot (plain loads, one tile ahead) and arrives on the stage's barrier
     if (lane == 0) {
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
-      if (has_ln) prefetch_tmap(&tmL);
       mbar_arrive_expect_tx(q_full, S::kTile);
 #pragma unroll
       for (int bx = 0; bx < S::kBoxes; ++bx)
         tma_load_2d(base + S::kQOff + bx * S::kBox, &tmQ, bx * 64, q_row0, q_full);
-      int issued_k = 0, issued_v = 0;
-      for (int i = 0; i < ntiles; ++i) {
-        const int s = i % ST;
-        const uint32_t ph = ((i / ST) - 1) & 1;
-        if (i >= ST && !mbar_wait_ab(&k_empty[s], ph, s_abort)) break;
-        mbar_arrive_expect_tx(&k_full[s], S::kTile);
+    }
+    auto ln4 = [&](int i) {
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (has_ln && i < ntiles) {
+        const int t = t0 + i * kFuKeys + 4 * lane;
+        v.x = t < t1 ? lnh[t] : 0.f;
+        v.y = t + 1 < t1 ? lnh[t + 1] : 0.f;
+        v.z = t + 2 < t1 ? lnh[t + 2] : 0.f;
+        v.w = t + 3 < t1 ? lnh[t + 3] : 0.f;
+      }
+      return v;
+    };
+    float4 ln_next = ln4(0);
+    int issued_k = 0, issued_v = 0;
+    for (int i = 0; i < ntiles; ++i) {
+      const int s = i % ST;
+      const uint32_t ph = ((i / ST) - 1) & 1;
+      bool ok = true;
+      if (lane == 0) {
+        ok = i < ST || mbar_wait_ab(&k_empty[s], ph, s_abort);
+        if (ok) {
+          mbar_arrive_expect_tx(&k_full[s], S::kTile);
 #pragma unroll
-        for (int bx = 0; bx < S::kBoxes; ++bx)
-          tma_load_2d(base + S::kKOff + s * S::kTile + bx * S::kBox, &tmK, bx * 64,
-                      k_row0 + i * kFuKeys, &k_full[s]);
-        issued_k = i + 1;
-        if (i >= ST && !mbar_wait_ab(&v_empty[s], ph, s_abort)) break;
-        mbar_arrive_expect_tx(&v_full[s], S::kTile + (has_ln ? S::kLnBox * 4 : 0));
+          for (int bx = 0; bx < S::kBoxes; ++bx)
+            tma_load_2d(base + S::kKOff + s * S::kTile + bx * S::kBox, &tmK, bx * 64,
+                        k_row0 + i * kFuKeys, &k_full[s]);
+        }
+      }
+      if (!__all_sync(0xffffffffu, ok)) break;
+      issued_k = i + 1;
+      ok = i < ST || mbar_wait_ab(&v_empty[s], ph, s_abort);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&v_full[s], S::kTile);
 #pragma unroll
         for (int bx = 0; bx < S::kBoxes; ++bx)
           tma_load_2d(base + S::kVOff + s * S::kTile + bx * S::kBox, &tmV, bx * 64,
                       k_row0 + i * kFuKeys, &v_full[s]);
-        if (has_ln) {
-          const uint64_t once = policy_evict_first();
-          tma_load_1d_hint(base + S::kLnOff + s * S::kLnSlot, &tmL,
-                           ln_lead + k_row0 + i * kFuKeys - ln_off, &v_full[s], once);
-        }
-        issued_v = i + 1;
       }
+      *reinterpret_cast<float4*>(base + S::kLnOff + s * S::kLnSlot + 16 * lane) = ln_next;
+      mbar_arrive(&v_full[s]);
+      ln_next = ln4(i + 1);
+      issued_v = i + 1;
+    }
+    if (lane == 0) {
       if (issued_v < ntiles) set_flag(flags, KVS_FLAG_TIMEOUT);
       // copies still in flight must land before the CTA ends (the plain bound, even after
       // an abort: these are this CTA's own copies)
@@ -289,7 +313,7 @@ window_fa_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       live = live && mbar_wait_ab(&s_full[g], k & 1, s_abort);
       live = live && mbar_wait_ab(&v_full[s], (i / ST) & 1, s_abort);   // log-counts, V
       live = __all_sync(0xffffffffu, live);          // tcgen05.ld / st are warp-collective
-      const float* lnb = reinterpret_cast<const float*>(base + S::kLnOff + s * S::kLnSlot) + ln_off;
+      const float* lnb = reinterpret_cast<const float*>(base + S::kLnOff + s * S::kLnSlot);
       // logits x = s q.k + log2(e) logn in the log2 domain; masks only on the split's last
       // tile and on keys the causal window hides from some queries
       const bool interior = tb + kFuKeys <= t1 && tb + kFuKeys - 1 <= L - W;
@@ -526,15 +550,22 @@ struct ScShape {
   static constexpr int kStageOff = kEOff + (PERQ ? 3 * kTile : 0);
   static constexpr int kStageBytes = 2 * kTile;              // K tile, then V tile
   static constexpr int kSmallOff = kStageOff + kStages * kStageBytes;
-  // barriers (128 B), Z_q = M_q + log2 L_q [128], o_bar [D], q mod W [128], and for the
+  // barriers (256 B), Z_q = M_q + log2 L_q [128], o_bar [D], q mod W [128], and for the
   // per-query form |e_q|^2 and o_bar . e_q [2][128]; tensor-memory address, abort flag
-  static constexpr int kZOff = kSmallOff + 128;
+  static constexpr int kZOff = kSmallOff + 256;
   static constexpr int kObOff = kZOff + 128 * 4;
   static constexpr int kQmodOff = kObOff + 128 * 4;
   static constexpr int kEqOff = kQmodOff + 128 * 4;
   static constexpr int kMiscOff = kEqOff + (PERQ ? 2 * 128 * 4 : 0);
   static constexpr int kSmem = kMiscOff + 16 + 1024;
   static_assert(kSmem <= 232448, "shared memory");
+  // TMA tile destinations with 128-byte swizzling start on 1024-byte boundaries; the
+  // barriers (1 + 2 ST + 8) fit the 256 bytes before Z_q; the float2 reads of Z_q and
+  // o_bar are 8-byte aligned
+  static_assert(kEOff % 1024 == 0 && kStageOff % 1024 == 0 && kStageBytes % 1024 == 0,
+                "tile alignment");
+  static_assert(8 * (1 + 2 * kStages + 8) <= kZOff - kSmallOff, "barrier room");
+  static_assert(kSmallOff % 8 == 0 && kZOff % 8 == 0 && kObOff % 8 == 0, "array alignment");
 };
 
 // Tensor memory of pass B, per softmax group g: S^T_g at [128 g, 128 g + 128) and, per
@@ -935,18 +966,12 @@ static cudaError_t launch_fused_t(const kvs_cache_desc& d, const void* K, const 
   bf16* e_hi = reinterpret_cast<bf16*>(ws + Ly.oq_hi);
   bf16* e_mid = reinterpret_cast<bf16*>(ws + Ly.oq_mid);
   bf16* e_lo = reinterpret_cast<bf16*>(ws + Ly.oq_lo);
-  CUtensorMap mQ, mK, mV, mL, mEh, mEm, mEl;
+  CUtensorMap mQ, mK, mV, mEh, mEm, mEl;
   const unsigned long long erows = (unsigned long long)units * 128;
   if (!encode_rows_map(&mQ, Qw, qrows, D, 128) || !encode_rows_map(&mK, K, rows, D, kFuKeys) ||
       !encode_rows_map(&mV, V, rows, D, kFuKeys) || !encode_rows_map(&mEh, e_hi, erows, D, 128) ||
       !encode_rows_map(&mEm, e_mid, erows, D, 128) || !encode_rows_map(&mEl, e_lo, erows, D, 128))
     return cudaErrorInvalidValue;
-  int ln_lead = 0;
-  if (logn) {
-    if (!encode_ln_map(&mL, logn, rows, FaShape<D>::kLnBox, &ln_lead)) return cudaErrorInvalidValue;
-  } else {
-    mL = mK;   // never read
-  }
   // pass A: two partials per CTA (one per softmax group), so at most half the layout's
   // partial slots worth of CTAs per head
   int nsa = fused_splits(units);
@@ -964,8 +989,7 @@ static cudaError_t launch_fused_t(const kvs_cache_desc& d, const void* K, const 
   auto ka = window_fa_kernel<D>;
   if (!ensure_smem_attr((const void*)ka, FaShape<D>::kSmem)) return cudaErrorInvalidValue;
   ka<<<dim3(nsa, units), kFuThreads, FaShape<D>::kSmem, st>>>(
-      mQ, mK, mV, mL, ln_lead, logn != nullptr, len, d.H_kv, d.H_q, W, d.T_cap, nsa, part_ml,
-      part_o, flags);
+      mQ, mK, mV, logn, len, d.H_kv, d.H_q, W, d.T_cap, nsa, part_ml, part_o, flags);
   const size_t csm = (size_t)Qn * 2 * nsa * sizeof(float);
   auto kc = fa_combine_kernel<D>;
   if (!ensure_smem_attr((const void*)kc, csm)) return cudaErrorInvalidValue;

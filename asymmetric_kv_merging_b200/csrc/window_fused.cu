@@ -30,8 +30,11 @@
 //     With e_q = o_q - o_bar, |v - o_q|^2 = |v - o_bar|^2 - 2 (v.e_q - o_bar.e_q) + |e_q|^2
 //     and |v_a + v_b - 2 o_q|^2 = |v_a + v_b - 2 o_bar|^2 - 4 (v_a.e_q + v_b.e_q
 //     - 2 o_bar.e_q) + 4 |e_q|^2: the row terms are taken directly in fp32 as in the mean
-//     form and U = V E^T (E as three bf16 parts) on the tensor cores. Centring on o_bar
-//     keeps the product small where v and o_q are close.
+//     form and U = V E^T (E as three bf16 parts) on the tensor cores. Where a query's
+//     output sits near the row (attention concentrated on it), the expansion cancels:
+//     its result is then far below the terms it is formed from, and the distance is
+//     recomputed directly from the value rows and e_q (rarely: at most a few keys per
+//     query can hold most of its attention).
 //
 // Warp roles (both passes): warp 0 issues the TMA loads (128-byte swizzle, no
 // multicast), warp 1 owns the tensor memory and one of its threads issues tcgen05.mma,
@@ -587,12 +590,52 @@ __device__ __forceinline__ void pair_weight_score(float n11, float n12, float n2
   }
 }
 
+// Per-query form, taken directly where the expansion around o_bar cancels:
+// |x - k e_q|^2 with x = (v_a - o_bar) (+ (v_b - o_bar) when vb is given), the value rows
+// read from the cache, o_bar and e_q = hi + mid + lo from shared memory (E tiles with
+// 128-byte swizzling, query q's row).
+template <int D>
+__device__ __noinline__ float direct_sq(const bf16* __restrict__ va, const bf16* __restrict__ vb,
+                                        const float* obs, const unsigned char* et, int q, float k) {
+  constexpr int kBox = 128 * 128, kTile = (D / 64) * kBox;
+  float acc = 0.f;
+#pragma unroll 2
+  for (int ch = 0; ch < D / 8; ++ch) {
+    const int dim = ch * 8, bx = dim >> 6, cc = (dim & 63) >> 3;
+    float fa[8], fb[8], eh[8], em[8], el[8];
+    load_vec(va + dim, fa);
+    if (vb) {
+      load_vec(vb + dim, fb);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) fb[e] = 0.f;
+    }
+    const uint32_t off = (uint32_t)(bx * kBox) + swz128(q, cc);
+    load_vec(reinterpret_cast<const bf16*>(et + off), eh);
+    load_vec(reinterpret_cast<const bf16*>(et + kTile + off), em);
+    load_vec(reinterpret_cast<const bf16*>(et + 2 * kTile + off), el);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float o = obs[dim + e];
+      const float x = vb ? (fa[e] - o) + (fb[e] - o) : fa[e] - o;
+      const float dlt = fmaf(-k, (el[e] + em[e]) + eh[e], x);
+      acc = fmaf(dlt, dlt, acc);
+    }
+  }
+  return acc;
+}
+
+// A squared distance from the expansion is recomputed directly when it is below this
+// fraction of the magnitude of the terms it was formed from (a bound on their error).
+constexpr float kRedoFrac = 1.f / 16.f;
+
 template <int D, bool PERQ>
 __global__ void __launch_bounds__(kFuThreads, 1)
 window_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmEh,
                     const __grid_constant__ CUtensorMap tmEm, const __grid_constant__ CUtensorMap tmEl,
-                    const float* __restrict__ logn, const int32_t* __restrict__ len,
+                    const bf16* __restrict__ Vg, const float* __restrict__ logn,
+                    const int32_t* __restrict__ len,
                     const int32_t* __restrict__ cand_begin, int n_recent, int H_kv, int H_q,
                     int W, int T_cap, int nsplit, int form, const float* __restrict__ stats,
                     const float* __restrict__ obar, const float* __restrict__ zqg,
@@ -798,7 +841,7 @@ window_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       // |v_b - o_bar|^2, |v_a + v_b - 2 o_bar|^2 (this lane's half of the dims)
       live = live && mbar_wait_ab(&full[s], (i / ST) & 1, s_abort);
       live = __all_sync(0xffffffffu, live);
-      float dd = 0.f, ea = 0.f, eb = 0.f, ec = 0.f;
+      float dd = 0.f, ea = 0.f, eb = 0.f, ec = 0.f, na = 0.f, nb = 0.f;
       if (live) {
         const unsigned char* kt = base + S::kStageOff + s * S::kStageBytes;
         const unsigned char* vt = kt + S::kTile;
@@ -823,6 +866,10 @@ window_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             ea = fmaf(ra2.x, ra2.x, fmaf(ra2.y, ra2.y, ea));
             eb = fmaf(rb2.x, rb2.x, fmaf(rb2.y, rb2.y, eb));
             ec = fmaf(rc2.x, rc2.x, fmaf(rc2.y, rc2.y, ec));
+            if (PERQ) {
+              na = fmaf(bf16_lo(vaw[e]), bf16_lo(vaw[e]), fmaf(bf16_hi(vaw[e]), bf16_hi(vaw[e]), na));
+              nb = fmaf(bf16_lo(vbw[e]), bf16_lo(vbw[e]), fmaf(bf16_hi(vbw[e]), bf16_hi(vbw[e]), nb));
+            }
           }
         }
       }
@@ -830,6 +877,10 @@ window_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       ea += __shfl_xor_sync(0xffffffffu, ea, 1);
       eb += __shfl_xor_sync(0xffffffffu, eb, 1);
       ec += __shfl_xor_sync(0xffffffffu, ec, 1);
+      if (PERQ) {
+        na += __shfl_xor_sync(0xffffffffu, na, 1);
+        nb += __shfl_xor_sync(0xffffffffu, nb, 1);
+      }
       // window probabilities p_qt = 2^(s q.k + lnt - Z_q), the key's row of S^T
       live = live && mbar_wait_ab(&s_full[g], k & 1, s_abort);
       if (PERQ) live = live && mbar_wait_ab(&u_full[g], k & 1, s_abort);
@@ -839,6 +890,12 @@ window_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       if (live) tc_fence_after();
       float acc = 0.f, n_self = 0.f, n_cpl = 0.f;
       const float t_own = is_a ? ea : eb;
+      // per query form: the magnitudes that bound the expansion's error (U carries the
+      // tensor cores' accumulation error, of order |v| |e_q|), and the value rows that a
+      // direct recomputation reads
+      const float vn_own = sqrtf(is_a ? na : nb), vn_pair = sqrtf(na) + sqrtf(nb);
+      const bf16* v_own = Vg + ((size_t)unit * T_cap + (kval ? t : 0)) * D;
+      const bf16* v_next = v_own + D;
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         float v[32];
@@ -880,17 +937,27 @@ window_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 #pragma unroll
             for (int j = 0; j < 32; ++j) u[j] = 0.f;
           }
-#pragma unroll 8
+          const unsigned char* et = base + S::kEOff;
+#pragma unroll 4
           for (int j = 0; j < 32; ++j) {
+            const int q = 32 * c + j;
             const float p = v[j], uu = u[j];
             const float p_o = __shfl_xor_sync(0xffffffffu, p, 1);
             const float u_o = __shfl_xor_sync(0xffffffffu, uu, 1);
-            const float z = eqs[32 * c + j], wq = eqs[128 + 32 * c + j];
-            n_self = fmaf(fabsf(p * (1.f - 2.f * p)),
-                          sqrtf(fmaxf(0.f, fmaf(-2.f, uu - wq, t_own) + z)), n_self);
-            if (is_a)
-              n_cpl = fmaf(p * p_o, sqrtf(fmaxf(0.f, fmaf(-4.f, uu + u_o - 2.f * wq, ec) + 4.f * z)),
-                           n_cpl);
+            const float z = eqs[q], wq = eqs[128 + q];
+            const float se = sqrtf(z);
+            // |v - o_q|^2 and |v_a + v_b - 2 o_q|^2 by the expansion; where that cancels
+            // (a query whose output sits near the row), directly from the rows
+            const float xs = uu - wq, xc = uu + u_o - 2.f * wq;
+            float rs = fmaf(-2.f, xs, t_own) + z;
+            float rc = fmaf(-4.f, xc, ec) + 4.f * z;
+            const float ms = t_own + z + 2.f * fabsf(xs) + 2.f * vn_own * se;
+            const float mc = ec + 4.f * z + 4.f * fabsf(xc) + 4.f * vn_pair * se;
+            if (p != 0.f && rs < kRedoFrac * ms) rs = direct_sq<D>(v_own, nullptr, obs, et, q, 1.f);
+            if (is_a && p * p_o != 0.f && rc < kRedoFrac * mc)
+              rc = direct_sq<D>(v_own, v_next, obs, et, q, 2.f);
+            n_self = fmaf(fabsf(p * (1.f - 2.f * p)), sqrtf(fmaxf(0.f, rs)), n_self);
+            if (is_a) n_cpl = fmaf(p * p_o, sqrtf(fmaxf(0.f, rc)), n_cpl);
           }
         }
       }
@@ -999,14 +1066,14 @@ static cudaError_t launch_fused_t(const kvs_cache_desc& d, const void* K, const 
     auto kb = window_score_kernel<D, true>;
     if (!ensure_smem_attr((const void*)kb, ScShape<D, true>::kSmem)) return cudaErrorInvalidValue;
     kb<<<dim3(nsb, units), kFuThreads, ScShape<D, true>::kSmem, st>>>(
-        mQ, mK, mV, mEh, mEm, mEl, logn, len, cand_begin, n_recent, d.H_kv, d.H_q, W, d.T_cap,
-        nsb, form, stats, obar, zq, wq, score, w_b, flags);
+        mQ, mK, mV, mEh, mEm, mEl, (const bf16*)V, logn, len, cand_begin, n_recent, d.H_kv,
+        d.H_q, W, d.T_cap, nsb, form, stats, obar, zq, wq, score, w_b, flags);
   } else {
     auto kb = window_score_kernel<D, false>;
     if (!ensure_smem_attr((const void*)kb, ScShape<D, false>::kSmem)) return cudaErrorInvalidValue;
     kb<<<dim3(nsb, units), kFuThreads, ScShape<D, false>::kSmem, st>>>(
-        mQ, mK, mV, mEh, mEm, mEl, logn, len, cand_begin, n_recent, d.H_kv, d.H_q, W, d.T_cap,
-        nsb, form, stats, obar, zq, wq, score, w_b, flags);
+        mQ, mK, mV, mEh, mEm, mEl, (const bf16*)V, logn, len, cand_begin, n_recent, d.H_kv,
+        d.H_q, W, d.T_cap, nsb, form, stats, obar, zq, wq, score, w_b, flags);
   }
   count_launches(3);
   return cudaGetLastError();

@@ -47,6 +47,9 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["kvs", "reference"], default="kvs")
     ap.add_argument("--workload", type=int, default=2)
+    ap.add_argument("--form", choices=["full", "diagonal", "per_query"], default="full",
+                    help="scoring form: the full coupled form with the window mean (default), "
+                         "the diagonal-only ablation, or the window read query by query")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--prefill", action="store_true",
@@ -215,12 +218,13 @@ class Runner:
     merged in place to 1/8 of their count after each such segment of decode steps.
     """
 
-    def __init__(self, w: inputs.Workload, rank: int, device):
+    def __init__(self, w: inputs.Workload, rank: int, device, form=None):
         import numpy as np
         from asymmetric_kv_merging_b200 import kvs
         self.kvs = kvs
         self.w = w
         self.dev = device
+        self.form = form
         B, H, d = w.B, w.H_kv, w.d
         seq = inputs.sequence_lengths(w).numpy()
         self.seq_lens = seq
@@ -301,7 +305,8 @@ class Runner:
                 dst = self.final[l] if r == self.rounds - 1 else self.scratch[r]
                 with _timed(timer, "score"):
                     kvs.score_pairs(self.descs[r], src["K"], src["V"], src["logn"], src["lens"],
-                                    self.cand, w.W, li.Q_win, w.W, self.score, self.w_b, self.ws)
+                                    self.cand, w.W, li.Q_win, w.W, self.score, self.w_b, self.ws,
+                                    form=self.form)
                 with _timed(timer, "merge"):
                     kvs.merge_compact(self.descs[r], src["K"], src["V"], src["logn"], src["lens"],
                                       self.cand, w.W, self.score, self.w_b, self.tgt,
@@ -327,7 +332,8 @@ class Runner:
                         f = self.final[l]
                         for sub in rm["subs"]:
                             kvs.score_pairs(dsc, f["K"], f["V"], f["logn"], f["lens"], sub["cand"],
-                                            0, rm["Qw"][l], w.W, self.score, self.w_b, self.ws)
+                                            0, rm["Qw"][l], w.W, self.score, self.w_b, self.ws,
+                                            form=self.form)
                             kvs.merge_compact(dsc, f["K"], f["V"], f["logn"], f["lens"],
                                               sub["cand"], 0, self.score, self.w_b, sub["tgt"],
                                               kvs.SCOPE_HEAD, self.caps[-1], f["K"], f["V"],
@@ -919,7 +925,10 @@ def main():
     w = inputs.workload(args.workload)
     if args.fp32:
         w = inputs.small_workload(w, dtype="f32", name=w.name + "_fp32")
-    rn = Runner(w, rank, dev)
+    from asymmetric_kv_merging_b200 import kvs
+    form_code = {"full": None, "diagonal": kvs.FORM_DIAGONAL,
+                 "per_query": kvs.FORM_FULL | kvs.FORM_PER_QUERY}[args.form]
+    rn = Runner(w, rank, dev, form=form_code)
     rn.capture()
     for _ in range(args.warmup):
         rn.step()
@@ -1020,7 +1029,7 @@ def main():
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-            "config": config_of(w, world),
+            "config": dict(config_of(w, world), form=args.form),
             "value_note": ("merged KV tokens per second of the whole step: the merge phase "
                            "(every layer to its budget) plus the decode phase"),
             "merge_ms_per_step": merge_ms, "decode_ms_per_step": decode_ms,

@@ -359,7 +359,7 @@ bool encode_rows_map(CUtensorMap* map, const void* base, unsigned long long rows
 // 1D map over the log-counts, starting at the 16-byte boundary at or below `logn`;
 // *lead = the elements between that boundary and logn (0..3). Elements past the end
 // read as zero; the few before logn lie in the same 16-byte chunk, so the same page.
-bool encode_ln_map(CUtensorMap* map, const float* logn, unsigned long long n, int box,
+static bool encode_ln_map(CUtensorMap* map, const float* logn, unsigned long long n, int box,
                           int* lead) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;

@@ -58,16 +58,6 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 bool encode_rows_map(CUtensorMap* map, const void* base, unsigned long long rows, int d,
                      int box_rows);
 
-// 1D fp32 map over `n` log-counts from the 16-byte boundary at or below logn, boxes of
-// `box` elements; *lead = elements between that boundary and logn (0..3).
-bool encode_ln_map(CUtensorMap* map, const float* logn, unsigned long long n, int box, int* lead);
-
-// Window statistics for bf16 caches on tcgen05 (G*W <= 128), same outputs as above.
-bool window_tc_supported(const kvs_cache_desc& d, int W);
-cudaError_t launch_window_stats_tc(const kvs_cache_desc& d, const void* K, const void* V,
-                                   const float* logn, const int32_t* len, const void* Qw, int W,
-                                   const ScoreLayout& Ly, char* ws, cudaStream_t st);
-
 // Window statistics and pair scores for bf16 caches in two fused tensor-core passes
 // (G*W <= 128): form is KVS_FORM_FULL or KVS_FORM_DIAGONAL; stats_form is 0 (window
 // mean) or KVS_FORM_PER_QUERY.

@@ -837,10 +837,16 @@ window_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         ln_next = kn < 2 * P ? lnh[c0 + kn] : 0.f;
       }
       const int hide = t - (L - W);               // queries with q mod W < hide miss the key
-      // the pair's row terms from the stage: |k_b - k_a|^2, |v_a - o_bar|^2,
-      // |v_b - o_bar|^2, |v_a + v_b - 2 o_bar|^2 (this lane's half of the dims)
+      // The tile's S^T first: its MMA was issued only after the stage's rows had landed,
+      // so once s_full completes the stage holds this tile, and the wait on `full` that
+      // follows can only match this tile's phase. (Waiting on `full` first could match the
+      // stage's previous phase: with an odd stage count consecutive uses of a stage go to
+      // different groups, and this group need not have seen the other's tile land.)
+      live = live && mbar_wait_ab(&s_full[g], k & 1, s_abort);
       live = live && mbar_wait_ab(&full[s], (i / ST) & 1, s_abort);
       live = __all_sync(0xffffffffu, live);
+      // the pair's row terms from the stage: |k_b - k_a|^2, |v_a - o_bar|^2,
+      // |v_b - o_bar|^2, |v_a + v_b - 2 o_bar|^2 (this lane's half of the dims)
       float dd = 0.f, ea = 0.f, eb = 0.f, ec = 0.f, na = 0.f, nb = 0.f;
       if (live) {
         const unsigned char* kt = base + S::kStageOff + s * S::kStageBytes;
@@ -882,7 +888,6 @@ window_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         nb += __shfl_xor_sync(0xffffffffu, nb, 1);
       }
       // window probabilities p_qt = 2^(s q.k + lnt - Z_q), the key's row of S^T
-      live = live && mbar_wait_ab(&s_full[g], k & 1, s_abort);
       if (PERQ) live = live && mbar_wait_ab(&u_full[g], k & 1, s_abort);
       live = __all_sync(0xffffffffu, live);
       // the stage's rows are read, here and by the tile's MMAs (done: S^T, U landed)

@@ -345,8 +345,6 @@ static cudaError_t launch_window_stats_t(const kvs_cache_desc& d, const void* K,
 cudaError_t launch_window_stats(const kvs_cache_desc& d, const void* K, const void* V,
                                 const float* logn, const int32_t* len, const void* Qw, int W,
                                 const ScoreLayout& Ly, char* ws, cudaStream_t st) {
-  // bf16 caches whose window fits one 128-row MMA tile take the tcgen05 kernels
-  if (window_tc_supported(d, W)) return launch_window_stats_tc(d, K, V, logn, len, Qw, W, Ly, ws, st);
   if (d.dtype == KVS_BF16) {
     if (d.d == 128) return launch_window_stats_t<bf16, 128>(d, K, V, logn, len, Qw, W, Ly, ws, st);
     return launch_window_stats_t<bf16, 64>(d, K, V, logn, len, Qw, W, Ly, ws, st);

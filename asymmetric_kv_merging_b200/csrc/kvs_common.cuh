@@ -118,7 +118,7 @@ struct HeadInfo {      // one (b, h)
 };
 
 struct ScoreLayout {
-  size_t part_ml, part_o, stats, obar, alpha, oq_hi, oq_mid, oq_lo, on2, owq, total;
+  size_t part_ml, part_o, stats, obar, alpha, oq, oq_hi, oq_mid, oq_lo, on2, owq, total;
   int nsplit, Qn;
   int part_slots;   // window partials per head the layout holds (>= nsplit, >= 2)
 };
@@ -176,9 +176,11 @@ inline ScoreLayout score_layout(const kvs_cache_desc& d, int W) {
   L.stats = align_up(L.part_o + units * L.part_slots * L.Qn * (size_t)d.d * sizeof(float), kWsAlign);
   L.obar = align_up(L.stats + units * L.Qn * 2 * sizeof(float), kWsAlign);
   L.alpha = align_up(L.obar + units * (size_t)d.d * sizeof(float), kWsAlign);
-  // window outputs of the bf16 path relative to their mean, e_q = o_q - o_bar: rows of
-  // 128 (padded) queries per head as bf16 hi / mid / lo parts, |e_q|^2 and o_bar . e_q
-  L.oq_hi = align_up(L.alpha + units * (size_t)d.T_cap * sizeof(float), kWsAlign);
+  // window outputs of the bf16 path: o_q (fp32, rows of 128 padded queries per head),
+  // and relative to their mean, e_q = o_q - o_bar, as bf16 hi / mid / lo parts with
+  // |e_q|^2 and o_bar . e_q
+  L.oq = align_up(L.alpha + units * (size_t)d.T_cap * sizeof(float), kWsAlign);
+  L.oq_hi = align_up(L.oq + units * 128 * (size_t)d.d * sizeof(float), kWsAlign);
   L.oq_mid = align_up(L.oq_hi + units * 128 * (size_t)d.d * 2, kWsAlign);
   L.oq_lo = align_up(L.oq_mid + units * 128 * (size_t)d.d * 2, kWsAlign);
   L.on2 = align_up(L.oq_lo + units * 128 * (size_t)d.d * 2, kWsAlign);

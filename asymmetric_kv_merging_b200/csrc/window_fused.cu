@@ -15,9 +15,9 @@
 //     memory over the tile's S and feeds the P V MMAs from there. The reference maximum
 //     of a row moves only when a tile exceeds it by 2^8 (the accumulator is then
 //     rescaled in tensor memory), so P <= 2^8 between moves.
-//   fa_combine_kernel (per KV head): the partials' (m, l, O) -> per query (M, L) and o_q,
-//     o_bar = mean_q o_q, and for pass B's per-query form e_q = o_q - o_bar as bf16
-//     hi / mid / lo rows with |e_q|^2 and o_bar . e_q.
+//   fa_query_kernel (per window query and KV head): the partials' (m, l, O) -> (M, L)
+//     and o_q; fa_center_kernel: o_bar = mean_q o_q, and for pass B's per-query form
+//     e_q = o_q - o_bar as bf16 hi / mid / lo rows with |e_q|^2 and o_bar . e_q.
 //   pass B (window_score_kernel, per KV head and candidate split): S^T = K Q^T with the
 //     keys on the tensor-memory lanes, so that a thread owns one key and its row of
 //     window probabilities p_qt = 2^(s_qt - M_q) / L_q: alpha_bar_t is a sum over the
@@ -61,16 +61,59 @@ __device__ __forceinline__ unsigned char* align1024(unsigned char* p) {
                                           ~static_cast<uintptr_t>(1023));
 }
 
-// 16 consecutive 32-bit columns of this thread's tensor-memory lane, stored from
-// registers (warp-collective), then wait until the stores are done.
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+// 16 consecutive 32-bit columns of this thread's tensor-memory lane, stored from registers
+// (warp-collective) without waiting; tmem_st_wait() waits for all of the thread's stores.
+__device__ __forceinline__ void tmem_st16_async(uint32_t taddr, const uint32_t (&v)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
       "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
       "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
       "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
       : "memory");
+}
+// The same from every other register of w, starting at w[OFF] (16 columns).
+template <int OFF>
+__device__ __forceinline__ void tmem_st16_pairs(uint32_t taddr, const uint32_t (&w)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(w[OFF]), "r"(w[OFF + 2]), "r"(w[OFF + 4]), "r"(w[OFF + 6]), "r"(w[OFF + 8]),
+      "r"(w[OFF + 10]), "r"(w[OFF + 12]), "r"(w[OFF + 14]), "r"(w[OFF + 16]), "r"(w[OFF + 18]),
+      "r"(w[OFF + 20]), "r"(w[OFF + 22]), "r"(w[OFF + 24]), "r"(w[OFF + 26]), "r"(w[OFF + 28]),
+      "r"(w[OFF + 30])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// 32 consecutive 32-bit columns of this thread's lane, loaded without waiting; the values
+// are defined only after tmem_ld_wait on the same registers (which ties them to the wait,
+// so that no use is scheduled before it).
+__device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+      "%28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+        "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                 "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                 "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]),
+                 "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+                 "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
+                 "+r"(r[30]), "+r"(r[31])
+               :
+               : "memory");
 }
 
 // ---------------------------------------------------------------------------
@@ -182,10 +225,10 @@ window_fa_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
       if (has_ln && i < ntiles) {
         const int t = t0 + i * kFuKeys + 4 * lane;
-        v.x = t < t1 ? lnh[t] : 0.f;
-        v.y = t + 1 < t1 ? lnh[t + 1] : 0.f;
-        v.z = t + 2 < t1 ? lnh[t + 2] : 0.f;
-        v.w = t + 3 < t1 ? lnh[t + 3] : 0.f;
+        v.x = t < t1 ? lnh[t] * kLog2e : 0.f;
+        v.y = t + 1 < t1 ? lnh[t + 1] * kLog2e : 0.f;
+        v.z = t + 2 < t1 ? lnh[t + 2] * kLog2e : 0.f;
+        v.w = t + 3 < t1 ? lnh[t + 3] * kLog2e : 0.f;
       }
       return v;
     };
@@ -320,84 +363,88 @@ window_fa_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       // logits x = s q.k + log2(e) logn in the log2 domain; masks only on the split's last
       // tile and on keys the causal window hides from some queries
       const bool interior = tb + kFuKeys <= t1 && tb + kFuKeys - 1 <= L - W;
-      auto logits = [&](float (&v)[32], int c) {
+      auto logits = [&](uint32_t (&w)[32], int c) {
         if (interior && row_ok) {
 #pragma unroll
           for (int j = 0; j < 32; j += 2) {
-            const float2 ln2 = has_ln ? make_float2(lnb[32 * c + j] * kLog2e, lnb[32 * c + j + 1] * kLog2e)
+            const float2 ln2 = has_ln ? *reinterpret_cast<const float2*>(lnb + 32 * c + j)
                                       : make_float2(0.f, 0.f);
-            const float2 x = ffma2(make_float2(v[j], v[j + 1]), make_float2(qscale, qscale), ln2);
-            v[j] = x.x;
-            v[j + 1] = x.y;
+            const float2 x = ffma2(make_float2(__uint_as_float(w[j]), __uint_as_float(w[j + 1])),
+                                   make_float2(qscale, qscale), ln2);
+            w[j] = __float_as_uint(x.x);
+            w[j + 1] = __float_as_uint(x.y);
           }
         } else {
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const int t = tb + 32 * c + j;
             const bool vis = row_ok && t < t1 && t <= pos;
-            v[j] = vis ? fmaf(v[j], qscale, has_ln ? lnb[32 * c + j] * kLog2e : 0.f) : -INFINITY;
+            w[j] = __float_as_uint(vis ? fmaf(__uint_as_float(w[j]), qscale, has_ln ? lnb[32 * c + j] : 0.f)
+                                       : -INFINITY);
           }
         }
       };
-      // sweep 1: the tile's row maximum
-      float mt = -INFINITY;
-      if (live) {
+      // P = 2^(x - m) as bf16 hi and lo parts over the chunk's own S columns, computed in
+      // place over the chunk's logits: pair j/2 leaves hi in w[j] and lo in w[j + 1]
+      auto exps = [&](uint32_t (&w)[32], int c, float m, float& lsum) {
+        float ps[2] = {0.f, 0.f};
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          const float pa = m > -INFINITY ? ex2_ftz(__uint_as_float(w[j]) - m) : 0.f;
+          const float pb = m > -INFINITY ? ex2_ftz(__uint_as_float(w[j + 1]) - m) : 0.f;
+          ps[0] += pa;
+          ps[1] += pb;
+          const uint32_t hh = pack_bf16x2(pa, pb);
+          w[j] = hh;
+          w[j + 1] = pack_bf16x2(pa - bf16_lo(hh), pb - bf16_hi(hh));
+        }
+        lsum += ps[0] + ps[1];
+        tmem_st16_pairs<0>(s_cols + 32 * c, w);
+        tmem_st16_pairs<1>(s_cols + 32 * c + 16, w);
+      };
+      float lsum = 0.f, cfac = 1.f, m_new = m_ref;
+      // a warp with no valid row leaves its P lanes as they are: an MMA row only feeds the
+      // same row of O, and those rows are never read
+      if (live && __any_sync(0xffffffffu, row_ok)) {
         tc_fence_after();
-#pragma unroll 1
+        // the whole row of S in registers (four loads in flight, one wait), the logits
+        // and their maximum, then P chunk by chunk
+        uint32_t r[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32_async(s_cols + 32 * c, r[c]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld_wait(r[c]);
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
         for (int c = 0; c < 4; ++c) {
-          float v[32];
-          tmem_ld32(s_cols + 32 * c, v);
-          logits(v, c);
-          float m4[4] = {v[0], v[1], v[2], v[3]};
+          logits(r[c], c);
 #pragma unroll
-          for (int j = 4; j < 32; ++j) m4[j & 3] = fmaxf(m4[j & 3], v[j]);
-          mt = fmaxf(mt, fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])));
+          for (int j = 0; j < 32; ++j) m4[j & 3] = fmaxf(m4[j & 3], __uint_as_float(r[c][j]));
         }
-      }
-      // the reference maximum moves only when the tile exceeds it by 2^8; O_g, which the
-      // group's previous P V MMAs update, is then rescaled
-      const float m_new = (mt > m_ref + kRescaleSlack) ? mt : m_ref;
-      const bool resc = m_new != m_ref && m_ref > -INFINITY;
-      const float cfac = resc ? ex2_ftz(m_ref - m_new) : 1.f;
-      if (__any_sync(0xffffffffu, resc)) {
-        live = live && mbar_wait_ab(&pv_done[g], (k - 1) & 1, s_abort);
-        live = __all_sync(0xffffffffu, live);
-        if (live) {
-          tc_fence_after();
-#pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
-            float ov[32];
-            tmem_ld32(o_cols + 32 * c, ov);
+        const float mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+        // the reference maximum moves only when the tile exceeds it by 2^8
+        m_new = (mt > m_ref + kRescaleSlack) ? mt : m_ref;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) ov[j] *= cfac;
-            tmem_st32(o_cols + 32 * c, ov);
+        for (int c = 0; c < 4; ++c) exps(r[c], c, m_new, lsum);
+        // O_g, which the group's previous P V MMAs update, follows a moved reference
+        const bool resc = m_new != m_ref && m_ref > -INFINITY;
+        cfac = resc ? ex2_ftz(m_ref - m_new) : 1.f;
+        if (__any_sync(0xffffffffu, resc)) {
+          live = live && mbar_wait_ab(&pv_done[g], (k - 1) & 1, s_abort);
+          live = __all_sync(0xffffffffu, live);
+          if (live) {
+            tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+              float ov[32];
+              tmem_ld32(o_cols + 32 * c, ov);
+#pragma unroll
+              for (int j = 0; j < 32; ++j) ov[j] *= cfac;
+              tmem_st32(o_cols + 32 * c, ov);
+            }
           }
         }
-      }
-      // sweep 2: P = 2^(x - m) as bf16 hi and lo parts over the chunk's own S columns
-      float lsum = 0.f;
-      if (live) {
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          float v[32];
-          tmem_ld32(s_cols + 32 * c, v);
-          logits(v, c);
-          uint32_t hi[16], lo[16];
-          float ps[2] = {0.f, 0.f};
-#pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            const float pa = m_new > -INFINITY ? ex2_ftz(v[j] - m_new) : 0.f;
-            const float pb = m_new > -INFINITY ? ex2_ftz(v[j + 1] - m_new) : 0.f;
-            ps[0] += pa;
-            ps[1] += pb;
-            const uint32_t hh = pack_bf16x2(pa, pb);
-            hi[j >> 1] = hh;
-            lo[j >> 1] = pack_bf16x2(pa - bf16_lo(hh), pb - bf16_hi(hh));
-          }
-          lsum += ps[0] + ps[1];
-          tmem_st16(s_cols + 32 * c, hi);
-          tmem_st16(s_cols + 32 * c + 16, lo);
-        }
+        tmem_st_wait();
       }
       l = l * cfac + lsum;
       // value rows past the split's end may hold anything (even non-finite): zero them,
@@ -460,81 +507,123 @@ window_fa_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 }
 
 // ---------------------------------------------------------------------------
-// Combine: per KV head, the partials' (m, l, O) -> (M, L) and o_q per window query,
-// o_bar, and for the per-query form e_q = o_q - o_bar as bf16 hi / mid / lo rows with
-// |e_q|^2 and o_bar . e_q
+// Combine, in two small kernels with many CTAs (a per-head CTA walking all partials of
+// all queries was latency-bound: one launch took longer than both passes together).
+//   fa_query_kernel (one CTA per window query and head): the partials' (m, l, O) ->
+//     (M, L) and o_q.
+//   fa_center_kernel (per head, and per block of queries in the per-query form):
+//     o_bar = mean_q o_q over the queries with a visible key, and e_q = o_q - o_bar as
+//     bf16 hi / mid / lo rows with |e_q|^2 and o_bar . e_q.
 // ---------------------------------------------------------------------------
 
 template <int D>
 __global__ void __launch_bounds__(D)
-fa_combine_kernel(const float* __restrict__ part_ml, const float* __restrict__ part_o, int Qn,
-                  int nparts, float* __restrict__ stats, float* __restrict__ obar,
-                  float* __restrict__ zq_out, float* __restrict__ wq_out, bf16* __restrict__ e_hi,
-                  bf16* __restrict__ e_mid, bf16* __restrict__ e_lo) {
-  extern __shared__ float fac[];                 // [Qn][nparts] weights 2^(m - M) / L
-  __shared__ float s_z[D / 32][128], s_w[D / 32][128];
-  __shared__ int s_valid;
-  const int unit = blockIdx.x, c = threadIdx.x, lane = c & 31, wid = c >> 5;
-  if (c == 0) s_valid = 0;
-  __syncthreads();
-  for (int q = c; q < Qn; q += D) {
-    const float* e = part_ml + (size_t)unit * nparts * Qn * 2;
+fa_query_kernel(const float* __restrict__ part_ml, const float* __restrict__ part_o, int Qn,
+                int nparts, float* __restrict__ stats, float* __restrict__ oq) {
+  extern __shared__ float fac[];                 // [nparts] weights 2^(m - M) / L
+  __shared__ float s_ml[2];
+  const int q = blockIdx.x, unit = blockIdx.y, c = threadIdx.x;
+  const float* e = part_ml + (size_t)unit * nparts * Qn * 2;
+  if (c < 32) {
     float M = -INFINITY;
-    for (int s = 0; s < nparts; ++s) {
+    for (int s = c; s < nparts; s += 32) {
       const float ls = e[((size_t)s * Qn + q) * 2 + 1];
       if (ls > 0.f) M = fmaxf(M, e[((size_t)s * Qn + q) * 2]);
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float Ls = 0.f;
     if (M > -INFINITY)
-      for (int s = 0; s < nparts; ++s) {
+      for (int s = c; s < nparts; s += 32) {
         const float ls = e[((size_t)s * Qn + q) * 2 + 1];
         if (ls > 0.f) Ls = fmaf(ls, exp2f(e[((size_t)s * Qn + q) * 2] - M), Ls);
       }
-    const bool valid = Ls > 0.f;
-    for (int s = 0; s < nparts; ++s) {
-      const float ls = e[((size_t)s * Qn + q) * 2 + 1];
-      fac[q * nparts + s] = (valid && ls > 0.f) ? exp2f(e[((size_t)s * Qn + q) * 2] - M) / Ls : 0.f;
+    Ls = warp_sum(Ls);
+    if (c == 0) {
+      s_ml[0] = M;
+      s_ml[1] = Ls;
+      stats[((size_t)unit * Qn + q) * 2 + 0] = M;
+      stats[((size_t)unit * Qn + q) * 2 + 1] = Ls;
     }
-    stats[((size_t)unit * Qn + q) * 2 + 0] = M;
-    stats[((size_t)unit * Qn + q) * 2 + 1] = Ls;
-    if (valid) atomicAdd(&s_valid, 1);
   }
   __syncthreads();
-  const float* po = part_o + (size_t)unit * nparts * Qn * D;
-  auto o_of = [&](int q) {
-    float o = 0.f;
-    for (int s = 0; s < nparts; ++s) o = fmaf(fac[q * nparts + s], po[((size_t)s * Qn + q) * D + c], o);
-    return o;
-  };
-  float acc = 0.f;
-  for (int q = 0; q < Qn; ++q) acc += o_of(q);
+  const float M = s_ml[0], Ls = s_ml[1];
+  const bool valid = Ls > 0.f;
+  for (int s = c; s < nparts; s += D) {
+    const float ls = e[((size_t)s * Qn + q) * 2 + 1];
+    fac[s] = (valid && ls > 0.f) ? exp2f(e[((size_t)s * Qn + q) * 2] - M) / Ls : 0.f;
+  }
+  __syncthreads();
+  // o_q = sum over partials of weight x O row: independent loads, four accumulators
+  const float* po = part_o + ((size_t)unit * nparts * Qn + q) * D + c;
+  const size_t stride = (size_t)Qn * D;
+  float a4[4] = {0.f, 0.f, 0.f, 0.f};
+  int s = 0;
+  for (; s + 4 <= nparts; s += 4) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) a4[j] = fmaf(fac[s + j], po[(s + j) * stride], a4[j]);
+  }
+  for (; s < nparts; ++s) a4[0] = fmaf(fac[s], po[s * stride], a4[0]);
+  oq[((size_t)unit * 128 + q) * D + c] = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+}
+
+constexpr int kCenterRows = 16;                  // queries per CTA of fa_center_kernel
+
+template <int D>
+__global__ void __launch_bounds__(D)
+fa_center_kernel(const float* __restrict__ stats, const float* __restrict__ oq, int Qn,
+                 int with_e, float* __restrict__ obar, float* __restrict__ zq_out,
+                 float* __restrict__ wq_out, bf16* __restrict__ e_hi, bf16* __restrict__ e_mid,
+                 bf16* __restrict__ e_lo) {
+  __shared__ float s_z[D / 32][kCenterRows], s_w[D / 32][kCenterRows];
+  const int unit = blockIdx.y, c = threadIdx.x, lane = c & 31, wid = c >> 5;
+  __shared__ int s_valid;                        // queries with a visible key
+  if (c == 0) s_valid = 0;
+  __syncthreads();
+  int nv = 0;
+  for (int q = c; q < Qn; q += D) nv += stats[((size_t)unit * Qn + q) * 2 + 1] > 0.f;
+  if (nv) atomicAdd(&s_valid, nv);
+  __syncthreads();
+  // o_bar in a fixed order (queries without a visible key have o_q = 0)
+  const float* col = oq + (size_t)unit * 128 * D + c;
+  float a8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  int q = 0;
+  for (; q + 8 <= Qn; q += 8) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) a8[j] += col[(size_t)(q + j) * D];
+  }
+  for (; q < Qn; ++q) a8[0] += col[(size_t)q * D];
+  const float acc = ((a8[0] + a8[1]) + (a8[2] + a8[3])) + ((a8[4] + a8[5]) + (a8[6] + a8[7]));
   const float ob = s_valid > 0 ? acc / (float)s_valid : 0.f;
-  obar[(size_t)unit * D + c] = ob;
-  for (int q = 0; q < 128; ++q) {
-    const float e = q < Qn ? o_of(q) - ob : 0.f;
+  if (blockIdx.x == 0) obar[(size_t)unit * D + c] = ob;
+  if (!with_e) return;
+  const int q0 = blockIdx.x * kCenterRows;
+  for (int r = 0; r < kCenterRows; ++r) {
+    const int qq = q0 + r;
+    const float e = qq < Qn ? col[(size_t)qq * D] - ob : 0.f;
     const bf16 hi = __float2bfloat16_rn(e);
     const float r1 = e - __bfloat162float(hi);
     const bf16 mid = __float2bfloat16_rn(r1);
-    const size_t at = ((size_t)unit * 128 + q) * D + c;
+    const size_t at = ((size_t)unit * 128 + qq) * D + c;
     e_hi[at] = hi;
     e_mid[at] = mid;
     e_lo[at] = __float2bfloat16_rn(r1 - __bfloat162float(mid));
     const float z = warp_sum(e * e), wv = warp_sum(ob * e);
     if (lane == 0) {
-      s_z[wid][q] = z;
-      s_w[wid][q] = wv;
+      s_z[wid][r] = z;
+      s_w[wid][r] = wv;
     }
   }
   __syncthreads();
-  for (int q = c; q < 128; q += D) {
+  if (c < kCenterRows) {
     float z = 0.f, wv = 0.f;
 #pragma unroll
     for (int w = 0; w < D / 32; ++w) {
-      z += s_z[w][q];
-      wv += s_w[w][q];
+      z += s_z[w][c];
+      wv += s_w[w][c];
     }
-    zq_out[(size_t)unit * 128 + q] = z;
-    wq_out[(size_t)unit * 128 + q] = wv;
+    zq_out[(size_t)unit * 128 + q0 + c] = z;
+    wq_out[(size_t)unit * 128 + q0 + c] = wv;
   }
 }
 
@@ -847,7 +936,9 @@ window_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       live = __all_sync(0xffffffffu, live);
       // the pair's row terms from the stage: |k_b - k_a|^2, |v_a - o_bar|^2,
       // |v_b - o_bar|^2, |v_a + v_b - 2 o_bar|^2 (this lane's half of the dims)
-      float dd = 0.f, ea = 0.f, eb = 0.f, ec = 0.f, na = 0.f, nb = 0.f;
+      // packed fp32 pairs: the two dims of a bf16 pair in one register pair
+      const float2 neg1 = make_float2(-1.f, -1.f);
+      float2 dd2 = make_float2(0.f, 0.f), ea2 = dd2, eb2 = dd2, ec2 = dd2, na2 = dd2, nb2 = dd2;
       if (live) {
         const unsigned char* kt = base + S::kStageOff + s * S::kStageBytes;
         const unsigned char* vt = kt + S::kTile;
@@ -864,21 +955,27 @@ window_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float2 o2 = *reinterpret_cast<const float2*>(obs + dim + 2 * e);
-            const float2 dk = make_float2(bf16_lo(kbw[e]) - bf16_lo(kaw[e]), bf16_hi(kbw[e]) - bf16_hi(kaw[e]));
-            const float2 ra2 = make_float2(bf16_lo(vaw[e]) - o2.x, bf16_hi(vaw[e]) - o2.y);
-            const float2 rb2 = make_float2(bf16_lo(vbw[e]) - o2.x, bf16_hi(vbw[e]) - o2.y);
+            const float2 ka2 = make_float2(bf16_lo(kaw[e]), bf16_hi(kaw[e]));
+            const float2 kb2 = make_float2(bf16_lo(kbw[e]), bf16_hi(kbw[e]));
+            const float2 va2 = make_float2(bf16_lo(vaw[e]), bf16_hi(vaw[e]));
+            const float2 vb2 = make_float2(bf16_lo(vbw[e]), bf16_hi(vbw[e]));
+            const float2 dk = ffma2(ka2, neg1, kb2);
+            const float2 ra2 = ffma2(o2, neg1, va2);
+            const float2 rb2 = ffma2(o2, neg1, vb2);
             const float2 rc2 = fadd2(ra2, rb2);
-            dd = fmaf(dk.x, dk.x, fmaf(dk.y, dk.y, dd));
-            ea = fmaf(ra2.x, ra2.x, fmaf(ra2.y, ra2.y, ea));
-            eb = fmaf(rb2.x, rb2.x, fmaf(rb2.y, rb2.y, eb));
-            ec = fmaf(rc2.x, rc2.x, fmaf(rc2.y, rc2.y, ec));
+            dd2 = ffma2(dk, dk, dd2);
+            ea2 = ffma2(ra2, ra2, ea2);
+            eb2 = ffma2(rb2, rb2, eb2);
+            ec2 = ffma2(rc2, rc2, ec2);
             if (PERQ) {
-              na = fmaf(bf16_lo(vaw[e]), bf16_lo(vaw[e]), fmaf(bf16_hi(vaw[e]), bf16_hi(vaw[e]), na));
-              nb = fmaf(bf16_lo(vbw[e]), bf16_lo(vbw[e]), fmaf(bf16_hi(vbw[e]), bf16_hi(vbw[e]), nb));
+              na2 = ffma2(va2, va2, na2);
+              nb2 = ffma2(vb2, vb2, nb2);
             }
           }
         }
       }
+      float dd = dd2.x + dd2.y, ea = ea2.x + ea2.y, eb = eb2.x + eb2.y, ec = ec2.x + ec2.y;
+      float na = na2.x + na2.y, nb = nb2.x + nb2.y;
       dd += __shfl_xor_sync(0xffffffffu, dd, 1);
       ea += __shfl_xor_sync(0xffffffffu, ea, 1);
       eb += __shfl_xor_sync(0xffffffffu, eb, 1);
@@ -1062,12 +1159,17 @@ static cudaError_t launch_fused_t(const kvs_cache_desc& d, const void* K, const 
   if (!ensure_smem_attr((const void*)ka, FaShape<D>::kSmem)) return cudaErrorInvalidValue;
   ka<<<dim3(nsa, units), kFuThreads, FaShape<D>::kSmem, st>>>(
       mQ, mK, mV, logn, len, d.H_kv, d.H_q, W, d.T_cap, nsa, part_ml, part_o, flags);
-  const size_t csm = (size_t)Qn * 2 * nsa * sizeof(float);
-  auto kc = fa_combine_kernel<D>;
-  if (!ensure_smem_attr((const void*)kc, csm)) return cudaErrorInvalidValue;
-  kc<<<units, D, csm, st>>>(part_ml, part_o, Qn, 2 * nsa, stats, obar, zq, wq, e_hi, e_mid, e_lo);
+  float* oq = reinterpret_cast<float*>(ws + Ly.oq);
+  const size_t qsm = (size_t)2 * nsa * sizeof(float);
+  auto kq = fa_query_kernel<D>;
+  if (!ensure_smem_attr((const void*)kq, qsm)) return cudaErrorInvalidValue;
+  kq<<<dim3(Qn, units), D, qsm, st>>>(part_ml, part_o, Qn, 2 * nsa, stats, oq);
+  const bool perq = stats_form == KVS_FORM_PER_QUERY;
+  const int ncb = perq ? (128 + kCenterRows - 1) / kCenterRows : 1;
+  fa_center_kernel<D><<<dim3(ncb, units), D, 0, st>>>(stats, oq, Qn, perq ? 1 : 0, obar, zq, wq,
+                                                      e_hi, e_mid, e_lo);
   const int nsb = fused_splits(units);
-  if (stats_form == KVS_FORM_PER_QUERY) {
+  if (perq) {
     auto kb = window_score_kernel<D, true>;
     if (!ensure_smem_attr((const void*)kb, ScShape<D, true>::kSmem)) return cudaErrorInvalidValue;
     kb<<<dim3(nsb, units), kFuThreads, ScShape<D, true>::kSmem, st>>>(
@@ -1080,7 +1182,7 @@ static cudaError_t launch_fused_t(const kvs_cache_desc& d, const void* K, const 
         mQ, mK, mV, mEh, mEm, mEl, (const bf16*)V, logn, len, cand_begin, n_recent, d.H_kv,
         d.H_q, W, d.T_cap, nsb, form, stats, obar, zq, wq, score, w_b, flags);
   }
-  count_launches(3);
+  count_launches(4);
   return cudaGetLastError();
 }
 

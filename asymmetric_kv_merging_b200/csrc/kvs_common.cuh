@@ -178,14 +178,14 @@ inline ScoreLayout score_layout(const kvs_cache_desc& d, int W) {
   L.alpha = align_up(L.obar + units * (size_t)d.d * sizeof(float), kWsAlign);
   // window outputs of the bf16 path: o_q (fp32, rows of 128 padded queries per head),
   // and relative to their mean, e_q = o_q - o_bar, as bf16 hi / mid / lo parts with
-  // |e_q|^2 and o_bar . e_q
+  // |e_q|^2 and o_bar . e_q in shares per block of 32 columns
   L.oq = align_up(L.alpha + units * (size_t)d.T_cap * sizeof(float), kWsAlign);
   L.oq_hi = align_up(L.oq + units * 128 * (size_t)d.d * sizeof(float), kWsAlign);
   L.oq_mid = align_up(L.oq_hi + units * 128 * (size_t)d.d * 2, kWsAlign);
   L.oq_lo = align_up(L.oq_mid + units * 128 * (size_t)d.d * 2, kWsAlign);
   L.on2 = align_up(L.oq_lo + units * 128 * (size_t)d.d * 2, kWsAlign);
-  L.owq = align_up(L.on2 + units * 128 * sizeof(float), kWsAlign);
-  L.total = align_up(L.owq + units * 128 * sizeof(float), kWsAlign);
+  L.owq = align_up(L.on2 + units * 128 * (size_t)(d.d / 32) * sizeof(float), kWsAlign);
+  L.total = align_up(L.owq + units * 128 * (size_t)(d.d / 32) * sizeof(float), kWsAlign);
   return L;
 }
 

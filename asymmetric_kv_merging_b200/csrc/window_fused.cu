@@ -83,6 +83,18 @@ __device__ __forceinline__ void tmem_st16_pairs(uint32_t taddr, const uint32_t (
       "r"(w[OFF + 30])
       : "memory");
 }
+// Two columns of this thread's lane: store (no wait), and load (waits).
+__device__ __forceinline__ void tmem_st2(uint32_t taddr, uint32_t a, uint32_t b) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x2.b32 [%0], {%1, %2};" ::"r"(taddr), "r"(a), "r"(b)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_ld2(uint32_t taddr, uint32_t (&r)[2]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0, %1}, [%2];"
+               : "=r"(r[0]), "=r"(r[1])
+               : "r"(taddr)
+               : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;" : "+r"(r[0]), "+r"(r[1]) : : "memory");
+}
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -407,26 +419,24 @@ window_fa_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       // same row of O, and those rows are never read
       if (live && __any_sync(0xffffffffu, row_ok)) {
         tc_fence_after();
-        // the whole row of S in registers (four loads in flight, one wait), the logits
-        // and their maximum, then P chunk by chunk
-        uint32_t r[4][32];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32_async(s_cols + 32 * c, r[c]);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld_wait(r[c]);
-        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
+        // sweep 1: the tile's row maximum (one chunk of S in registers at a time: a whole
+        // row does not fit beside the rest without spilling)
+        float mt = -INFINITY;
+#pragma unroll 1
         for (int c = 0; c < 4; ++c) {
-          logits(r[c], c);
+          uint32_t w[32];
+          tmem_ld32_async(s_cols + 32 * c, w);
+          tmem_ld_wait(w);
+          logits(w, c);
+          float m4[4] = {__uint_as_float(w[0]), __uint_as_float(w[1]), __uint_as_float(w[2]),
+                         __uint_as_float(w[3])};
 #pragma unroll
-          for (int j = 0; j < 32; ++j) m4[j & 3] = fmaxf(m4[j & 3], __uint_as_float(r[c][j]));
+          for (int j = 4; j < 32; ++j) m4[j & 3] = fmaxf(m4[j & 3], __uint_as_float(w[j]));
+          mt = fmaxf(mt, fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])));
         }
-        const float mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-        // the reference maximum moves only when the tile exceeds it by 2^8
+        // the reference maximum moves only when the tile exceeds it by 2^8; O_g, which the
+        // group's previous P V MMAs update, is then rescaled
         m_new = (mt > m_ref + kRescaleSlack) ? mt : m_ref;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) exps(r[c], c, m_new, lsum);
-        // O_g, which the group's previous P V MMAs update, follows a moved reference
         const bool resc = m_new != m_ref && m_ref > -INFINITY;
         cfac = resc ? ex2_ftz(m_ref - m_new) : 1.f;
         if (__any_sync(0xffffffffu, resc)) {
@@ -442,6 +452,17 @@ window_fa_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
               for (int j = 0; j < 32; ++j) ov[j] *= cfac;
               tmem_st32(o_cols + 32 * c, ov);
             }
+          }
+        }
+        // sweep 2: P chunk by chunk (stores in flight until the one wait below)
+        if (live) {
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t w[32];
+            tmem_ld32_async(s_cols + 32 * c, w);
+            tmem_ld_wait(w);
+            logits(w, c);
+            exps(w, c, m_new, lsum);
           }
         }
         tmem_st_wait();
@@ -467,33 +488,65 @@ window_fa_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       m_ref = m_new;
     }
     if (!live) set_flag(flags, KVS_FLAG_TIMEOUT);
-    // this group's partial: (m, l) per query row and the unnormalised O row, stored as
-    // partial 2 split + g
+    // The CTA's partial, the two groups merged: group 1 leaves its (m, l) per row in two
+    // columns of its S buffer (free once its last P V MMAs are done; the same lanes), and
+    // the group-0 warp of the same lane quarter combines both O rows from tensor memory
+    // (the two warps meet at a named barrier of their own).
     bool got = n_mine > 0 && live && mbar_wait_ab(&pv_done[g], (n_mine - 1) & 1, s_abort);
     got = __all_sync(0xffffffffu, got);
     if (n_mine > 0 && !got) set_flag(flags, KVS_FLAG_TIMEOUT);
     const bool any = got && row_ok && m_ref > -INFINITY && l > 0.f;
-    const size_t prow = ((size_t)unit * (2 * nsplit) + 2 * split + g) * Qn + r;
-    if (r < Qn) {
-      part_ml[prow * 2 + 0] = any ? m_ref : -INFINITY;
-      part_ml[prow * 2 + 1] = any ? l : 0.f;
+    const uint32_t ml1_cols = tmem + lane_base + (uint32_t)kFuKeys;   // S_1, columns 0-1
+    if (g == 1) {
+      tmem_st2(ml1_cols, __float_as_uint(any ? m_ref : -INFINITY), __float_as_uint(any ? l : 0.f));
+      tmem_st_wait();
+      tc_fence_before();
     }
-    if (got) tc_fence_after();
-#pragma unroll 1
-    for (int c = 0; c < D / 32; ++c) {
-      float ov[32];
-      if (got) {
-        tmem_ld32(o_cols + 32 * c, ov);
-      } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) ov[j] = 0.f;
-      }
+    named_bar(1 + quarter, 2 * 32);
+    if (g == 0) {
+      tc_fence_after();
+      uint32_t ml[2];
+      tmem_ld2(ml1_cols, ml);
+      const float m1 = __uint_as_float(ml[0]), l1 = __uint_as_float(ml[1]);
+      const bool any1 = l1 > 0.f;
+      const float m0 = any ? m_ref : -INFINITY;
+      const float M = fmaxf(m0, m1);
+      const float f0 = any ? ex2_ftz(m0 - M) : 0.f, f1 = any1 ? ex2_ftz(m1 - M) : 0.f;
+      const bool both = any || any1;
+      const float Ls = (any ? f0 * l : 0.f) + (any1 ? f1 * l1 : 0.f);
+      const size_t prow = ((size_t)unit * nsplit + split) * Qn + r;
       if (r < Qn) {
-        float* po = part_o + prow * D + 32 * c;
+        part_ml[prow * 2 + 0] = both ? M : -INFINITY;
+        part_ml[prow * 2 + 1] = both ? Ls : 0.f;
+      }
+      const uint32_t o1_cols = tmem + lane_base + 256 + (uint32_t)D;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        float o0[32], o1[32];
+        if (__any_sync(0xffffffffu, any)) {
+          tmem_ld32(o_cols + 32 * c, o0);
+        } else {
 #pragma unroll
-        for (int j = 0; j < 32; j += 4)
-          *reinterpret_cast<float4*>(po + j) =
-              any ? make_float4(ov[j], ov[j + 1], ov[j + 2], ov[j + 3]) : make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int j = 0; j < 32; ++j) o0[j] = 0.f;
+        }
+        if (__any_sync(0xffffffffu, any1)) {
+          tmem_ld32(o1_cols + 32 * c, o1);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) o1[j] = 0.f;
+        }
+        if (r < Qn) {
+          float* po = part_o + prow * D + 32 * c;
+#pragma unroll
+          for (int j = 0; j < 32; j += 4) {
+            float4 v4;
+            v4.x = (any ? f0 * o0[j] : 0.f) + (any1 ? f1 * o1[j] : 0.f);
+            v4.y = (any ? f0 * o0[j + 1] : 0.f) + (any1 ? f1 * o1[j + 1] : 0.f);
+            v4.z = (any ? f0 * o0[j + 2] : 0.f) + (any1 ? f1 * o1[j + 2] : 0.f);
+            v4.w = (any ? f0 * o0[j + 3] : 0.f) + (any1 ? f1 * o1[j + 3] : 0.f);
+            *reinterpret_cast<float4*>(po + j) = v4;
+          }
+        }
       }
     }
   }
@@ -557,73 +610,71 @@ fa_query_kernel(const float* __restrict__ part_ml, const float* __restrict__ par
   // o_q = sum over partials of weight x O row: independent loads, four accumulators
   const float* po = part_o + ((size_t)unit * nparts * Qn + q) * D + c;
   const size_t stride = (size_t)Qn * D;
-  float a4[4] = {0.f, 0.f, 0.f, 0.f};
+  float a8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   int s = 0;
-  for (; s + 4 <= nparts; s += 4) {
+  for (; s + 8 <= nparts; s += 8) {
 #pragma unroll
-    for (int j = 0; j < 4; ++j) a4[j] = fmaf(fac[s + j], po[(s + j) * stride], a4[j]);
+    for (int j = 0; j < 8; ++j) a8[j] = fmaf(fac[s + j], po[(s + j) * stride], a8[j]);
   }
-  for (; s < nparts; ++s) a4[0] = fmaf(fac[s], po[s * stride], a4[0]);
-  oq[((size_t)unit * 128 + q) * D + c] = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+  for (; s < nparts; ++s) a8[s & 7] = fmaf(fac[s], po[s * stride], a8[s & 7]);
+  oq[((size_t)unit * 128 + q) * D + c] =
+      ((a8[0] + a8[1]) + (a8[2] + a8[3])) + ((a8[4] + a8[5]) + (a8[6] + a8[7]));
 }
 
-constexpr int kCenterRows = 16;                  // queries per CTA of fa_center_kernel
+// One CTA per 32 columns of a head: 8 warps x 32 columns, warp w summing the queries
+// q = w, w + 8, ... in a fixed order, so o_bar is the same on every run.
+constexpr int kCenterWarps = 8;
 
 template <int D>
-__global__ void __launch_bounds__(D)
+__global__ void __launch_bounds__(kCenterWarps * 32)
 fa_center_kernel(const float* __restrict__ stats, const float* __restrict__ oq, int Qn,
-                 int with_e, float* __restrict__ obar, float* __restrict__ zq_out,
-                 float* __restrict__ wq_out, bf16* __restrict__ e_hi, bf16* __restrict__ e_mid,
+                 int with_e, float* __restrict__ obar, float* __restrict__ zpart,
+                 float* __restrict__ wpart, bf16* __restrict__ e_hi, bf16* __restrict__ e_mid,
                  bf16* __restrict__ e_lo) {
-  __shared__ float s_z[D / 32][kCenterRows], s_w[D / 32][kCenterRows];
-  const int unit = blockIdx.y, c = threadIdx.x, lane = c & 31, wid = c >> 5;
+  __shared__ float s_sum[kCenterWarps][32];
+  __shared__ float s_ob[32];
   __shared__ int s_valid;                        // queries with a visible key
-  if (c == 0) s_valid = 0;
+  const int cb = blockIdx.x, unit = blockIdx.y, tid = threadIdx.x;
+  const int lane = tid & 31, qg = tid >> 5;
+  const int c = 32 * cb + lane;
+  if (tid == 0) s_valid = 0;
   __syncthreads();
   int nv = 0;
-  for (int q = c; q < Qn; q += D) nv += stats[((size_t)unit * Qn + q) * 2 + 1] > 0.f;
+  for (int q = tid; q < Qn; q += kCenterWarps * 32) nv += stats[((size_t)unit * Qn + q) * 2 + 1] > 0.f;
   if (nv) atomicAdd(&s_valid, nv);
-  __syncthreads();
-  // o_bar in a fixed order (queries without a visible key have o_q = 0)
   const float* col = oq + (size_t)unit * 128 * D + c;
-  float a8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  int q = 0;
-  for (; q + 8 <= Qn; q += 8) {
+  float a = 0.f;
+#pragma unroll 4
+  for (int q = qg; q < Qn; q += kCenterWarps) a += col[(size_t)q * D];
+  s_sum[qg][lane] = a;
+  __syncthreads();
+  if (qg == 0) {
+    float t = 0.f;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) a8[j] += col[(size_t)(q + j) * D];
+    for (int w = 0; w < kCenterWarps; ++w) t += s_sum[w][lane];
+    const float ob = s_valid > 0 ? t / (float)s_valid : 0.f;
+    s_ob[lane] = ob;
+    obar[(size_t)unit * D + c] = ob;
   }
-  for (; q < Qn; ++q) a8[0] += col[(size_t)q * D];
-  const float acc = ((a8[0] + a8[1]) + (a8[2] + a8[3])) + ((a8[4] + a8[5]) + (a8[6] + a8[7]));
-  const float ob = s_valid > 0 ? acc / (float)s_valid : 0.f;
-  if (blockIdx.x == 0) obar[(size_t)unit * D + c] = ob;
   if (!with_e) return;
-  const int q0 = blockIdx.x * kCenterRows;
-  for (int r = 0; r < kCenterRows; ++r) {
-    const int qq = q0 + r;
-    const float e = qq < Qn ? col[(size_t)qq * D] - ob : 0.f;
+  __syncthreads();
+  // e_q = o_q - o_bar for this CTA's 32 columns of every (padded) query row, and the
+  // column block's share of |e_q|^2 and o_bar . e_q (pass B adds the D / 32 shares)
+  const float ob = s_ob[lane];
+  for (int q = qg; q < 128; q += kCenterWarps) {
+    const float e = q < Qn ? col[(size_t)q * D] - ob : 0.f;
     const bf16 hi = __float2bfloat16_rn(e);
     const float r1 = e - __bfloat162float(hi);
     const bf16 mid = __float2bfloat16_rn(r1);
-    const size_t at = ((size_t)unit * 128 + qq) * D + c;
+    const size_t at = ((size_t)unit * 128 + q) * D + c;
     e_hi[at] = hi;
     e_mid[at] = mid;
     e_lo[at] = __float2bfloat16_rn(r1 - __bfloat162float(mid));
     const float z = warp_sum(e * e), wv = warp_sum(ob * e);
     if (lane == 0) {
-      s_z[wid][r] = z;
-      s_w[wid][r] = wv;
+      zpart[((size_t)unit * (D / 32) + cb) * 128 + q] = z;
+      wpart[((size_t)unit * (D / 32) + cb) * 128 + q] = wv;
     }
-  }
-  __syncthreads();
-  if (c < kCenterRows) {
-    float z = 0.f, wv = 0.f;
-#pragma unroll
-    for (int w = 0; w < D / 32; ++w) {
-      z += s_z[w][c];
-      wv += s_w[w][c];
-    }
-    zq_out[(size_t)unit * 128 + q0 + c] = z;
-    wq_out[(size_t)unit * 128 + q0 + c] = wv;
   }
 }
 
@@ -648,7 +699,7 @@ struct ScShape {
   static constexpr int kObOff = kZOff + 128 * 4;
   static constexpr int kQmodOff = kObOff + 128 * 4;
   static constexpr int kEqOff = kQmodOff + 128 * 4;
-  static constexpr int kMiscOff = kEqOff + (PERQ ? 2 * 128 * 4 : 0);
+  static constexpr int kMiscOff = kEqOff + (PERQ ? 3 * 128 * 4 : 0);
   static constexpr int kSmem = kMiscOff + 16 + 1024;
   static_assert(kSmem <= 232448, "shared memory");
   // TMA tile destinations with 128-byte swizzling start on 1024-byte boundaries; the
@@ -677,6 +728,14 @@ __device__ __forceinline__ void pair_weight_score(float n11, float n12, float n2
     w = 0.5f;
     s = dd * (n11 + 2.f * n12 + n22) * 0.25f;
   }
+}
+
+// Square root on the special-function unit (PTX sqrt.approx.ftz: relative error of a few
+// units in the last place of fp32, far inside the score tolerance; subnormals flush to 0).
+__device__ __forceinline__ float sqrt_approx(float x) {
+  float y;
+  asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 // Per-query form, taken directly where the expansion around o_bar cancels:
@@ -745,7 +804,7 @@ window_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
   float* zq = reinterpret_cast<float*>(base + S::kZOff);
   float* obs = reinterpret_cast<float*>(base + S::kObOff);
   int* qmod = reinterpret_cast<int*>(base + S::kQmodOff);
-  float* eqs = reinterpret_cast<float*>(base + S::kEqOff);        // |e_q|^2, o_bar.e_q
+  float* eqs = reinterpret_cast<float*>(base + S::kEqOff);        // |e_q|^2, o_bar.e_q, |e_q|
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(base + S::kMiscOff);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
 
@@ -793,8 +852,15 @@ window_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     qmod[q] = q % W;
     obs[q] = q < D ? obar[(size_t)unit * D + q] : 0.f;
     if (PERQ) {
-      eqs[q] = zqg[(size_t)unit * 128 + q];
-      eqs[128 + q] = wqg[(size_t)unit * 128 + q];
+      float z = 0.f, wv = 0.f;
+#pragma unroll
+      for (int cb = 0; cb < D / 32; ++cb) {
+        z += zqg[((size_t)unit * (D / 32) + cb) * 128 + q];
+        wv += wqg[((size_t)unit * (D / 32) + cb) * 128 + q];
+      }
+      eqs[q] = z;
+      eqs[128 + q] = wv;
+      eqs[256 + q] = sqrtf(z);
     }
   }
   if (warp == 1) tmem_alloc(s_tmem, kFuTmemCols);
@@ -1046,8 +1112,7 @@ window_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             const float p = v[j], uu = u[j];
             const float p_o = __shfl_xor_sync(0xffffffffu, p, 1);
             const float u_o = __shfl_xor_sync(0xffffffffu, uu, 1);
-            const float z = eqs[q], wq = eqs[128 + q];
-            const float se = sqrtf(z);
+            const float z = eqs[q], wq = eqs[128 + q], se = eqs[256 + q];
             // |v - o_q|^2 and |v_a + v_b - 2 o_q|^2 by the expansion; where that cancels
             // (a query whose output sits near the row), directly from the rows
             const float xs = uu - wq, xc = uu + u_o - 2.f * wq;
@@ -1058,8 +1123,8 @@ window_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             if (p != 0.f && rs < kRedoFrac * ms) rs = direct_sq<D>(v_own, nullptr, obs, et, q, 1.f);
             if (is_a && p * p_o != 0.f && rc < kRedoFrac * mc)
               rc = direct_sq<D>(v_own, v_next, obs, et, q, 2.f);
-            n_self = fmaf(fabsf(p * (1.f - 2.f * p)), sqrtf(fmaxf(0.f, rs)), n_self);
-            if (is_a) n_cpl = fmaf(p * p_o, sqrtf(fmaxf(0.f, rc)), n_cpl);
+            n_self = fmaf(fabsf(p * (1.f - 2.f * p)), sqrt_approx(fmaxf(0.f, rs)), n_self);
+            if (is_a) n_cpl = fmaf(p * p_o, sqrt_approx(fmaxf(0.f, rc)), n_cpl);
           }
         }
       }
@@ -1141,11 +1206,10 @@ static cudaError_t launch_fused_t(const kvs_cache_desc& d, const void* K, const 
       !encode_rows_map(&mV, V, rows, D, kFuKeys) || !encode_rows_map(&mEh, e_hi, erows, D, 128) ||
       !encode_rows_map(&mEm, e_mid, erows, D, 128) || !encode_rows_map(&mEl, e_lo, erows, D, 128))
     return cudaErrorInvalidValue;
-  // pass A: two partials per CTA (one per softmax group), so at most half the layout's
-  // partial slots worth of CTAs per head
+  // pass A: one partial per CTA (its two softmax groups merged), as many CTAs per head as
+  // the layout has partial slots at most
   int nsa = fused_splits(units);
-  const int cap = Ly.part_slots / 2;
-  if (nsa > cap) nsa = cap;
+  if (nsa > Ly.part_slots) nsa = Ly.part_slots;
   const int Qn = Ly.Qn;
   int32_t* flags = reinterpret_cast<int32_t*>(ws);
   float* part_ml = reinterpret_cast<float*>(ws + Ly.part_ml);
@@ -1160,14 +1224,13 @@ static cudaError_t launch_fused_t(const kvs_cache_desc& d, const void* K, const 
   ka<<<dim3(nsa, units), kFuThreads, FaShape<D>::kSmem, st>>>(
       mQ, mK, mV, logn, len, d.H_kv, d.H_q, W, d.T_cap, nsa, part_ml, part_o, flags);
   float* oq = reinterpret_cast<float*>(ws + Ly.oq);
-  const size_t qsm = (size_t)2 * nsa * sizeof(float);
+  const size_t qsm = (size_t)nsa * sizeof(float);
   auto kq = fa_query_kernel<D>;
   if (!ensure_smem_attr((const void*)kq, qsm)) return cudaErrorInvalidValue;
-  kq<<<dim3(Qn, units), D, qsm, st>>>(part_ml, part_o, Qn, 2 * nsa, stats, oq);
+  kq<<<dim3(Qn, units), D, qsm, st>>>(part_ml, part_o, Qn, nsa, stats, oq);
   const bool perq = stats_form == KVS_FORM_PER_QUERY;
-  const int ncb = perq ? (128 + kCenterRows - 1) / kCenterRows : 1;
-  fa_center_kernel<D><<<dim3(ncb, units), D, 0, st>>>(stats, oq, Qn, perq ? 1 : 0, obar, zq, wq,
-                                                      e_hi, e_mid, e_lo);
+  fa_center_kernel<D><<<dim3(D / 32, units), kCenterWarps * 32, 0, st>>>(
+      stats, oq, Qn, perq ? 1 : 0, obar, zq, wq, e_hi, e_mid, e_lo);
   const int nsb = fused_splits(units);
   if (perq) {
     auto kb = window_score_kernel<D, true>;

@@ -967,8 +967,8 @@ def main():
         names = {
             "decode": "decode_tc_kernel (GQA decode; thread-block clusters per KV head when "
                       "they fit the GPU, else the split grid)",
-            "score": "kvs_score_pairs: window_fa_kernel (S = Q K^T, O += P V), fa_combine_kernel, "
-                     "window_score_kernel (window mass and pair scores)",
+            "score": "kvs_score_pairs: window_fa_kernel (S = Q K^T, O += P V), fa_query_kernel, "
+                     "fa_center_kernel, window_score_kernel (window mass and pair scores)",
         }
     else:
         names = {

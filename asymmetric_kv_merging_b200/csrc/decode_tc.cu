@@ -118,12 +118,16 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     const int g = i / D, c = i - g * D;
     qs[g][c] = to_f32(q[((size_t)head * G + g) * D + c]) * qscale;
   }
-  const bool append = k_new != nullptr && v_new != nullptr && !bad;
-  if (kCluster && append) {
+  // the appended row is staged whatever the length turns out to be, so that its loads
+  // go out with the length's and the query's (one round trip before the stream starts,
+  // not two); `append` then gates its use
+  const bool want_append = k_new != nullptr && v_new != nullptr;
+  if (kCluster && want_append) {
     // element loads: the API does not require these rows to be 16-byte aligned
     for (int i = tid; i < 2 * D; i += kThreads)
       s_kvnew[i / D][i % D] = (i < D ? k_new : v_new)[(size_t)head * D + i % D];
   }
+  const bool append = want_append && !bad;
   if (tid == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);

@@ -50,6 +50,10 @@ def parse_args():
     ap.add_argument("--form", choices=["full", "diagonal", "per_query"], default="full",
                     help="scoring form: the full coupled form with the window mean (default), "
                          "the diagonal-only ablation, or the window read query by query")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="fewer layers than the workload has (reduced runs for profiler captures)")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="fewer sequences than the workload has (reduced runs for profiler captures)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--prefill", action="store_true",
@@ -153,6 +157,20 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # the timed workload
 # ---------------------------------------------------------------------------
+
+def reduced(w, args):
+    """The workload with fewer layers or sequences, when asked for (profiler captures of
+    a small case); its name says so."""
+    ch = {}
+    if args.layers is not None and args.layers < w.layers:
+        ch["layers"] = args.layers
+    if args.batch is not None and args.batch < w.B:
+        ch["B"] = args.batch
+    if not ch:
+        return w
+    tag = "".join(f"_{k}{v}" for k, v in ch.items())
+    return inputs.small_workload(w, name=w.name + "_reduced" + tag, **ch)
+
 
 def plan_rounds(T, target, sink, n_recent):
     """Per-head lengths after each merge round (a round merges R = min(P, len - target))."""
@@ -925,6 +943,7 @@ def main():
     w = inputs.workload(args.workload)
     if args.fp32:
         w = inputs.small_workload(w, dtype="f32", name=w.name + "_fp32")
+    w = reduced(w, args)
     from asymmetric_kv_merging_b200 import kvs
     form_code = {"full": None, "diagonal": kvs.FORM_DIAGONAL,
                  "per_query": kvs.FORM_FULL | kvs.FORM_PER_QUERY}[args.form]

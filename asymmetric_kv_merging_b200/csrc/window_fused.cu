@@ -569,17 +569,22 @@ window_fa_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 //     bf16 hi / mid / lo rows with |e_q|^2 and o_bar . e_q.
 // ---------------------------------------------------------------------------
 
+// One CTA per block of QB window queries of a head (QB grows with the number of heads,
+// so that the grid stays near a thousand CTAs): the warps take the block's queries in
+// turn for (M, L), then every thread (one column) sums its column of the partials' O rows
+// for each query of the block, the loads independent of one another.
 template <int D>
 __global__ void __launch_bounds__(D)
 fa_query_kernel(const float* __restrict__ part_ml, const float* __restrict__ part_o, int Qn,
-                int nparts, float* __restrict__ stats, float* __restrict__ oq) {
-  extern __shared__ float fac[];                 // [nparts] weights 2^(m - M) / L
-  __shared__ float s_ml[2];
-  const int q = blockIdx.x, unit = blockIdx.y, c = threadIdx.x;
+                int nparts, int QB, float* __restrict__ stats, float* __restrict__ oq) {
+  extern __shared__ float fac[];                 // [QB][nparts] weights 2^(m - M) / L
+  const int unit = blockIdx.y, c = threadIdx.x, lane = c & 31, warp = c >> 5;
+  const int q0 = blockIdx.x * QB, nq = min(QB, Qn - q0);
   const float* e = part_ml + (size_t)unit * nparts * Qn * 2;
-  if (c < 32) {
+  for (int j = warp; j < nq; j += D / 32) {
+    const int q = q0 + j;
     float M = -INFINITY;
-    for (int s = c; s < nparts; s += 32) {
+    for (int s = lane; s < nparts; s += 32) {
       const float ls = e[((size_t)s * Qn + q) * 2 + 1];
       if (ls > 0.f) M = fmaxf(M, e[((size_t)s * Qn + q) * 2]);
     }
@@ -587,38 +592,38 @@ fa_query_kernel(const float* __restrict__ part_ml, const float* __restrict__ par
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float Ls = 0.f;
     if (M > -INFINITY)
-      for (int s = c; s < nparts; s += 32) {
+      for (int s = lane; s < nparts; s += 32) {
         const float ls = e[((size_t)s * Qn + q) * 2 + 1];
         if (ls > 0.f) Ls = fmaf(ls, exp2f(e[((size_t)s * Qn + q) * 2] - M), Ls);
       }
     Ls = warp_sum(Ls);
-    if (c == 0) {
-      s_ml[0] = M;
-      s_ml[1] = Ls;
+    const bool valid = Ls > 0.f;
+    for (int s = lane; s < nparts; s += 32) {
+      const float ls = e[((size_t)s * Qn + q) * 2 + 1];
+      fac[j * nparts + s] = (valid && ls > 0.f) ? exp2f(e[((size_t)s * Qn + q) * 2] - M) / Ls : 0.f;
+    }
+    if (lane == 0) {
       stats[((size_t)unit * Qn + q) * 2 + 0] = M;
       stats[((size_t)unit * Qn + q) * 2 + 1] = Ls;
     }
   }
   __syncthreads();
-  const float M = s_ml[0], Ls = s_ml[1];
-  const bool valid = Ls > 0.f;
-  for (int s = c; s < nparts; s += D) {
-    const float ls = e[((size_t)s * Qn + q) * 2 + 1];
-    fac[s] = (valid && ls > 0.f) ? exp2f(e[((size_t)s * Qn + q) * 2] - M) / Ls : 0.f;
-  }
-  __syncthreads();
-  // o_q = sum over partials of weight x O row: independent loads, four accumulators
-  const float* po = part_o + ((size_t)unit * nparts * Qn + q) * D + c;
+  // o_q = sum over partials of weight x O row
   const size_t stride = (size_t)Qn * D;
-  float a8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  int s = 0;
-  for (; s + 8 <= nparts; s += 8) {
+  for (int j = 0; j < nq; ++j) {
+    const int q = q0 + j;
+    const float* po = part_o + ((size_t)unit * nparts * Qn + q) * D + c;
+    const float* f = fac + j * nparts;
+    float a8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    int s = 0;
+    for (; s + 8 <= nparts; s += 8) {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) a8[j] = fmaf(fac[s + j], po[(s + j) * stride], a8[j]);
+      for (int k = 0; k < 8; ++k) a8[k] = fmaf(f[s + k], po[(s + k) * stride], a8[k]);
+    }
+    for (; s < nparts; ++s) a8[s & 7] = fmaf(f[s], po[s * stride], a8[s & 7]);
+    oq[((size_t)unit * 128 + q) * D + c] =
+        ((a8[0] + a8[1]) + (a8[2] + a8[3])) + ((a8[4] + a8[5]) + (a8[6] + a8[7]));
   }
-  for (; s < nparts; ++s) a8[s & 7] = fmaf(fac[s], po[s * stride], a8[s & 7]);
-  oq[((size_t)unit * 128 + q) * D + c] =
-      ((a8[0] + a8[1]) + (a8[2] + a8[3])) + ((a8[4] + a8[5]) + (a8[6] + a8[7]));
 }
 
 // One CTA per 32 columns of a head: 8 warps x 32 columns, warp w summing the queries
@@ -1224,10 +1229,13 @@ static cudaError_t launch_fused_t(const kvs_cache_desc& d, const void* K, const 
   ka<<<dim3(nsa, units), kFuThreads, FaShape<D>::kSmem, st>>>(
       mQ, mK, mV, logn, len, d.H_kv, d.H_q, W, d.T_cap, nsa, part_ml, part_o, flags);
   float* oq = reinterpret_cast<float*>(ws + Ly.oq);
-  const size_t qsm = (size_t)nsa * sizeof(float);
+  // queries per CTA: about a thousand CTAs in all
+  int QB = 1;
+  while (QB < 16 && (long long)units * Qn / (2 * QB) >= 1024) QB *= 2;
+  const size_t qsm = (size_t)QB * nsa * sizeof(float);
   auto kq = fa_query_kernel<D>;
   if (!ensure_smem_attr((const void*)kq, qsm)) return cudaErrorInvalidValue;
-  kq<<<dim3(Qn, units), D, qsm, st>>>(part_ml, part_o, Qn, nsa, stats, oq);
+  kq<<<dim3((Qn + QB - 1) / QB, units), D, qsm, st>>>(part_ml, part_o, Qn, nsa, QB, stats, oq);
   const bool perq = stats_form == KVS_FORM_PER_QUERY;
   fa_center_kernel<D><<<dim3(D / 32, units), kCenterWarps * 32, 0, st>>>(
       stats, oq, Qn, perq ? 1 : 0, obar, zq, wq, e_hi, e_mid, e_lo);

@@ -7,8 +7,9 @@
 //
 //   window_partial_kernel : per (KV head, key split): online softmax of the G*W
 //                           window queries over the split's keys -> (m, l, o) partials
-//   window_combine_kernel : per KV head: merge the splits -> per-query (m, l) and
-//                           o_bar = mean_q o_q
+//   window_combine_kernel : per (KV head, block of queries): merge the splits ->
+//                           per-query (m, l), and sums of o_q over the block
+//   obar_kernel           : per KV head: o_bar = mean_q o_q from the block sums
 //   alpha_bar_kernel      : per (KV head, 64 keys): alpha_bar_t = mean_q 2^(s_qt - m_q) / l_q
 //
 // Logits are kept in the log2 domain: s = (q log2(e)/sqrt(d)) . k + log2(e) logn.
@@ -159,62 +160,92 @@ window_partial_kernel(const T* __restrict__ K, const T* __restrict__ V,
   }
 }
 
+// Combine, with many CTAs (one CTA per head walking every partial of every query was
+// latency-bound). window_combine_kernel: one CTA per block of kCombQ queries of a head;
+// each warp takes queries in turn for (M, L), then every thread (one column) sums its
+// column of o_q over the block's queries into one row of block sums. obar_kernel: per
+// head, o_bar = (sum of the block rows, in order) / number of queries with a finite
+// normaliser.
+constexpr int kCombQ = 4;
+
 template <int D>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(D)
 window_combine_kernel(const float* __restrict__ part_ml, const float* __restrict__ part_o,
-                      int Qn, int nsplit, float* __restrict__ stats, float* __restrict__ obar,
+                      int Qn, int nsplit, float* __restrict__ stats, float* __restrict__ osum,
                       int32_t* __restrict__ flags) {
-  extern __shared__ __align__(16) float csm[];
-  float* fac = csm;                    // [Qn][nsplit]
-  float* red = fac + Qn * nsplit;      // [256]
-  __shared__ int s_valid;
-  const int unit = blockIdx.x, tid = threadIdx.x;
-  if (tid == 0) s_valid = 0;
-  __syncthreads();
+  extern __shared__ __align__(16) float fac[];   // [kCombQ][nsplit]
+  const int unit = blockIdx.y, qb = blockIdx.x, c = threadIdx.x;
+  const int lane = c & 31, warp = c >> 5;
+  const int q0 = qb * kCombQ, nq = min(kCombQ, Qn - q0);
   const float* ml = part_ml + (size_t)unit * nsplit * Qn * 2;
-  for (int q = tid; q < Qn; q += blockDim.x) {
+  for (int j = warp; j < nq; j += D / 32) {
+    const int q = q0 + j;
     float M = -INFINITY;
-    for (int s = 0; s < nsplit; ++s) {
-      float ls = ml[((size_t)s * Qn + q) * 2 + 1];
+    for (int s = lane; s < nsplit; s += 32) {
+      const float ls = ml[((size_t)s * Qn + q) * 2 + 1];
       if (ls > 0.f) M = fmaxf(M, ml[((size_t)s * Qn + q) * 2]);
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float Lsum = 0.f;
-    if (M > -INFINITY) {
-      for (int s = 0; s < nsplit; ++s) {
-        float ls = ml[((size_t)s * Qn + q) * 2 + 1];
+    if (M > -INFINITY)
+      for (int s = lane; s < nsplit; s += 32) {
+        const float ls = ml[((size_t)s * Qn + q) * 2 + 1];
         if (ls > 0.f) Lsum += ls * exp2f(ml[((size_t)s * Qn + q) * 2] - M);
       }
-    }
-    stats[((size_t)unit * Qn + q) * 2 + 0] = M;
-    stats[((size_t)unit * Qn + q) * 2 + 1] = Lsum;
+    Lsum = warp_sum(Lsum);
     const bool ok = Lsum > 0.f && isfinite(Lsum) && isfinite(M);
-    if (!ok && M > -INFINITY) set_flag(flags, KVS_FLAG_NONFINITE_STATS);
     const float inv = ok ? 1.f / Lsum : 0.f;
-    if (ok) atomicAdd(&s_valid, 1);
-    for (int s = 0; s < nsplit; ++s) {
-      float ls = ml[((size_t)s * Qn + q) * 2 + 1];
-      fac[q * nsplit + s] = (ok && ls > 0.f) ? exp2f(ml[((size_t)s * Qn + q) * 2] - M) * inv : 0.f;
+    for (int s = lane; s < nsplit; s += 32) {
+      const float ls = ml[((size_t)s * Qn + q) * 2 + 1];
+      fac[j * nsplit + s] = (ok && ls > 0.f) ? exp2f(ml[((size_t)s * Qn + q) * 2] - M) * inv : 0.f;
+    }
+    if (lane == 0) {
+      stats[((size_t)unit * Qn + q) * 2 + 0] = M;
+      stats[((size_t)unit * Qn + q) * 2 + 1] = ok ? Lsum : 0.f;
+      if (!ok && M > -INFINITY) set_flag(flags, KVS_FLAG_NONFINITE_STATS);
     }
   }
   __syncthreads();
-  const int ngrp = blockDim.x / D;
-  const int c = tid % D, grp = tid / D;
   float acc = 0.f;
-  if (grp < ngrp) {
-    for (int q = grp; q < Qn; q += ngrp) {
-      for (int s = 0; s < nsplit; ++s) {
-        float f = fac[q * nsplit + s];
-        if (f != 0.f) acc = fmaf(f, part_o[(((size_t)unit * nsplit + s) * Qn + q) * D + c], acc);
-      }
+  for (int j = 0; j < nq; ++j) {
+    const float* po = part_o + ((size_t)unit * nsplit * Qn + q0 + j) * D + c;
+    const float* f = fac + j * nsplit;
+    float a4[4] = {0.f, 0.f, 0.f, 0.f};
+    int s = 0;
+    for (; s + 4 <= nsplit; s += 4) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) a4[k] = fmaf(f[s + k], po[(size_t)(s + k) * Qn * D], a4[k]);
     }
+    for (; s < nsplit; ++s) a4[0] = fmaf(f[s], po[(size_t)s * Qn * D], a4[0]);
+    acc += (a4[0] + a4[1]) + (a4[2] + a4[3]);
   }
-  red[tid] = acc;
+  osum[((size_t)unit * 128 + qb) * D + c] = acc;
+}
+
+template <int D>
+__global__ void __launch_bounds__(D)
+obar_kernel(const float* __restrict__ stats, const float* __restrict__ osum, int Qn,
+            float* __restrict__ obar) {
+  __shared__ int s_valid;
+  const int unit = blockIdx.x, c = threadIdx.x;
+  if (c == 0) s_valid = 0;
   __syncthreads();
-  if (tid < D) {
-    float t = 0.f;
-    for (int g2 = 0; g2 < ngrp; ++g2) t += red[g2 * D + tid];
-    obar[(size_t)unit * D + tid] = s_valid > 0 ? t / (float)s_valid : 0.f;
+  int nv = 0;
+  for (int q = c; q < Qn; q += D) nv += stats[((size_t)unit * Qn + q) * 2 + 1] > 0.f;
+  if (nv) atomicAdd(&s_valid, nv);
+  const int nb = (Qn + kCombQ - 1) / kCombQ;
+  const float* col = osum + (size_t)unit * 128 * D + c;
+  float a8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  int b = 0;
+  for (; b + 8 <= nb; b += 8) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) a8[k] += col[(size_t)(b + k) * D];
   }
+  for (; b < nb; ++b) a8[b & 7] += col[(size_t)b * D];
+  __syncthreads();
+  const float t = ((a8[0] + a8[1]) + (a8[2] + a8[3])) + ((a8[4] + a8[5]) + (a8[6] + a8[7]));
+  obar[(size_t)unit * D + c] = s_valid > 0 ? t / (float)s_valid : 0.f;
 }
 
 template <typename T, int D>
@@ -326,10 +357,14 @@ static cudaError_t launch_window_stats_t(const kvs_cache_desc& d, const void* K,
       (const T*)K, (const T*)V, logn, len, (const T*)Qw, d.H_kv, d.H_q, d.T_cap, W, Ly.nsplit,
       part_ml, part_o, flags);
 
-  size_t sm2 = (size_t)(Qn * Ly.nsplit + 256) * sizeof(float);
+  // block sums of o_q in the fp32 window-output rows (ceil(Qn / kCombQ) <= 128 rows a head)
+  float* osum = reinterpret_cast<float*>(ws + Ly.oq);
+  size_t sm2 = (size_t)kCombQ * Ly.nsplit * sizeof(float);
   auto k2 = window_combine_kernel<D>;
   if (!ensure_smem_attr((const void*)k2, sm2)) return cudaErrorInvalidValue;
-  k2<<<units, 256, sm2, st>>>(part_ml, part_o, Qn, Ly.nsplit, stats, obar, flags);
+  k2<<<dim3((Qn + kCombQ - 1) / kCombQ, units), D, sm2, st>>>(part_ml, part_o, Qn, Ly.nsplit,
+                                                               stats, osum, flags);
+  obar_kernel<D><<<units, D, 0, st>>>(stats, osum, Qn, obar);
 
   size_t sm3 = (size_t)(Qn * DP + kAlphaTokens * DP + 2 * Qn + kAlphaTokens + kAlphaThreads) *
                sizeof(float);
@@ -338,7 +373,7 @@ static cudaError_t launch_window_stats_t(const kvs_cache_desc& d, const void* K,
   dim3 g3((d.T_cap + kAlphaTokens - 1) / kAlphaTokens, units);
   k3<<<g3, kAlphaThreads, sm3, st>>>((const T*)K, logn, len, (const T*)Qw, d.H_kv, d.H_q,
                                      d.T_cap, W, stats, alpha);
-  count_launches(3);
+  count_launches(4);
   return cudaGetLastError();
 }
 

@@ -573,8 +573,10 @@ window_fa_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 // so that the grid stays near a thousand CTAs): the warps take the block's queries in
 // turn for (M, L), then every thread (one column) sums its column of the partials' O rows
 // for each query of the block, the loads independent of one another.
+constexpr int kQueryBlockMax = 16;
+
 template <int D>
-__global__ void __launch_bounds__(D)
+__global__ void __launch_bounds__(D, 8)
 fa_query_kernel(const float* __restrict__ part_ml, const float* __restrict__ part_o, int Qn,
                 int nparts, int QB, float* __restrict__ stats, float* __restrict__ oq) {
   extern __shared__ float fac[];                 // [QB][nparts] weights 2^(m - M) / L
@@ -608,21 +610,37 @@ fa_query_kernel(const float* __restrict__ part_ml, const float* __restrict__ par
     }
   }
   __syncthreads();
-  // o_q = sum over partials of weight x O row
+  // o_q = sum over partials of weight x O row, with the loads of a batch independent of
+  // one another: eight partials of one query at a time when there are many partials, all
+  // the block's queries of one partial at a time when there are few
   const size_t stride = (size_t)Qn * D;
-  for (int j = 0; j < nq; ++j) {
-    const int q = q0 + j;
-    const float* po = part_o + ((size_t)unit * nparts * Qn + q) * D + c;
-    const float* f = fac + j * nparts;
-    float a8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    int s = 0;
-    for (; s + 8 <= nparts; s += 8) {
+  const float* pb = part_o + ((size_t)unit * nparts * Qn + q0) * D + c;
+  if (nparts >= 8 || nq == 1) {
+    for (int j = 0; j < nq; ++j) {
+      const float* po = pb + (size_t)j * D;
+      const float* f = fac + j * nparts;
+      float a8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      int s = 0;
+      for (; s + 8 <= nparts; s += 8) {
 #pragma unroll
-      for (int k = 0; k < 8; ++k) a8[k] = fmaf(f[s + k], po[(s + k) * stride], a8[k]);
+        for (int k = 0; k < 8; ++k) a8[k] = fmaf(f[s + k], po[(s + k) * stride], a8[k]);
+      }
+      for (; s < nparts; ++s) a8[s & 7] = fmaf(f[s], po[s * stride], a8[s & 7]);
+      oq[((size_t)unit * 128 + q0 + j) * D + c] =
+          ((a8[0] + a8[1]) + (a8[2] + a8[3])) + ((a8[4] + a8[5]) + (a8[6] + a8[7]));
     }
-    for (; s < nparts; ++s) a8[s & 7] = fmaf(f[s], po[s * stride], a8[s & 7]);
-    oq[((size_t)unit * 128 + q) * D + c] =
-        ((a8[0] + a8[1]) + (a8[2] + a8[3])) + ((a8[4] + a8[5]) + (a8[6] + a8[7]));
+  } else {
+    float acc[kQueryBlockMax];
+#pragma unroll
+    for (int j = 0; j < kQueryBlockMax; ++j) acc[j] = 0.f;
+    for (int s = 0; s < nparts; ++s) {
+#pragma unroll
+      for (int j = 0; j < kQueryBlockMax; ++j)
+        if (j < nq) acc[j] = fmaf(fac[j * nparts + s], pb[s * stride + (size_t)j * D], acc[j]);
+    }
+#pragma unroll
+    for (int j = 0; j < kQueryBlockMax; ++j)
+      if (j < nq) oq[((size_t)unit * 128 + q0 + j) * D + c] = acc[j];
   }
 }
 
@@ -1231,7 +1249,7 @@ static cudaError_t launch_fused_t(const kvs_cache_desc& d, const void* K, const 
   float* oq = reinterpret_cast<float*>(ws + Ly.oq);
   // queries per CTA: about a thousand CTAs in all
   int QB = 1;
-  while (QB < 16 && (long long)units * Qn / (2 * QB) >= 1024) QB *= 2;
+  while (QB < kQueryBlockMax && (long long)units * Qn / (2 * QB) >= 1024) QB *= 2;
   const size_t qsm = (size_t)QB * nsa * sizeof(float);
   auto kq = fa_query_kernel<D>;
   if (!ensure_smem_attr((const void*)kq, qsm)) return cudaErrorInvalidValue;

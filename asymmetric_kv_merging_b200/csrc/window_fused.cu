@@ -83,6 +83,41 @@ __device__ __forceinline__ void tmem_st16_pairs(uint32_t taddr, const uint32_t (
       "r"(w[OFF + 30])
       : "memory");
 }
+// CW (16 or 32) consecutive fp32 columns of this thread's lane, loaded and waited for.
+template <int CW>
+__device__ __forceinline__ void tmem_ld_n(uint32_t taddr, float (&v)[CW]) {
+  if constexpr (CW == 32) {
+    tmem_ld32(taddr, v);
+  } else {
+    static_assert(CW == 16, "chunk width");
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                   "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                   "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+                 :
+                 : "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+  }
+}
+
+// One fp32 column of this thread's lane (warp-collective), waited for.
+__device__ __forceinline__ float tmem_ld1(uint32_t taddr) {
+  uint32_t r;
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr) : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;" : "+r"(r) : : "memory");
+  return __uint_as_float(r);
+}
+
 // Two columns of this thread's lane: store (no wait), and load (waits).
 __device__ __forceinline__ void tmem_st2(uint32_t taddr, uint32_t a, uint32_t b) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x2.b32 [%0], {%1, %2};" ::"r"(taddr), "r"(a), "r"(b)
@@ -1087,19 +1122,22 @@ window_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       const float vn_own = sqrtf(is_a ? na : nb), vn_pair = sqrtf(na) + sqrtf(nb);
       const bf16* v_own = Vg + ((size_t)unit * T_cap + (kval ? t : 0)) * D;
       const bf16* v_next = v_own + D;
+      // chunks of CW window queries (16 in the per-query form, whose per-element work
+      // keeps two chunk-wide arrays live: a narrower chunk keeps them in registers)
+      constexpr int CW = PERQ ? 16 : 32;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        float v[32];
+      for (int c = 0; c < 128 / CW; ++c) {
+        float v[CW];
         if (live) {
-          tmem_ld32(s_cols + 32 * c, v);
+          tmem_ld_n<CW>(s_cols + CW * c, v);
         } else {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = 0.f;
+          for (int j = 0; j < CW; ++j) v[j] = 0.f;
         }
         if (kval) {
 #pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            const float2 z = *reinterpret_cast<const float2*>(&zq[32 * c + j]);
+          for (int j = 0; j < CW; j += 2) {
+            const float2 z = *reinterpret_cast<const float2*>(&zq[CW * c + j]);
             const float2 x = ffma2(make_float2(v[j], v[j + 1]), make_float2(qscale, qscale),
                                    make_float2(lnt - z.x, lnt - z.y));
             v[j] = ex2_ftz(x.x);
@@ -1107,47 +1145,74 @@ window_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
           }
           if (hide > 0) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (qmod[32 * c + j] < hide) v[j] = 0.f;
+            for (int j = 0; j < CW; ++j)
+              if (qmod[CW * c + j] < hide) v[j] = 0.f;
           }
         } else {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = 0.f;
+          for (int j = 0; j < CW; ++j) v[j] = 0.f;
         }
         if constexpr (!PERQ) {
           float a4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int j = 0; j < 32; ++j) a4[j & 3] += v[j];
+          for (int j = 0; j < CW; ++j) a4[j & 3] += v[j];
           acc += (a4[0] + a4[1]) + (a4[2] + a4[3]);
         } else {
           // per window query: lane a (even key) takes N11 and N12, lane b N22
-          float u[32];
+          float u[CW];
           if (live) {
-            tmem_ld32(u_cols + 32 * c, u);
+            tmem_ld_n<CW>(u_cols + CW * c, u);
           } else {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) u[j] = 0.f;
+            for (int j = 0; j < CW; ++j) u[j] = 0.f;
           }
-          const unsigned char* et = base + S::kEOff;
-#pragma unroll 4
-          for (int j = 0; j < 32; ++j) {
-            const int q = 32 * c + j;
+          // fully unrolled: v[] and u[] stay in registers (a partly unrolled loop indexes
+          // them at run time, which puts them in local memory). The terms whose expansion
+          // cancels are only marked here and taken directly afterwards, outside the loop.
+          uint32_t redo_s = 0u, redo_c = 0u;
+#pragma unroll
+          for (int j = 0; j < CW; ++j) {
+            const int q = CW * c + j;
             const float p = v[j], uu = u[j];
             const float p_o = __shfl_xor_sync(0xffffffffu, p, 1);
             const float u_o = __shfl_xor_sync(0xffffffffu, uu, 1);
             const float z = eqs[q], wq = eqs[128 + q], se = eqs[256 + q];
-            // |v - o_q|^2 and |v_a + v_b - 2 o_q|^2 by the expansion; where that cancels
-            // (a query whose output sits near the row), directly from the rows
+            // |v - o_q|^2 and |v_a + v_b - 2 o_q|^2 by the expansion, unless it cancels
+            // (a query whose output sits near the row)
             const float xs = uu - wq, xc = uu + u_o - 2.f * wq;
-            float rs = fmaf(-2.f, xs, t_own) + z;
-            float rc = fmaf(-4.f, xc, ec) + 4.f * z;
+            const float rs = fmaf(-2.f, xs, t_own) + z;
+            const float rc = fmaf(-4.f, xc, ec) + 4.f * z;
             const float ms = t_own + z + 2.f * fabsf(xs) + 2.f * vn_own * se;
             const float mc = ec + 4.f * z + 4.f * fabsf(xc) + 4.f * vn_pair * se;
-            if (p != 0.f && rs < kRedoFrac * ms) rs = direct_sq<D>(v_own, nullptr, obs, et, q, 1.f);
-            if (is_a && p * p_o != 0.f && rc < kRedoFrac * mc)
-              rc = direct_sq<D>(v_own, v_next, obs, et, q, 2.f);
-            n_self = fmaf(fabsf(p * (1.f - 2.f * p)), sqrt_approx(fmaxf(0.f, rs)), n_self);
-            if (is_a) n_cpl = fmaf(p * p_o, sqrt_approx(fmaxf(0.f, rc)), n_cpl);
+            const bool ds = p != 0.f && rs < kRedoFrac * ms;
+            const bool dc = is_a && p * p_o != 0.f && rc < kRedoFrac * mc;
+            redo_s |= (uint32_t)ds << j;
+            redo_c |= (uint32_t)dc << j;
+            n_self = fmaf(ds ? 0.f : fabsf(p * (1.f - 2.f * p)), sqrt_approx(fmaxf(0.f, rs)), n_self);
+            if (is_a) n_cpl = fmaf(dc ? 0.f : p * p_o, sqrt_approx(fmaxf(0.f, rc)), n_cpl);
+          }
+          // the marked terms, directly from the value rows and e_q (rare: only keys that
+          // hold much of some query's attention); the query's column of S^T is loaded
+          // again by the whole warp and p recomputed with the same arithmetic
+          uint32_t todo = __reduce_or_sync(0xffffffffu, redo_s | redo_c);
+          const unsigned char* et = base + S::kEOff;
+          while (todo) {
+            const int j = __ffs(todo) - 1;
+            todo &= todo - 1u;
+            const int q = CW * c + j;
+            float sv = tmem_ld1(s_cols + q);
+            float p = 0.f;
+            if (kval) {
+              p = ex2_ftz(fmaf(sv, qscale, lnt - zq[q]));
+              if (hide > 0 && qmod[q] < hide) p = 0.f;
+            }
+            const float p_o = __shfl_xor_sync(0xffffffffu, p, 1);
+            if ((redo_s >> j) & 1u)
+              n_self = fmaf(fabsf(p * (1.f - 2.f * p)),
+                            sqrt_approx(direct_sq<D>(v_own, nullptr, obs, et, q, 1.f)), n_self);
+            if ((redo_c >> j) & 1u)
+              n_cpl = fmaf(p * p_o, sqrt_approx(direct_sq<D>(v_own, v_next, obs, et, q, 2.f)),
+                           n_cpl);
           }
         }
       }

@@ -153,7 +153,7 @@ def planted_sinks(w, plants, layer=0):
 
 
 @pytest.mark.parametrize("dtype,d,form", [("f32", 64, None), ("bf16", 128, None),
-                                          ("bf16", 128, "per_query")])
+                                          ("bf16", 128, "per_query"), ("bf16", 64, "per_query")])
 def test_peaked_attention_exercises_degenerate_pairs(kvs, dtype, d, form):
     """Planted attention sinks: a pair at alpha_bar ~ 0.35 per row (D < 0, the
     plain-average branch) in KV head 0 and a row at alpha_bar ~ 0.7 (> 1/2) in KV head 1.
@@ -207,6 +207,22 @@ def test_per_query_window_form(kvs, wl, T, H_kv):
     g, o = decode_both(kvs, w, li, g, o, range(w.n_decode), stats=stats, ws=ws)
     stats.report(f"per-query window form T={T} H_kv={H_kv}")
     assert stats.scores_compared > 0
+    assert stats.near_threshold <= 8
+
+
+@pytest.mark.parametrize("form", ["full", "diagonal", "per_query"])
+def test_head_dim_64_tensor_core_passes(kvs, form):
+    """bf16 caches with d = 64 take the d = 64 instantiations of both tensor-core window
+    passes (four-stage rings, one 64-column box per row): every form, several tiles per
+    CTA in both passes, every round compared, then decode."""
+    w = inputs.small_workload(inputs.workload(1), T=32768, H_kv=2, H_q=8, d=64, n_decode=4)
+    li = inputs.make_layer(w, 0, device="cuda")
+    code = {"full": kvs.FORM_FULL, "diagonal": kvs.FORM_DIAGONAL,
+            "per_query": kvs.FORM_FULL | kvs.FORM_PER_QUERY}[form]
+    g, o, stats, ws = compress_both(kvs, w, li, form=code)
+    g, o = decode_both(kvs, w, li, g, o, range(w.n_decode), stats=stats, ws=ws)
+    stats.report(f"bf16 d=64 {form} form T=32768 H_kv=2")
+    assert stats.scores_compared > 0 and stats.merged_compared > 0
     assert stats.near_threshold <= 8
 
 

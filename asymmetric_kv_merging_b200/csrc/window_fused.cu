@@ -197,7 +197,7 @@ __global__ void __launch_bounds__(kFuThreads, 1)
 window_fa_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const float* __restrict__ logn,
                  const int32_t* __restrict__ len, int H_kv, int H_q, int W, int T_cap, int nsplit,
-                 float* __restrict__ part_ml, float* __restrict__ part_o,
+                 int cap_chunks, float* __restrict__ part_ml, float* __restrict__ part_o,
                  int32_t* __restrict__ flags) {
   using S = FaShape<D>;
   constexpr int ST = S::kStages;
@@ -224,10 +224,23 @@ window_fa_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     if (split == 0 && tid == 0) set_flag(flags, KVS_FLAG_BAD_LENGTH);
     L = 0;
   }
-  int chunk = (L + nsplit - 1) / nsplit;
+  // split s takes one chunk of the head's rows: a share of its length, or (cap_chunks) of
+  // the capacity, so that a head shorter than the capacity leaves its last CTAs idle
+  int chunk = ((cap_chunks ? T_cap : L) + nsplit - 1) / nsplit;
   chunk = (chunk + kFuKeys - 1) / kFuKeys * kFuKeys;
   const int t0 = split * chunk, t1 = min(L, t0 + chunk);
   const int ntiles = t1 > t0 ? (t1 - t0 + kFuKeys - 1) / kFuKeys : 0;
+  if (ntiles == 0) {   // nothing of the head in this split: an empty partial (uniform over the CTA)
+    float* pm = part_ml + ((size_t)unit * nsplit + split) * Qn * 2;
+    float* po = part_o + ((size_t)unit * nsplit + split) * Qn * D;
+    for (int i = tid; i < Qn; i += kFuThreads) {
+      pm[2 * i] = -INFINITY;
+      pm[2 * i + 1] = 0.f;
+    }
+    for (int i = tid; i < Qn * D / 4; i += kFuThreads)
+      reinterpret_cast<float4*>(po)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    return;
+  }
   const int q_row0 = (b * H_q + h * G) * W;
   const int k_row0 = unit * T_cap + t0;
   const bool has_ln = logn != nullptr;
@@ -843,7 +856,8 @@ window_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     const bf16* __restrict__ Vg, const float* __restrict__ logn,
                     const int32_t* __restrict__ len,
                     const int32_t* __restrict__ cand_begin, int n_recent, int H_kv, int H_q,
-                    int W, int T_cap, int nsplit, int form, const float* __restrict__ stats,
+                    int W, int T_cap, int nsplit, int cap_chunks, int form,
+                    const float* __restrict__ stats,
                     const float* __restrict__ obar, const float* __restrict__ zqg,
                     const float* __restrict__ wqg, float* __restrict__ score,
                     float* __restrict__ w_b, int32_t* __restrict__ flags) {
@@ -876,8 +890,18 @@ window_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
   const int span = L - n_recent - c0;
   const int P = (L >= 0 && span > 0) ? span / 2 : 0;
   const int ntot = (2 * P + kFuKeys - 1) / kFuKeys;   // candidate tiles of the head
-  const int tbeg = (int)((long long)split * ntot / nsplit);
-  const int tend = (int)((long long)(split + 1) * ntot / nsplit);
+  // split s takes a share of the head's candidate tiles, or (cap_chunks) a fixed number of
+  // tiles of the capacity's, so that a short head leaves its last CTAs idle
+  int tbeg, tend;
+  if (cap_chunks) {
+    const int cap_tiles = (T_cap / 2 + kFuKeys / 2 - 1) / (kFuKeys / 2);
+    const int per = (cap_tiles + nsplit - 1) / nsplit;
+    tbeg = min(ntot, split * per);
+    tend = min(ntot, tbeg + per);
+  } else {
+    tbeg = (int)((long long)split * ntot / nsplit);
+    tend = (int)((long long)(split + 1) * ntot / nsplit);
+  }
   const int ntiles = tend - tbeg;
   if (ntiles <= 0) return;                           // uniform over the CTA
   const int q_row0 = (b * H_q + h * G) * W;
@@ -1267,6 +1291,14 @@ static int fused_splits(int units) {
   return s;
 }
 
+// Many heads over a large capacity: a few splits per head over fixed chunks of the
+// capacity instead of one share of each head's length. With ragged lengths (a serving
+// batch) a head's CTAs then carry at most a chunk each and the short heads' spare CTAs
+// return at once, so the SMs even the load out over the waves; a single CTA per head
+// would leave the longest heads setting the time.
+static bool cap_chunked(int units, int T_cap) { return units >= 74 && T_cap >= 8192; }
+static int cap_splits(int T_cap) { return T_cap / 2048 < 4 ? T_cap / 2048 : 4; }
+
 bool window_fused_supported(const kvs_cache_desc& d, int W) {
   const unsigned long long rows = (unsigned long long)d.B * d.H_kv * (unsigned long long)d.T_cap;
   const unsigned long long qrows = (unsigned long long)d.B * d.H_q * (unsigned long long)W;
@@ -1296,7 +1328,8 @@ static cudaError_t launch_fused_t(const kvs_cache_desc& d, const void* K, const 
     return cudaErrorInvalidValue;
   // pass A: one partial per CTA (its two softmax groups merged), as many CTAs per head as
   // the layout has partial slots at most
-  int nsa = fused_splits(units);
+  const bool capc = cap_chunked(units, d.T_cap);
+  int nsa = capc ? cap_splits(d.T_cap) : fused_splits(units);
   if (nsa > Ly.part_slots) nsa = Ly.part_slots;
   const int Qn = Ly.Qn;
   int32_t* flags = reinterpret_cast<int32_t*>(ws);
@@ -1310,7 +1343,8 @@ static cudaError_t launch_fused_t(const kvs_cache_desc& d, const void* K, const 
   auto ka = window_fa_kernel<D>;
   if (!ensure_smem_attr((const void*)ka, FaShape<D>::kSmem)) return cudaErrorInvalidValue;
   ka<<<dim3(nsa, units), kFuThreads, FaShape<D>::kSmem, st>>>(
-      mQ, mK, mV, logn, len, d.H_kv, d.H_q, W, d.T_cap, nsa, part_ml, part_o, flags);
+      mQ, mK, mV, logn, len, d.H_kv, d.H_q, W, d.T_cap, nsa, capc ? 1 : 0, part_ml, part_o,
+      flags);
   float* oq = reinterpret_cast<float*>(ws + Ly.oq);
   // queries per CTA: about a thousand CTAs in all
   int QB = 1;
@@ -1322,19 +1356,19 @@ static cudaError_t launch_fused_t(const kvs_cache_desc& d, const void* K, const 
   const bool perq = stats_form == KVS_FORM_PER_QUERY;
   fa_center_kernel<D><<<dim3(D / 32, units), kCenterWarps * 32, 0, st>>>(
       stats, oq, Qn, perq ? 1 : 0, obar, zq, wq, e_hi, e_mid, e_lo);
-  const int nsb = fused_splits(units);
+  const int nsb = capc ? cap_splits(d.T_cap) : fused_splits(units);
   if (perq) {
     auto kb = window_score_kernel<D, true>;
     if (!ensure_smem_attr((const void*)kb, ScShape<D, true>::kSmem)) return cudaErrorInvalidValue;
     kb<<<dim3(nsb, units), kFuThreads, ScShape<D, true>::kSmem, st>>>(
         mQ, mK, mV, mEh, mEm, mEl, (const bf16*)V, logn, len, cand_begin, n_recent, d.H_kv,
-        d.H_q, W, d.T_cap, nsb, form, stats, obar, zq, wq, score, w_b, flags);
+        d.H_q, W, d.T_cap, nsb, capc ? 1 : 0, form, stats, obar, zq, wq, score, w_b, flags);
   } else {
     auto kb = window_score_kernel<D, false>;
     if (!ensure_smem_attr((const void*)kb, ScShape<D, false>::kSmem)) return cudaErrorInvalidValue;
     kb<<<dim3(nsb, units), kFuThreads, ScShape<D, false>::kSmem, st>>>(
         mQ, mK, mV, mEh, mEm, mEl, (const bf16*)V, logn, len, cand_begin, n_recent, d.H_kv,
-        d.H_q, W, d.T_cap, nsb, form, stats, obar, zq, wq, score, w_b, flags);
+        d.H_q, W, d.T_cap, nsb, capc ? 1 : 0, form, stats, obar, zq, wq, score, w_b, flags);
   }
   count_launches(4);
   return cudaGetLastError();

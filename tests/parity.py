@@ -48,6 +48,7 @@ class Stats:
     degenerate_pairs: int = 0        # the oracle took the plain-average branch
     degenerate_boundary: int = 0     # D within 2x of the branch threshold: either branch
     alpha_over_half: int = 0         # candidate rows with alpha_bar > 1/2
+    extrapolating: int = 0           # pairs whose w_b lies outside [0, 1] (used as printed)
     selected: int = 0
     near_threshold: int = 0          # selection differences within 1e-5 of the threshold
     merged_compared: int = 0
@@ -172,6 +173,7 @@ def _check_scores(hs, sg, wg, dd, form, stats, where):
         boundary = ~np.isfinite(ratio) | ((ratio > 0.5e-6) & (ratio < 2e-6))
     stats.degenerate_pairs += int(hs.degenerate.sum())
     stats.degenerate_boundary += int(boundary.sum())
+    stats.extrapolating += int(((hs.w_b < 0.0) | (hs.w_b > 1.0)).sum())
     strict = ~boundary
     scale = np.max(np.abs(hs.score[np.isfinite(hs.score)]), initial=0.0)
     np.testing.assert_allclose(sg[strict], hs.score[strict], rtol=2e-4, atol=1e-7 * scale,

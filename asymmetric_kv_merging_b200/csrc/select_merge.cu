@@ -435,25 +435,20 @@ merge_kernel(const T* __restrict__ K, const T* __restrict__ V, const float* __re
   if constexpr (LPR <= 16) {
     constexpr int PPI = 16 / LPR;                   // pairs per warp iteration
     const int slot = lane / (2 * LPR), r = (lane / LPR) & 1, c = lane % LPR;
-    for (int base = warp * PPI; base < nvalid; base += WARPS * PPI) {
-      const int t = base + slot;
+    // U warp iterations per batch: every load of the batch is issued before the first is
+    // used, so a warp keeps U times the bytes in flight (one iteration's 32 x 32 bytes
+    // would leave the kernel bound by memory latency)
+    constexpr int U = 4;
+    auto pair_rows = [&](int t, const uint4& kr, const uint4& vr, float lr) {
       const bool valid = t < nvalid;
       const int p = pbase + t;
-      const int row = c0 + 2 * p + r;
-      uint4 kr = make_uint4(0, 0, 0, 0), vr = make_uint4(0, 0, 0, 0);
-      float lr = 0.f;
-      if (valid) {
-        kr = load_raw(Kh + (size_t)row * D + c * VN);
-        vr = load_raw(Vh + (size_t)row * D + c * VN);
-        lr = lnh ? lnh[row] : 0.f;
-      }
       uint4 kp, vp;
       kp.x = __shfl_xor_sync(0xffffffffu, kr.x, LPR); kp.y = __shfl_xor_sync(0xffffffffu, kr.y, LPR);
       kp.z = __shfl_xor_sync(0xffffffffu, kr.z, LPR); kp.w = __shfl_xor_sync(0xffffffffu, kr.w, LPR);
       vp.x = __shfl_xor_sync(0xffffffffu, vr.x, LPR); vp.y = __shfl_xor_sync(0xffffffffu, vr.y, LPR);
       vp.z = __shfl_xor_sync(0xffffffffu, vr.z, LPR); vp.w = __shfl_xor_sync(0xffffffffu, vr.w, LPR);
       const float lp = __shfl_xor_sync(0xffffffffu, lr, LPR);
-      if (!valid) continue;
+      if (!valid) return;
       const int off = s_off[t];
       if (s_sel[t]) {
         if (r == 0) {
@@ -484,6 +479,25 @@ merge_kernel(const T* __restrict__ K, const T* __restrict__ V, const float* __re
         store_raw(Vo + (size_t)(off + r) * D + c * VN, vr);
         if (c == 0) lno[off + r] = lr;
       }
+    };
+    for (int base0 = warp * PPI; base0 < nvalid; base0 += WARPS * PPI * U) {
+      uint4 krs[U], vrs[U];
+      float lrs[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int t = base0 + u * WARPS * PPI + slot;
+        krs[u] = make_uint4(0, 0, 0, 0);
+        vrs[u] = make_uint4(0, 0, 0, 0);
+        lrs[u] = 0.f;
+        if (t < nvalid) {
+          const int row = c0 + 2 * (pbase + t) + r;
+          krs[u] = load_raw(Kh + (size_t)row * D + c * VN);
+          vrs[u] = load_raw(Vh + (size_t)row * D + c * VN);
+          lrs[u] = lnh ? lnh[row] : 0.f;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) pair_rows(base0 + u * WARPS * PPI + slot, krs[u], vrs[u], lrs[u]);
     }
   } else {
     // LPR == 32: one lane holds the same 16-byte slice of both rows.

@@ -16,7 +16,7 @@
 //   the protected prefix and suffix; a block-level ballot scan gives each pair's
 //   output row; rows move as 16-byte vectors, merged rows are computed in fp32.
 // merge_inplace_kernel: one CTA per head walks the span in order, staging each
-//   chunk in shared memory (double-buffered, the next chunk's copies in flight)
+//   chunk in shared memory (a ring of three stages, the next chunks' copies in flight)
 //   before writing it to lower (or equal) rows.
 #include "kvs_common.cuh"
 #include "kvs_kernels.h"
@@ -557,13 +557,21 @@ __device__ __forceinline__ void cp_async4(void* smem, const void* gmem) {
                : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+// Shared-memory stages of the in-place merge's walk: item k is copied in while items
+// k - 1 and k - 2 are processed.
+constexpr int kInplaceStages = 3;
+// Wait until at most kInplaceStages - 1 of this thread's copy groups are pending: with
+// one group committed per item (and kInplaceStages - 1 before the walk), item k's landed.
+__device__ __forceinline__ void cp_async_wait_stages() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(kInplaceStages - 1) : "memory");
+}
 
 // In-place merge of one head per CTA. Items are the pair chunks of the span (CH pairs,
 // 2 CH rows), then the suffix chunks (2 CH rows). Every output row lies at or below its
 // input row, so no item writes a row that a later item still has to read: the rows of
-// item k + 1 are copied into the other shared-memory stage while item k is written back,
-// and the planning warp loads the scores of chunk k + 1 while it plans chunk k.
+// items k + 1 and k + 2 are being copied into the other shared-memory stages while item k
+// is written back (reading ahead never conflicts: rows only move down), and the planning
+// warp loads the scores of chunk k + 1 while it plans chunk k.
 template <typename T, int D>
 __global__ void __launch_bounds__(kMergeThreads)
 merge_inplace_kernel(T* __restrict__ K, T* __restrict__ V, float* __restrict__ logn,
@@ -577,9 +585,9 @@ merge_inplace_kernel(T* __restrict__ K, T* __restrict__ V, float* __restrict__ l
   constexpr int VPR = D * (int)sizeof(T) / 16;
   constexpr int VN = Vec16<T>::n;
   extern __shared__ __align__(16) unsigned char ism[];
-  uint4* sK = reinterpret_cast<uint4*>(ism);                   // [2][SROWS][VPR]
-  uint4* sV = sK + 2 * SROWS * VPR;                            // [2][SROWS][VPR]
-  float* sL = reinterpret_cast<float*>(sV + 2 * SROWS * VPR);  // [2][SROWS]
+  uint4* sK = reinterpret_cast<uint4*>(ism);                             // [ST][SROWS][VPR]
+  uint4* sV = sK + kInplaceStages * SROWS * VPR;                         // [ST][SROWS][VPR]
+  float* sL = reinterpret_cast<float*>(sV + kInplaceStages * SROWS * VPR);  // [ST][SROWS]
   __shared__ int s_off[32];
   __shared__ unsigned char s_sel[32];
   __shared__ float s_w[32];
@@ -624,8 +632,11 @@ merge_inplace_kernel(T* __restrict__ K, T* __restrict__ V, float* __restrict__ l
       }
       for (int r = tid; r < nr; r += blockDim.x) cp_async4(dl + r, lnh + r0 + r);
     };
-    load_stage(0, 0);
-    cp_async_commit();
+    // the first kInplaceStages - 1 items in flight before the walk starts
+    for (int k = 0; k < kInplaceStages - 1; ++k) {
+      if (k < n_items) load_stage(k, k);
+      cp_async_commit();                                       // (possibly empty)
+    }
     // the planning warp's scores and weights of the current pair chunk
     float sc_cur = 0.f, w_cur = 0.f;
     if (tid < 32 && lane < min(CH, P)) {
@@ -634,9 +645,11 @@ merge_inplace_kernel(T* __restrict__ K, T* __restrict__ V, float* __restrict__ l
     }
     __syncthreads();                                           // s_lt / s_eq initialised
     for (int k = 0; k < n_items; ++k) {
-      const int b = k & 1;
-      if (k + 1 < n_items) load_stage(b ^ 1, k + 1);
-      cp_async_commit();                                       // (empty on the last item)
+      const int b = k % kInplaceStages;
+      // the stage freed by item k - 1 takes item k + ST - 1
+      if (k + kInplaceStages - 1 < n_items)
+        load_stage((k + kInplaceStages - 1) % kInplaceStages, k + kInplaceStages - 1);
+      cp_async_commit();                                       // (empty near the end)
       if (k < n_pc && tid < 32) {                              // one warp plans the chunk
         const int pb = CH * k, np = min(CH, P - pb);
         float sc_next = 0.f, w_next = 0.f;
@@ -669,7 +682,7 @@ merge_inplace_kernel(T* __restrict__ K, T* __restrict__ V, float* __restrict__ l
         sc_cur = sc_next;
         w_cur = w_next;
       }
-      cp_async_wait1();                                        // this thread's copies of item k landed
+      cp_async_wait_stages();                                  // this thread's copies of item k landed
       __syncthreads();                                         // everyone's, and the plan
       const uint4* cK = sK + b * SROWS * VPR;
       const uint4* cV = sV + b * SROWS * VPR;
@@ -759,8 +772,9 @@ static cudaError_t launch_merge_t(const kvs_cache_desc& d, const void* K, const 
   if (inplace) {
     constexpr int VPR = D * (int)sizeof(T) / 16;
     constexpr int CH = inplace_chunk<T, D>();
-    // two stages of K, V (2 CH rows each) and log-counts
-    constexpr size_t smem = (size_t)2 * 2 * (2 * CH * VPR) * 16 + 2 * 2 * CH * sizeof(float);
+    // kInplaceStages stages of K, V (2 CH rows each) and log-counts
+    constexpr size_t smem = (size_t)kInplaceStages * 2 * (2 * CH * VPR) * 16 +
+                            (size_t)kInplaceStages * 2 * CH * sizeof(float);
     static_assert(smem <= 100 * 1024, "in-place staging");
     auto kfn = merge_inplace_kernel<T, D>;
     if (!ensure_smem_attr((const void*)kfn, smem)) return cudaErrorInvalidValue;

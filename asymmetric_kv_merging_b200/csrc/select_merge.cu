@@ -16,7 +16,7 @@
 //   the protected prefix and suffix; a block-level ballot scan gives each pair's
 //   output row; rows move as 16-byte vectors, merged rows are computed in fp32.
 // merge_inplace_kernel: one CTA per head walks the span in order, staging each
-//   chunk in shared memory (a ring of three stages, the next chunks' copies in flight)
+//   chunk in shared memory (a ring of stages, the next chunk's copies in flight)
 //   before writing it to lower (or equal) rows.
 #include "kvs_common.cuh"
 #include "kvs_kernels.h"
@@ -557,9 +557,11 @@ __device__ __forceinline__ void cp_async4(void* smem, const void* gmem) {
                : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-// Shared-memory stages of the in-place merge's walk: item k is copied in while items
-// k - 1 and k - 2 are processed.
-constexpr int kInplaceStages = 3;
+// Shared-memory stages of the in-place merge's walk: items k + 1 .. k + ST - 1 are copied
+// in while item k is processed. Two stages: three measured the same on the 32-layer
+// prefill (the walk is not bound by its copies' latency there) with half again the
+// shared memory per CTA.
+constexpr int kInplaceStages = 2;
 // Wait until at most kInplaceStages - 1 of this thread's copy groups are pending: with
 // one group committed per item (and kInplaceStages - 1 before the walk), item k's landed.
 __device__ __forceinline__ void cp_async_wait_stages() {
@@ -569,8 +571,8 @@ __device__ __forceinline__ void cp_async_wait_stages() {
 // In-place merge of one head per CTA. Items are the pair chunks of the span (CH pairs,
 // 2 CH rows), then the suffix chunks (2 CH rows). Every output row lies at or below its
 // input row, so no item writes a row that a later item still has to read: the rows of
-// items k + 1 and k + 2 are being copied into the other shared-memory stages while item k
-// is written back (reading ahead never conflicts: rows only move down), and the planning
+// the next items are being copied into the other shared-memory stages while item k is
+// written back (reading ahead never conflicts: rows only move down), and the planning
 // warp loads the scores of chunk k + 1 while it plans chunk k.
 template <typename T, int D>
 __global__ void __launch_bounds__(kMergeThreads)

@@ -67,7 +67,7 @@ __device__ __forceinline__ int block_excl_scan(int v, int* warp_tot, int& total)
   return r;
 }
 
-__global__ void __launch_bounds__(kSelThreads)
+__global__ void __launch_bounds__(kSelThreads, 1)
 select_kernel(const float* __restrict__ score, const int32_t* __restrict__ len,
               const int32_t* __restrict__ cand_begin, int n_recent,
               const int32_t* __restrict__ target, int scope, int H_kv, int T_cap, int nblk,
@@ -199,15 +199,26 @@ select_kernel(const float* __restrict__ score, const int32_t* __restrict__ len,
         const int hh = h_first + i;
         const int P = hinfo[hh].P;
         const float* sc = score + (size_t)hh * pstride;
-        for (int p0 = 0; p0 < P; p0 += kSelThreads) {
-          const int p = p0 + tid;
-          const uint32_t key = p < P ? score_key(sc[p]) : 0u;
-          const bool match = p < P && (key & pmask) == prefix;
-          const unsigned ball = __ballot_sync(0xffffffffu, match);
-          int base = 0;
-          if (lane == 0 && ball) base = atomicAdd(&s_ncand, __popc(ball));
-          base = __shfl_sync(0xffffffffu, base, 0);
-          if (match) cand[base + __popc(ball & ((1u << lane) - 1u))] = key;
+        // eight independent loads per thread in flight, as in the histogram pass
+        constexpr int kBatch = 8;
+        for (int p0 = 0; p0 < P; p0 += kSelThreads * kBatch) {
+          float v[kBatch];
+#pragma unroll
+          for (int k = 0; k < kBatch; ++k) {
+            const int p = p0 + k * kSelThreads + tid;
+            v[k] = p < P ? sc[p] : 0.f;
+          }
+#pragma unroll
+          for (int k = 0; k < kBatch; ++k) {
+            const int p = p0 + k * kSelThreads + tid;
+            const uint32_t key = p < P ? score_key(v[k]) : 0u;
+            const bool match = p < P && (key & pmask) == prefix;
+            const unsigned ball = __ballot_sync(0xffffffffu, match);
+            int base = 0;
+            if (lane == 0 && ball) base = atomicAdd(&s_ncand, __popc(ball));
+            base = __shfl_sync(0xffffffffu, base, 0);
+            if (match) cand[base + __popc(ball & ((1u << lane) - 1u))] = key;
+          }
         }
       }
       __syncthreads();

@@ -25,19 +25,26 @@ def merge_bytes(n_in, n_out, head_dim, elem_bytes):
     return int(n_in) * row + int(n_out) * row
 
 
-def score_bytes(n_rows, n_pairs, head_dim, elem_bytes):
-    """Algorithmic bytes of one scoring pass over one KV head of n_rows rows: window
-    pass A reads K and the log-counts, pass B reads K, V and the log-counts and writes
-    the window mass, pair scoring reads K, V and the window mass and writes a score and
-    a weight per pair."""
+def score_bytes(n_rows, n_pairs, head_dim, elem_bytes, fused=True):
+    """Algorithmic bytes of one scoring call over one KV head of n_rows rows with n_pairs
+    candidate pairs (2 n_pairs candidate rows).
+
+    fused (the tensor-core passes of bf16 caches): window pass A reads every row's K, V and
+    log-count (the window outputs need V); pass B reads the candidate rows' K, V and
+    log-counts (the window mass needs K, the pair terms V) and writes a score and a weight
+    per pair. Not fused (the CUDA-core path of fp32 caches): the window pass reads every
+    row's K, V and log-count, the window-mass pass every row's K and log-count and writes
+    the mass, and pair scoring reads the candidate rows' K, V and mass and writes the
+    score and weight."""
     k_row = int(head_dim) * int(elem_bytes)
-    pass_a = int(n_rows) * (k_row + 4)
-    pass_b = int(n_rows) * (2 * k_row + 4 + 4)
-    pairs = int(n_rows) * (2 * k_row + 4) + int(n_pairs) * 8
-    return pass_a + pass_b + pairs
+    rows, cand = int(n_rows), 2 * int(n_pairs)
+    out = int(n_pairs) * 8
+    if fused:
+        return rows * (2 * k_row + 4) + cand * (2 * k_row + 4) + out
+    return rows * (2 * k_row + 4) + rows * (k_row + 4 + 4) + cand * (2 * k_row + 4) + out
 
 
-def prefill_chunk_bytes(L, n, budget, sink, W, head_dim, elem_bytes):
+def prefill_chunk_bytes(L, n, budget, sink, W, head_dim, elem_bytes, fused=True):
     """Algorithmic bytes of one chunked-prefill step over one KV head that holds L rows:
     append n rows (read the chunk's K and V, write them and their log-counts), then
     the merge rounds back to `budget` (each a scoring pass and an in-place merge over
@@ -50,7 +57,7 @@ def prefill_chunk_bytes(L, n, budget, sink, W, head_dim, elem_bytes):
         R = min(P, length - budget)
         if R <= 0:
             raise ValueError("budget unreachable")
-        total += score_bytes(length, P, head_dim, elem_bytes)
+        total += score_bytes(length, P, head_dim, elem_bytes, fused)
         total += merge_bytes(length - sink, length - R - sink, head_dim, elem_bytes)
         length -= R
         rounds += 1

@@ -407,7 +407,7 @@ class Runner:
         tot = 0
         for (L_in, _, _) in self.plan:
             P = (L_in - w.W - w.sink) // 2
-            tot += sum(accounting.score_bytes(int(a), max(0, int(p)), w.d, eb)
+            tot += sum(accounting.score_bytes(int(a), max(0, int(p)), w.d, eb, w.dtype == "bf16")
                        for a, p in zip(L_in.reshape(-1), P.reshape(-1)))
         return tot * w.layers
 
@@ -442,7 +442,7 @@ class Runner:
                 n, L = sub["n"], sub["L"]
                 P, R = n // 2, n // 2
                 for Lh in L.reshape(-1):
-                    tot += accounting.score_bytes(int(Lh), P, w.d, eb)
+                    tot += accounting.score_bytes(int(Lh), P, w.d, eb, w.dtype == "bf16")
                     tot += accounting.merge_bytes(n, n - R, w.d, eb)
         return tot * w.layers
 

@@ -67,8 +67,11 @@ def test_prefill_chunk_accounting():
     assert rounds == 1
     row = 2 * 128 * 2
     want = (512 * (2 * row + 4)                                           # append
-            + 2560 * (256 + 4) + 2560 * (row + 8) + 2560 * (row + 4) + 1248 * 8  # scoring
+            + 2560 * (row + 4) + 2 * 1248 * (row + 4) + 1248 * 8         # the two window passes
             + (2560 - 32) * (row + 4) + (2048 - 32) * (row + 4))           # in-place merge
     assert b == want
+    # the CUDA-core path of fp32 caches reads K once more for the window mass
+    bf, _ = accounting.prefill_chunk_bytes(2048, 512, 2048, 32, 32, 128, 2, fused=False)
+    assert bf - b == 2560 * (256 + 4 + 4)
     # under the budget: the append only
     assert accounting.prefill_chunk_bytes(0, 512, 2048, 32, 32, 128, 2) == (512 * (2 * row + 4), 0)

@@ -173,7 +173,7 @@ struct FaShape {
   static constexpr int kBox = 128 * 128;                 // 128 rows x 128 bytes
   static constexpr int kTile = kBoxes * kBox;            // a Q, K or V tile
   static constexpr int kStages = D == 128 ? 3 : 4;
-  static constexpr int kLnSlot = kFuKeys * 4;            // log-counts of a tile (bytes)
+  static constexpr int kLnSlot = kFuKeys * 4 + 16;       // log-counts of a tile + their maximum
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kQOff + kTile;
   static constexpr int kVOff = kKOff + kStages * kTile;
@@ -320,6 +320,15 @@ window_fa_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                       k_row0 + i * kFuKeys, &v_full[s]);
       }
       *reinterpret_cast<float4*>(base + S::kLnOff + s * S::kLnSlot + 16 * lane) = ln_next;
+      {
+        // the tile's largest log-count (entries past the split read as 0 <= every
+        // log-count): with the row maximum of S it bounds the tile's logits from above
+        float lm = fmaxf(fmaxf(ln_next.x, ln_next.y), fmaxf(ln_next.z, ln_next.w));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) lm = fmaxf(lm, __shfl_xor_sync(0xffffffffu, lm, o));
+        if (lane == 0)
+          *reinterpret_cast<float*>(base + S::kLnOff + s * S::kLnSlot + kFuKeys * 4) = lm;
+      }
       mbar_arrive(&v_full[s]);
       ln_next = ln4(i + 1);
       issued_v = i + 1;
@@ -447,18 +456,19 @@ window_fa_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       // P = 2^(x - m) as bf16 hi and lo parts over the chunk's own S columns, computed in
       // place over the chunk's logits: pair j/2 leaves hi in w[j] and lo in w[j + 1]
       auto exps = [&](uint32_t (&w)[32], int c, float m, float& lsum) {
-        float ps[2] = {0.f, 0.f};
+        float2 ps = make_float2(0.f, 0.f);
 #pragma unroll
         for (int j = 0; j < 32; j += 2) {
           const float pa = m > -INFINITY ? ex2_ftz(__uint_as_float(w[j]) - m) : 0.f;
           const float pb = m > -INFINITY ? ex2_ftz(__uint_as_float(w[j + 1]) - m) : 0.f;
-          ps[0] += pa;
-          ps[1] += pb;
+          const float2 p2 = make_float2(pa, pb);
+          ps = fadd2(ps, p2);
           const uint32_t hh = pack_bf16x2(pa, pb);
+          const float2 r2 = ffma2(make_float2(bf16_lo(hh), bf16_hi(hh)), make_float2(-1.f, -1.f), p2);
           w[j] = hh;
-          w[j + 1] = pack_bf16x2(pa - bf16_lo(hh), pb - bf16_hi(hh));
+          w[j + 1] = pack_bf16x2(r2.x, r2.y);
         }
-        lsum += ps[0] + ps[1];
+        lsum += ps.x + ps.y;
         tmem_st16_pairs<0>(s_cols + 32 * c, w);
         tmem_st16_pairs<1>(s_cols + 32 * c + 16, w);
       };
@@ -469,19 +479,24 @@ window_fa_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         tc_fence_after();
         // sweep 1: the tile's row maximum (one chunk of S in registers at a time: a whole
         // row does not fit beside the rest without spilling)
+        // On a tile without masked keys an upper bound serves as well as the maximum (the
+        // reference only has to be at least every logit): the row maximum of the raw S
+        // times the scale, plus the tile's largest log-count, costs one max per element.
         float mt = -INFINITY;
+        const bool bound = interior;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t w[32];
           tmem_ld32_async(s_cols + 32 * c, w);
           tmem_ld_wait(w);
-          logits(w, c);
+          if (!bound) logits(w, c);
           float m4[4] = {__uint_as_float(w[0]), __uint_as_float(w[1]), __uint_as_float(w[2]),
                          __uint_as_float(w[3])};
 #pragma unroll
           for (int j = 4; j < 32; ++j) m4[j & 3] = fmaxf(m4[j & 3], __uint_as_float(w[j]));
           mt = fmaxf(mt, fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])));
         }
+        if (bound) mt = fmaf(mt, qscale, lnb[kFuKeys]);
         // the reference maximum moves only when the tile exceeds it by 2^8; O_g, which the
         // group's previous P V MMAs update, is then rescaled
         m_new = (mt > m_ref + kRescaleSlack) ? mt : m_ref;

@@ -1089,12 +1089,15 @@ window_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         ln_next = kn < 2 * P ? lnh[c0 + kn] : 0.f;
       }
       const int hide = t - (L - W);               // queries with q mod W < hide miss the key
-      // The tile's S^T first: its MMA was issued only after the stage's rows had landed,
-      // so once s_full completes the stage holds this tile, and the wait on `full` that
-      // follows can only match this tile's phase. (Waiting on `full` first could match the
-      // stage's previous phase: with an odd stage count consecutive uses of a stage go to
-      // different groups, and this group need not have seen the other's tile land.)
-      live = live && mbar_wait_ab(&s_full[g], k & 1, s_abort);
+      // With an even stage count every use of a stage is this group's (tiles i, i + ST,
+      // ... have i's parity), so the group has seen the stage's previous phase and may wait
+      // on `full` first: the row terms below then overlap the tile's S^T MMA. With an odd
+      // count consecutive uses of a stage go to different groups and a parity wait on
+      // `full` could match the previous phase, so the group waits for its S^T first (the
+      // MMA was issued only after the stage's rows had landed, so the stage then holds
+      // this tile and the wait on `full` can only match this tile's phase).
+      constexpr bool kOwnStages = (ST % 2) == 0;
+      if (!kOwnStages) live = live && mbar_wait_ab(&s_full[g], k & 1, s_abort);
       live = live && mbar_wait_ab(&full[s], (i / ST) & 1, s_abort);
       live = __all_sync(0xffffffffu, live);
       // the pair's row terms from the stage: |k_b - k_a|^2, |v_a - o_bar|^2,
@@ -1148,6 +1151,7 @@ window_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         nb += __shfl_xor_sync(0xffffffffu, nb, 1);
       }
       // window probabilities p_qt = 2^(s q.k + lnt - Z_q), the key's row of S^T
+      if (kOwnStages) live = live && mbar_wait_ab(&s_full[g], k & 1, s_abort);
       if (PERQ) live = live && mbar_wait_ab(&u_full[g], k & 1, s_abort);
       live = __all_sync(0xffffffffu, live);
       // the stage's rows are read, here and by the tile's MMAs (done: S^T, U landed)

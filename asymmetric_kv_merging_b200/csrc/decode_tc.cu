@@ -36,6 +36,10 @@
 namespace kvs {
 
 
+// Lazy reference of the decode's online softmax: it moves when a logit exceeds it by this
+// much (log2 units), so probabilities stay <= 2^8 between moves.
+constexpr float kDecodeSlack = 8.f;
+
 template <int D, int NC, int STAGES, int EXTRA>
 struct TcShape {
   static constexpr int kTile = 16 * NC;                    // cache rows per stage
@@ -254,23 +258,39 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
         const float x1 = v0 ? fmaf(sa[1] + sb[1], qscale, ln_cur.x * kLog2e) : -INFINITY;
         const float x2 = v1 ? fmaf(sa[2] + sb[2], qscale, ln_cur.y * kLog2e) : -INFINITY;
         const float x3 = v1 ? fmaf(sa[3] + sb[3], qscale, ln_cur.y * kLog2e) : -INFINITY;
-        // column maxima over the 16 rows: the 8 lanes sharing tig
-        float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+        // The reference maximum of a column moves only when a logit exceeds it by 2^8
+        // (so P <= 2^8 between moves); the column maxima over the 16 rows (the 8 lanes
+        // sharing tig) and the rescale of l and O are taken only when some lane's logit
+        // does, which after the first stages is rare.
+        const bool up = x0 > m0 + kDecodeSlack || x2 > m0 + kDecodeSlack ||
+                        x1 > m1 + kDecodeSlack || x3 > m1 + kDecodeSlack;
+        if (__any_sync(0xffffffffu, up)) {
+          float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
 #pragma unroll
-        for (int off = 4; off < 32; off <<= 1) {
-          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+          for (int off = 4; off < 32; off <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+          }
+          const float mn0 = mx0 > m0 + kDecodeSlack ? mx0 : m0;
+          const float mn1 = mx1 > m1 + kDecodeSlack ? mx1 : m1;
+          // factors of the old reference (0 when there was none: l and O are still 0)
+          const float c0 = mn0 == m0 ? 1.f : ex2_ftz(m0 - mn0);
+          const float c1 = mn1 == m1 ? 1.f : ex2_ftz(m1 - mn1);
+          l0 *= c0;
+          l1 *= c1;
+#pragma unroll
+          for (int j = 0; j < D / 16; ++j) {
+            O[j][0] *= c0; O[j][1] *= c1; O[j][2] *= c0; O[j][3] *= c1;
+          }
+          m0 = mn0;
+          m1 = mn1;
         }
-        const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-        const float b0 = mn0 == -INFINITY ? 0.f : mn0;     // all -inf so far: keep zeros
-        const float b1 = mn1 == -INFINITY ? 0.f : mn1;
-        const float c0 = exp2f(m0 - b0), c1 = exp2f(m1 - b1);
-        const float p0 = exp2f(x0 - b0), p1 = exp2f(x1 - b1);
-        const float p2 = exp2f(x2 - b0), p3 = exp2f(x3 - b1);
-        l0 = fmaf(l0, c0, p0 + p2);
-        l1 = fmaf(l1, c1, p1 + p3);
-        m0 = mn0;
-        m1 = mn1;
+        const float b0 = m0 == -INFINITY ? 0.f : m0;       // all -inf so far: keep zeros
+        const float b1 = m1 == -INFINITY ? 0.f : m1;
+        const float p0 = ex2_ftz(x0 - b0), p1 = ex2_ftz(x1 - b1);
+        const float p2 = ex2_ftz(x2 - b0), p3 = ex2_ftz(x3 - b1);
+        l0 += p0 + p2;
+        l1 += p1 + p3;
         // P^T as the B operand: transpose the two 8x8 bf16 blocks (rows 0-7, 8-15)
         const uint32_t pb0 = movmatrix_trans(pack_bf16x2(p0, p1));
         const uint32_t pb1 = movmatrix_trans(pack_bf16x2(p2, p3));
@@ -280,7 +300,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
           const int el = j * 16 + ((mi & 1) << 3);
           uint32_t a0, a1, a2, a3;
           ldsm_x4_trans(vb + (el >> 6) * S::kBoxBytes + swz128(row, (el & 63) >> 3), a0, a1, a2, a3);
-          O[j][0] *= c0; O[j][1] *= c1; O[j][2] *= c0; O[j][3] *= c1;
           mma_bf16_16816(O[j], a0, a1, a2, a3, pb0, pb1);
         }
       }

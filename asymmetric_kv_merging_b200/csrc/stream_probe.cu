@@ -1,8 +1,9 @@
 // Measurement helper, not part of the method: the device-memory read ceiling of the
 // decode step's access pattern. One thread per CTA streams consecutive 128-row boxes of
-// a [rows, d] bf16 array through a 3-stage shared-memory ring with 2D TMA loads (128-byte
-// swizzle, L2 evict-first), exactly as the decode kernel feeds its K and V rows, and a
-// consumer warp only waits for each stage and releases it. Timing it over as many bytes
+// a [rows, d] bf16 array through a shared-memory ring with 2D TMA loads (128-byte
+// swizzle, L2 evict-first), as the decode kernel feeds its K and V rows, with as many
+// bytes in flight as the decode's ring holds (six 32 KB stages = its three stages of K and
+// V), and a consumer warp only waits for each stage and releases it. Timing it over as many bytes
 // as one decode step reads, on as many SMs as the decode launch uses, gives the time the
 // decode kernel would take if its MMAs, softmax and combine were free.
 #include <cudaTypedefs.h>
@@ -14,7 +15,7 @@
 namespace kvs {
 
 constexpr int kProbeRows = 128;
-constexpr int kProbeStages = 3;
+constexpr int kProbeStages = 6;
 
 template <int D>
 __global__ void __launch_bounds__(64, 1)
@@ -82,7 +83,8 @@ cudaError_t launch_stream_probe(const void* buf, long long rows, int d, int ctas
     return cudaErrorInvalidValue;
   CUtensorMap m;
   if (!encode_rows_map(&m, buf, (unsigned long long)rows, d, kProbeRows)) return cudaErrorInvalidValue;
-  const size_t smem = (size_t)kProbeStages * (d / 64) * kProbeRows * 128 + 64 + 1024;
+  // the ring, then the full / empty barriers (2 x kProbeStages x 8 bytes), 1024-byte alignment
+  const size_t smem = (size_t)kProbeStages * (d / 64) * kProbeRows * 128 + 256 + 1024;
   const void* fn = d == 128 ? (const void*)stream_probe_kernel<128> : (const void*)stream_probe_kernel<64>;
   if (!ensure_smem_attr(fn, smem)) return cudaErrorInvalidValue;
   if (d == 128)

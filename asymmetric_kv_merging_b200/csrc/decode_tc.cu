@@ -233,6 +233,18 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
           fence_proxy_async_smem();
           __syncwarp();
         }
+        // The warp's V fragments (A operands of O^T += V^T P^T) first, kept in registers,
+        // then its K fragments straight into the S^T MMAs, and the stage's log-counts: the
+        // warp is then done with the stage's shared memory and releases it before its
+        // softmax and P V MMAs, so the producer refills it while they run.
+        uint32_t vf[D / 16][4];
+#pragma unroll
+        for (int j = 0; j < D / 16; ++j) {
+          const int row = r0 + ((mi >> 1) << 3) + ri;
+          const int el = j * 16 + ((mi & 1) << 3);
+          ldsm_x4_trans(vb + (el >> 6) * S::kBoxBytes + swz128(row, (el & 63) >> 3), vf[j][0],
+                        vf[j][1], vf[j][2], vf[j][3]);
+        }
         // S^T (16 rows x 8 columns): A = the K rows, two accumulators to halve the chain
         float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -252,7 +264,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
           const float* lns = reinterpret_cast<const float*>(ln_ring + s * S::kLnSlot) + ln_off + r0;
           ln_cur = make_float2(lns[grp], lns[grp + 8]);
         }
-        // this lane: rows grp (x0: n0, x1: n1) and grp + 8 (x2: n0, x3: n1)
+        // every shared-memory read of the stage is issued (the arrive orders them before it)
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
         const bool v0 = grp < nval, v1 = grp + 8 < nval;
         const float x0 = v0 ? fmaf(sa[0] + sb[0], qscale, ln_cur.x * kLog2e) : -INFINITY;
         const float x1 = v0 ? fmaf(sa[1] + sb[1], qscale, ln_cur.x * kLog2e) : -INFINITY;
@@ -295,16 +309,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
         const uint32_t pb0 = movmatrix_trans(pack_bf16x2(p0, p1));
         const uint32_t pb1 = movmatrix_trans(pack_bf16x2(p2, p3));
 #pragma unroll
-        for (int j = 0; j < D / 16; ++j) {
-          const int row = r0 + ((mi >> 1) << 3) + ri;
-          const int el = j * 16 + ((mi & 1) << 3);
-          uint32_t a0, a1, a2, a3;
-          ldsm_x4_trans(vb + (el >> 6) * S::kBoxBytes + swz128(row, (el & 63) >> 3), a0, a1, a2, a3);
-          mma_bf16_16816(O[j], a0, a1, a2, a3, pb0, pb1);
-        }
+        for (int j = 0; j < D / 16; ++j) mma_bf16_16816(O[j], vf[j][0], vf[j][1], vf[j][2], vf[j][3], pb0, pb1);
+      } else {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);   // no rows of this warp in the stage
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
     }
     // the lanes sharing tig hold disjoint rows' shares of the column sums
 #pragma unroll

@@ -98,6 +98,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
 
   const int head = blockIdx.y, split = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == NC * 32) {   // the producer: descriptor fetches overlap the length load
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+    if (logn != nullptr) prefetch_tmap(&tmL);
+  }
   int L = len[head];
   const bool bad = L < 0 || L > T_cap;
   if (bad) {
@@ -132,13 +137,36 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
       s_kvnew[i / D][i % D] = (i < D ? k_new : v_new)[(size_t)head * D + i % D];
   }
   const bool append = want_append && !bad;
-  if (tid == 0) {
+  // One thread issues every TMA load of the ring: stage i % STAGES takes the K and V rows
+  // of tile i (and its log-counts) and signals full[s] when they have landed.
+  const bool producer = tid == NC * 32;
+  const uint64_t once = policy_evict_first();   // K and V are read once per step
+  auto issue = [&](int i) {
+    const int s = i % STAGES;
+    unsigned char* st = base + s * S::kStageBytes;
+    mbar_arrive_expect_tx(&full[s], S::kStageBytes + (has_ln ? S::kLnBox * 4 : 0));
+    if (has_ln)
+      tma_load_1d_hint(ln_ring + s * S::kLnSlot, &tmL, ln_lead + row0 + i * kTile - ln_off,
+                       &full[s], once);
+#pragma unroll
+    for (int bx = 0; bx < S::kBoxes; ++bx) {
+      tma_load_2d_hint(st + bx * S::kBoxBytes, &tmK, bx * 64, row0 + i * kTile, &full[s], once);
+      tma_load_2d_hint(st + S::kTileBytes + bx * S::kBoxBytes, &tmV, bx * 64, row0 + i * kTile,
+                       &full[s], once);
+    }
+  };
+  // The producer sets up the barriers and fills the ring as soon as the length is known,
+  // without waiting for the query and appended-row loads that the CTA barrier below waits
+  // for: the first stages are in flight while those loads complete.
+  int issued = 0;
+  if (producer) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], NC);
     }
     mbar_init(cbar, 1);
     fence_mbar_init();
+    for (; issued < STAGES && issued < ntiles; ++issued) issue(issued);
   }
   __syncthreads();
 
@@ -160,29 +188,14 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
   } else if (warp == NC) {
     // ---------------- producer: one thread issues every TMA load ----------------
     if (lane == 0) {
-      prefetch_tmap(&tmK);
-      prefetch_tmap(&tmV);
-      if (has_ln) prefetch_tmap(&tmL);
-      const uint64_t once = policy_evict_first();   // K and V are read once per step
-      int issued = 0;
-      for (int i = 0; i < ntiles; ++i) {
+      // the first STAGES tiles went out before the CTA barrier; the rest wait for a free stage
+      for (int i = issued; i < ntiles; ++i) {
         const int s = i % STAGES;
-        if (i >= STAGES && !mbar_wait(&empty[s], ((i / STAGES) - 1) & 1)) {
+        if (!mbar_wait(&empty[s], ((i / STAGES) - 1) & 1)) {
           set_flag(flags, KVS_FLAG_TIMEOUT);
           break;
         }
-        unsigned char* st = base + s * S::kStageBytes;
-        mbar_arrive_expect_tx(&full[s], S::kStageBytes + (has_ln ? S::kLnBox * 4 : 0));
-        if (has_ln)
-          tma_load_1d_hint(ln_ring + s * S::kLnSlot, &tmL, ln_lead + row0 + i * kTile - ln_off,
-                           &full[s], once);
-#pragma unroll
-        for (int bx = 0; bx < S::kBoxes; ++bx) {
-          tma_load_2d_hint(st + bx * S::kBoxBytes, &tmK, bx * 64, row0 + i * kTile, &full[s],
-                           once);
-          tma_load_2d_hint(st + S::kTileBytes + bx * S::kBoxBytes, &tmV, bx * 64,
-                           row0 + i * kTile, &full[s], once);
-        }
+        issue(i);
         issued = i + 1;
       }
       // the last load issued into each stage must land before the buffers are reused

@@ -291,105 +291,166 @@ __device__ __forceinline__ void decode_epilogue_staged(const DecodeSmem<D, G, NW
 // the ring), because peers may push while this CTA is still streaming.
 template <int D, int G>
 struct __align__(16) ClusterInbox {
-  float acc[G * D + kMaxClusterSize];                   // [C][G*D/C + 1]
+  float acc[G * D + 4 * kMaxClusterSize];               // [C][G*D/(4C) + 1] 4-column units
   float ml[kMaxClusterSize][G][2];                      // [C][G] (m, l)
 };
 
-// Output slice of rank r among C CTAs: columns [G*D*r/C, G*D*(r+1)/C).
+// Output slice of rank r among C CTAs: units [n*r/C, n*(r+1)/C) of n.
 __device__ __forceinline__ int slice_lo(int n, int r, int C) { return (int)((unsigned)n * r / C); }
 __device__ __forceinline__ int slice_owner(int n, int col, int C) {
   return (int)(((unsigned)(col + 1) * C - 1) / n);
 }
+// Bytes that land in the inbox of rank r: every CTA's units of r's slice, and every
+// CTA's (m, l) per query head.
+template <int G>
+__device__ __forceinline__ uint32_t inbox_bytes(int n, int C, int r) {
+  return (uint32_t)(C * (slice_lo(n, r + 1, C) - slice_lo(n, r, C)) * 16 + C * G * 8);
+}
+// Bytes the dry run pushes into its own scratch inbox: all n units and C copies of (m, l).
+template <int G>
+__device__ __forceinline__ uint32_t dry_inbox_bytes(int n, int C) {
+  return (uint32_t)(n * 16 + C * G * 8);
+}
 
 // Cluster combine of a decode step in which the C CTAs of a cluster are all the splits
 // of one KV head: no global partials, no arrival counter, no last CTA. Every CTA
-// merges its warp partials and pushes each column to the CTA owning that column's
-// output slice (distributed shared-memory stores into the owner's inbox), and its
-// (m, l) to every CTA; after one cluster barrier each CTA combines its slice from its
-// own inbox, and the CTA of rank 0 appends the new row. Nothing is read remotely, so
-// a CTA may leave as soon as its slice is written.
+// merges its warp partials, four output columns per thread, and pushes each 4-column
+// unit to the CTA owning that unit's output slice, and its (m, l) to every CTA, with
+// asynchronous distributed shared-memory stores that count their bytes on the
+// receiver's inbox barrier. Each CTA combines its slice as soon as its own inbox
+// barrier says every push into it has landed (no cluster-wide barrier on that path), and
+// the CTA of rank 0 appends the new row. The cluster barrier's arrive follows the pushes
+// and its wait ends the function, so no CTA leaves while a push into it may still be in
+// flight. The loop over warps is unrolled, so that its shared-memory loads and
+// exponentials overlap; the slice takes one lane per source CTA and unit.
 //
-// kn, vn: the appended row of this head (nullable when !append); the caller stages it
-// in shared memory at kernel start, so the combine waits on no global load.
+// Protocol with the caller: every CTA initialises `inbar` (count 1) at kernel start and
+// arrives on it once with expect_tx = inbox_bytes<G>(NU, C, rank), then every thread
+// arrives (relaxed, after the barrier-init fence) on the cluster barrier; the combine
+// begins with the matching wait.
+// s_new: the appended row's logit per query head (read when append && L < T_cap);
+// vn: its value row, staged in shared memory at kernel start (nullable when !append).
 // `dry`: run the same instructions with every store aimed at this CTA's scratch
-// (`inbox` and `out` point there, head is 0) and without barriers or the append,
-// from a single warp while the other warps stream (its loads of the warp partials see
-// stage data in flight; the values are discarded). A kernel launch starts with cold
-// instruction caches; the dry run pulls this code in before the real combine needs it.
+// (`inbox`, `inbar` and `out` point there, head is 0) and without the barriers, the
+// inbox wait or the append, from a single warp while the other warps stream (its loads
+// of the warp partials see stage data in flight; the values are discarded). A kernel
+// launch starts with cold instruction caches; the dry run pulls this code in before the
+// real combine needs it. The scratch barrier expects dry_inbox_bytes<G>(NU, C).
 template <typename T, int D, int G, int NW>
 __device__ __noinline__ void cluster_combine(
-    float (*sm)[G], float (*sl)[G], float (*sacc)[G][D], float (*qs)[D], float* s_cml,
-    float* s_new, ClusterInbox<D, G>* inbox, int C, int rank, int tid, int nthreads, bool dry,
-    int head, int L, int T_cap, bool append, T* K, T* V, float* logn, int32_t* len,
-    const T* kn, const T* vn, T* out, int32_t* flags) {
-  constexpr int N = G * D;
-  const int lane = tid & 31, warp = tid >> 5, nwarps = nthreads / 32;
+    float (*sm)[G], float (*sl)[G], float (*sacc)[G][D], const float* s_new,
+    ClusterInbox<D, G>* inbox, uint64_t* inbar, int C, int rank, int tid, int nthreads, bool dry,
+    int head, int L, int T_cap, bool append, T* K, T* V, float* logn, int32_t* len, const T* kn,
+    const T* vn, T* out, int32_t* flags) {
+  constexpr int NU = G * D / 4;                        // 4-column output units
   const bool fits = L < T_cap;
   const bool attend_new = append && fits;
-  const int slice_w = N / C + 1;                       // inbox row stride (>= any slice)
-  // this CTA's (m, l) per query head
-  for (int g = tid; g < G; g += nthreads) {
+  const int slice_w = NU / C + 1;                      // inbox row stride in units (>= any slice)
+  const uint32_t in_acc = smem_u32(inbox->acc), in_ml = smem_u32(&inbox->ml[0][0][0]);
+  const uint32_t in_bar = smem_u32(inbar);
+  if (!dry) cluster_wait();                            // every CTA's inbox barrier is set up
+  // merge the warps unit by unit and push each unit to its owner
+  for (int u = tid; u < NU; u += nthreads) {
+    const int g = (u * 4) / D, c = u * 4 - g * D;
+    float mw[NW];
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < NW; ++w) M = fmaxf(M, sm[w][g]);
+    for (int w = 0; w < NW; ++w) {
+      mw[w] = sm[w][g];
+      M = fmaxf(M, mw[w]);
+    }
+    float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (M > -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < NW; ++w) {
+        const float f = exp2f(mw[w] - M);
+        const float4 v = *reinterpret_cast<const float4*>(&sacc[w][g][c]);
+        A.x = fmaf(v.x, f, A.x); A.y = fmaf(v.y, f, A.y);
+        A.z = fmaf(v.z, f, A.z); A.w = fmaf(v.w, f, A.w);
+      }
+    }
+    const int owner = slice_owner(NU, u, C);
+    const int at = rank * slice_w + (u - slice_lo(NU, owner, C));
+    const uint32_t dst = dry ? rank : owner;
+    st_async_f32x4(cluster_map(in_acc + (uint32_t)at * 16u, dst), A, cluster_map(in_bar, dst));
+  }
+  // push (m, l) of every query head to every CTA: ml[rank][g] in CTA j (the threads past
+  // the unit loop's last take these first)
+  const int k0 = (tid + nthreads - NU % nthreads) % nthreads;
+  for (int k = k0; k < C * G; k += nthreads) {
+    const int j = k / G, g = k - j * G;
+    float mw[NW];
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      mw[w] = sm[w][g];
+      M = fmaxf(M, mw[w]);
+    }
     float Ls = 0.f;
     if (M > -INFINITY) {
 #pragma unroll
-      for (int w = 0; w < NW; ++w) Ls = fmaf(sl[w][g], exp2f(sm[w][g] - M), Ls);
+      for (int w = 0; w < NW; ++w) Ls = fmaf(sl[w][g], exp2f(mw[w] - M), Ls);
     }
-    s_cml[2 * g] = M;
-    s_cml[2 * g + 1] = Ls;
+    const uint32_t dst = dry ? rank : j;
+    st_async_f32x2(cluster_map(in_ml + (uint32_t)((rank * G + g) * 2) * 4u, dst), M, Ls,
+                   cluster_map(in_bar, dst));
   }
-  if (attend_new) appended_logits<T, D, G, NW>(DecodeSmem<D, G, NW>{sm, sl, sacc, qs, s_new, nullptr, nullptr, nullptr},
-                                               kn, warp, lane, nwarps);
-  if (!dry) __syncthreads();
-  const uint32_t in_acc = smem_u32(inbox->acc), in_ml = smem_u32(&inbox->ml[0][0][0]);
-  // push (m, l) of every query head to every CTA: ml[rank][g] in CTA j
-  for (int k = tid; k < C * G; k += nthreads) {
-    const int j = k / G, g = k - j * G;
-    const uint32_t dst = cluster_map(in_ml + (uint32_t)((rank * G + g) * 2) * 4u, dry ? rank : j);
-    st_cluster_f32x2(dst, s_cml[2 * g], s_cml[2 * g + 1]);
-  }
-  // merge the warps column by column and push each column to its owner
-  for (int i = tid; i < N; i += nthreads) {
-    const int g = i / D, c = i - g * D;
-    const float M = s_cml[2 * g];
-    float A = 0.f;
-    if (M > -INFINITY) {
-#pragma unroll
-      for (int w = 0; w < NW; ++w) A = fmaf(sacc[w][g][c], exp2f(sm[w][g] - M), A);
+  if (!dry) cluster_arrive();                          // this CTA's pushes; the wait is at the end
+  // combine this CTA's slice from its inbox, once every push into it has landed: 16
+  // lanes per unit, lane j of a half-warp taking source CTA j (C <= 16), max and sums
+  // by shuffles within the half-warp; whole warps take part, so that the shuffles are
+  // warp-uniform
+  const int lo = slice_lo(NU, rank, C), hi = slice_lo(NU, rank + 1, C);
+  const int nunits = hi - lo, warp = tid >> 5, nwarps = nthreads >> 5;
+  // (thread 0 waits whatever its share, so the CTA outlives every push into it)
+  if (!dry && (tid == 0 || 2 * warp < nunits) && !mbar_wait(inbar, 0))
+    set_flag(flags, KVS_FLAG_TIMEOUT);
+  const int j = tid & 15;
+  for (int b0 = 2 * warp; b0 < nunits; b0 += 2 * nwarps) {
+    const int b = b0 + ((tid >> 4) & 1);
+    const bool act = b < nunits;
+    const int u = lo + (act ? b : 0);
+    const int g = (u * 4) / D, c = u * 4 - g * D;
+    float m = -INFINITY, l = 0.f;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (act && j < C) {
+      const float2 ml = *reinterpret_cast<const float2*>(&inbox->ml[j][g][0]);
+      v = *reinterpret_cast<const float4*>(&inbox->acc[(j * slice_w + b) * 4]);
+      if (ml.y > 0.f) {
+        m = ml.x;
+        l = ml.y;
+      }
     }
-    const int owner = slice_owner(N, i, C);
-    const int at = rank * slice_w + (i - slice_lo(N, owner, C));
-    st_cluster_f32(cluster_map(in_acc + (uint32_t)at * 4u, dry ? rank : owner), A);
-  }
-  if (!dry) {
-    cluster_arrive();
-    cluster_wait();                                    // every push to this CTA landed
-  }
-  // combine this CTA's slice from its inbox
-  const int lo = slice_lo(N, rank, C), hi = slice_lo(N, rank + 1, C);
-  for (int col = lo + tid; col < hi; col += nthreads) {
-    const int g = col / D, c = col - g * D;
     const float sn = attend_new ? s_new[g] : -INFINITY;
-    float M = sn;
-    for (int j = 0; j < C; ++j)
-      if (inbox->ml[j][g][1] > 0.f) M = fmaxf(M, inbox->ml[j][g][0]);
-    float Ls = 0.f, A = 0.f;
-    if (M > -INFINITY) {
-      for (int j = 0; j < C; ++j) {
-        const float lj = inbox->ml[j][g][1];
-        const float f = lj > 0.f ? exp2f(inbox->ml[j][g][0] - M) : 0.f;
-        Ls = fmaf(lj, f, Ls);
-        A = fmaf(inbox->acc[j * slice_w + (col - lo)], f, A);
-      }
-      if (attend_new) {
-        const float f = exp2f(sn - M);
-        Ls += f;
-        A = fmaf(to_f32(vn[c]), f, A);
-      }
+    float M = fmaxf(m, sn);
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    const float f = (l > 0.f && M > -INFINITY) ? exp2f(m - M) : 0.f;
+    float Ls = l * f;
+    float4 A = make_float4(v.x * f, v.y * f, v.z * f, v.w * f);
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) {
+      Ls += __shfl_xor_sync(0xffffffffu, Ls, off);
+      A.x += __shfl_xor_sync(0xffffffffu, A.x, off);
+      A.y += __shfl_xor_sync(0xffffffffu, A.y, off);
+      A.z += __shfl_xor_sync(0xffffffffu, A.z, off);
+      A.w += __shfl_xor_sync(0xffffffffu, A.w, off);
     }
-    store_out<T>(out + ((size_t)head * G + g) * D + c, Ls > 0.f ? A / Ls : 0.f);
+    if (act && j == 0) {
+      if (attend_new && M > -INFINITY) {
+        const float fn = exp2f(sn - M);
+        Ls += fn;
+        A.x = fmaf(to_f32(vn[c]), fn, A.x);
+        A.y = fmaf(to_f32(vn[c + 1]), fn, A.y);
+        A.z = fmaf(to_f32(vn[c + 2]), fn, A.z);
+        A.w = fmaf(to_f32(vn[c + 3]), fn, A.w);
+      }
+      T* o = out + ((size_t)head * G + g) * D + c;
+      store_out<T>(o, Ls > 0.f ? A.x / Ls : 0.f);
+      store_out<T>(o + 1, Ls > 0.f ? A.y / Ls : 0.f);
+      store_out<T>(o + 2, Ls > 0.f ? A.z / Ls : 0.f);
+      store_out<T>(o + 3, Ls > 0.f ? A.w / Ls : 0.f);
+    }
   }
   if (!dry && rank == 0 && append) {
     if (fits) {
@@ -403,6 +464,7 @@ __device__ __noinline__ void cluster_combine(
       set_flag(flags, KVS_FLAG_OUT_CAPACITY);
     }
   }
+  if (!dry) cluster_wait();                            // every push of the cluster has landed
 }
 
 }  // namespace kvs

@@ -86,13 +86,13 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
   __shared__ float s_new[G];
   __shared__ float s_fac[G][kMaxDecodeSplits];
   __shared__ float s_gstat[G][2];
-  __shared__ float s_cml[G][2];
   __shared__ int s_last;
   // cluster shape: the inbox peers push into, the scratch of the warm-up run, and the
   // appended row (k, v) staged at kernel start
   using Inbox = std::conditional_t<kCluster, ClusterInbox<D, G>, char>;
   __shared__ Inbox s_inbox[2];
   __shared__ __align__(16) bf16 s_kvnew[kCluster ? 2 : 1][kCluster ? D : 8];
+  __shared__ uint64_t s_inbar[2];   // cluster shape: the inbox's barrier, the scratch inbox's
   // after the main loop the stage buffers hold the consumer warps' partial outputs
   float(*s_acc)[G][D] = reinterpret_cast<float(*)[G][D]>(base);
 
@@ -102,6 +102,39 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
     if (logn != nullptr) prefetch_tmap(&tmL);
+  }
+  // Every global load of the prologue goes out before the length comes back: this
+  // thread's share of the query (staged in shared memory below), the appended row (the
+  // cluster shape stages it whatever the length turns out to be; `append` gates its
+  // use) and, in the consumer warps, the query fragments of the S^T MMAs.
+  constexpr int kQPer = (G * D + kThreads - 1) / kThreads;
+  float qv[kQPer];
+#pragma unroll
+  for (int r = 0; r < kQPer; ++r) {
+    const int i = tid + r * kThreads;
+    qv[r] = i < G * D ? to_f32(q[(size_t)head * G * D + i]) : 0.f;
+  }
+  const bool want_append = k_new != nullptr && v_new != nullptr;
+  static_assert(!kCluster || 2 * D <= kThreads, "one appended element per thread");
+  bf16 kvv = __float2bfloat16_rn(0.f);
+  // element loads: the API does not require these rows to be 16-byte aligned
+  if (kCluster && want_append && tid < 2 * D)
+    kvv = (tid < D ? k_new : v_new)[(size_t)head * D + tid % D];
+  // B operand of S^T = K Q^T in consumer lane (grp, tig): column n = grp holds query
+  // head grp (zero past G)
+  uint32_t qb[D / 16][2];
+  {
+    const int grp = lane >> 2, tig = lane & 3;
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+      if (warp < NC && grp < G) {
+        const bf16* qr = q + ((size_t)head * G + grp) * D + ks * 16 + tig * 2;
+        qb[ks][0] = *reinterpret_cast<const uint32_t*>(qr);
+        qb[ks][1] = *reinterpret_cast<const uint32_t*>(qr + 8);
+      } else {
+        qb[ks][0] = qb[ks][1] = 0u;
+      }
+    }
   }
   int L = len[head];
   const bool bad = L < 0 || L > T_cap;
@@ -122,20 +155,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
   const bool has_ln = logn != nullptr;
   const int ln_off = (ln_lead + row0) & 3;
 
-  const float qscale = kLog2e / sqrtf((float)D);
-  for (int i = tid; i < G * D; i += kThreads) {
-    const int g = i / D, c = i - g * D;
-    qs[g][c] = to_f32(q[((size_t)head * G + g) * D + c]) * qscale;
-  }
-  // the appended row is staged whatever the length turns out to be, so that its loads
-  // go out with the length's and the query's (one round trip before the stream starts,
-  // not two); `append` then gates its use
-  const bool want_append = k_new != nullptr && v_new != nullptr;
-  if (kCluster && want_append) {
-    // element loads: the API does not require these rows to be 16-byte aligned
-    for (int i = tid; i < 2 * D; i += kThreads)
-      s_kvnew[i / D][i % D] = (i < D ? k_new : v_new)[(size_t)head * D + i % D];
-  }
   const bool append = want_append && !bad;
   // One thread issues every TMA load of the ring: stage i % STAGES takes the K and V rows
   // of tile i (and its log-counts) and signals full[s] when they have landed.
@@ -156,8 +175,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     }
   };
   // The producer sets up the barriers and fills the ring as soon as the length is known,
-  // without waiting for the query and appended-row loads that the CTA barrier below waits
-  // for: the first stages are in flight while those loads complete.
+  // before it takes its share of the query and appended-row staging that the CTA barrier
+  // below waits for: the first stages are in flight while those loads complete.
   int issued = 0;
   if (producer) {
     for (int s = 0; s < STAGES; ++s) {
@@ -165,10 +184,29 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
       mbar_init(&empty[s], NC);
     }
     mbar_init(cbar, 1);
+    if constexpr (kCluster) {
+      mbar_init(&s_inbar[0], 1);
+      mbar_init(&s_inbar[1], 1);
+    }
     fence_mbar_init();
     for (; issued < STAGES && issued < ntiles; ++issued) issue(issued);
+    if constexpr (kCluster) {
+      constexpr int NU = G * D / 4;
+      mbar_arrive_expect_tx(&s_inbar[0], inbox_bytes<G>(NU, nsplit, (int)cluster_ctarank()));
+      mbar_arrive_expect_tx(&s_inbar[1], dry_inbox_bytes<G>(NU, nsplit));
+    }
   }
+  const float qscale = kLog2e / sqrtf((float)D);
+#pragma unroll
+  for (int r = 0; r < kQPer; ++r) {
+    const int i = tid + r * kThreads;
+    if (i < G * D) qs[i / D][i % D] = qv[r] * qscale;
+  }
+  if (kCluster && want_append && tid < 2 * D) s_kvnew[tid / D][tid % D] = kvv;
   __syncthreads();
+  // every CTA's inbox barrier is initialised before any peer pushes into it (the combine
+  // opens with the matching wait)
+  if constexpr (kCluster) cluster_arrive_relaxed();
 
   // per consumer lane: two query-head columns n0 = 2 tig, n1 = 2 tig + 1 of the
   // transposed problem (running max, this lane's share of the sum) and the
@@ -179,12 +217,24 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
   for (int j = 0; j < D / 16; ++j) O[j][0] = O[j][1] = O[j][2] = O[j][3] = 0.f;
 
   if (kCluster && warp == NC + 1) {
-    // ---------------- warm-up: the combine's code, dry, while the others stream ----
-    if constexpr (kCluster)
-      cluster_combine<bf16, D, G, NC>(s_m, s_l, s_acc, qs, &s_cml[0][0], s_new, &s_inbox[1], nsplit,
+    // ---------------- the extra warp, while the others stream: the appended row's
+    // logits (read by the combine), then the combine's code run dry ----------------
+    if constexpr (kCluster) {
+      if (append && L < T_cap) {
+        for (int g = 0; g < G; ++g) {
+          float sp = 0.f;
+          for (int c = lane; c < D; c += 32) sp = fmaf(qs[g][c], to_f32(s_kvnew[0][c]), sp);
+          sp = warp_sum(sp);
+          if (lane == 0) s_new[g] = sp;
+        }
+      }
+      cluster_combine<bf16, D, G, NC>(s_m, s_l, s_acc, s_new, &s_inbox[1], &s_inbar[1], nsplit,
                                       (int)cluster_ctarank(), lane, 32, /*dry=*/true, 0, L, T_cap,
                                       append, K, V, logn, len, s_kvnew[0], s_kvnew[kCluster ? 1 : 0],
                                       reinterpret_cast<bf16*>(&s_inbox[1]), flags);
+      // its pushes into the scratch inbox have all landed before the CTA can leave
+      if (lane == 0 && !mbar_wait(&s_inbar[1], 0)) set_flag(flags, KVS_FLAG_TIMEOUT);
+    }
   } else if (warp == NC) {
     // ---------------- producer: one thread issues every TMA load ----------------
     if (lane == 0) {
@@ -205,20 +255,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     __syncwarp();   // reconverge before the CTA-wide barrier after the main loop
   } else if (warp < NC) {
     // ---------------- consumers: 16 rows of each stage per warp ----------------
-    const int grp = lane >> 2, tig = lane & 3;       // fragment row / column pair
+    const int grp = lane >> 2;                       // fragment row
     const int mi = lane >> 3, ri = lane & 7;         // ldmatrix: matrix index, row in matrix
-    // B operand of S^T = K Q^T: column n = grp holds query head grp (zero past G)
-    uint32_t qb[D / 16][2];
-#pragma unroll
-    for (int ks = 0; ks < D / 16; ++ks) {
-      if (grp < G) {
-        const bf16* qr = q + ((size_t)head * G + grp) * D + ks * 16 + tig * 2;
-        qb[ks][0] = *reinterpret_cast<const uint32_t*>(qr);
-        qb[ks][1] = *reinterpret_cast<const uint32_t*>(qr + 8);
-      } else {
-        qb[ks][0] = qb[ks][1] = 0u;
-      }
-    }
     const int r0 = warp * 16;                        // this warp's rows inside a stage
     const uint32_t ring = smem_u32(base);
     for (int i = 0; i < ntiles; ++i) {
@@ -361,7 +399,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
   const DecodeArgs<bf16> a{head, split, nsplit, L, T_cap, bad, K, V, logn, len, k_new, v_new,
                            out, counters, part, flags};
   if constexpr (kCluster) {
-    cluster_combine<bf16, D, G, NC>(s_m, s_l, s_acc, qs, &s_cml[0][0], s_new, &s_inbox[0], nsplit,
+    cluster_combine<bf16, D, G, NC>(s_m, s_l, s_acc, s_new, &s_inbox[0], &s_inbar[0], nsplit,
                                     (int)cluster_ctarank(), tid, kThreads, /*dry=*/false, head, L,
                                     T_cap, append, K, V, logn, len, s_kvnew[0],
                                     s_kvnew[kCluster ? 1 : 0], out, flags);

@@ -270,6 +270,12 @@ __device__ __forceinline__ void cluster_wait() {
   asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
 }
 
+// The first half of a cluster barrier without ordering of memory (pair it with a fence,
+// e.g. fence_mbar_init, where ordering is wanted).
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");
+}
+
 // Address of the same shared-memory location in the CTA of rank `rank`.
 __device__ __forceinline__ uint32_t cluster_map(uint32_t smem_addr, uint32_t rank) {
   uint32_t r;
@@ -281,6 +287,26 @@ __device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
 }
 __device__ __forceinline__ void st_cluster_f32x2(uint32_t addr, float a, float b) {
   asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(a), "f"(b) : "memory");
+}
+// Asynchronous stores into the shared memory of a CTA of the cluster (`addr` and `mbar`
+// are shared::cluster addresses in the same CTA): on completion each counts its bytes
+// against the transaction count of the mbarrier at `mbar`, so the receiving CTA learns
+// from its own barrier that the data has landed.
+__device__ __forceinline__ void st_async_f32x4(uint32_t addr, float4 v, uint32_t mbar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];"
+      ::"r"(addr), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(mbar)
+      : "memory");
+}
+__device__ __forceinline__ void st_async_f32x2(uint32_t addr, float a, float b, uint32_t mbar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];"
+               ::"r"(addr), "f"(a), "f"(b), "r"(mbar)
+               : "memory");
+}
+__device__ __forceinline__ void st_cluster_f32x4(uint32_t addr, float4 v) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x), "f"(v.y),
+               "f"(v.z), "f"(v.w)
+               : "memory");
 }
 
 // Transpose an 8x8 matrix of 16-bit elements held one row pair per lane (lane l:

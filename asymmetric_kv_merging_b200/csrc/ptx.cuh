@@ -270,6 +270,13 @@ __device__ __forceinline__ void cluster_wait() {
   asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
 }
 
+// Programmatic dependent launch: wait for the preceding grid of the stream to complete
+// (and its memory to be visible); let the next grid of the stream be scheduled.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // The first half of a cluster barrier without ordering of memory (pair it with a fence,
 // e.g. fence_mbar_init, where ordering is wanted).
 __device__ __forceinline__ void cluster_arrive_relaxed() {

@@ -444,71 +444,74 @@ merge_kernel(const T* __restrict__ K, const T* __restrict__ V, const float* __re
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   constexpr int WARPS = kMergeThreads / 32;
   if constexpr (LPR <= 16) {
-    constexpr int PPI = 16 / LPR;                   // pairs per warp iteration
-    const int slot = lane / (2 * LPR), r = (lane / LPR) & 1, c = lane % LPR;
+    // LPR lanes per pair, each holding the same 16-byte slice of both rows of its pair (no
+    // exchange between lanes; every lane of a merged pair computes its slice)
+    constexpr int PPI = 32 / LPR;                   // pairs per warp iteration
+    const int slot = lane / LPR, c = lane % LPR;
     // U warp iterations per batch: every load of the batch is issued before the first is
-    // used, so a warp keeps U times the bytes in flight (one iteration's 32 x 32 bytes
-    // would leave the kernel bound by memory latency)
-    constexpr int U = 4;
-    auto pair_rows = [&](int t, const uint4& kr, const uint4& vr, float lr) {
-      const bool valid = t < nvalid;
+    // used, so that a warp keeps several rows' bytes in flight
+    constexpr int U = 2;
+    auto pair_rows = [&](int t, const uint4& ka_r, const uint4& kb_r, const uint4& va_r,
+                         const uint4& vb_r, float la, float lb) {
+      if (t >= nvalid) return;
       const int p = pbase + t;
-      uint4 kp, vp;
-      kp.x = __shfl_xor_sync(0xffffffffu, kr.x, LPR); kp.y = __shfl_xor_sync(0xffffffffu, kr.y, LPR);
-      kp.z = __shfl_xor_sync(0xffffffffu, kr.z, LPR); kp.w = __shfl_xor_sync(0xffffffffu, kr.w, LPR);
-      vp.x = __shfl_xor_sync(0xffffffffu, vr.x, LPR); vp.y = __shfl_xor_sync(0xffffffffu, vr.y, LPR);
-      vp.z = __shfl_xor_sync(0xffffffffu, vr.z, LPR); vp.w = __shfl_xor_sync(0xffffffffu, vr.w, LPR);
-      const float lp = __shfl_xor_sync(0xffffffffu, lr, LPR);
-      if (!valid) return;
       const int off = s_off[t];
       if (s_sel[t]) {
-        if (r == 0) {
-          float ka[VN], kb[VN], va[VN], vb[VN], ko[VN], vo[VN];
-          load_vec(reinterpret_cast<const T*>(&kr), ka);
-          load_vec(reinterpret_cast<const T*>(&kp), kb);
-          load_vec(reinterpret_cast<const T*>(&vr), va);
-          load_vec(reinterpret_cast<const T*>(&vp), vb);
-          const float w = s_w[t];
-          const float na = expf(lr), nb = expf(lp);
-          const float inv = 1.f / (na + nb);
+        float ka[VN], kb[VN], va[VN], vb[VN], ko[VN], vo[VN];
+        load_vec(reinterpret_cast<const T*>(&ka_r), ka);
+        load_vec(reinterpret_cast<const T*>(&kb_r), kb);
+        load_vec(reinterpret_cast<const T*>(&va_r), va);
+        load_vec(reinterpret_cast<const T*>(&vb_r), vb);
+        const float w = s_w[t];
+        const float na = expf(la), nb = expf(lb);
+        const float inv = 1.f / (na + nb);
 #pragma unroll
-          for (int e = 0; e < VN; ++e) {
-            ko[e] = fmaf(w, kb[e] - ka[e], ka[e]);
-            vo[e] = (na * va[e] + nb * vb[e]) * inv;
-          }
-          store_vec(Ko + (size_t)off * D + c * VN, ko);
-          store_vec(Vo + (size_t)off * D + c * VN, vo);
-          if (c == 0) lno[off] = logf(na + nb);
-          if (dbg_km) {
-            float* dk = dbg_km + ((size_t)head * (T_cap / 2) + p) * D + c * VN;
+        for (int e = 0; e < VN; ++e) {
+          ko[e] = fmaf(w, kb[e] - ka[e], ka[e]);
+          vo[e] = (na * va[e] + nb * vb[e]) * inv;
+        }
+        store_vec(Ko + (size_t)off * D + c * VN, ko);
+        store_vec(Vo + (size_t)off * D + c * VN, vo);
+        if (c == 0) lno[off] = logf(na + nb);
+        if (dbg_km) {
+          float* dk = dbg_km + ((size_t)head * (T_cap / 2) + p) * D + c * VN;
 #pragma unroll
-            for (int e = 0; e < VN; e += 4) *reinterpret_cast<float4*>(dk + e) = make_float4(ko[e], ko[e + 1], ko[e + 2], ko[e + 3]);
-          }
+          for (int e = 0; e < VN; e += 4) *reinterpret_cast<float4*>(dk + e) = make_float4(ko[e], ko[e + 1], ko[e + 2], ko[e + 3]);
         }
       } else {
-        store_raw(Ko + (size_t)(off + r) * D + c * VN, kr);
-        store_raw(Vo + (size_t)(off + r) * D + c * VN, vr);
-        if (c == 0) lno[off + r] = lr;
+        store_raw(Ko + (size_t)off * D + c * VN, ka_r);
+        store_raw(Ko + (size_t)(off + 1) * D + c * VN, kb_r);
+        store_raw(Vo + (size_t)off * D + c * VN, va_r);
+        store_raw(Vo + (size_t)(off + 1) * D + c * VN, vb_r);
+        if (c == 0) {
+          lno[off] = la;
+          lno[off + 1] = lb;
+        }
       }
     };
     for (int base0 = warp * PPI; base0 < nvalid; base0 += WARPS * PPI * U) {
-      uint4 krs[U], vrs[U];
-      float lrs[U];
+      uint4 kas[U], kbs[U], vas[U], vbs[U];
+      float las[U], lbs[U];
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int t = base0 + u * WARPS * PPI + slot;
-        krs[u] = make_uint4(0, 0, 0, 0);
-        vrs[u] = make_uint4(0, 0, 0, 0);
-        lrs[u] = 0.f;
+        kas[u] = kbs[u] = vas[u] = vbs[u] = make_uint4(0, 0, 0, 0);
+        las[u] = lbs[u] = 0.f;
         if (t < nvalid) {
-          const int row = c0 + 2 * (pbase + t) + r;
-          krs[u] = load_raw(Kh + (size_t)row * D + c * VN);
-          vrs[u] = load_raw(Vh + (size_t)row * D + c * VN);
-          lrs[u] = lnh ? lnh[row] : 0.f;
+          const int row = c0 + 2 * (pbase + t);
+          kas[u] = load_raw(Kh + (size_t)row * D + c * VN);
+          kbs[u] = load_raw(Kh + (size_t)(row + 1) * D + c * VN);
+          vas[u] = load_raw(Vh + (size_t)row * D + c * VN);
+          vbs[u] = load_raw(Vh + (size_t)(row + 1) * D + c * VN);
+          if (lnh) {
+            las[u] = lnh[row];
+            lbs[u] = lnh[row + 1];
+          }
         }
       }
 #pragma unroll
-      for (int u = 0; u < U; ++u) pair_rows(base0 + u * WARPS * PPI + slot, krs[u], vrs[u], lrs[u]);
+      for (int u = 0; u < U; ++u)
+        pair_rows(base0 + u * WARPS * PPI + slot, kas[u], kbs[u], vas[u], vbs[u], las[u], lbs[u]);
     }
   } else {
     // LPR == 32: one lane holds the same 16-byte slice of both rows.

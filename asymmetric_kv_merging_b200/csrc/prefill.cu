@@ -32,20 +32,36 @@ append_rows_kernel(T* __restrict__ K, T* __restrict__ V, float* __restrict__ log
   const int head = blockIdx.y;
   const int r0 = blockIdx.x * kAppendRowsPerBlock;
   const int r1 = min(n, r0 + kAppendRowsPerBlock);
+  // this thread's vectors of the new rows are loaded together with the length check (the
+  // loads do not depend on it), so the block waits one round trip, not one per vector
+  constexpr int kPer = (kAppendRowsPerBlock * VPR + kAppendThreads - 1) / kAppendThreads;
+  const uint4* ks = reinterpret_cast<const uint4*>(k_rows + ((size_t)head * n + r0) * D);
+  const uint4* vs = reinterpret_cast<const uint4*>(v_rows + ((size_t)head * n + r0) * D);
+  const int nv = (r1 - r0) * VPR;
+  uint4 kv[kPer], vv[kPer];
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    const int i = threadIdx.x + j * kAppendThreads;
+    if (i < nv) {
+      kv[j] = __ldcs(ks + i);
+      vv[j] = __ldcs(vs + i);
+    }
+  }
   if (threadIdx.x == 0) {
     s_ok = (len[head] == L);
     if (!s_ok && blockIdx.x == 0) set_flag(flags, KVS_FLAG_BAD_LENGTH);
   }
   __syncthreads();
   if (!s_ok) return;                                // the whole head is left as it is
-  const uint4* ks = reinterpret_cast<const uint4*>(k_rows + ((size_t)head * n + r0) * D);
-  const uint4* vs = reinterpret_cast<const uint4*>(v_rows + ((size_t)head * n + r0) * D);
   uint4* kd = reinterpret_cast<uint4*>(K + ((size_t)head * T_cap + L + r0) * D);
   uint4* vd = reinterpret_cast<uint4*>(V + ((size_t)head * T_cap + L + r0) * D);
-  const int nv = (r1 - r0) * VPR;
-  for (int i = threadIdx.x; i < nv; i += kAppendThreads) {
-    kd[i] = __ldcs(ks + i);
-    vd[i] = __ldcs(vs + i);
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    const int i = threadIdx.x + j * kAppendThreads;
+    if (i < nv) {
+      kd[i] = kv[j];
+      vd[i] = vv[j];
+    }
   }
   if (logn)
     for (int r = r0 + threadIdx.x; r < r1; r += kAppendThreads)

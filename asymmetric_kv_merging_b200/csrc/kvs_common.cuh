@@ -21,6 +21,27 @@ typedef __nv_bfloat16 bf16;
 // Host-side count of kernel launches (see kvs_launch_count).
 void count_launches(int n);
 
+// Launch with programmatic stream serialisation: the grid may be scheduled while the
+// previous kernel of the stream is still running, so the kernel must execute
+// griddepcontrol.wait (griddep_wait) before its first access to memory that earlier work
+// writes -- the kernels launched this way do so first thing -- and it triggers its own
+// dependents right after. Returns the launch's error.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kfn)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kfn, static_cast<Args&&>(args)...);
+}
+
 __host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Elements of T that fit one 16-byte vector.

@@ -73,6 +73,10 @@ select_kernel(const float* __restrict__ score, const int32_t* __restrict__ len,
               const int32_t* __restrict__ target, int scope, int H_kv, int T_cap, int nblk,
               SelUnit* __restrict__ sel, HeadInfo* __restrict__ hinfo, int2* __restrict__ blk,
               int32_t* __restrict__ flags) {
+  // launched with programmatic stream serialisation: wait for the preceding grid (and its
+  // memory) before any access, then let the next grid be scheduled
+  griddep_wait();
+  griddep_launch_dependents();
   __shared__ int hist[4096];
   __shared__ uint32_t cand[kSelCand];
   __shared__ int warp_tot[33];
@@ -382,6 +386,10 @@ merge_kernel(const T* __restrict__ K, const T* __restrict__ V, const float* __re
              int32_t* __restrict__ len_out, uint8_t* __restrict__ dbg_sel,
              int32_t* __restrict__ dbg_off, float* __restrict__ dbg_km,
              int32_t* __restrict__ flags) {
+  // launched with programmatic stream serialisation: wait for the preceding grid (and its
+  // memory) before any access, then let the next grid be scheduled
+  griddep_wait();
+  griddep_launch_dependents();
   constexpr int MB = kMergePairsPerBlock;
   constexpr int VN = Vec16<T>::n;
   constexpr int LPR = D / VN;
@@ -765,12 +773,13 @@ cudaError_t launch_select(const kvs_cache_desc& d, const float* score, const int
                           const int32_t* cand_begin, int n_recent, const int32_t* target,
                           int scope, const MergeLayout& Ly, char* ws, cudaStream_t st) {
   const int units = scope == KVS_SCOPE_POOLED ? d.B : d.B * d.H_kv;
-  select_kernel<<<units, kSelThreads, 0, st>>>(
-      score, len, cand_begin, n_recent, target, scope, d.H_kv, d.T_cap, Ly.nblk,
-      reinterpret_cast<SelUnit*>(ws + Ly.sel), reinterpret_cast<HeadInfo*>(ws + Ly.head),
-      reinterpret_cast<int2*>(ws + Ly.blk), reinterpret_cast<int32_t*>(ws));
+  const cudaError_t e = launch_pdl(
+      select_kernel, dim3(units), dim3(kSelThreads), 0, st, score, len, cand_begin, n_recent,
+      target, scope, d.H_kv, d.T_cap, Ly.nblk, reinterpret_cast<SelUnit*>(ws + Ly.sel),
+      reinterpret_cast<HeadInfo*>(ws + Ly.head), reinterpret_cast<int2*>(ws + Ly.blk),
+      reinterpret_cast<int32_t*>(ws));
   count_launches(1);
-  return cudaGetLastError();
+  return e;
 }
 
 template <typename T, int D>
@@ -802,11 +811,12 @@ static cudaError_t launch_merge_t(const kvs_cache_desc& d, const void* K, const 
   }
   const int ncopy = (d.T_cap + kCopyRows - 1) / kCopyRows;
   dim3 grid(Ly.nblk + ncopy, heads);
-  merge_kernel<T, D><<<grid, kMergeThreads, 0, st>>>(
-      (const T*)K, (const T*)V, logn, score, w_b, scope, d.H_kv, d.T_cap, T_cap_out, Ly.nblk,
-      sel, hinfo, blk, (T*)K_out, (T*)V_out, logn_out, len_out, dbg_sel, dbg_off, dbg_km, flags);
+  const cudaError_t e = launch_pdl(
+      merge_kernel<T, D>, grid, dim3(kMergeThreads), 0, st, (const T*)K, (const T*)V, logn, score,
+      w_b, scope, d.H_kv, d.T_cap, T_cap_out, Ly.nblk, sel, hinfo, blk, (T*)K_out, (T*)V_out,
+      logn_out, len_out, dbg_sel, dbg_off, dbg_km, flags);
   count_launches(1);
-  return cudaGetLastError();
+  return e;
 }
 
 cudaError_t launch_merge(const kvs_cache_desc& d, const void* K, const void* V, const float* logn,

@@ -185,6 +185,9 @@ kvs_status kvs_score_pairs_form(const kvs_cache_desc* desc, const void* K, const
  *      dbg_out_offset [B,H_kv,T_cap/2] i32 (output row of the pair's first row);
  *      dbg_kmerged_f32 [B,H_kv,T_cap/2,d] fp32 (merged key before rounding).
  * Workspace: kvs_workspace_size(desc, 0, KVS_OP_MERGE) bytes.
+ * The selection and the out-of-place merge kernels are launched with programmatic
+ * stream serialisation; each waits for the preceding kernel's completion and memory
+ * before any access, so the call keeps plain stream order.
  */
 kvs_status kvs_merge_compact(const kvs_cache_desc* desc, const void* K, const void* V,
                              const float* logn, const int32_t* len, const int32_t* cand_begin,
@@ -264,6 +267,9 @@ kvs_status kvs_plan_rounds(int32_t len, int32_t target, int32_t cand_begin, int3
  * outside any stream capture. Launch shape: one thread-block cluster per KV head that
  * combines the head's splits in distributed shared memory, when every head's cluster
  * fits the GPU at once; else a grid of splits combined by the last one to finish.
+ * The kernel is launched with programmatic stream serialisation: it may be scheduled
+ * while the previous kernel of the stream runs, but it waits for that kernel's
+ * completion and memory before any access, so the call keeps plain stream order.
  */
 kvs_status kvs_decode_attn(const kvs_cache_desc* desc, const void* q, void* K, void* V,
                            float* logn, int32_t* len, const void* k_new, const void* v_new,
